@@ -1,0 +1,379 @@
+"""Pins of the CPU oracle against things other than itself.
+
+Library routines (scipy's Hadamard), closed forms, invariants that the
+definitions force, brute force on tiny inputs and hand-derived fixtures under
+tests/golden/.  Each test names the plausible oracle mistake it would catch.
+"""
+
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.linalg
+
+from oracle import kvq_oracle as o
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def outlier_tile(rng, t, d=128, n_out=4, mult=20.0):
+    x = rng.standard_normal((t, d))
+    ch = rng.choice(d, size=n_out, replace=False)
+    x[:, ch] *= mult
+    return x.astype(np.float16)
+
+
+# --------------------------------------------------------------------------- Hadamard
+
+@pytest.mark.parametrize("d", [2, 4, 8, 16, 32, 64, 128])
+def test_hadamard_equals_scipy(d):
+    # wrong recursion / order / sign -> differs from the library matrix
+    h = o.sylvester_hadamard(d)
+    np.testing.assert_array_equal(np.rint(h * math.sqrt(d)), scipy.linalg.hadamard(d))
+
+
+def test_hadamard_popcount_closed_form():
+    h = o.sylvester_hadamard(128) * math.sqrt(128)
+    for j, k in itertools.product(range(0, 128, 7), range(128)):
+        assert h[j, k] == (-1) ** bin(j & k).count("1")
+
+
+def test_hadamard_orthonormal_symmetric():
+    h = o.sylvester_hadamard(128)
+    np.testing.assert_allclose(h @ h, np.eye(128), atol=1e-13)
+    np.testing.assert_array_equal(h, h.T)
+
+
+def test_rotation_side_and_norm():
+    # X' = X H acts on token rows: row e_k maps to row k of H; e_0 maps to
+    # the constant vector 1/sqrt(d); norms are preserved.
+    h = o.sylvester_hadamard(128)
+    for k in (0, 1, 37, 127):
+        e = np.zeros((1, 128))
+        e[0, k] = 1.0
+        np.testing.assert_allclose(o.rotate(e)[0], h[k], atol=0)
+    np.testing.assert_allclose(o.rotate(np.eye(1, 128))[0], np.full(128, 1 / math.sqrt(128)), atol=1e-15)
+    x = np.random.default_rng(1).standard_normal((64, 128))
+    np.testing.assert_allclose(np.linalg.norm(o.rotate(x), axis=1), np.linalg.norm(x, axis=1), rtol=1e-13)
+
+
+# --------------------------------------------------------------------------- normalization
+
+def pop_std(a, axis):
+    m = a.mean(axis=axis, keepdims=True)
+    return np.sqrt(((a - m) ** 2).mean(axis=axis))
+
+
+@pytest.mark.parametrize("iters", [1, 2, 3, 8])
+def test_rows_unit_std_after_token_step(iters):
+    # channel step first, token step last; ddof 0.  A swapped order, ddof 1
+    # or a dropped division leaves some row std away from 1.
+    rng = np.random.default_rng(10 + iters)
+    xr = o.rotate(outlier_tile(rng, 64))
+    y, c, r = o.sinkhorn_normalize(xr, iters)
+    np.testing.assert_allclose(pop_std(y, 1), 1.0, rtol=1e-12)
+
+
+def test_reconstruction_identity():
+    # Y_ij R_i C_j == X'_ij: catches C / R accumulated by division or on the wrong axis
+    rng = np.random.default_rng(3)
+    xr = o.rotate(outlier_tile(rng, 64))
+    y, c, r = o.sinkhorn_normalize(xr, 5)
+    np.testing.assert_allclose(y * r[:, None] * c[None, :], xr, rtol=1e-12, atol=1e-12)
+
+
+def test_energy_identity_of_channel_stds():
+    # After a token step every row has unit std, so summing squares by rows
+    # and by columns gives mean_j sigma_j^2 = 1 + mean_i mu_i^2 - mean_j nu_j^2
+    # (mu = row means, nu = column means).  A wrong axis or ddof breaks it.
+    rng = np.random.default_rng(4)
+    for t in (32, 64, 128):
+        y, _, _ = o.sinkhorn_normalize(o.rotate(outlier_tile(rng, t)), 3)
+        mu = y.mean(axis=1)
+        nu = y.mean(axis=0)
+        lhs = (pop_std(y, 0) ** 2).mean()
+        rhs = 1.0 + (mu ** 2).mean() - (nu ** 2).mean()
+        assert abs(lhs - rhs) < 1e-12
+
+
+@pytest.mark.parametrize("t", [32, 64, 128])
+def test_channel_variances_equalized_at_large_n(t):
+    # The method equalizes the channels' variances.  With the centred std the
+    # fixed point has one common channel std (not necessarily 1, see the
+    # energy identity); at n = 32 they agree to 1e-3.
+    rng = np.random.default_rng(20 + t)
+    y, _, _ = o.sinkhorn_normalize(o.rotate(outlier_tile(rng, t)), 32)
+    s = pop_std(y, 0)
+    assert s.max() / s.min() - 1.0 < 1e-3
+    # For plain N(0,1) tiles the common value sits next to 1.
+    x = rng.standard_normal((t, 128)).astype(np.float16)
+    y, _, _ = o.sinkhorn_normalize(o.rotate(x), 32)
+    s = pop_std(y, 0)
+    assert s.max() / s.min() - 1.0 < 1e-3
+    assert abs(s.mean() - 1.0) < 0.02
+
+
+def test_clamp_on_zero_variance_channel():
+    # Tile whose rotated image is k_i * sqrt(d)/2 * (e0 + e1), k_i = 1..64:
+    # channels 2..127 are exactly zero, so the first channel step clamps them
+    # to sigma = eps while channels 0, 1 get the closed-form std
+    # std(1..64) * sqrt(d)/2 = sqrt((64^2 - 1)/12) * sqrt(128)/2.
+    d = 128
+    h = o.sylvester_hadamard(d)
+    v = (h[:, 0] + h[:, 1]) * math.sqrt(d) / 2   # entries in {0, 1}
+    k = np.arange(1, 65, dtype=np.float64)
+    x = (k[:, None] * v[None, :])                  # exact integers in fp16
+    xr = o.rotate(x)
+    assert not xr[:, 2:].any()
+    y, c, r = o.sinkhorn_normalize(xr, 1)
+    sigma0 = math.sqrt((64 ** 2 - 1) / 12) * math.sqrt(d) / 2
+    np.testing.assert_allclose(c[2:] / c[0], 1e-6 / sigma0, rtol=1e-12)
+    np.testing.assert_allclose(c[1], c[0], rtol=0)
+
+
+def test_renormalization_keeps_metadata_finite():
+    # degenerate tiles: all zero, and 64 identical tokens (every rotated
+    # channel is constant over the tile, so the clamp fires on every channel in
+    # every iteration).  max C stays in [1, 2), the metadata stays finite, the
+    # zero tile comes back exactly and the constant tile as well as 4-bit RTN
+    # of its one row allows.
+    rng = np.random.default_rng(14)
+    row = rng.standard_normal(128).astype(np.float16)
+    for x in (np.zeros((64, 128), np.float16), np.tile(row, (64, 1))):
+        for n in (1, 2, 8):
+            for dt in (np.float64, np.float32):
+                q = o.quantize_tile(x, 4, n, dtype=dt, return_parts=True)
+                assert 1.0 <= q["c"].max() < 2.0
+                for key in ("s_t", "z_t", "c_t"):
+                    assert np.all(np.isfinite(q[key]))
+                _, xh = o.dequantize_tile(q["codes"], q["s_t"], q["z_t"], q["c_t"])
+                ref = x.astype(np.float64)
+                if not ref.any():
+                    assert not xh.any()
+                else:
+                    assert np.linalg.norm(xh - ref) / np.linalg.norm(ref) < 0.15
+                    np.testing.assert_allclose(xh, xh[:1].repeat(64, 0), rtol=0, atol=0)
+
+
+def test_scale_equivariance():
+    # X -> 2^k X (exact in fp16): codes and C~ unchanged (C is renormalized to
+    # max in [1, 2)), s~ and z~ scaled by 2^k
+    rng = np.random.default_rng(5)
+    x = outlier_tile(rng, 64, mult=5.0)
+    a = o.quantize_tile(x, 4, 4)
+    b = o.quantize_tile((x.astype(np.float32) * 4).astype(np.float16), 4, 4)
+    np.testing.assert_array_equal(a["codes"], b["codes"])
+    np.testing.assert_array_equal(a["c_t"], b["c_t"])
+    np.testing.assert_array_equal(a["s_t"].astype(np.float32) * 4, b["s_t"].astype(np.float32))
+    np.testing.assert_array_equal(a["z_t"].astype(np.float32) * 4, b["z_t"].astype(np.float32))
+
+
+def test_token_permutation_equivariance():
+    rng = np.random.default_rng(6)
+    x = outlier_tile(rng, 64)
+    perm = rng.permutation(64)
+    a = o.quantize_tile(x, 4, 4)
+    b = o.quantize_tile(x[perm], 4, 4)
+    np.testing.assert_array_equal(a["codes"][perm], b["codes"])
+    np.testing.assert_array_equal(a["s_t"][perm], b["s_t"])
+    np.testing.assert_array_equal(a["c_t"], b["c_t"])
+
+
+# --------------------------------------------------------------------------- RTN
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_rtn_brute_force_and_bounds(bits):
+    # brute force: each code is the nearest grid point c*s + z (fp64, no ties);
+    # min row entry -> 0, max -> 2^b - 1, error <= s/2, codes in range.
+    rng = np.random.default_rng(30 + bits)
+    y = rng.standard_normal((16, 128)) * rng.uniform(0.1, 3, size=(16, 1))
+    codes, s, z = o.asymmetric_rtn(y, bits)
+    qmax = (1 << bits) - 1
+    grid = np.arange(qmax + 1)[None, None, :] * s[:, None, None] + z[:, None, None]
+    brute = np.abs(y[:, :, None] - grid).argmin(axis=2)
+    np.testing.assert_array_equal(codes, brute)
+    assert codes.max() <= qmax
+    np.testing.assert_array_equal(codes[np.arange(16), y.argmin(1)], 0)
+    np.testing.assert_array_equal(codes[np.arange(16), y.argmax(1)], qmax)
+    err = np.abs(y - (codes * s[:, None] + z[:, None]))
+    assert np.all(err <= s[:, None] / 2 * (1 + 1e-12))
+
+
+def test_rtn_golden_rows():
+    # hand-derived rows, tests/golden/rtn_worked_examples.txt
+    path = os.path.join(GOLDEN, "rtn_worked_examples.txt")
+    cases = []
+    with open(path) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            bits, vals, codes = line.split("|")
+            cases.append((int(bits), [float(v) for v in vals.split()], [int(c) for c in codes.split()]))
+    assert cases
+    for bits, vals, want in cases:
+        codes, s, z = o.asymmetric_rtn(np.array([vals]), bits)
+        assert codes[0].tolist() == want, (bits, vals)
+
+
+def test_constant_row_gives_zero_scale():
+    y = np.full((2, 128), 0.75)
+    codes, s, z = o.asymmetric_rtn(y, 4)
+    assert np.all(codes == 0) and np.all(s == 0) and np.all(z == 0.75)
+
+
+# --------------------------------------------------------------------------- tile quantizer
+
+@pytest.mark.parametrize("t,bits,iters", [(32, 2, 1), (64, 4, 4), (128, 3, 8), (64, 2, 0)])
+def test_dequantized_tile_within_half_step(t, bits, iters):
+    # X^' - X' is bounded by (s/2) R_i C_j plus the fp16 rounding of the
+    # metadata; a missing R or C factor in s~, z~ or C~ breaks it by orders of magnitude.
+    rng = np.random.default_rng(40 + t + bits)
+    x = outlier_tile(rng, t)
+    q = o.quantize_tile(x, bits, iters, return_parts=True)
+    xr_hat, x_hat = o.dequantize_tile(q["codes"], q["s_t"], q["z_t"], q["c_t"])
+    half = (q["s"] * q["r"])[:, None] * q["c"][None, :] / 2
+    fp16_slack = 2.0 ** -10 * (np.abs(q["xr"]) + (q["s"] * q["r"])[:, None] * q["c"][None, :] * ((1 << bits) - 1))
+    assert np.all(np.abs(xr_hat - q["xr"]) <= half + 3 * fp16_slack)
+    # original domain: the inverse rotation is exact up to rounding
+    np.testing.assert_allclose(x_hat, xr_hat @ o.sylvester_hadamard(128), rtol=0, atol=1e-12)
+    err = np.linalg.norm(x_hat - x.astype(np.float64)) / np.linalg.norm(x.astype(np.float64))
+    assert err < {2: 0.7, 3: 0.3, 4: 0.15}[bits]
+
+
+@pytest.mark.parametrize("t,bits,iters", [(t, b, n) for t in (32, 64, 128) for b in (2, 3, 4) for n in (1, 4, 8)])
+def test_method_beats_plain_rtn_on_outliers(t, bits, iters):
+    # the method's point: lower reconstruction MSE than plain per-token RTN
+    rng = np.random.default_rng(1000 + 7 * t + 3 * bits + iters)
+    d = 128
+    x = rng.standard_normal((t, d))
+    k = max(1, round(rng.uniform(0.01, 0.05) * d))
+    ch = rng.choice(d, size=k, replace=False)
+    x[:, ch] *= np.exp(rng.uniform(np.log(5), np.log(50), size=k))
+    x = x.astype(np.float16)
+    q = o.quantize_tile(x, bits, iters)
+    _, x_hat = o.dequantize_tile(q["codes"], q["s_t"], q["z_t"], q["c_t"])
+    ref = x.astype(np.float64)
+    mse_method = ((x_hat - ref) ** 2).mean()
+    mse_plain = ((o.plain_rtn_baseline(x, bits) - ref) ** 2).mean()
+    assert mse_method < mse_plain
+
+
+def test_float32_mode_agrees_with_fp64():
+    # the parity tests run the quantizer in float32 (the GPU's precision for
+    # the code decision); it must agree with fp64 except at rare near-ties
+    rng = np.random.default_rng(8)
+    x = outlier_tile(rng, 64)
+    a = o.quantize_tile(x, 4, 4)
+    b = o.quantize_tile(x, 4, 4, dtype=np.float32)
+    diff = a["codes"].astype(int) - b["codes"].astype(int)
+    assert np.abs(diff).max() <= 1 and (diff != 0).mean() < 1e-3
+
+
+# --------------------------------------------------------------------------- format
+
+@pytest.mark.parametrize("bits,is_v", [(2, False), (3, False), (4, False), (2, True), (3, True), (4, True)])
+def test_code_positions_are_a_bijection(bits, is_v):
+    pos = sorted(o.code_bit_position(c, p, bits, is_v) for p in range(16) for c in range(128))
+    assert pos == list(range(0, 16 * 128 * bits, bits))
+
+
+def test_layout_sizes_hand_computed():
+    # K, T=64, b=4: 16*128*4/8 = 1024 codes + 64 meta + 32 channels*2 B = 1152
+    assert o.page_layout(4, 64)["page_bytes"] == 1152
+    # V, T=128, b=2: 512 + 64 + 16*2 = 608;  T=32, b=3: 768 + 64 + 64*2 = 960
+    assert o.page_layout(2, 128)["page_bytes"] == 608
+    assert o.page_layout(3, 32)["page_bytes"] == 960
+    assert o.page_layout(4, 64)["cslice_channels"] == 32
+
+
+def test_code_positions_golden():
+    # hand-derived positions from the written layout, tests/golden/format_positions.txt
+    path = os.path.join(GOLDEN, "format_positions.txt")
+    n = 0
+    with open(path) as f:
+        for line in f:
+            line = line.split("#")[0].strip()
+            if not line:
+                continue
+            kind, bits, ch, tok, want = line.split()
+            got = o.code_bit_position(int(ch), int(tok), int(bits), kind == "V")
+            assert got == int(want), line
+            n += 1
+    assert n >= 8
+
+
+@pytest.mark.parametrize("bits,is_v", [(2, True), (4, True), (3, False), (4, False)])
+def test_pack_unpack_roundtrip(bits, is_v):
+    rng = np.random.default_rng(bits + 10 * is_v)
+    codes = rng.integers(0, 1 << bits, size=(16, 128)).astype(np.uint8)
+    region = o.pack_page_codes(codes, bits, is_v)
+    assert region.size == 16 * 128 * bits // 8
+    np.testing.assert_array_equal(o.unpack_page_codes(region, bits, is_v), codes)
+
+
+def test_tile_pages_roundtrip():
+    rng = np.random.default_rng(9)
+    x = outlier_tile(rng, 64)
+    q = o.quantize_tile(x, 4, 2)
+    lay = o.page_layout(4, 64)
+    pool = np.zeros((10, 2, lay["page_bytes"]), dtype=np.uint8)
+    blocks = [7, 2, 9, 0]
+    o.write_tile_pages(pool, blocks, 1, q, 4, 64, True)
+    back = o.read_tile_pages(pool, blocks, 1, 4, 64, True)
+    for key in ("codes", "s_t", "z_t", "c_t"):
+        np.testing.assert_array_equal(back[key], q[key])
+    assert not pool[:, 0].any()
+
+
+# --------------------------------------------------------------------------- decode
+
+def brute_attention(q, k, v, scale):
+    # pure-Python loops, tiny sizes only
+    logits = [scale * sum(q[j] * k[i][j] for j in range(len(q))) for i in range(len(k))]
+    m = max(logits)
+    w = [math.exp(a - m) for a in logits]
+    tot = sum(w)
+    return [sum(w[i] * v[i][j] for i in range(len(k))) / tot for j in range(len(q))]
+
+
+def test_attention_brute_force():
+    rng = np.random.default_rng(11)
+    q = rng.standard_normal(128)
+    k = rng.standard_normal((9, 128))
+    v = rng.standard_normal((9, 128))
+    want = brute_attention(q.tolist(), k.tolist(), v.tolist(), 1 / math.sqrt(128))
+    np.testing.assert_allclose(o.attention_fp64(q, k, v), want, rtol=1e-12, atol=1e-14)
+
+
+def test_attention_special_cases():
+    rng = np.random.default_rng(12)
+    k = rng.standard_normal((5, 128))
+    v = rng.standard_normal((5, 128))
+    np.testing.assert_allclose(o.attention_fp64(rng.standard_normal(128), k[:1], v[:1]), v[0], rtol=1e-15)
+    np.testing.assert_allclose(o.attention_fp64(np.zeros(128), k, v), v.mean(axis=0), rtol=1e-13)
+
+
+def test_decode_gqa_mapping_and_tail():
+    # query head h reads KV head h // g; the raw tail follows the tiles
+    rng = np.random.default_rng(13)
+    g, hkv, t = 4, 2, 32
+    rows_k = [rng.standard_normal((t + 3, 128)).astype(np.float16) for _ in range(hkv)]
+    rows_v = [(float(4 * h) + rng.standard_normal((t + 3, 128))).astype(np.float16) for h in range(hkv)]
+    k_hat, v_hat = [], []
+    for h in range(hkv):
+        tk, tail_k = o.quantize_sequence(rows_k[h], t, 4, 2)
+        tv, tail_v = o.quantize_sequence(rows_v[h], t, 4, 2)
+        assert tail_k.shape[0] == 3
+        k_hat.append(o.sequence_kv_hat(tk, tail_k))
+        v_hat.append(o.sequence_kv_hat(tv, tail_v))
+        assert k_hat[-1].shape == (t + 3, 128)
+        np.testing.assert_array_equal(k_hat[-1][t:], rows_k[h][t:].astype(np.float64))
+    qh = rng.standard_normal((g * hkv, 128))
+    out = o.decode_sequence(qh, k_hat, v_hat, g)
+    for h in range(g * hkv):
+        # KV head 1's values sit near 4, KV head 0's near 0
+        assert abs(out[h].mean() - 4.0 * (h // g)) < 0.6
+        np.testing.assert_array_equal(out[h], o.attention_fp64(qh[h], k_hat[h // g], v_hat[h // g]))
