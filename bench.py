@@ -1,0 +1,463 @@
+#!/usr/bin/env python
+"""Benchmark of the quantized paged KV-cache hot path on B200.
+
+One step = one pass of the whole path over one batch of the Qwen3-4B-shaped
+workload (6 sequences x 131072 cached tokens, 8 KV heads, 32 query heads,
+d=128, T=64, 4-bit K and V, n=4):
+  1. kvq_quantize_tiles   every full tile of the batch (rotation,
+                          normalization, RTN, packing into scattered pages)
+  2. kvq_append_tokens    the step's new token per sequence (fp16 tail)
+  3. kvq_paged_decode_attention  one decode query per sequence over the
+                          packed pages plus the tail (split-K + merge)
+``value`` is the step's algorithmic bytes (what the method must move: fp16
+rows read and packed pages written by 1, tail rows by 2, packed pages,
+tables, tail, q and out by 3) per second over the timed steps; the
+``decode`` and ``quantize`` objects break it down per call (CUDA events on
+the launching stream).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kvq|reference]
+
+Under torchrun each rank runs an independent replica batch (weak scaling,
+no data-path collective); rank 0 prints one JSON line.  ``--impl
+reference`` times the CPU oracle on a bounded sample of the same workload
+(rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import multiprocessing as mp
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+METRIC = "paged decode attn GB/s & tok/s over quantized KV (% HBM peak); quantize GB/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# --------------------------------------------------------------------------- helpers
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_digest() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "quantized_paged_kv_tile_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, units_now: float):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, scaled
+    to this launch's units, or None when the kernel changed since the capture."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)[kernel]
+    except (OSError, KeyError, ValueError):
+        return None
+    if rec.get("source_digest") != source_digest():
+        return None
+    return rec["dram_bytes_per_launch"] * units_now / rec["units_per_launch"]
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.gpu = gpu_index
+        self.path = os.path.join("/tmp", f"kvq_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.out, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        load = [s for s in sm if s > 0.5 * max(sm)] if sm else []
+        return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def byte_model(w, cfg_layout_k, cfg_layout_v):
+    """Algorithmic bytes of one step (see the module docstring)."""
+    d, t, p, h = 128, w.tile_tokens, 16, w.num_kv_heads
+    lens0 = np.asarray(w.lens, dtype=np.int64)
+    per_tok_head = d * (w.bits_k + w.bits_v) / 8 + 8 + 4 * d / t   # codes + meta + C slices, K+V
+    full0 = (lens0 // t) * t
+    quant = float(full0.sum()) * h * (2 * d * 2 + per_tok_head)
+    rest = lens0 - full0 + w.append_tokens
+    append = float(rest.sum()) * h * d * 2 * 2 * 2
+    lens1 = lens0 + w.append_tokens
+    full1 = (lens1 // t) * t
+    tau1 = lens1 - full1
+    decode = (float(full1.sum()) * h * per_tok_head + float(full1.sum()) // p * 4
+              + float(tau1.sum()) * h * d * 2 * 2 + w.num_seqs * w.num_q_heads * d * 2 * 2)
+    return {"quantize": quant, "append": append, "decode": decode, "kv_tokens": float(lens1.sum()),
+            "quant_units": float(full0.sum()) * h * 2 * d}
+
+
+# --------------------------------------------------------------------------- oracle sample
+
+def _oracle_pair(task):
+    """One (sequence, KV head) of the workload through the oracle: quantize
+    its K and V tiles, dequantize, decode its query group.  Returns bytes."""
+    wname, overrides, head, seq = task
+    from threadpoolctl import threadpool_limits
+    sys.path.insert(0, ROOT)
+    from oracle import kvq_oracle as o
+    from quantized_paged_kv_tile_b200 import synth
+    w = synth.workload(wname, **overrides)
+    L0 = w.lens[seq]
+    L1 = L0 + w.append_tokens
+    with threadpool_limits(1):
+        rk = synth.kv_rows_one_head(w, "k", L1, head, stream_id=seq)
+        rv = synth.kv_rows_one_head(w, "v", L1, head, stream_id=seq)
+        tk, tail_k = o.quantize_sequence(rk, w.tile_tokens, w.bits_k, w.iters)
+        tv, tail_v = o.quantize_sequence(rv, w.tile_tokens, w.bits_v, w.iters)
+        kh, vh = o.sequence_kv_hat(tk, tail_k), o.sequence_kv_hat(tv, tail_v)
+        q = np.random.default_rng(seq * 131 + head).standard_normal((w.group_size, 128))
+        o.decode_sequence(q, [kh], [vh], w.group_size)
+    return 0
+
+
+def _warm(_):
+    sys.path.insert(0, ROOT)
+    import oracle.kvq_oracle  # noqa: F401
+    import quantized_paged_kv_tile_b200.synth  # noqa: F401
+    return 0
+
+
+class OraclePool:
+    """Spawned worker processes (safe after CUDA init) running oracle pairs."""
+
+    def __init__(self, procs):
+        self.procs = procs
+        self.pool = mp.get_context("spawn").Pool(procs)
+        self.pool.map(_warm, range(procs))
+
+    def time(self, wname, overrides, pairs):
+        tasks = [(wname, overrides, h, s) for (s, h) in pairs]
+        t0 = time.perf_counter()
+        self.pool.map(_oracle_pair, tasks, chunksize=1)
+        return time.perf_counter() - t0
+
+    def close(self):
+        self.pool.close()
+        self.pool.join()
+
+
+def oracle_pairs(w, n):
+    return [(i % w.num_seqs, (i // w.num_seqs) % w.num_kv_heads) for i in range(n)]
+
+
+def cpu_sample_bytes(w, bm, n_pairs):
+    return (bm["quantize"] + bm["append"] + bm["decode"]) * n_pairs / (w.num_seqs * w.num_kv_heads)
+
+
+# --------------------------------------------------------------------------- GPU arm
+
+def run_kvq(args, ranks):
+    import torch
+    from quantized_paged_kv_tile_b200 import build, kvq, synth
+
+    build.build()
+    kvq.load_library()
+    dev = torch.device("cuda", ranks.local_rank)
+    torch.cuda.set_device(dev)
+    w = synth.workload(args.workload, replica=ranks.rank)
+    cfg = kvq.Config(num_kv_heads=w.num_kv_heads, group_size=w.group_size, tile_tokens=w.tile_tokens,
+                     bits_k=w.bits_k, bits_v=w.bits_v, iters=w.iters)
+    lay = kvq.get_layout(cfg)
+    B, H, T = w.num_seqs, w.num_kv_heads, w.tile_tokens
+    lens0 = np.asarray(w.lens, dtype=np.int64)
+    lens1 = lens0 + w.append_tokens
+    bps = int(math.ceil(lens1.max() / 16))
+    bt_np = synth.block_table(w, bps)
+    nblocks = int(bt_np.max()) + 1
+    bt = torch.from_numpy(bt_np).to(dev)
+    total0 = int(lens0.sum())
+    rows_k = synth.kv_rows(w, "k", total0, device=dev)
+    rows_v = synth.kv_rows(w, "v", total0, device=dev)
+    starts = np.concatenate([[0], np.cumsum(lens0)[:-1]])
+    full0 = (lens0 // T) * T
+    desc_np = np.asarray([(starts[s] + i * T, s, i) for s in range(B) for i in range(lens0[s] // T)],
+                         dtype=np.int32).reshape(-1, 3)
+    desc = torch.from_numpy(desc_np).to(dev)
+    # the step's appended rows: the unfinished prefill rows plus the new tokens
+    new_k = torch.cat([rows_k[starts[s] + full0[s]:starts[s] + lens0[s]] for s in range(B)] +
+                      [synth.kv_rows(w, "k", B * w.append_tokens, device=dev, stream_id=1)])
+    new_v = torch.cat([rows_v[starts[s] + full0[s]:starts[s] + lens0[s]] for s in range(B)] +
+                      [synth.kv_rows(w, "v", B * w.append_tokens, device=dev, stream_id=1)])
+    counts = lens1 - full0
+    # reorder so each sequence's rows are contiguous: rest rows then new rows
+    order = []
+    rest_start = np.concatenate([[0], np.cumsum(lens0 - full0)[:-1]])
+    new_base = int((lens0 - full0).sum())
+    for s in range(B):
+        order += list(range(rest_start[s], rest_start[s] + lens0[s] - full0[s]))
+        order += list(range(new_base + s * w.append_tokens, new_base + (s + 1) * w.append_tokens))
+    order_t = torch.tensor(order, dtype=torch.long, device=dev)
+    new_k, new_v = new_k.index_select(0, order_t).contiguous(), new_v.index_select(0, order_t).contiguous()
+    cu_new = torch.from_numpy(np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)).to(dev)
+    before = torch.from_numpy(full0.astype(np.int32)).to(dev)
+    seq_lens = torch.from_numpy(lens1.astype(np.int32)).to(dev)
+    k_pool = torch.zeros((nblocks, H, lay["page_bytes_k"]), dtype=torch.uint8, device=dev)
+    v_pool = torch.zeros((nblocks, H, lay["page_bytes_v"]), dtype=torch.uint8, device=dev)
+    k_tail = torch.zeros((B, H, T, 128), dtype=torch.float16, device=dev)
+    v_tail = torch.zeros_like(k_tail)
+    q = synth.queries(w, device=dev)
+    out = torch.empty_like(q)
+    ws = torch.empty(kvq.decode_workspace_bytes(cfg, B, 0), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    max_new = int(counts.max())
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        kvq.quantize_tiles(cfg, rows_k, rows_v, desc, bt, k_pool, v_pool, num_blocks=nblocks, dev_status=status,
+                           stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        kvq.append_tokens(cfg, new_k, new_v, cu_new, before, max_new, bt, k_pool, v_pool, k_tail, v_tail,
+                          num_blocks=nblocks, dev_status=status, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+        kvq.paged_decode_attention(cfg, q, out, seq_lens, bt, k_pool, v_pool, k_tail, v_tail, ws,
+                                   num_blocks=nblocks, dev_status=status, stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} after warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    visible = [x for x in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if x.strip()]
+    clocks = ClockSampler(visible[ranks.local_rank] if len(visible) > ranks.local_rank else ranks.local_rank)
+    clocks.start()
+    ranks.barrier()
+    torch.cuda.synchronize(dev)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    ranks.barrier()
+    clk = clocks.stop()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    max_ms = ranks.max(elapsed_ms)
+    q_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    a_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    d_ms = [e[2].elapsed_time(e[3]) for e in evs]
+
+    bm = byte_model(w, lay["page_bytes_k"], lay["page_bytes_v"])
+    step_bytes = bm["quantize"] + bm["append"] + bm["decode"]
+    all_bytes = ranks.sum(step_bytes) * args.steps
+    value = all_bytes / (max_ms * 1e-3) / 1e9
+    peak, peak_kind = hbm_peak()
+    q_avg, d_avg = statistics.mean(q_ms), statistics.mean(d_ms)
+    q_gbs = bm["quantize"] / (q_avg * 1e-3) / 1e9
+    d_gbs = bm["decode"] / (d_avg * 1e-3) / 1e9
+
+    # end to end through the public calls with host buffers: H2D of the step's
+    # inputs (fp16 rows, new rows, q) from pinned memory, the three calls,
+    # D2H of the output
+    e2e = None
+    if not args.no_e2e:
+        host = {name: t.cpu().pin_memory() for name, t in
+                dict(rows_k=rows_k, rows_v=rows_v, new_k=new_k, new_v=new_v, q=q).items()}
+        out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = out_host.numel() * out_host.element_size()
+        e2e_steps = max(1, min(args.steps, 3))
+
+        def e2e_step():
+            rows_k.copy_(host["rows_k"], non_blocking=True)
+            rows_v.copy_(host["rows_v"], non_blocking=True)
+            new_k.copy_(host["new_k"], non_blocking=True)
+            new_v.copy_(host["new_v"], non_blocking=True)
+            q.copy_(host["q"], non_blocking=True)
+            step()
+            out_host.copy_(out, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        ranks.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ranks.barrier()
+        e_ms = ranks.max(e0.elapsed_time(e1))
+        e2e = {"value": ranks.sum(step_bytes) * e2e_steps / (e_ms * 1e-3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": e2e_steps,
+               "ms_per_step": e_ms / e2e_steps}
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} after the timed steps")
+
+    cpu = None
+    if ranks.rank == 0 and ranks.world == 1 and not args.no_cpu_baseline:
+        procs = max(1, min(os.cpu_count() or 1, 8))
+        pairs = oracle_pairs(w, procs)
+        pool = OraclePool(procs)
+        try:
+            secs = pool.time(args.workload, {}, pairs)
+        finally:
+            pool.close()
+        cpu = {"value": cpu_sample_bytes(w, bm, len(pairs)) / secs / 1e9, "unit": "GB/s", "cores": procs,
+               "kind": "oracle",
+               "sample": f"{len(pairs)} of {B * H} (sequence, KV head) pairs: fp64 quantize of every K and V "
+                         f"tile, dequantize, fp64 decode of the query group; {secs:.1f} s wall on {procs} "
+                         f"processes, same byte model"}
+
+    launches_per_step = 1 + 1 + 2
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": ranks.world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": f"{w.name}: {B} seqs x {int(lens0[0])} cached tokens + {w.append_tokens} appended, "
+                               f"{H} KV heads, {w.num_q_heads} query heads, d=128, T={T}, P=16, "
+                               f"b_K={w.bits_k}, b_V={w.bits_v}, n={w.iters}, pages scattered by a seeded "
+                               f"permutation",
+                   "global_batch": B * ranks.world, "seq_len": int(lens1.max()),
+                   "parallelism": f"replicas x{ranks.world} (no data-path collective)",
+                   "l2": "inputs larger than L2 (fp16 rows 3.2 GB, pages 0.9 GB per replica)"},
+        "decode": {"gbs": d_gbs, "ms": d_avg, "frac": d_gbs / peak, "tok_per_s": B / (d_avg * 1e-3),
+                   "kv_tok_per_s": bm["kv_tokens"] / (d_avg * 1e-3), "bytes": bm["decode"],
+                   "fp16_bytes_equiv": bm["kv_tokens"] * H * 512},
+        "quantize": {"gbs": q_gbs, "ms": q_avg, "frac": q_gbs / peak, "bytes": bm["quantize"]},
+        "append": {"ms": statistics.mean(a_ms), "bytes": bm["append"]},
+        "roofline": {"bound": "hbm", "kernel": "quantize_tiles_kernel", "achieved": q_gbs, "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": q_gbs / peak,
+                     "traffic": ncu_traffic("quantize_tiles_kernel", bm["quant_units"])},
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps, "clocks": clk,
+    }
+    return line
+
+
+# --------------------------------------------------------------------------- reference arm
+
+def run_reference(args, ranks):
+    from quantized_paged_kv_tile_b200 import synth
+    w = synth.workload(args.workload)
+    bm = byte_model(w, 0, 0)
+    procs = max(1, min(os.cpu_count() or 1, 8))
+    pairs = oracle_pairs(w, procs)
+    times = []
+    pool = OraclePool(procs)
+    try:
+        for i in range(args.warmup + args.steps):
+            secs = pool.time(args.workload, {}, pairs)
+            if i >= args.warmup:
+                times.append(secs)
+    finally:
+        pool.close()
+    nbytes = cpu_sample_bytes(w, bm, len(pairs))
+    value = nbytes * len(times) / sum(times) / 1e9
+    sample = (f"per step {len(pairs)} of {w.num_seqs * w.num_kv_heads} (sequence, KV head) pairs: fp64 quantize "
+              f"of every K and V tile, dequantize, fp64 decode of the query group, {procs} processes")
+    lens1 = np.asarray(w.lens) + w.append_tokens
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": ranks.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{w.name} (oracle sample)", "global_batch": w.num_seqs,
+                   "seq_len": int(lens1.max()), "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": procs, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["kvq", "reference"], default="kvq")
+    ap.add_argument("--workload", default="qwen3_4b")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    sys.path.insert(0, ROOT)
+    from quantized_paged_kv_tile_b200.dist import Ranks
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        if rank != 0:
+            return 0
+        class _Solo:
+            world = int(os.environ.get("WORLD_SIZE", str(args.gpus)))
+        line = run_reference(args, _Solo())
+        print(json.dumps(line), flush=True)
+        return 0
+    ranks = Ranks()
+    if ranks.world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={ranks.world}", file=sys.stderr)
+    try:
+        line = run_kvq(args, ranks)
+        if ranks.rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        ranks.close()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,224 @@
+/*
+ * kvq.h - C ABI of the B200 (sm_100a) quantized paged KV-cache library.
+ *
+ * What the library computes
+ * -------------------------
+ * The method is the one described on axbrief.com, "Huawei's KVarN boosts
+ * vLLM KV-cache capacity by 5x without accuracy loss", section "What
+ * differs from existing methods" (the four-step paragraph): the fp16 K/V
+ * cache is quantized in fixed-size token tiles; each tile gets a Hadamard
+ * rotation along the head-dim channels, then Sinkhorn-like alternating
+ * channel / token variance normalization, then asymmetric round-to-nearest
+ * to b-bit codes.  Attention reads the packed pages directly (aitrends.kr
+ * article 74976, "TL;DR" and glossary "attention backend"); pages follow
+ * PagedAttention's fixed-size blocks with a logical -> physical block table
+ * (ttj.kr KVarN explainer, "Dieting the cache with quantization";
+ * narnarhi.com "SwiftKV ...", main part 2).
+ *
+ * Definitions (the pages give the outline only; these are the concrete
+ * readings the library implements):
+ *   d = head_dim = 128, P = page_tokens = 16, T = tile_tokens in {32,64,128},
+ *   b = bits in {2,3,4}, n = iters >= 0, eps = std_eps (1e-6).
+ *   H = orthonormal Sylvester Hadamard, H[j][k] = (-1)^popcount(j&k)/sqrt(d).
+ *   For one tile X (T x d fp16, one sequence, one KV head, K or V):
+ *     Y = X H;  C = 1_d;  R = 1_T;  repeat n times:
+ *       sigma_j = max(std_i Y_ij, eps);  Y_:j /= sigma_j;  C_j *= sigma_j
+ *       rho_i   = max(std_j Y_ij, eps);  Y_i: /= rho_i;    R_i *= rho_i
+ *       (C, R) <- (C / 2^k, R * 2^k), 2^k the power of two with max C in [1,2)
+ *     std = centred population standard deviation (ddof 0).
+ *     Per token i: z_i = min_j Y_ij, s_i = (max_j Y_ij - z_i) / (2^b - 1),
+ *     code_ij = clamp(round_half_even((Y_ij - z_i) / s_i), 0, 2^b - 1)
+ *     (all codes 0 when s_i == 0).
+ *     Stored: s~_i = fp16(s_i R_i), z~_i = fp16(z_i R_i), C~_j = fp16(C_j).
+ *   Dequantization: X^'_ij = (code_ij s~_i + z~_i) C~_j and X^ = X^' H.
+ *   A sequence of L tokens holds floor(L/T) quantized tiles, tile t covering
+ *   tokens [tT, (t+1)T); the last L mod T tokens stay raw fp16 in a tail
+ *   buffer until their tile fills.
+ *   Decode: out_h = softmax(q_h K^T * scale) V over the dequantized tiles and
+ *   the raw tail of KV head h / g, computed as: q' = H q (once), scores and
+ *   P V on the packed codes in the rotated domain, one inverse rotation H of
+ *   the accumulated output, plus the raw-domain tail; split-K over tiles
+ *   with a log-sum-exp merge.
+ *
+ * Page format (version 1)
+ * -----------------------
+ *   K pool and V pool are separate device buffers, each
+ *     uint8 pool[num_blocks][num_kv_heads][page_bytes]
+ *   One page region (block, head) holds P tokens of one KV head:
+ *     [codes | meta | C slice], each region starting on a 16-byte boundary.
+ *   codes: P*d*b/8 bytes (1024 at b=4, 768 at b=3, 512 at b=2), a little-
+ *     endian bitstream; a code occupies b bits at the bit offset below.
+ *   meta:  P entries of {fp16 s~, fp16 z~} (64 bytes), token-major.
+ *   C slice: page k of its tile (k = logical block index mod T/P) carries
+ *     fp16 C~ of channels [k*d*P/T, (k+1)*d*P/T)  (2*d*P/T bytes).
+ *   page_bytes = codes + 64 + 2*d*P/T  (1152 for T=64, b=4).
+ *   Bit offset of the code of (channel c, token p of the page):
+ *     K, and V at b=3:   (p*d + c) * b                (token-major)
+ *     V at b in {2,4}:   the decode kernel's grouped order.  With
+ *       n = c/8, g = c%8, t = (p%8)/2, u = p/8, s = p%2, F = 32/b,
+ *       h = F/2, k = 2*(n/h) + u, e = n%h, lane = 4*g + t:
+ *       byte of word = ((k/4)*32 + lane)*16 + (k%4)*4,
+ *       bit offset   = 8*(byte of word) + b*(e + h*s).
+ *   Tails: fp16 [num_seqs][num_kv_heads][T][d], one for K and one for V;
+ *     token position q of a sequence lives in row q mod T.
+ *   Query / output: fp16 [num_seqs][num_kv_heads*group_size][d]; query head
+ *     h reads KV head h / group_size.
+ *
+ * Conventions
+ * -----------
+ *  - Every pointer argument marked "device" is a device pointer of the
+ *    current CUDA device; every such pointer must be 16-byte aligned.
+ *  - The caller owns every buffer (pools, tails, tables, workspace, status
+ *    word).  The library allocates no device memory and keeps no state
+ *    beyond a thread-local error message.
+ *  - Every call is asynchronous on `stream` (0 = legacy default stream) and
+ *    never synchronizes.  Arguments are validated on the host first; an
+ *    invalid call returns an error and launches nothing.
+ *  - Errors the device detects (a block id outside [0, num_blocks), a
+ *    missing page) are written once into *dev_status (device int32, may be
+ *    NULL; the first error wins) and the affected work item is skipped.
+ *    Nothing traps.  A launch failure returns KVQ_ERR_CUDA.
+ *  - The caller allocates pages before appending and owns seq_lens.
+ */
+#ifndef KVQ_H_
+#define KVQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KVQ_API __attribute__((visibility("default")))
+#else
+#define KVQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KVQ_OK = 0,
+  KVQ_ERR_INVALID_ARG = 1,   /* bad pointer, size, or configuration value   */
+  KVQ_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. decode b=3) */
+  KVQ_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed        */
+  KVQ_ERR_WORKSPACE = 4,     /* decode workspace smaller than required      */
+  KVQ_ERR_DEVICE_BOUNDS = 5, /* device saw a block id out of range          */
+  KVQ_ERR_DEVICE_TIMEOUT = 6 /* a bounded device wait gave up               */
+} kvq_status;
+
+typedef struct {
+  int head_dim;      /* d: must be 128                                   */
+  int num_kv_heads;  /* H_kv >= 1                                        */
+  int group_size;    /* g = query heads per KV head, 1..8                */
+  int tile_tokens;   /* T: 32, 64 or 128                                 */
+  int page_tokens;   /* P: must be 16                                    */
+  int bits_k;        /* b for K codes: 2, 3 or 4                         */
+  int bits_v;        /* b for V codes: 2, 3 or 4                         */
+  int iters;         /* n: normalization iterations, 0..64               */
+  float std_eps;     /* std clamp, > 0 (1e-6 in the method)              */
+} kvq_config;
+
+typedef struct {
+  size_t page_bytes_k, page_bytes_v;     /* one (block, head) page region   */
+  size_t codes_bytes_k, codes_bytes_v;   /* codes region = meta offset      */
+  size_t cslice_off_k, cslice_off_v;     /* C-slice offset in the region    */
+  size_t block_stride_k, block_stride_v; /* num_kv_heads * page_bytes       */
+  size_t tail_bytes;                     /* one tail buffer (K or V) per sequence:
+                                            num_kv_heads * T * d * 2        */
+  int cslice_channels;                   /* d * P / T                       */
+  int pages_per_tile;                    /* T / P                           */
+} kvq_layout;
+
+/* Fill *out with the byte layout of config *cfg.
+ * cfg, out: host pointers.  Returns KVQ_ERR_INVALID_ARG for a bad config. */
+KVQ_API kvq_status kvq_get_layout(const kvq_config* cfg, kvq_layout* out);
+
+/* Bytes of device workspace kvq_paged_decode_attention needs for num_seqs
+ * sequences and num_splits (0 = automatic) on the current device.
+ * cfg, bytes: host pointers. */
+KVQ_API kvq_status kvq_decode_workspace_bytes(const kvq_config* cfg, int num_seqs, int num_splits,
+                                      size_t* bytes);
+
+/* Write path, prefill: quantize full tiles of raw rows into the pools.
+ *   src_k, src_v : device fp16 [num_rows][num_kv_heads][d]; either may be NULL
+ *                  to skip K or V.
+ *   tile_desc    : device int32 [num_tiles][3] = {src_row, seq, tile_idx}:
+ *                  tile tokens are rows src_row .. src_row+T-1 and land in the
+ *                  pages of logical blocks tile_idx*T/P .. +T/P-1 of seq.
+ *   block_tables : device int32 [num_seqs][max_blocks_per_seq].
+ *   k_pool/v_pool: device uint8 pools (layout above).
+ * Every KV head of every listed tile is quantized (one work item per tile,
+ * head and K/V).  A descriptor with rows outside [0, num_rows), a sequence
+ * outside [0, num_seqs) or pages outside the table is skipped and reported
+ * through dev_status (KVQ_ERR_DEVICE_BOUNDS). */
+KVQ_API kvq_status kvq_quantize_tiles(const kvq_config* cfg, const void* src_k, const void* src_v,
+                              int num_rows, const int32_t* tile_desc, int num_tiles,
+                              const int32_t* block_tables, int num_seqs, int max_blocks_per_seq,
+                              int num_blocks, void* k_pool, void* v_pool,
+                              int32_t* dev_status, void* stream);
+
+/* Write path, decode / chunked prefill: append new tokens.
+ *   new_k, new_v     : device fp16 [cu_new[num_seqs]][num_kv_heads][d].
+ *   cu_new           : device int32 [num_seqs+1], prefix sums of new tokens.
+ *   seq_lens_before  : device int32 [num_seqs], tokens already cached.
+ *   max_new_per_seq  : host bound on cu_new[s+1]-cu_new[s] (>= 0).
+ *   k_tail, v_tail   : device fp16 tails [num_seqs][num_kv_heads][T][d].
+ * Every tile completed by the new tokens is quantized (from the old tail
+ * rows and the new rows) into its pages; the remaining new tokens land in
+ * the tail.  The result is bit-identical to kvq_quantize_tiles on the same
+ * tokens.  seq_lens is not updated (the caller owns it). */
+KVQ_API kvq_status kvq_append_tokens(const kvq_config* cfg, const void* new_k, const void* new_v,
+                             const int32_t* cu_new, const int32_t* seq_lens_before,
+                             int num_seqs, int max_new_per_seq,
+                             const int32_t* block_tables, int max_blocks_per_seq,
+                             int num_blocks, void* k_pool, void* v_pool,
+                             void* k_tail, void* v_tail, int32_t* dev_status, void* stream);
+
+/* Read path: one decode step of paged attention over the quantized cache.
+ *   q, out       : device fp16 [num_seqs][num_kv_heads*group_size][d]; q is
+ *                  not rotated (the kernel rotates it).
+ *   seq_lens     : device int32 [num_seqs], tokens in the cache (including
+ *                  any token appended for this step); full tiles come from
+ *                  the pools, the last seq_len mod T tokens from the tails.
+ *   softmax_scale: scale of q.k (1/sqrt(d) in the method).
+ *   workspace    : device, >= kvq_decode_workspace_bytes(cfg, num_seqs,
+ *                  num_splits) bytes; contents on entry are ignored.
+ *   num_splits   : split-K factor over tiles per (sequence, KV head); 0 picks
+ *                  one from the device size.  The output does not depend on it
+ *                  beyond rounding.
+ * Decode supports b in {2, 4} for K and V (KVQ_ERR_UNSUPPORTED for 3). */
+KVQ_API kvq_status kvq_paged_decode_attention(const kvq_config* cfg, const void* q, void* out,
+                                      const int32_t* seq_lens, int num_seqs,
+                                      const int32_t* block_tables, int max_blocks_per_seq,
+                                      int num_blocks, const void* k_pool, const void* v_pool,
+                                      const void* k_tail, const void* v_tail,
+                                      float softmax_scale, void* workspace,
+                                      size_t workspace_bytes, int num_splits,
+                                      int32_t* dev_status, void* stream);
+
+/* Inspection (tests, tools): read num_tiles tiles back out of a pool.
+ *   tile_desc : device int32 [num_tiles][2] = {seq, tile_idx}; all heads.
+ *   is_v      : 0 = K pool / bits_k, 1 = V pool / bits_v.
+ *   codes     : device uint8 [num_tiles][num_kv_heads][T][d]      (may be NULL)
+ *   meta      : device fp16  [num_tiles][num_kv_heads][T][2] {s~, z~} (may be NULL)
+ *   cvec      : device fp16  [num_tiles][num_kv_heads][d]        (may be NULL)
+ *   out_rot   : device fp32  [num_tiles][num_kv_heads][T][d] dequantized,
+ *               rotated domain (X^')                             (may be NULL)
+ *   out_orig  : device fp32, same shape, original domain (X^' H)  (may be NULL) */
+KVQ_API kvq_status kvq_unpack_tiles(const kvq_config* cfg, const int32_t* tile_desc, int num_tiles,
+                            const int32_t* block_tables, int num_seqs, int max_blocks_per_seq, int num_blocks,
+                            const void* pool, int is_v, uint8_t* codes, void* meta, void* cvec,
+                            float* out_rot, float* out_orig, int32_t* dev_status, void* stream);
+
+/* Static text for a status code. */
+KVQ_API const char* kvq_status_string(kvq_status s);
+/* Detail of the last error on the calling host thread ("" if none). */
+KVQ_API const char* kvq_last_error(void);
+/* Library version string ("kvq <major>.<minor> format 1 sm_100a"). */
+KVQ_API const char* kvq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H_ */

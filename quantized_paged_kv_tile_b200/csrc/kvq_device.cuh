@@ -1,0 +1,87 @@
+// Device helpers shared by the kernels: the page-format bit positions,
+// device error reporting, warp reductions and the warp-wide 128-point
+// Walsh-Hadamard butterfly.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "kvq_internal.h"
+
+namespace kvq {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+// First device-detected error wins; the work item that saw it is skipped.
+__device__ __forceinline__ void report_error(int32_t* status, int code) {
+  if (status) atomicCAS(reinterpret_cast<int*>(status), 0, code);
+}
+
+// Bit offset of the code of (channel c, token p of the page) inside a page's
+// codes region.  K, and V at 3 bits: token-major bitstream.  V at 2 / 4
+// bits: grouped so that decode lane (4*g + t) owns one contiguous run of
+// 32-bit words holding channels 8n+g (n = 0..15) for the token pairs
+// {2t, 2t+1} and {2t+8, 2t+9}.
+__device__ __forceinline__ int code_bit(int c, int p, int bits, bool is_v) {
+  if (!is_v || bits == 3) return (p * kHeadDim + c) * bits;
+  const int n = c >> 3, g = c & 7;
+  const int t = (p & 7) >> 1, u = p >> 3, s = p & 1;
+  const int h = 16 / bits;             // code pairs per 32-bit word
+  const int k = 2 * (n / h) + u;       // word index inside the lane's run
+  const int e = n % h;
+  const int lane = 4 * g + t;
+  const int word_byte = ((k >> 2) * 32 + lane) * 16 + (k & 3) * 4;
+  return word_byte * 8 + bits * (e + h * s);
+}
+
+// Read one b-bit code at `bit` from a byte array (may straddle a byte).
+__device__ __forceinline__ int read_code(const uint8_t* base, int bit, int bits) {
+  const int byte = bit >> 3, off = bit & 7;
+  unsigned v = base[byte];
+  if (off + bits > 8) v |= static_cast<unsigned>(base[byte + 1]) << 8;
+  return static_cast<int>((v >> off) & ((1u << bits) - 1u));
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) v += __shfl_xor_sync(kFull, v, m);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, m));
+  return v;
+}
+__device__ __forceinline__ float warp_min(float v) {
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) v = fminf(v, __shfl_xor_sync(kFull, v, m));
+  return v;
+}
+
+// Unnormalized Walsh-Hadamard transform of one 128-vector held by a warp,
+// lane L holding channels 4L..4L+3 in v[0..3].  Natural (Sylvester) order:
+// the result is sum_k x_k (-1)^popcount(j & k).  Channel bits 0-1 are
+// in-register butterflies, bits 2-6 pair lanes differing in bit 0-4.
+__device__ __forceinline__ void fwht128_warp(float v[4], int lane) {
+  const float a0 = v[0] + v[1], a1 = v[0] - v[1];
+  const float a2 = v[2] + v[3], a3 = v[2] - v[3];
+  v[0] = a0 + a2;
+  v[2] = a0 - a2;
+  v[1] = a1 + a3;
+  v[3] = a1 - a3;
+#pragma unroll
+  for (int k = 0; k < 5; ++k) {
+    const int m = 1 << k;
+    const bool upper = lane & m;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float o = __shfl_xor_sync(kFull, v[i], m);
+      v[i] = upper ? (o - v[i]) : (v[i] + o);
+    }
+  }
+}
+
+constexpr float kSqrtHeadDim = 11.313708498984761f;  // sqrt(128) rounded to fp32
+constexpr float kLog2e = 1.4426950408889634f;
+
+}  // namespace kvq

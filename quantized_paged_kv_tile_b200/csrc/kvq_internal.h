@@ -1,0 +1,115 @@
+// Internal declarations shared by the library's translation units.
+// Host-side launchers: each validates nothing (the C-ABI layer in
+// kvq_api.cu has done that) and returns the cudaError_t of its launches.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/kvq.h"
+
+namespace kvq {
+
+constexpr int kHeadDim = 128;
+constexpr int kPageTokens = 16;
+constexpr int kMaxGroup = 8;
+
+// Layout numbers of one pool (K or V), derived from the config.
+struct PoolGeom {
+  int bits;            // code width
+  int codes_bytes;     // P*d*b/8
+  int meta_off;        // == codes_bytes
+  int cslice_off;      // codes_bytes + 64
+  int page_bytes;      // one (block, head) region
+  int cs_channels;     // d*P/T channels of C per page
+  int pages_per_tile;  // T/P
+};
+
+PoolGeom pool_geom(const kvq_config& cfg, bool is_v);
+
+// Quantize work: one item per (tile, head, K/V).
+struct QuantizeArgs {
+  kvq_config cfg;
+  PoolGeom gk, gv;
+  const void* src_k;
+  const void* src_v;
+  int num_rows;
+  const int32_t* tile_desc;  // [num_tiles][3]
+  int num_tiles;
+  const int32_t* block_tables;
+  int num_seqs;
+  int max_blocks_per_seq;
+  int num_blocks;
+  void* k_pool;
+  void* v_pool;
+  int32_t* dev_status;
+};
+cudaError_t launch_quantize_tiles(const QuantizeArgs& a, cudaStream_t s);
+
+struct AppendArgs {
+  kvq_config cfg;
+  PoolGeom gk, gv;
+  const void* new_k;
+  const void* new_v;
+  const int32_t* cu_new;
+  const int32_t* seq_lens_before;
+  int num_seqs;
+  int max_new_per_seq;
+  const int32_t* block_tables;
+  int max_blocks_per_seq;
+  int num_blocks;
+  void* k_pool;
+  void* v_pool;
+  void* k_tail;
+  void* v_tail;
+  int32_t* dev_status;
+};
+cudaError_t launch_append_tokens(const AppendArgs& a, cudaStream_t s);
+
+struct UnpackArgs {
+  kvq_config cfg;
+  PoolGeom g;
+  const int32_t* tile_desc;  // [num_tiles][2]
+  int num_tiles;
+  const int32_t* block_tables;
+  int num_seqs;
+  int max_blocks_per_seq;
+  int num_blocks;
+  const void* pool;
+  int is_v;
+  uint8_t* codes;
+  void* meta;
+  void* cvec;
+  float* out_rot;
+  float* out_orig;
+  int32_t* dev_status;
+};
+cudaError_t launch_unpack_tiles(const UnpackArgs& a, cudaStream_t s);
+
+struct DecodeArgs {
+  kvq_config cfg;
+  PoolGeom gk, gv;
+  const void* q;
+  void* out;
+  const int32_t* seq_lens;
+  int num_seqs;
+  const int32_t* block_tables;
+  int max_blocks_per_seq;
+  int num_blocks;
+  const void* k_pool;
+  const void* v_pool;
+  const void* k_tail;
+  const void* v_tail;
+  float softmax_scale;
+  void* workspace;
+  int num_splits;  // resolved (> 0)
+  int32_t* dev_status;
+};
+// Workspace bytes for a resolved split count.
+size_t decode_workspace_bytes(const kvq_config& cfg, int num_seqs, int num_splits);
+// Split count used when the caller passes 0.
+int decode_auto_splits(const kvq_config& cfg, int num_seqs, int num_sms);
+cudaError_t launch_paged_decode(const DecodeArgs& a, cudaStream_t s);
+
+}  // namespace kvq

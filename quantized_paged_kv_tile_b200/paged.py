@@ -1,0 +1,122 @@
+"""Host-side bookkeeping of a quantized paged KV cache (one attention layer).
+
+``PagedKVCache`` owns the device buffers the C ABI works on (K/V page
+pools, fp16 tails, block tables, sequence lengths, decode workspace) and
+turns user-level operations into the three library calls:
+  prefill(rows)  -> kvq_quantize_tiles for every full tile, then
+                    kvq_append_tokens for the unfinished last tile
+  append(rows)   -> kvq_append_tokens (quantizes tiles as they fill)
+  decode(q)      -> kvq_paged_decode_attention
+All arithmetic runs in the library's kernels; this module only sizes and
+indexes buffers (PyTorch provides the memory and the stream).
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+from . import kvq
+
+
+class PagedKVCache:
+    def __init__(self, cfg: kvq.Config, num_seqs: int, max_tokens_per_seq: int, device="cuda",
+                 block_table: np.ndarray | None = None, num_splits: int = 0):
+        self.cfg = cfg
+        self.num_seqs = num_seqs
+        self.device = torch.device(device)
+        self.layout = kvq.get_layout(cfg)
+        self.blocks_per_seq = math.ceil(max_tokens_per_seq / cfg.page_tokens)
+        if block_table is None:
+            block_table = np.arange(num_seqs * self.blocks_per_seq, dtype=np.int32).reshape(num_seqs, -1)
+        if block_table.shape != (num_seqs, self.blocks_per_seq):
+            raise ValueError(f"block table shape {block_table.shape} != {(num_seqs, self.blocks_per_seq)}")
+        self.num_blocks = int(block_table.max()) + 1
+        self.block_tables = torch.from_numpy(np.ascontiguousarray(block_table, dtype=np.int32)).to(self.device)
+        h = cfg.num_kv_heads
+        self.k_pool = torch.zeros((self.num_blocks, h, self.layout["page_bytes_k"]), dtype=torch.uint8,
+                                  device=self.device)
+        self.v_pool = torch.zeros((self.num_blocks, h, self.layout["page_bytes_v"]), dtype=torch.uint8,
+                                  device=self.device)
+        tail_shape = (num_seqs, h, cfg.tile_tokens, cfg.head_dim)
+        self.k_tail = torch.zeros(tail_shape, dtype=torch.float16, device=self.device)
+        self.v_tail = torch.zeros(tail_shape, dtype=torch.float16, device=self.device)
+        self.seq_lens = torch.zeros(num_seqs, dtype=torch.int32, device=self.device)
+        self.host_lens = np.zeros(num_seqs, dtype=np.int64)
+        self.num_splits = num_splits
+        self.workspace = torch.empty(kvq.decode_workspace_bytes(cfg, num_seqs, num_splits), dtype=torch.uint8,
+                                     device=self.device)
+        self.dev_status = torch.zeros(1, dtype=torch.int32, device=self.device)
+
+    # ------------------------------------------------------------------ write
+    def prefill_tile_desc(self, lens) -> np.ndarray:
+        """{src_row, seq, tile_idx} for every full tile of packed rows with
+        per-sequence lengths ``lens`` (rows of seq s start at sum(lens[:s]))."""
+        t = self.cfg.tile_tokens
+        starts = np.concatenate([[0], np.cumsum(lens)[:-1]]).astype(np.int64)
+        desc = [(starts[s] + i * t, s, i) for s in range(len(lens)) for i in range(int(lens[s]) // t)]
+        return np.asarray(desc, dtype=np.int32).reshape(-1, 3)
+
+    def prefill(self, rows_k: torch.Tensor, rows_v: torch.Tensor, lens, stream=None) -> None:
+        """Load an empty cache with packed rows [sum(lens)][H_kv][d]."""
+        lens = np.asarray(lens, dtype=np.int64)
+        if np.any(self.host_lens):
+            raise RuntimeError("prefill expects an empty cache")
+        desc = torch.from_numpy(self.prefill_tile_desc(lens)).to(self.device)
+        kvq.quantize_tiles(self.cfg, rows_k, rows_v, desc, self.block_tables, self.k_pool, self.v_pool,
+                           num_blocks=self.num_blocks, dev_status=self.dev_status, stream=stream)
+        t = self.cfg.tile_tokens
+        full = (lens // t) * t
+        rest = lens - full
+        if rest.any():
+            starts = np.concatenate([[0], np.cumsum(lens)[:-1]])
+            idx = np.concatenate([np.arange(starts[s] + full[s], starts[s] + lens[s]) for s in range(len(lens))])
+            idx_t = torch.from_numpy(idx).to(self.device)
+            self._append(rows_k.index_select(0, idx_t), rows_v.index_select(0, idx_t), full, rest, stream)
+        self.host_lens = lens.copy()
+        self.seq_lens.copy_(torch.from_numpy(lens.astype(np.int32)))
+
+    def _append(self, new_k, new_v, before, counts, stream=None) -> None:
+        cu = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+        kvq.append_tokens(self.cfg, new_k, new_v, torch.from_numpy(cu).to(self.device),
+                          torch.from_numpy(np.asarray(before, dtype=np.int32)).to(self.device),
+                          int(np.max(counts)), self.block_tables, self.k_pool, self.v_pool, self.k_tail,
+                          self.v_tail, num_blocks=self.num_blocks, dev_status=self.dev_status, stream=stream)
+
+    def append(self, new_k: torch.Tensor, new_v: torch.Tensor, counts=None, stream=None) -> None:
+        """Append packed rows (``counts`` per sequence, default one each)."""
+        if counts is None:
+            counts = np.ones(self.num_seqs, dtype=np.int64)
+        counts = np.asarray(counts, dtype=np.int64)
+        if np.any(self.host_lens + counts > self.blocks_per_seq * self.cfg.page_tokens):
+            raise ValueError("append past the allocated pages")
+        self._append(new_k, new_v, self.host_lens, counts, stream)
+        self.host_lens = self.host_lens + counts
+        self.seq_lens.copy_(torch.from_numpy(self.host_lens.astype(np.int32)))
+
+    # ------------------------------------------------------------------- read
+    def decode(self, q: torch.Tensor, out: torch.Tensor | None = None, num_splits: int | None = None,
+               stream=None) -> torch.Tensor:
+        """One decode step: q fp16 [B][H_q][d] -> out fp16 [B][H_q][d]."""
+        if out is None:
+            out = torch.empty_like(q)
+        splits = self.num_splits if num_splits is None else num_splits
+        ws = self.workspace
+        need = kvq.decode_workspace_bytes(self.cfg, self.num_seqs, splits)
+        if ws.numel() < need:
+            ws = torch.empty(need, dtype=torch.uint8, device=self.device)
+        kvq.paged_decode_attention(self.cfg, q, out, self.seq_lens, self.block_tables, self.k_pool, self.v_pool,
+                                   self.k_tail, self.v_tail, ws, num_splits=splits, num_blocks=self.num_blocks,
+                                   dev_status=self.dev_status, stream=stream)
+        return out
+
+    def status(self) -> int:
+        """Device status word (0 = no device-detected error); synchronizes."""
+        return int(self.dev_status.item())
+
+    def bytes_per_token_head(self) -> float:
+        """Stored bytes per (token, KV head) for K+V, pages only."""
+        p = self.cfg.page_tokens
+        return (self.layout["page_bytes_k"] + self.layout["page_bytes_v"]) / p

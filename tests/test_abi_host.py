@@ -1,0 +1,157 @@
+"""CPU-only checks of the C ABI library and the host-side helpers.
+
+No compute call reaches the GPU here: the library is loaded, its exported
+symbols are compared with include/kvq.h, and only host-side entry points
+(layout, workspace sizing with an explicit split count, argument
+validation that fails before any launch) are called.
+"""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import kvq_oracle as o
+from quantized_paged_kv_tile_b200 import build, kvq, synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return kvq.load_library()
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "kvq.h")).read()
+    return sorted(set(re.findall(r"KVQ_API\s+[^;(]*?\b(kvq_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_symbols():
+    assert declared_symbols() == sorted(kvq.EXPORTED_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", kvq.library_path()], capture_output=True, text=True,
+                         check=True).stdout
+    exported = sorted(set(re.findall(r"\bT (kvq_\w+)", out)))
+    assert exported == declared_symbols()
+    for name in declared_symbols():
+        assert hasattr(lib, name)
+
+
+def test_version_and_status_strings(lib):
+    assert kvq.version().startswith("kvq ") and "sm_100a" in kvq.version()
+    assert lib.kvq_status_string(kvq.KVQ_ERR_WORKSPACE).decode() == "workspace too small"
+
+
+@pytest.mark.parametrize("t", [32, 64, 128])
+@pytest.mark.parametrize("bk,bv", [(4, 4), (4, 2), (3, 2), (2, 3)])
+def test_layout_matches_oracle(lib, t, bk, bv):
+    cfg = kvq.Config(num_kv_heads=8, group_size=4, tile_tokens=t, bits_k=bk, bits_v=bv, iters=4)
+    lay = kvq.get_layout(cfg)
+    ok_, ov = o.page_layout(bk, t), o.page_layout(bv, t)
+    assert lay["page_bytes_k"] == ok_["page_bytes"] and lay["page_bytes_v"] == ov["page_bytes"]
+    assert lay["codes_bytes_k"] == ok_["codes"] and lay["cslice_off_k"] == ok_["cslice_off"]
+    assert lay["cslice_channels"] == ok_["cslice_channels"] and lay["pages_per_tile"] == t // 16
+    assert lay["tail_bytes"] == 8 * t * 128 * 2
+    assert lay["block_stride_v"] == 8 * ov["page_bytes"]
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("head_dim", 64, kvq.KVQ_ERR_UNSUPPORTED), ("tile_tokens", 48, kvq.KVQ_ERR_UNSUPPORTED),
+    ("bits_k", 5, kvq.KVQ_ERR_UNSUPPORTED), ("group_size", 9, kvq.KVQ_ERR_UNSUPPORTED),
+    ("iters", -1, kvq.KVQ_ERR_INVALID_ARG), ("std_eps", 0.0, kvq.KVQ_ERR_INVALID_ARG),
+    ("page_tokens", 32, kvq.KVQ_ERR_UNSUPPORTED), ("num_kv_heads", 0, kvq.KVQ_ERR_INVALID_ARG),
+])
+def test_config_validation(lib, field, value, status):
+    base = dict(num_kv_heads=2, group_size=4, tile_tokens=64, bits_k=4, bits_v=4, iters=4)
+    cfg = kvq.Config(**base)
+    cfg = kvq.Config(**{**cfg.__dict__, field: value})
+    with pytest.raises(kvq.KvqError) as ei:
+        kvq.get_layout(cfg)
+    assert ei.value.status == status
+
+
+def test_argument_errors_launch_nothing(lib):
+    cfg = kvq.Config(num_kv_heads=2, group_size=4, tile_tokens=64, bits_k=4, bits_v=4, iters=4)
+    c = cfg.c()
+    # both sources NULL
+    st = lib.kvq_quantize_tiles(ctypes.byref(c), None, None, 10, 16, 1, 16, 1, 4, 8, 16, 16, None, None)
+    assert st == kvq.KVQ_ERR_INVALID_ARG
+    # misaligned pointer
+    st = lib.kvq_quantize_tiles(ctypes.byref(c), 17, None, 10, 16, 1, 16, 1, 4, 8, 16, 16, None, None)
+    assert st == kvq.KVQ_ERR_INVALID_ARG and "aligned" in kvq.load_library().kvq_last_error().decode()
+    # 3-bit decode is storage-only
+    c3 = kvq.Config(num_kv_heads=2, group_size=4, tile_tokens=64, bits_k=3, bits_v=4, iters=4).c()
+    st = lib.kvq_paged_decode_attention(ctypes.byref(c3), 16, 16, 16, 1, 16, 4, 8, 16, 16, 16, 16, 0.1, 16,
+                                        1 << 20, 1, None, None)
+    assert st == kvq.KVQ_ERR_UNSUPPORTED
+    # workspace too small (explicit split count: no device query)
+    need = kvq.decode_workspace_bytes(cfg, 3, 2)
+    assert need == 3 * 2 * 2 * 4 * 130 * 4
+    st = lib.kvq_paged_decode_attention(ctypes.byref(c), 16, 16, 16, 3, 16, 4, 8, 16, 16, 16, 16, 0.1, 16,
+                                        need - 1, 2, None, None)
+    assert st == kvq.KVQ_ERR_WORKSPACE
+    # zero-sized work is a no-op
+    assert lib.kvq_quantize_tiles(ctypes.byref(c), 16, None, 0, None, 0, None, 0, 0, 0, None, None, None,
+                                  None) == kvq.KVQ_OK
+
+
+def test_binding_rejects_cpu_tensors(lib):
+    cfg = kvq.Config(num_kv_heads=1, group_size=1, tile_tokens=64, bits_k=4, bits_v=4, iters=1)
+    x = torch.zeros((64, 1, 128), dtype=torch.float16)
+    with pytest.raises(TypeError):
+        kvq.quantize_tiles(cfg, x, None, torch.zeros((1, 3), dtype=torch.int32), torch.zeros((1, 4), dtype=torch.int32),
+                           torch.zeros((4, 1, 1152), dtype=torch.uint8), None)
+
+
+# ------------------------------------------------------------------ synth
+
+def test_synth_is_seeded_and_shaped():
+    w = synth.workload("qwen3_4b", num_seqs=2, lens=(256, 256))
+    a = synth.kv_rows(w, "k", 64)
+    b = synth.kv_rows(w, "k", 64)
+    assert a.shape == (64, 8, 128) and a.dtype == torch.float16
+    assert torch.equal(a, b)
+    assert not torch.equal(a, synth.kv_rows(w, "v", 64))
+    sc = synth.channel_scales(w, "k")
+    # 3 outlier channels per head scaled by 10 on top of lognormal(0,1)
+    assert sc.shape == (8, 128) and np.all(sc > 0)
+    assert np.all(synth.channel_scales(w, "v") == 1.0)
+
+
+def test_synth_tiny_uses_same_outlier_channels_for_k_and_v():
+    w = synth.workload("tiny")
+    k, v = synth.channel_scales(w, "k"), synth.channel_scales(w, "v")
+    assert (k == 20).sum() == 4 and np.array_equal(k, v)
+
+
+def test_synth_sweep_outlier_counts():
+    w = synth.workload("prefill_sweep")
+    for which in ("k", "v"):
+        sc = synth.channel_scales(w, which)
+        n = (sc != 1.0).sum(axis=1)
+        assert np.all(n >= 1) and np.all(n <= 7)
+        big = sc[sc != 1.0]
+        assert big.min() >= 5.0 and big.max() <= 50.0
+
+
+def test_mixed_lengths_log_uniform():
+    lens = np.array(synth.workload("mixed").lens)
+    assert lens.shape == (256,) and lens.min() >= 1024 and lens.max() <= 131072
+    # log-uniform: the median sits near the geometric mean of the range
+    assert 6000 < np.median(lens) < 24000
+
+
+def test_block_table_is_a_permutation():
+    w = synth.workload("qwen3_4b")
+    bt = synth.block_table(w, 8193)
+    assert bt.shape == (6, 8193)
+    assert np.array_equal(np.sort(bt.ravel()), np.arange(6 * 8193))
+    assert not np.array_equal(bt.ravel(), np.arange(6 * 8193))
