@@ -125,10 +125,13 @@ def sinkhorn_normalize(xr: np.ndarray, iters: int, eps: float = EPS):
     c = np.ones(d, dtype=y.dtype)
     r = np.ones(t, dtype=y.dtype)
     for _ in range(iters):
-        sigma = np.maximum(y.std(axis=0), dt(eps))      # each channel over the tile's tokens
+        # std is shift-invariant; taking it of the values minus the first
+        # sample makes an exactly constant channel (or token) give exactly 0
+        # in any precision, so the clamp decides as the definition says
+        sigma = np.maximum((y - y[:1, :]).std(axis=0), dt(eps))   # each channel over the tile's tokens
         y = y / sigma[None, :]
         c = c * sigma
-        rho = np.maximum(y.std(axis=1), dt(eps))        # each token over the channels
+        rho = np.maximum((y - y[:, :1]).std(axis=1), dt(eps))     # each token over the channels
         y = y / rho[:, None]
         r = r * rho
         _, e = np.frexp(c.max())                        # max C = m 2^e, m in [0.5, 1)

@@ -65,14 +65,16 @@ __device__ void quantize_tile_block(QuantSmem<T>& sm, const PoolGeom g, bool is_
 
   // 2. normalization
   for (int it = 0; it < iters; ++it) {
-    {  // channel step: thread = channel
+    {  // channel step: thread = channel.  Deviations are taken from the
+       // column's first value, so a constant column has exactly zero std.
       const int j = tid;
+      const float y0 = sm.y[0][j];
       float s = 0.f;
-      for (int i = 0; i < T; ++i) s += sm.y[i][j];
+      for (int i = 0; i < T; ++i) s += sm.y[i][j] - y0;
       const float mean = s / static_cast<float>(T);
       float q = 0.f;
       for (int i = 0; i < T; ++i) {
-        const float d = sm.y[i][j] - mean;
+        const float d = (sm.y[i][j] - y0) - mean;
         q += d * d;
       }
       const float sigma = fmaxf(sqrtf(q / static_cast<float>(T)), eps);
@@ -80,15 +82,17 @@ __device__ void quantize_tile_block(QuantSmem<T>& sm, const PoolGeom g, bool is_
       sm.c[j] *= sigma;
     }
     __syncthreads();
-    for (int i = warp; i < T; i += 4) {  // token step: warp = row
+    for (int i = warp; i < T; i += 4) {  // token step: warp = row, shifted by the row's first value
       float v[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) v[k] = sm.y[i][4 * lane + k];
-      const float mean = warp_sum((v[0] + v[1]) + (v[2] + v[3])) / static_cast<float>(kHeadDim);
+      const float y0 = __shfl_sync(kFull, v[0], 0);
+      const float mean =
+          warp_sum(((v[0] - y0) + (v[1] - y0)) + ((v[2] - y0) + (v[3] - y0))) / static_cast<float>(kHeadDim);
       float q = 0.f;
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const float d = v[k] - mean;
+        const float d = (v[k] - y0) - mean;
         q += d * d;
       }
       const float rho = fmaxf(sqrtf(warp_sum(q) / static_cast<float>(kHeadDim)), eps);

@@ -157,6 +157,17 @@ def test_renormalization_keeps_metadata_finite():
                     np.testing.assert_allclose(xh, xh[:1].repeat(64, 0), rtol=0, atol=0)
 
 
+@pytest.mark.parametrize("dt", [np.float64, np.float32])
+def test_identical_tokens_clamp_every_channel(dt):
+    # 64 identical tokens: every rotated channel is exactly constant over the
+    # tile, so every channel std is 0 and every sigma is the clamp eps; all C
+    # come out equal and every token row is the same.
+    row = np.random.default_rng(15).standard_normal(128).astype(np.float16)
+    q = o.quantize_tile(np.tile(row, (64, 1)), 4, 3, dtype=dt, return_parts=True)
+    assert np.all(q["c"] == q["c"][0])
+    assert np.all(q["codes"] == q["codes"][:1])
+
+
 def test_scale_equivariance():
     # X -> 2^k X (exact in fp16): codes and C~ unchanged (C is renormalized to
     # max in [1, 2)), s~ and z~ scaled by 2^k
