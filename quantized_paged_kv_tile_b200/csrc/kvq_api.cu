@@ -115,19 +115,21 @@ kvq_status kvq_get_layout(const kvq_config* cfg, kvq_layout* out) {
   return ok();
 }
 
+kvq_status device_sm_count(int* sms) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_status(e, "querying the SM count");
+  return KVQ_OK;
+}
+
 kvq_status kvq_decode_workspace_bytes(const kvq_config* cfg, int num_seqs, int num_splits, size_t* bytes) {
   KVQ_TRY(check_config(cfg));
   if (bytes == nullptr) return fail(KVQ_ERR_INVALID_ARG, "bytes output is NULL");
   if (num_seqs < 0 || num_splits < 0) return fail(KVQ_ERR_INVALID_ARG, "negative num_seqs or num_splits");
-  int splits = num_splits;
-  if (splits == 0) {
-    int dev = 0, sms = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return cuda_status(e, "querying the SM count");
-    splits = kvq::decode_auto_splits(*cfg, num_seqs, sms);
-  }
-  *bytes = kvq::decode_workspace_bytes(*cfg, num_seqs, splits);
+  int sms = 0;
+  if (num_splits == 0) KVQ_TRY(device_sm_count(&sms));
+  *bytes = kvq::decode_workspace_bytes(*cfg, num_seqs, num_splits, sms);
   return ok();
 }
 
@@ -231,16 +233,10 @@ kvq_status kvq_paged_decode_attention(const kvq_config* cfg, const void* q, void
   KVQ_TRY(check_ptr(v_tail, "v_tail"));
   KVQ_TRY(check_ptr(workspace, "workspace"));
   KVQ_TRY(check_ptr(dev_status, "dev_status", true));
-  int splits = num_splits;
-  if (splits == 0) {
-    int dev = 0, sms = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return cuda_status(e, "querying the SM count");
-    splits = kvq::decode_auto_splits(*cfg, num_seqs, sms);
-  }
-  if (splits > 65535) return fail(KVQ_ERR_INVALID_ARG, "num_splits > 65535");
-  const size_t need = kvq::decode_workspace_bytes(*cfg, num_seqs, splits);
+  if (num_splits > 65535) return fail(KVQ_ERR_INVALID_ARG, "num_splits > 65535");
+  int sms = 0;
+  if (num_splits == 0) KVQ_TRY(device_sm_count(&sms));
+  const size_t need = kvq::decode_workspace_bytes(*cfg, num_seqs, num_splits, sms);
   if (workspace_bytes < need)
     return fail(KVQ_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, need);
   kvq::DecodeArgs a{};
@@ -260,7 +256,7 @@ kvq_status kvq_paged_decode_attention(const kvq_config* cfg, const void* q, void
   a.v_tail = v_tail;
   a.softmax_scale = softmax_scale;
   a.workspace = workspace;
-  a.num_splits = splits;
+  a.num_splits_fixed = num_splits;
   a.dev_status = dev_status;
   return cuda_status(kvq::launch_paged_decode(a, static_cast<cudaStream_t>(stream)),
                      "kvq_paged_decode_attention launch");

@@ -2,14 +2,27 @@
 //
 // The attention backend reads the compressed pages directly (aitrends.kr
 // article 74976, "TL;DR"; glossary "attention backend").  Per (sequence,
-// KV head) the g query heads are rotated once, q' = H q; each tile t then
-// contributes, in the rotated domain,
-//   score_i = s~K_i (q'' . codeK_i) + z~K_i sum_j q''_j,  q'' = q' * C~K_t
+// KV head) the g query heads are rotated once, q' = H q, and each tile t
+// contributes in the rotated domain
+//   score_i = s~K_i (q'' . codeK_i) + z~K_i sum_j q''_j,   q'' = q' * C~K_t
 //   acc'_j += C~V_tj (sum_i p_i s~V_i codeV_ij + sum_i p_i z~V_i)
-// which equals softmax over q' . K^'_i and P V^' exactly in real arithmetic.
-// Tiles are split into `num_splits` chunks (split-K); the merge kernel adds
-// the raw fp16 tail, combines the chunks by log-sum-exp, applies the one
-// inverse rotation and writes fp16.
+// which equals softmax(q' . K^'_i) P V^' exactly in real arithmetic.
+//
+// Kernels (three launches per call):
+//   decode_schedule_kernel  one CTA: tiles per sequence, chunk size, the
+//                           prefix of work units (sequence, KV head, chunk)
+//   decode_tiles_kernel     persistent warps, one work unit at a time:
+//                           per-warp double-buffered cp.async.bulk staging
+//                           of whole tiles (all pages, K and V) into shared
+//                           memory; scores and P.V on the legacy tensor
+//                           cores (mma.sync m16n8k16, f16 -> f32) with the
+//                           16 MMA rows = 8 query heads x {hi, lo} fp16
+//                           halves (fp32-accurate operands at no extra MMA)
+//                           and the packed codes unpacked in registers;
+//                           online softmax per tile; rotated-domain partial
+//   decode_merge_kernel     per (sequence, KV head): raw fp16 tail, log-sum-
+//                           exp merge of the chunks, the one inverse rotation,
+//                           fp16 output
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -22,168 +35,513 @@ namespace kvq {
 
 namespace {
 
-constexpr int kThreads = 128;
 constexpr int kPartFloats = 2 + kHeadDim;  // m, l, acc[d] per query head
+constexpr int kDecWarps = 4;               // warps per decode CTA
+constexpr int kUnitsPerSm = 32;            // work-unit budget of the automatic split
+constexpr long long kWaitLimitNs = 2000000000LL;  // bounded mbarrier waits: 2 s
 
-template <int T>
-struct DecSmem {
-  float qr[kMaxGroup][kHeadDim];  // rotated query * scale * log2(e)
-  float qq[kMaxGroup][kHeadDim];  // q'' = q' * C~K of the current tile
-  float sc[kMaxGroup][T];         // scores, then P_i = p_i * s~V_i
-  float sig[kMaxGroup];
-  float m[kMaxGroup], l[kMaxGroup], alpha[kMaxGroup], w[kMaxGroup];
-  float ks[T], kz[T], vs[T], vz[T];
-  const uint8_t* kpg[T / kPageTokens];
-  const uint8_t* vpg[T / kPageTokens];
-  int bad;
+// ------------------------------------------------------------------ workspace
+// [0]        int32 U (total work units)
+// [4..]      int32 prefix[B+1]: chunks of sequences 0..b-1 (per KV head)
+// then       int32 chunk[B]: tiles per chunk of each sequence
+// at 256-B   float partial[U][G][2 + d]
+struct WsLayout {
+  size_t prefix_off, chunk_off, part_off;
 };
+__host__ __device__ inline WsLayout ws_layout(int num_seqs) {
+  WsLayout l;
+  l.prefix_off = 4;
+  l.chunk_off = l.prefix_off + 4 * static_cast<size_t>(num_seqs + 1);
+  l.part_off = (l.chunk_off + 4 * static_cast<size_t>(num_seqs) + 255) / 256 * 256;
+  return l;
+}
 
-template <int T>
-__global__ void __launch_bounds__(kThreads) decode_split_kernel(DecodeArgs a) {
-  __shared__ DecSmem<T> sm;
-  constexpr int kPages = T / kPageTokens;
-  const int sp = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int G = a.cfg.group_size, nh = a.cfg.num_kv_heads, S = a.num_splits;
-  const PoolGeom gk = a.gk, gv = a.gv;
-  const int L = a.seq_lens[b];
-  const int F = L > 0 ? L / T : 0;
-  const int chunk = (F + S - 1) / S;
-  const int t0 = sp * chunk, t1 = min(F, t0 + chunk);
-  float* part = static_cast<float*>(a.workspace) +
-                ((static_cast<size_t>(b) * nh + h) * S + sp) * G * kPartFloats;
-  if (t0 >= t1) {
-    if (tid < G) {
-      part[tid * kPartFloats + 0] = -INFINITY;
-      part[tid * kPartFloats + 1] = 0.f;
-    }
-    return;
+// ------------------------------------------------------------------ PTX helpers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ long long global_ns() {
+  long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Wait for a phase with a time bound; false on timeout.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = global_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_ns() - t0 > kWaitLimitNs) return false;
   }
-  const float qscale = a.softmax_scale * kLog2e / kSqrtHeadDim;
-  const __half* q = static_cast<const __half*>(a.q) + (static_cast<size_t>(b) * nh + h) * G * kHeadDim;
-  for (int hh = warp; hh < G; hh += 4) {
-    const uint2 raw = *reinterpret_cast<const uint2*>(q + hh * kHeadDim + 4 * lane);
-    const __half2 h01 = *reinterpret_cast<const __half2*>(&raw.x);
-    const __half2 h23 = *reinterpret_cast<const __half2*>(&raw.y);
-    float v[4] = {__low2float(h01), __high2float(h01), __low2float(h23), __high2float(h23)};
-    fwht128_warp(v, lane);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) sm.qr[hh][4 * lane + k] = v[k] * qscale;
-  }
-  if (tid < G) {
-    sm.m[tid] = -INFINITY;
-    sm.l[tid] = 0.f;
-  }
-  float acc[kMaxGroup];
-#pragma unroll
-  for (int hh = 0; hh < kMaxGroup; ++hh) acc[hh] = 0.f;
-  const uint8_t* kpool = static_cast<const uint8_t*>(a.k_pool);
-  const uint8_t* vpool = static_cast<const uint8_t*>(a.v_pool);
+  return true;
+}
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;  // (a & b) | c
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ void mma16816(float d[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+__device__ __forceinline__ __half2 u32_as_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
 
-  for (int t = t0; t < t1; ++t) {
-    if (tid == 0) sm.bad = 0;
-    __syncthreads();
-    if (tid < kPages) {
-      const int lb = t * kPages + tid;
-      const int blk = lb < a.max_blocks_per_seq
-                          ? a.block_tables[static_cast<size_t>(b) * a.max_blocks_per_seq + lb]
-                          : -1;
-      if (blk < 0 || blk >= a.num_blocks) {
-        sm.bad = 1;
-        report_error(a.dev_status, KVQ_ERR_DEVICE_BOUNDS);
-      } else {
-        sm.kpg[tid] = kpool + (static_cast<size_t>(blk) * nh + h) * gk.page_bytes;
-        sm.vpg[tid] = vpool + (static_cast<size_t>(blk) * nh + h) * gv.page_bytes;
-      }
-    }
-    __syncthreads();
-    if (sm.bad) continue;
-    const int j = tid;
-    const float ck = __half2float(*reinterpret_cast<const __half*>(sm.kpg[j / gk.cs_channels] + gk.cslice_off +
-                                                                    2 * (j % gk.cs_channels)));
-    const float cv = __half2float(*reinterpret_cast<const __half*>(sm.vpg[j / gv.cs_channels] + gv.cslice_off +
-                                                                    2 * (j % gv.cs_channels)));
-    for (int hh = 0; hh < G; ++hh) sm.qq[hh][j] = sm.qr[hh][j] * ck;
-    for (int i = tid; i < T; i += kThreads) {
-      const int pg = i / kPageTokens, p = i % kPageTokens;
-      const __half2 km = *reinterpret_cast<const __half2*>(sm.kpg[pg] + gk.meta_off + 4 * p);
-      const __half2 vm = *reinterpret_cast<const __half2*>(sm.vpg[pg] + gv.meta_off + 4 * p);
-      sm.ks[i] = __low2float(km);
-      sm.kz[i] = __high2float(km);
-      sm.vs[i] = __low2float(vm);
-      sm.vz[i] = __high2float(vm);
-    }
-    __syncthreads();
-    for (int hh = warp; hh < G; hh += 4) {
-      const float s4 = (sm.qq[hh][4 * lane] + sm.qq[hh][4 * lane + 1]) +
-                       (sm.qq[hh][4 * lane + 2] + sm.qq[hh][4 * lane + 3]);
-      const float s = warp_sum(s4);
-      if (lane == 0) sm.sig[hh] = s;
-    }
-    __syncthreads();
-    for (int i = tid; i < T; i += kThreads) {  // scores: thread = token
-      const uint8_t* pg = sm.kpg[i / kPageTokens];
-      const int p = i % kPageTokens;
-      float dot[kMaxGroup];
+// A 32-bit word of b-bit codes -> fp16 pairs holding exact small integers.
+// b = 4: pair e (0..3) = (nibble e, nibble e+4);  b = 2: pair e (0..7) =
+// (field e, field e+8).  The fields land in fp16 mantissas under the
+// exponent of 1024 (0x6400) and are rebased with one fused multiply-add.
+template <int B>
+__device__ __forceinline__ void unpack_word(uint32_t w, uint32_t out[16 / B]) {
+  const uint32_t magic = 0x64006400u;
+  if constexpr (B == 4) {
+    const uint32_t w8 = w >> 8;
+    const __half2 k1024 = __float2half2_rn(1024.f);
+    const __half2 s16 = __float2half2_rn(1.f / 16.f), o64 = __float2half2_rn(-64.f);
+    out[0] = h2_as_u32(__hsub2(u32_as_h2(lop3_and_or(w, 0x000F000Fu, magic)), k1024));
+    out[1] = h2_as_u32(__hfma2(u32_as_h2(lop3_and_or(w, 0x00F000F0u, magic)), s16, o64));
+    out[2] = h2_as_u32(__hsub2(u32_as_h2(lop3_and_or(w8, 0x000F000Fu, magic)), k1024));
+    out[3] = h2_as_u32(__hfma2(u32_as_h2(lop3_and_or(w8, 0x00F000F0u, magic)), s16, o64));
+  } else {
+    const uint32_t w8 = w >> 8;
+    const __half2 k1024 = __float2half2_rn(1024.f);
+    const __half2 s4 = __float2half2_rn(0.25f), o256 = __float2half2_rn(-256.f);
+    const __half2 s16 = __float2half2_rn(1.f / 16.f), o64 = __float2half2_rn(-64.f);
+    const __half2 s64 = __float2half2_rn(1.f / 64.f), o16 = __float2half2_rn(-16.f);
 #pragma unroll
-      for (int hh = 0; hh < kMaxGroup; ++hh) dot[hh] = 0.f;
-      for (int c = 0; c < kHeadDim; ++c) {
-        const float code = static_cast<float>(read_code(pg, code_bit(c, p, gk.bits, false), gk.bits));
-#pragma unroll
-        for (int hh = 0; hh < kMaxGroup; ++hh)
-          if (hh < G) dot[hh] += sm.qq[hh][c] * code;
-      }
-      for (int hh = 0; hh < G; ++hh) sm.sc[hh][i] = sm.ks[i] * dot[hh] + sm.kz[i] * sm.sig[hh];
+    for (int half = 0; half < 2; ++half) {
+      const uint32_t x = half ? w8 : w;
+      out[4 * half + 0] = h2_as_u32(__hsub2(u32_as_h2(lop3_and_or(x, 0x00030003u, magic)), k1024));
+      out[4 * half + 1] = h2_as_u32(__hfma2(u32_as_h2(lop3_and_or(x, 0x000C000Cu, magic)), s4, o256));
+      out[4 * half + 2] = h2_as_u32(__hfma2(u32_as_h2(lop3_and_or(x, 0x00300030u, magic)), s16, o64));
+      out[4 * half + 3] = h2_as_u32(__hfma2(u32_as_h2(lop3_and_or(x, 0x00C000C0u, magic)), s64, o16));
     }
-    __syncthreads();
-    for (int hh = warp; hh < G; hh += 4) {  // online softmax over this tile
-      float mt = -INFINITY;
-      for (int i = lane; i < T; i += 32) mt = fmaxf(mt, sm.sc[hh][i]);
-      mt = warp_max(mt);
-      const float m_old = sm.m[hh];
-      const float m_new = fmaxf(m_old, mt);
-      float ps = 0.f, pz = 0.f;
-      for (int i = lane; i < T; i += 32) {
-        const float p = exp2f(sm.sc[hh][i] - m_new);
-        ps += p;
-        pz += p * sm.vz[i];
-        sm.sc[hh][i] = p * sm.vs[i];
-      }
-      ps = warp_sum(ps);
-      pz = warp_sum(pz);
-      if (lane == 0) {
-        const float al = exp2f(m_old - m_new);
-        sm.alpha[hh] = al;
-        sm.l[hh] = sm.l[hh] * al + ps;
-        sm.m[hh] = m_new;
-        sm.w[hh] = pz;
-      }
-    }
-    __syncthreads();
-    {  // P V: thread = channel
-      float u[kMaxGroup];
-#pragma unroll
-      for (int hh = 0; hh < kMaxGroup; ++hh) u[hh] = 0.f;
-      for (int i = 0; i < T; ++i) {
-        const float code = static_cast<float>(
-            read_code(sm.vpg[i / kPageTokens], code_bit(j, i % kPageTokens, gv.bits, true), gv.bits));
-#pragma unroll
-        for (int hh = 0; hh < kMaxGroup; ++hh)
-          if (hh < G) u[hh] += sm.sc[hh][i] * code;
-      }
-#pragma unroll
-      for (int hh = 0; hh < kMaxGroup; ++hh)
-        if (hh < G) acc[hh] = acc[hh] * sm.alpha[hh] + cv * (u[hh] + sm.w[hh]);
-    }
-    __syncthreads();
-  }
-  for (int hh = 0; hh < G; ++hh) part[hh * kPartFloats + 2 + tid] = acc[hh];
-  if (tid < G) {
-    part[tid * kPartFloats + 0] = sm.m[tid];
-    part[tid * kPartFloats + 1] = sm.l[tid];
   }
 }
 
+// Channel pair p (0..15) of lane-quad t in the K register order:
+// b = 4: word p/4, nibbles (p%4, p%4+4) -> channels 32t + 8(p/4) + p%4 + {0, 4}
+// b = 2: word p/8, fields (p%8, p%8+8) -> channels 32t + 16(p/8) + p%8 + {0, 8}
+template <int B>
+__device__ __forceinline__ constexpr int pair_ch0(int p) {
+  return B == 4 ? 8 * (p / 4) + (p % 4) : 16 * (p / 8) + (p % 8);
+}
+template <int B>
+__device__ __forceinline__ constexpr int pair_gap() {
+  return B == 4 ? 4 : 8;
+}
+
+// ------------------------------------------------------------------ schedule
+__global__ void __launch_bounds__(1024) decode_schedule_kernel(const int32_t* seq_lens, int num_seqs, int tile_tokens,
+                                                               int num_kv_heads, int num_splits, int target_units,
+                                                               void* workspace) {
+  __shared__ long long s_total;
+  __shared__ int s_scan[1024];
+  __shared__ int s_carry;
+  const WsLayout wl = ws_layout(num_seqs);
+  int32_t* ws_i = static_cast<int32_t*>(workspace);
+  int32_t* prefix = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + wl.prefix_off);
+  int32_t* chunk = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + wl.chunk_off);
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    s_total = 0;
+    s_carry = 0;
+  }
+  __syncthreads();
+  long long part = 0;
+  for (int b = tid; b < num_seqs; b += blockDim.x) part += max(seq_lens[b], 0) / tile_tokens;
+  atomicAdd(reinterpret_cast<unsigned long long*>(&s_total), static_cast<unsigned long long>(part));
+  __syncthreads();
+  const long long total = s_total;
+  long long ch_auto = 1;
+  if (num_splits == 0 && total > 0)
+    ch_auto = std::max(1LL, (total * num_kv_heads + target_units - 1) / target_units);
+  for (int base = 0; base < num_seqs; base += blockDim.x) {
+    const int b = base + tid;
+    int units = 0;
+    if (b < num_seqs) {
+      const int f = max(seq_lens[b], 0) / tile_tokens;
+      int ch;
+      if (num_splits > 0) {
+        const int s = min(num_splits, f);
+        ch = s > 0 ? (f + s - 1) / s : 1;
+      } else {
+        ch = static_cast<int>(std::min<long long>(ch_auto, 1 << 30));
+      }
+      units = f > 0 ? (f + ch - 1) / ch : 0;
+      chunk[b] = ch;
+    }
+    s_scan[tid] = units;
+    __syncthreads();
+    for (int off = 1; off < static_cast<int>(blockDim.x); off <<= 1) {  // inclusive scan
+      const int v = tid >= off ? s_scan[tid - off] : 0;
+      __syncthreads();
+      s_scan[tid] += v;
+      __syncthreads();
+    }
+    if (b < num_seqs) prefix[b] = s_carry + s_scan[tid] - units;
+    __syncthreads();
+    if (tid == blockDim.x - 1) s_carry += s_scan[tid];
+    __syncthreads();
+  }
+  if (tid == 0) {
+    prefix[num_seqs] = s_carry;
+    ws_i[0] = s_carry * num_kv_heads;
+  }
+}
+
+// ------------------------------------------------------------------ main decode
+template <int T, int BK, int BV>
+struct DecodeGeom {
+  static constexpr int kPages = T / kPageTokens;
+  static constexpr int kCodesK = kPageTokens * kHeadDim * BK / 8;
+  static constexpr int kCodesV = kPageTokens * kHeadDim * BV / 8;
+  static constexpr int kCs = kHeadDim * kPageTokens / T;        // C-slice channels per page
+  static constexpr int kCsBytes = (2 * kCs + 15) / 16 * 16;
+  static constexpr int kPageK = kCodesK + 64 + kCsBytes;
+  static constexpr int kPageV = kCodesV + 64 + kCsBytes;
+  static constexpr int kStage = kPages * (kPageK + kPageV);    // one tile, K pages then V pages
+  static constexpr int kSmem = kDecWarps * (2 * kStage + 16);
+};
+
+template <int T, int BK, int BV>
+__global__ void __launch_bounds__(kDecWarps * 32) decode_tiles_kernel(DecodeArgs a) {
+  using Geo = DecodeGeom<T, BK, BV>;
+  constexpr int NP = Geo::kPages;
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  unsigned char* stage_base = smem + warp * 2 * Geo::kStage;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kDecWarps * 2 * Geo::kStage) + 2 * warp;
+  if (lane == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncwarp();
+
+  const int G = a.cfg.group_size, nh = a.cfg.num_kv_heads;
+  const WsLayout wl = ws_layout(a.num_seqs);
+  const int32_t* ws_i = static_cast<const int32_t*>(a.workspace);
+  const int32_t* prefix = reinterpret_cast<const int32_t*>(static_cast<const char*>(a.workspace) + wl.prefix_off);
+  const int32_t* chunk = reinterpret_cast<const int32_t*>(static_cast<const char*>(a.workspace) + wl.chunk_off);
+  float* parts = reinterpret_cast<float*>(static_cast<char*>(a.workspace) + wl.part_off);
+  const int U = ws_i[0];
+  const uint8_t* kpool = static_cast<const uint8_t*>(a.k_pool);
+  const uint8_t* vpool = static_cast<const uint8_t*>(a.v_pool);
+  const float qscale = a.softmax_scale * kLog2e / kSqrtHeadDim;
+  const bool head_live = g < G;
+  uint32_t phase[2] = {0u, 0u};
+  bool pending[2] = {false, false};  // copies issued into the stage and not yet waited for
+  bool failed = false;
+
+  const int total_warps = gridDim.x * kDecWarps;
+  for (int u = blockIdx.x * kDecWarps + warp; u < U && !failed; u += total_warps) {
+    // ---- locate the unit: sequence b (binary search), head h, chunk c
+    int lo = 0, hi = a.num_seqs;  // find the largest b with nh*prefix[b] <= u
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (nh * prefix[mid] <= u) lo = mid; else hi = mid;
+    }
+    const int b = lo;
+    const int S = prefix[b + 1] - prefix[b];
+    const int r = u - nh * prefix[b];
+    const int h = r / S, c = r % S;
+    const int F = max(a.seq_lens[b], 0) / T;
+    const int ch = chunk[b];
+    const int t0 = c * ch, t1 = min(F, t0 + ch);
+
+    // ---- rotated, scaled query: lane (g, t) holds channels 32t..32t+31 of head g
+    float qs[32];
+    if (head_live) {
+      const __half* qp = static_cast<const __half*>(a.q) +
+                         ((static_cast<size_t>(b) * nh + h) * G + g) * kHeadDim + 32 * t;
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const uint4 raw = *reinterpret_cast<const uint4*>(qp + 8 * v);
+        const __half2* hp = reinterpret_cast<const __half2*>(&raw);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 f = __half22float2(hp[k]);
+          qs[8 * v + 2 * k] = f.x;
+          qs[8 * v + 2 * k + 1] = f.y;
+        }
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) qs[i] = 0.f;
+    }
+#pragma unroll
+    for (int bit = 0; bit < 5; ++bit) {  // channel bits 0..4: in-register butterflies
+      const int m = 1 << bit;
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (!(i & m)) {
+          const float x = qs[i], y = qs[i | m];
+          qs[i] = x + y;
+          qs[i | m] = x - y;
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {  // channel bits 5, 6: lanes with t differing in bit k
+      const int m = 1 << k;
+      const bool upper = t & m;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float o = __shfl_xor_sync(kFull, qs[i], m);
+        qs[i] = upper ? (o - qs[i]) : (qs[i] + o);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 32; ++i) qs[i] *= qscale;
+
+    float m_run = -INFINITY, l_part = 0.f;
+    float acc[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+
+    // ---- issue the first two tiles
+    auto issue = [&](int tile, int st) {
+      // lanes 0..NP-1 read and check the block ids of the tile's pages
+      const int lb = tile * NP + lane;
+      int blk = -1;
+      if (lane < NP)
+        blk = lb < a.max_blocks_per_seq ? a.block_tables[static_cast<size_t>(b) * a.max_blocks_per_seq + lb] : -1;
+      const bool bad = lane < NP && (blk < 0 || blk >= a.num_blocks);
+      if (__any_sync(kFull, bad)) {
+        if (lane == 0) report_error(a.dev_status, KVQ_ERR_DEVICE_BOUNDS);
+        pending[st] = false;
+        return;
+      }
+      if (lane == 0) mbar_arrive_expect_tx(&bars[st], NP * (Geo::kPageK + Geo::kPageV));
+      __syncwarp();
+      unsigned char* dst = stage_base + st * Geo::kStage;
+      if (lane < NP) {
+        const size_t reg = static_cast<size_t>(blk) * nh + h;
+        bulk_g2s(dst + lane * Geo::kPageK, kpool + reg * Geo::kPageK, Geo::kPageK, &bars[st]);
+        bulk_g2s(dst + NP * Geo::kPageK + lane * Geo::kPageV, vpool + reg * Geo::kPageV, Geo::kPageV, &bars[st]);
+      }
+      pending[st] = true;
+    };
+    if (t0 < t1) issue(t0, 0);
+    if (t0 + 1 < t1) issue(t0 + 1, 1);
+
+    for (int i = t0; i < t1; ++i) {
+      const int st = (i - t0) & 1;
+      if (!pending[st]) {  // tile skipped (bad block id, already reported)
+        if (i + 2 < t1) issue(i + 2, st);
+        continue;
+      }
+      if (!mbar_wait_bounded(&bars[st], phase[st])) {
+        if (lane == 0) report_error(a.dev_status, KVQ_ERR_DEVICE_TIMEOUT);
+        failed = true;
+        break;
+      }
+      phase[st] ^= 1u;
+      pending[st] = false;
+      const unsigned char* sK = stage_base + st * Geo::kStage;
+      const unsigned char* sV = sK + NP * Geo::kPageK;
+
+      // -- q'' = q' * C~K in hi/lo fp16 pairs (A operand rows g and g+8) and sigma
+      uint32_t qa_hi[16], qa_lo[16];
+      float sig = 0.f;
+      {
+        float ck[32];
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const int c0 = 32 * t + 8 * v;  // channels c0..c0+7, within one page slice
+          const unsigned char* src = sK + (c0 / Geo::kCs) * Geo::kPageK + Geo::kCodesK + 64 + 2 * (c0 % Geo::kCs);
+          const uint4 raw = *reinterpret_cast<const uint4*>(src);
+          const __half2* hp = reinterpret_cast<const __half2*>(&raw);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 f = __half22float2(hp[k]);
+            ck[8 * v + 2 * k] = f.x;
+            ck[8 * v + 2 * k + 1] = f.y;
+          }
+        }
+#pragma unroll
+        for (int p = 0; p < 16; ++p) {
+          const int c0 = pair_ch0<BK>(p), c1 = c0 + pair_gap<BK>();
+          const float x0 = qs[c0] * ck[c0], x1 = qs[c1] * ck[c1];
+          sig += x0 + x1;
+          const __half2 hv = __floats2half2_rn(x0, x1);
+          const float2 hf = __half22float2(hv);
+          qa_hi[p] = h2_as_u32(hv);
+          qa_lo[p] = h2_as_u32(__floats2half2_rn(x0 - hf.x, x1 - hf.y));
+        }
+        sig += __shfl_xor_sync(kFull, sig, 1);
+        sig += __shfl_xor_sync(kFull, sig, 2);
+      }
+
+      // -- scores: D[16 rows][8 tokens] per (page, n-block); rows g / g+8 = head g hi / lo
+      float sd[NP][2][4];
+#pragma unroll
+      for (int pg = 0; pg < NP; ++pg)
+#pragma unroll
+        for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+          for (int k = 0; k < 4; ++k) sd[pg][nb][k] = 0.f;
+      constexpr int kWords = BK;  // 32-bit words per lane per token record
+#pragma unroll
+      for (int wd = 0; wd < kWords; ++wd) {
+#pragma unroll
+        for (int pg = 0; pg < NP; ++pg) {
+#pragma unroll
+          for (int nb = 0; nb < 2; ++nb) {
+            const int tok = 8 * nb + g;
+            const uint32_t w = *reinterpret_cast<const uint32_t*>(sK + pg * Geo::kPageK + tok * (16 * BK) +
+                                                                  t * (4 * BK) + 4 * wd);
+            uint32_t pr[16 / BK];
+            unpack_word<BK>(w, pr);
+            constexpr int kbPerWord = 8 / BK;  // k-blocks per word: 2 (b=4) or 4 (b=2)
+#pragma unroll
+            for (int j = 0; j < kbPerWord; ++j) {
+              const int kb = wd * kbPerWord + j;
+              const uint32_t afr[4] = {qa_hi[2 * kb], qa_lo[2 * kb], qa_hi[2 * kb + 1], qa_lo[2 * kb + 1]};
+              mma16816(sd[pg][nb], afr, pr[2 * j], pr[2 * j + 1]);
+            }
+          }
+        }
+      }
+
+      // -- scores in the log2 domain; tokens (8nb + 2t, 8nb + 2t + 1) of each page
+      float sc[NP][2][2];
+      float mt = -INFINITY;
+#pragma unroll
+      for (int pg = 0; pg < NP; ++pg) {
+        const unsigned char* meta = sK + pg * Geo::kPageK + Geo::kCodesK;
+#pragma unroll
+        for (int nb = 0; nb < 2; ++nb) {
+          const uint2 mm = *reinterpret_cast<const uint2*>(meta + 4 * (8 * nb + 2 * t));
+          const float2 m0 = __half22float2(u32_as_h2(mm.x)), m1 = __half22float2(u32_as_h2(mm.y));
+          sc[pg][nb][0] = m0.x * (sd[pg][nb][0] + sd[pg][nb][2]) + m0.y * sig;
+          sc[pg][nb][1] = m1.x * (sd[pg][nb][1] + sd[pg][nb][3]) + m1.y * sig;
+          mt = fmaxf(mt, fmaxf(sc[pg][nb][0], sc[pg][nb][1]));
+        }
+      }
+      mt = fmaxf(mt, __shfl_xor_sync(kFull, mt, 1));
+      mt = fmaxf(mt, __shfl_xor_sync(kFull, mt, 2));
+      const float m_new = fmaxf(m_run, mt);
+      const float alpha = exp2f(m_run - m_new);
+      m_run = m_new;
+      l_part *= alpha;
+
+      // -- P = p * s~V as hi/lo fp16 A fragments per page; w = sum p z~V
+      uint32_t pa[NP][4];
+      float wsum = 0.f;
+#pragma unroll
+      for (int pg = 0; pg < NP; ++pg) {
+        const unsigned char* meta = sV + pg * Geo::kPageV + Geo::kCodesV;
+#pragma unroll
+        for (int nb = 0; nb < 2; ++nb) {
+          const uint2 mm = *reinterpret_cast<const uint2*>(meta + 4 * (8 * nb + 2 * t));
+          const float2 m0 = __half22float2(u32_as_h2(mm.x)), m1 = __half22float2(u32_as_h2(mm.y));
+          const float p0 = exp2f(sc[pg][nb][0] - m_new), p1 = exp2f(sc[pg][nb][1] - m_new);
+          l_part += p0 + p1;
+          wsum += p0 * m0.y + p1 * m1.y;
+          const float x0 = p0 * m0.x, x1 = p1 * m1.x;
+          const __half2 hv = __floats2half2_rn(x0, x1);
+          const float2 hf = __half22float2(hv);
+          pa[pg][2 * nb] = h2_as_u32(hv);
+          pa[pg][2 * nb + 1] = h2_as_u32(__floats2half2_rn(x0 - hf.x, x1 - hf.y));
+        }
+      }
+      wsum += __shfl_xor_sync(kFull, wsum, 1);
+      wsum += __shfl_xor_sync(kFull, wsum, 2);
+
+      // -- P V: D[16 rows][8 channels] per n-block (channels 8nv..8nv+7)
+      float dv[16][4];
+#pragma unroll
+      for (int nv = 0; nv < 16; ++nv)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) dv[nv][k] = 0.f;
+      constexpr int kWordsV = 2 * BV;       // words per lane per page
+      constexpr int kPairsV = 16 / BV;      // pairs per word
+#pragma unroll
+      for (int pg = 0; pg < NP; ++pg) {
+        const uint32_t afr[4] = {pa[pg][0], pa[pg][1], pa[pg][2], pa[pg][3]};
+        const unsigned char* vrec = sV + pg * Geo::kPageV;
+#pragma unroll
+        for (int kw = 0; kw < kWordsV; kw += 2) {
+          // words kw (tokens 2t, 2t+1) and kw+1 (tokens 2t+8, 2t+9) of the same n-blocks
+          const uint32_t w0 = *reinterpret_cast<const uint32_t*>(vrec + ((kw >> 2) * 32 + lane) * 16 + (kw & 3) * 4);
+          const uint32_t w1 =
+              *reinterpret_cast<const uint32_t*>(vrec + (((kw + 1) >> 2) * 32 + lane) * 16 + ((kw + 1) & 3) * 4);
+          uint32_t p0[kPairsV], p1[kPairsV];
+          unpack_word<BV>(w0, p0);
+          unpack_word<BV>(w1, p1);
+#pragma unroll
+          for (int e = 0; e < kPairsV; ++e) {
+            const int nv = kPairsV * (kw >> 1) + e;
+            mma16816(dv[nv], afr, p0[e], p1[e]);
+          }
+        }
+      }
+
+      // -- acc' = alpha acc' + C~V (u + w); lane (g,t) owns channels 8nv + 2t, 8nv + 2t + 1
+#pragma unroll
+      for (int nv = 0; nv < 16; ++nv) {
+        const int c0 = 8 * nv + 2 * t;
+        const __half2 cvh = *reinterpret_cast<const __half2*>(sV + (c0 / Geo::kCs) * Geo::kPageV + Geo::kCodesV + 64 +
+                                                              2 * (c0 % Geo::kCs));
+        const float2 cv = __half22float2(cvh);
+        acc[2 * nv] = alpha * acc[2 * nv] + cv.x * (dv[nv][0] + dv[nv][2] + wsum);
+        acc[2 * nv + 1] = alpha * acc[2 * nv + 1] + cv.y * (dv[nv][1] + dv[nv][3] + wsum);
+      }
+      __syncwarp();
+      if (i + 2 < t1) issue(i + 2, st);
+    }
+    if (failed) break;
+
+    // ---- partial of this unit
+    float l_tot = l_part + __shfl_xor_sync(kFull, l_part, 1);
+    l_tot += __shfl_xor_sync(kFull, l_tot, 2);
+    if (head_live) {
+      float* part = parts + (static_cast<size_t>(u) * G + g) * kPartFloats;
+      if (t == 0) {
+        part[0] = m_run;
+        part[1] = l_tot;
+      }
+#pragma unroll
+      for (int nv = 0; nv < 16; ++nv) {
+        const int c0 = 8 * nv + 2 * t;
+        *reinterpret_cast<float2*>(part + 2 + c0) = make_float2(acc[2 * nv], acc[2 * nv + 1]);
+      }
+    }
+  }
+  if (failed) {  // let copies already in flight land before the CTA's shared memory is released
+    for (int st = 0; st < 2; ++st)
+      if (pending[st]) (void)mbar_wait_bounded(&bars[st], phase[st]);
+  }
+}
+
+// ------------------------------------------------------------------ merge
 template <int T>
 struct MergeSmem {
   float qraw[kMaxGroup][kHeadDim];
@@ -193,23 +551,28 @@ struct MergeSmem {
   float mt[kMaxGroup], lt[kMaxGroup], big_m[kMaxGroup], inv_l[kMaxGroup], et[kMaxGroup];
 };
 
-// One CTA per (sequence, KV head): raw tail, log-sum-exp merge of the
-// split partials, inverse rotation, fp16 output.
+// One CTA of 128 threads per (sequence, KV head): raw tail, log-sum-exp
+// merge of the chunk partials, inverse rotation, fp16 output.
 template <int T>
-__global__ void __launch_bounds__(kThreads) decode_merge_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(128) decode_merge_kernel(DecodeArgs a) {
   __shared__ MergeSmem<T> sm;
   const int h = blockIdx.x, b = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int G = a.cfg.group_size, nh = a.cfg.num_kv_heads, S = a.num_splits;
+  const int G = a.cfg.group_size, nh = a.cfg.num_kv_heads;
   const int L = max(a.seq_lens[b], 0);
   const int F = L / T, tau = L - F * T;
+  const WsLayout wl = ws_layout(a.num_seqs);
+  const int32_t* prefix = reinterpret_cast<const int32_t*>(static_cast<const char*>(a.workspace) + wl.prefix_off);
+  const float* parts = reinterpret_cast<const float*>(static_cast<const char*>(a.workspace) + wl.part_off);
+  const int S = prefix[b + 1] - prefix[b];
+  const size_t ubase = static_cast<size_t>(nh) * prefix[b] + static_cast<size_t>(h) * S;
   const float qscale = a.softmax_scale * kLog2e;
   const __half* q = static_cast<const __half*>(a.q) + (static_cast<size_t>(b) * nh + h) * G * kHeadDim;
   const __half* kt = static_cast<const __half*>(a.k_tail) + (static_cast<size_t>(b) * nh + h) * T * kHeadDim;
   const __half* vt = static_cast<const __half*>(a.v_tail) + (static_cast<size_t>(b) * nh + h) * T * kHeadDim;
   for (int hh = 0; hh < G; ++hh) sm.qraw[hh][tid] = __half2float(q[hh * kHeadDim + tid]) * qscale;
   __syncthreads();
-  for (int i = tid; i < tau; i += kThreads) {
+  for (int i = tid; i < tau; i += 128) {
     float dot[kMaxGroup];
 #pragma unroll
     for (int hh = 0; hh < kMaxGroup; ++hh) dot[hh] = 0.f;
@@ -251,17 +614,16 @@ __global__ void __launch_bounds__(kThreads) decode_merge_kernel(DecodeArgs a) {
     }
     for (int hh = 0; hh < G; ++hh) sm.tl[hh][tid] = at[hh];
   }
-  const float* parts = static_cast<const float*>(a.workspace) + (static_cast<size_t>(b) * nh + h) * S * G * kPartFloats;
   if (tid < G) {
     const int hh = tid;
     float m = sm.mt[hh];
     for (int s = 0; s < S; ++s) {
-      const float* pp = parts + (static_cast<size_t>(s) * G + hh) * kPartFloats;
+      const float* pp = parts + ((ubase + s) * G + hh) * kPartFloats;
       if (pp[1] > 0.f) m = fmaxf(m, pp[0]);
     }
     float l = sm.lt[hh] > 0.f ? sm.lt[hh] * exp2f(sm.mt[hh] - m) : 0.f;
     for (int s = 0; s < S; ++s) {
-      const float* pp = parts + (static_cast<size_t>(s) * G + hh) * kPartFloats;
+      const float* pp = parts + ((ubase + s) * G + hh) * kPartFloats;
       if (pp[1] > 0.f) l += pp[1] * exp2f(pp[0] - m);
     }
     sm.big_m[hh] = m;
@@ -272,7 +634,7 @@ __global__ void __launch_bounds__(kThreads) decode_merge_kernel(DecodeArgs a) {
   for (int hh = 0; hh < G; ++hh) {
     float accr = 0.f;
     for (int s = 0; s < S; ++s) {
-      const float* pp = parts + (static_cast<size_t>(s) * G + hh) * kPartFloats;
+      const float* pp = parts + ((ubase + s) * G + hh) * kPartFloats;
       if (pp[1] > 0.f) accr += exp2f(pp[0] - sm.big_m[hh]) * pp[2 + tid];
     }
     sm.fin[hh][tid] = accr;
@@ -293,28 +655,55 @@ __global__ void __launch_bounds__(kThreads) decode_merge_kernel(DecodeArgs a) {
   }
 }
 
+int device_sms() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
+}
+
+template <int T, int BK, int BV>
+cudaError_t launch_tiles_t(const DecodeArgs& a, cudaStream_t s, int grid) {
+  using Geo = DecodeGeom<T, BK, BV>;
+  auto kern = decode_tiles_kernel<T, BK, BV>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Geo::kSmem);
+  if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kDecWarps * 32, Geo::kSmem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid * std::max(per_sm, 1), kDecWarps * 32, Geo::kSmem, s>>>(a);
+  return cudaGetLastError();
+}
+
+template <int T>
+cudaError_t launch_tiles_bits(const DecodeArgs& a, cudaStream_t s, int grid) {
+  if (a.cfg.bits_k == 4 && a.cfg.bits_v == 4) return launch_tiles_t<T, 4, 4>(a, s, grid);
+  if (a.cfg.bits_k == 4 && a.cfg.bits_v == 2) return launch_tiles_t<T, 4, 2>(a, s, grid);
+  if (a.cfg.bits_k == 2 && a.cfg.bits_v == 4) return launch_tiles_t<T, 2, 4>(a, s, grid);
+  return launch_tiles_t<T, 2, 2>(a, s, grid);
+}
+
 template <int T>
 cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t s) {
-  dim3 g1(a.num_splits, a.cfg.num_kv_heads, a.num_seqs);
-  decode_split_kernel<T><<<g1, kThreads, 0, s>>>(a);
+  const int sms = device_sms();
+  decode_schedule_kernel<<<1, 1024, 0, s>>>(a.seq_lens, a.num_seqs, T, a.cfg.num_kv_heads, a.num_splits_fixed,
+                                            kUnitsPerSm * sms, a.workspace);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  e = launch_tiles_bits<T>(a, s, sms);
+  if (e != cudaSuccess) return e;
   dim3 g2(a.cfg.num_kv_heads, a.num_seqs);
-  decode_merge_kernel<T><<<g2, kThreads, 0, s>>>(a);
+  decode_merge_kernel<T><<<g2, 128, 0, s>>>(a);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-size_t decode_workspace_bytes(const kvq_config& cfg, int num_seqs, int num_splits) {
-  return static_cast<size_t>(num_seqs) * cfg.num_kv_heads * num_splits * cfg.group_size * kPartFloats *
-         sizeof(float);
-}
-
-int decode_auto_splits(const kvq_config& cfg, int num_seqs, int num_sms) {
-  const long pairs = std::max(1L, static_cast<long>(num_seqs) * cfg.num_kv_heads);
-  const long want = (4L * num_sms + pairs - 1) / pairs;
-  return static_cast<int>(std::min(256L, std::max(1L, want)));
+size_t decode_workspace_bytes(const kvq_config& cfg, int num_seqs, int num_splits, int num_sms) {
+  const WsLayout wl = ws_layout(num_seqs);
+  const size_t units = num_splits > 0
+                           ? static_cast<size_t>(num_seqs) * cfg.num_kv_heads * num_splits
+                           : static_cast<size_t>(kUnitsPerSm) * num_sms + static_cast<size_t>(num_seqs) * cfg.num_kv_heads;
+  return wl.part_off + units * cfg.group_size * kPartFloats * sizeof(float);
 }
 
 cudaError_t launch_paged_decode(const DecodeArgs& a, cudaStream_t s) {

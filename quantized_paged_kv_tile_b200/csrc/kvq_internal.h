@@ -103,13 +103,11 @@ struct DecodeArgs {
   const void* v_tail;
   float softmax_scale;
   void* workspace;
-  int num_splits;  // resolved (> 0)
+  int num_splits_fixed;  // > 0: chunks per (sequence, KV head); 0: automatic
   int32_t* dev_status;
 };
-// Workspace bytes for a resolved split count.
-size_t decode_workspace_bytes(const kvq_config& cfg, int num_seqs, int num_splits);
-// Split count used when the caller passes 0.
-int decode_auto_splits(const kvq_config& cfg, int num_seqs, int num_sms);
+// Workspace bytes for a split setting on a device with num_sms SMs.
+size_t decode_workspace_bytes(const kvq_config& cfg, int num_seqs, int num_splits, int num_sms);
 cudaError_t launch_paged_decode(const DecodeArgs& a, cudaStream_t s);
 
 }  // namespace kvq
