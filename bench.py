@@ -212,7 +212,8 @@ def run_kvq(args, ranks):
     kvq.load_library()
     dev = torch.device("cuda", ranks.local_rank)
     torch.cuda.set_device(dev)
-    w = synth.workload(args.workload, replica=ranks.rank)
+    over = {"num_seqs": args.num_seqs} if args.num_seqs > 0 else {}
+    w = synth.workload(args.workload, replica=ranks.rank, **over)
     cfg = kvq.Config(num_kv_heads=w.num_kv_heads, group_size=w.group_size, tile_tokens=w.tile_tokens,
                      bits_k=w.bits_k, bits_v=w.bits_v, iters=w.iters)
     lay = kvq.get_layout(cfg)
@@ -430,6 +431,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["kvq", "reference"], default="kvq")
     ap.add_argument("--workload", default="qwen3_4b")
+    ap.add_argument("--num-seqs", type=int, default=0,
+                    help="override the workload's sequence count (smaller inputs for profiler captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()

@@ -35,7 +35,10 @@ namespace kvq {
 
 namespace {
 
-constexpr int kPartFloats = 2 + kHeadDim;  // m, l, acc[d] per query head
+// Partial record per (work unit, query head): m, l, two pad floats, acc[d];
+// 132 floats = 528 bytes, so every record and its acc start 16-byte aligned.
+constexpr int kPartFloats = 4 + kHeadDim;
+constexpr int kPartAcc = 4;
 constexpr int kDecWarps = 4;               // warps per decode CTA
 constexpr int kUnitsPerSm = 32;            // work-unit budget of the automatic split
 constexpr long long kWaitLimitNs = 2000000000LL;  // bounded mbarrier waits: 2 s
@@ -44,7 +47,7 @@ constexpr long long kWaitLimitNs = 2000000000LL;  // bounded mbarrier waits: 2 s
 // [0]        int32 U (total work units)
 // [4..]      int32 prefix[B+1]: chunks of sequences 0..b-1 (per KV head)
 // then       int32 chunk[B]: tiles per chunk of each sequence
-// at 256-B   float partial[U][G][2 + d]
+// at 256-B   float partial[U][G][4 + d]  (m, l, pad, pad, acc)
 struct WsLayout {
   size_t prefix_off, chunk_off, part_off;
 };
@@ -103,7 +106,7 @@ __device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t b, uint32_t
   return d;
 }
 __device__ __forceinline__ void mma16816(float d[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
@@ -230,7 +233,7 @@ struct DecodeGeom {
 };
 
 template <int T, int BK, int BV>
-__global__ void __launch_bounds__(kDecWarps * 32) decode_tiles_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(kDecWarps * 32, T == 128 ? 2 : 3) decode_tiles_kernel(DecodeArgs a) {
   using Geo = DecodeGeom<T, BK, BV>;
   constexpr int NP = Geo::kPages;
   extern __shared__ __align__(128) unsigned char smem[];
@@ -407,25 +410,38 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_tiles_kernel(DecodeArgs
         for (int nb = 0; nb < 2; ++nb)
 #pragma unroll
           for (int k = 0; k < 4; ++k) sd[pg][nb][k] = 0.f;
-      constexpr int kWords = BK;  // 32-bit words per lane per token record
+      {
+        // lane (g, t) reads its 4*BK-byte chunk (channels 32t..32t+31) of tokens g and 8+g
+        uint32_t rec[NP][2][BK];
 #pragma unroll
-      for (int wd = 0; wd < kWords; ++wd) {
-#pragma unroll
-        for (int pg = 0; pg < NP; ++pg) {
+        for (int pg = 0; pg < NP; ++pg)
 #pragma unroll
           for (int nb = 0; nb < 2; ++nb) {
-            const int tok = 8 * nb + g;
-            const uint32_t w = *reinterpret_cast<const uint32_t*>(sK + pg * Geo::kPageK + tok * (16 * BK) +
-                                                                  t * (4 * BK) + 4 * wd);
-            uint32_t pr[16 / BK];
-            unpack_word<BK>(w, pr);
-            constexpr int kbPerWord = 8 / BK;  // k-blocks per word: 2 (b=4) or 4 (b=2)
-#pragma unroll
-            for (int j = 0; j < kbPerWord; ++j) {
-              const int kb = wd * kbPerWord + j;
-              const uint32_t afr[4] = {qa_hi[2 * kb], qa_lo[2 * kb], qa_hi[2 * kb + 1], qa_lo[2 * kb + 1]};
-              mma16816(sd[pg][nb], afr, pr[2 * j], pr[2 * j + 1]);
+            const unsigned char* src = sK + pg * Geo::kPageK + (8 * nb + g) * (16 * BK) + t * (4 * BK);
+            if constexpr (BK == 4) {
+              const uint4 v = *reinterpret_cast<const uint4*>(src);
+              rec[pg][nb][0] = v.x; rec[pg][nb][1] = v.y; rec[pg][nb][2] = v.z; rec[pg][nb][3] = v.w;
+            } else {
+              const uint2 v = *reinterpret_cast<const uint2*>(src);
+              rec[pg][nb][0] = v.x; rec[pg][nb][1] = v.y;
             }
+          }
+        constexpr int kbPerWord = 8 / BK;  // k-blocks per word: 2 (b=4) or 4 (b=2)
+#pragma unroll
+        for (int wd = 0; wd < BK; ++wd) {
+          uint32_t pr[NP][2][16 / BK];
+#pragma unroll
+          for (int pg = 0; pg < NP; ++pg)
+#pragma unroll
+            for (int nb = 0; nb < 2; ++nb) unpack_word<BK>(rec[pg][nb][wd], pr[pg][nb]);
+#pragma unroll
+          for (int j = 0; j < kbPerWord; ++j) {
+            const int kb = wd * kbPerWord + j;
+            const uint32_t afr[4] = {qa_hi[2 * kb], qa_lo[2 * kb], qa_hi[2 * kb + 1], qa_lo[2 * kb + 1]};
+#pragma unroll
+            for (int pg = 0; pg < NP; ++pg)
+#pragma unroll
+              for (int nb = 0; nb < 2; ++nb) mma16816(sd[pg][nb], afr, pr[pg][nb][2 * j], pr[pg][nb][2 * j + 1]);
           }
         }
       }
@@ -475,44 +491,42 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_tiles_kernel(DecodeArgs
       wsum += __shfl_xor_sync(kFull, wsum, 1);
       wsum += __shfl_xor_sync(kFull, wsum, 2);
 
-      // -- P V: D[16 rows][8 channels] per n-block (channels 8nv..8nv+7)
-      float dv[16][4];
+      // -- P V: D[16 rows][8 channels] per n-block (channels 8nv..8nv+7).  Lane
+      // words 2q, 2q+1 (token pairs {2t,2t+1} and {2t+8,2t+9}) hold the n-blocks
+      // kPairsV*q .. kPairsV*q + kPairsV-1; a group's accumulators are folded
+      // into acc' (times C~V) as soon as all pages of the tile are in.
+      constexpr int kPairsV = 16 / BV;      // n-blocks per word pair
+      constexpr int kGroups = 16 / kPairsV;  // word pairs per lane (4 at b=4, 2 at b=2)
 #pragma unroll
-      for (int nv = 0; nv < 16; ++nv)
+      for (int q = 0; q < kGroups; ++q) {
+        float dv[kPairsV][4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) dv[nv][k] = 0.f;
-      constexpr int kWordsV = 2 * BV;       // words per lane per page
-      constexpr int kPairsV = 16 / BV;      // pairs per word
+        for (int e = 0; e < kPairsV; ++e)
 #pragma unroll
-      for (int pg = 0; pg < NP; ++pg) {
-        const uint32_t afr[4] = {pa[pg][0], pa[pg][1], pa[pg][2], pa[pg][3]};
-        const unsigned char* vrec = sV + pg * Geo::kPageV;
+          for (int k = 0; k < 4; ++k) dv[e][k] = 0.f;
 #pragma unroll
-        for (int kw = 0; kw < kWordsV; kw += 2) {
-          // words kw (tokens 2t, 2t+1) and kw+1 (tokens 2t+8, 2t+9) of the same n-blocks
-          const uint32_t w0 = *reinterpret_cast<const uint32_t*>(vrec + ((kw >> 2) * 32 + lane) * 16 + (kw & 3) * 4);
-          const uint32_t w1 =
-              *reinterpret_cast<const uint32_t*>(vrec + (((kw + 1) >> 2) * 32 + lane) * 16 + ((kw + 1) & 3) * 4);
+        for (int pg = 0; pg < NP; ++pg) {
+          const uint32_t afr[4] = {pa[pg][0], pa[pg][1], pa[pg][2], pa[pg][3]};
+          // words 2q and 2q+1 sit in the same 16-byte row of the lane; the whole
+          // row is loaded (lanes read consecutive 16-byte rows: no bank conflict)
+          const uint4 row = *reinterpret_cast<const uint4*>(sV + pg * Geo::kPageV + (((2 * q) >> 2) * 32 + lane) * 16);
+          const uint32_t w0 = (q & 1) ? row.z : row.x, w1 = (q & 1) ? row.w : row.y;
           uint32_t p0[kPairsV], p1[kPairsV];
           unpack_word<BV>(w0, p0);
           unpack_word<BV>(w1, p1);
 #pragma unroll
-          for (int e = 0; e < kPairsV; ++e) {
-            const int nv = kPairsV * (kw >> 1) + e;
-            mma16816(dv[nv], afr, p0[e], p1[e]);
-          }
+          for (int e = 0; e < kPairsV; ++e) mma16816(dv[e], afr, p0[e], p1[e]);
         }
-      }
-
-      // -- acc' = alpha acc' + C~V (u + w); lane (g,t) owns channels 8nv + 2t, 8nv + 2t + 1
 #pragma unroll
-      for (int nv = 0; nv < 16; ++nv) {
-        const int c0 = 8 * nv + 2 * t;
-        const __half2 cvh = *reinterpret_cast<const __half2*>(sV + (c0 / Geo::kCs) * Geo::kPageV + Geo::kCodesV + 64 +
-                                                              2 * (c0 % Geo::kCs));
-        const float2 cv = __half22float2(cvh);
-        acc[2 * nv] = alpha * acc[2 * nv] + cv.x * (dv[nv][0] + dv[nv][2] + wsum);
-        acc[2 * nv + 1] = alpha * acc[2 * nv + 1] + cv.y * (dv[nv][1] + dv[nv][3] + wsum);
+        for (int e = 0; e < kPairsV; ++e) {
+          const int nv = kPairsV * q + e;
+          const int c0 = 8 * nv + 2 * t;
+          const __half2 cvh = *reinterpret_cast<const __half2*>(sV + (c0 / Geo::kCs) * Geo::kPageV + Geo::kCodesV +
+                                                                64 + 2 * (c0 % Geo::kCs));
+          const float2 cv = __half22float2(cvh);
+          acc[2 * nv] = alpha * acc[2 * nv] + cv.x * (dv[e][0] + dv[e][2] + wsum);
+          acc[2 * nv + 1] = alpha * acc[2 * nv + 1] + cv.y * (dv[e][1] + dv[e][3] + wsum);
+        }
       }
       __syncwarp();
       if (i + 2 < t1) issue(i + 2, st);
@@ -531,7 +545,7 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_tiles_kernel(DecodeArgs
 #pragma unroll
       for (int nv = 0; nv < 16; ++nv) {
         const int c0 = 8 * nv + 2 * t;
-        *reinterpret_cast<float2*>(part + 2 + c0) = make_float2(acc[2 * nv], acc[2 * nv + 1]);
+        *reinterpret_cast<float2*>(part + kPartAcc + c0) = make_float2(acc[2 * nv], acc[2 * nv + 1]);
       }
     }
   }
@@ -542,20 +556,24 @@ __global__ void __launch_bounds__(kDecWarps * 32) decode_tiles_kernel(DecodeArgs
 }
 
 // ------------------------------------------------------------------ merge
+constexpr int kMergeThreads = 256;
+
 template <int T>
-struct MergeSmem {
+struct __align__(16) MergeSmem {
   float qraw[kMaxGroup][kHeadDim];
   float sc[kMaxGroup][T];
-  float fin[kMaxGroup][kHeadDim];
-  float tl[kMaxGroup][kHeadDim];
-  float mt[kMaxGroup], lt[kMaxGroup], big_m[kMaxGroup], inv_l[kMaxGroup], et[kMaxGroup];
+  float tl[kMaxGroup][kHeadDim];                 // raw-domain tail accumulator
+  float red[kMergeThreads / 32][kHeadDim];       // per-warp partial sums of one head
+  float big_m[kMaxGroup], inv_l[kMaxGroup], et[kMaxGroup], mt[kMaxGroup], lt[kMaxGroup];
 };
 
-// One CTA of 128 threads per (sequence, KV head): raw tail, log-sum-exp
-// merge of the chunk partials, inverse rotation, fp16 output.
+// One CTA of 256 threads per (sequence, KV head): raw fp16 tail, log-sum-
+// exp merge of the chunk partials (warps split the chunks, lanes own four
+// channels), the inverse rotation of the merged accumulator, fp16 output.
 template <int T>
-__global__ void __launch_bounds__(128) decode_merge_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(DecodeArgs a) {
   __shared__ MergeSmem<T> sm;
+  constexpr int kWarps = kMergeThreads / 32;
   const int h = blockIdx.x, b = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = a.cfg.group_size, nh = a.cfg.num_kv_heads;
@@ -570,9 +588,12 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(DecodeArgs a) {
   const __half* q = static_cast<const __half*>(a.q) + (static_cast<size_t>(b) * nh + h) * G * kHeadDim;
   const __half* kt = static_cast<const __half*>(a.k_tail) + (static_cast<size_t>(b) * nh + h) * T * kHeadDim;
   const __half* vt = static_cast<const __half*>(a.v_tail) + (static_cast<size_t>(b) * nh + h) * T * kHeadDim;
-  for (int hh = 0; hh < G; ++hh) sm.qraw[hh][tid] = __half2float(q[hh * kHeadDim + tid]) * qscale;
+
+  // 1. raw tail: scores (thread = token), softmax (warp = head), P V (thread = channel)
+  for (int idx = tid; idx < G * kHeadDim; idx += kMergeThreads)
+    sm.qraw[idx / kHeadDim][idx % kHeadDim] = __half2float(q[idx]) * qscale;
   __syncthreads();
-  for (int i = tid; i < tau; i += 128) {
+  for (int i = tid; i < tau; i += kMergeThreads) {
     float dot[kMaxGroup];
 #pragma unroll
     for (int hh = 0; hh < kMaxGroup; ++hh) dot[hh] = 0.f;
@@ -585,7 +606,7 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(DecodeArgs a) {
     for (int hh = 0; hh < G; ++hh) sm.sc[hh][i] = dot[hh];
   }
   __syncthreads();
-  for (int hh = warp; hh < G; hh += 4) {
+  for (int hh = warp; hh < G; hh += kWarps) {
     float m = -INFINITY;
     for (int i = lane; i < tau; i += 32) m = fmaxf(m, sm.sc[hh][i]);
     m = warp_max(m);
@@ -596,62 +617,73 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(DecodeArgs a) {
       ps += p;
     }
     ps = warp_sum(ps);
+    // merge statistics over the chunks: the warp's lanes stride over them
+    float mm = m;
+    for (int s = lane; s < S; s += 32) {
+      const float* pp = parts + ((ubase + s) * G + hh) * kPartFloats;
+      if (pp[1] > 0.f) mm = fmaxf(mm, pp[0]);
+    }
+    mm = warp_max(mm);
+    float ll = 0.f;
+    for (int s = lane; s < S; s += 32) {
+      const float* pp = parts + ((ubase + s) * G + hh) * kPartFloats;
+      if (pp[1] > 0.f) ll += pp[1] * exp2f(pp[0] - mm);
+    }
+    ll = warp_sum(ll);
     if (lane == 0) {
-      sm.mt[hh] = m;
-      sm.lt[hh] = ps;
+      const float et = ps > 0.f ? exp2f(m - mm) : 0.f;
+      const float l = ll + ps * et;
+      sm.big_m[hh] = mm;
+      sm.et[hh] = et;
+      sm.inv_l[hh] = l > 0.f ? 1.f / l : 0.f;
     }
+  }
+  __syncthreads();  // tail weights in sm.sc are read by every thread below
+  for (int idx = tid; idx < G * kHeadDim; idx += kMergeThreads) {
+    const int hh = idx / kHeadDim, c = idx % kHeadDim;
+    float at = 0.f;
+    for (int i = 0; i < tau; ++i) at += sm.sc[hh][i] * __half2float(vt[i * kHeadDim + c]);
+    sm.tl[hh][c] = at;
   }
   __syncthreads();
-  {
-    float at[kMaxGroup];
-#pragma unroll
-    for (int hh = 0; hh < kMaxGroup; ++hh) at[hh] = 0.f;
-    for (int i = 0; i < tau; ++i) {
-      const float vv = __half2float(vt[i * kHeadDim + tid]);
-#pragma unroll
-      for (int hh = 0; hh < kMaxGroup; ++hh)
-        if (hh < G) at[hh] += sm.sc[hh][i] * vv;
-    }
-    for (int hh = 0; hh < G; ++hh) sm.tl[hh][tid] = at[hh];
-  }
-  if (tid < G) {
-    const int hh = tid;
-    float m = sm.mt[hh];
-    for (int s = 0; s < S; ++s) {
-      const float* pp = parts + ((ubase + s) * G + hh) * kPartFloats;
-      if (pp[1] > 0.f) m = fmaxf(m, pp[0]);
-    }
-    float l = sm.lt[hh] > 0.f ? sm.lt[hh] * exp2f(sm.mt[hh] - m) : 0.f;
-    for (int s = 0; s < S; ++s) {
-      const float* pp = parts + ((ubase + s) * G + hh) * kPartFloats;
-      if (pp[1] > 0.f) l += pp[1] * exp2f(pp[0] - m);
-    }
-    sm.big_m[hh] = m;
-    sm.inv_l[hh] = l > 0.f ? 1.f / l : 0.f;
-    sm.et[hh] = sm.lt[hh] > 0.f ? exp2f(sm.mt[hh] - m) : 0.f;
-  }
-  __syncthreads();
-  for (int hh = 0; hh < G; ++hh) {
-    float accr = 0.f;
-    for (int s = 0; s < S; ++s) {
-      const float* pp = parts + ((ubase + s) * G + hh) * kPartFloats;
-      if (pp[1] > 0.f) accr += exp2f(pp[0] - sm.big_m[hh]) * pp[2 + tid];
-    }
-    sm.fin[hh][tid] = accr;
-  }
-  __syncthreads();
+
+  // 2. per head: warps split the chunks, lane owns channels 4*lane .. 4*lane+3
   __half* out = static_cast<__half*>(a.out) + (static_cast<size_t>(b) * nh + h) * G * kHeadDim;
-  for (int hh = warp; hh < G; hh += 4) {
-    float v[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) v[k] = sm.fin[hh][4 * lane + k];
-    fwht128_warp(v, lane);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int c = 4 * lane + k;
-      const float o = (v[k] / kSqrtHeadDim + sm.et[hh] * sm.tl[hh][c]) * sm.inv_l[hh];
-      out[hh * kHeadDim + c] = __float2half_rn(o);
+  for (int hh = 0; hh < G; ++hh) {
+    const float mm = sm.big_m[hh];
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int s = warp; s < S; s += kWarps) {
+      const float* pp = parts + ((ubase + s) * G + hh) * kPartFloats;
+      const float2 ml = *reinterpret_cast<const float2*>(pp);
+      const float4 v = *reinterpret_cast<const float4*>(pp + kPartAcc + 4 * lane);
+      if (ml.y > 0.f) {
+        const float wgt = exp2f(ml.x - mm);
+        acc.x += wgt * v.x;
+        acc.y += wgt * v.y;
+        acc.z += wgt * v.z;
+        acc.w += wgt * v.w;
+      }
     }
+    *reinterpret_cast<float4*>(&sm.red[warp][4 * lane]) = acc;
+    __syncthreads();
+    if (warp == 0) {
+      float v[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float x = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) x += sm.red[w][4 * lane + k];
+        v[k] = x;
+      }
+      fwht128_warp(v, lane);  // the one inverse rotation (H = H^T = H^-1)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int c = 4 * lane + k;
+        out[hh * kHeadDim + c] = __float2half_rn((v[k] / kSqrtHeadDim + sm.et[hh] * sm.tl[hh][c]) * sm.inv_l[hh]);
+      }
+    }
+    __syncthreads();
   }
 }
 
@@ -692,7 +724,7 @@ cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t s) {
   e = launch_tiles_bits<T>(a, s, sms);
   if (e != cudaSuccess) return e;
   dim3 g2(a.cfg.num_kv_heads, a.num_seqs);
-  decode_merge_kernel<T><<<g2, 128, 0, s>>>(a);
+  decode_merge_kernel<T><<<g2, kMergeThreads, 0, s>>>(a);
   return cudaGetLastError();
 }
 

@@ -94,7 +94,7 @@ def test_argument_errors_launch_nothing(lib):
     assert st == kvq.KVQ_ERR_UNSUPPORTED
     # workspace too small (explicit split count: no device query)
     need = kvq.decode_workspace_bytes(cfg, 3, 2)
-    assert need == 256 + 3 * 2 * 2 * 4 * 130 * 4      # schedule header, then the partials
+    assert need == 256 + 3 * 2 * 2 * 4 * 132 * 4      # schedule header, then 528-byte partial records
     st = lib.kvq_paged_decode_attention(ctypes.byref(c), 16, 16, 16, 3, 16, 4, 8, 16, 16, 16, 16, 0.1, 16,
                                         need - 1, 2, None, None)
     assert st == kvq.KVQ_ERR_WORKSPACE
