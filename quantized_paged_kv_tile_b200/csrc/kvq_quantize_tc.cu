@@ -39,7 +39,8 @@ namespace kvq {
 
 namespace {
 
-constexpr int kQThreads = 256;          // 8 warps: warps w and w+4 share TMEM lane quadrant w, split the columns
+constexpr int kMathThreads = 256;       // 8 math warps: warps w and w+4 share TMEM lane quadrant w, split the columns
+constexpr int kQThreads = kMathThreads + 32;  // + 1 producer warp (metadata, TMA, MMA) in the quantize kernel
 constexpr int kRows = 128;                 // token rows per MMA group
 constexpr int kMaxPageBytes = 1024 + 64 + 128;
 constexpr int kStageBytes = 8 * kMaxPageBytes;  // the group's 8 pages
@@ -50,12 +51,12 @@ constexpr int kOffH = 0;                   // +-1 Sylvester matrix, 2 x 16 KB SW
 constexpr int kOffX = 32768;               // the group's rows, same layout
 constexpr int kOffStage = 65536;           // 2 staging buffers
 constexpr int kOffRr = kOffStage + 2 * kStageBytes;   // float r[128]  (token reciprocals)
-constexpr int kOffCc = kOffRr + 512;                  // float c[4][128] (channel reciprocals per tile)
-constexpr int kOffRed = kOffCc + 2048;                // float [8 warps][4 tiles] partial maxima
+constexpr int kOffCc = kOffRr + 512;                  // float c[2][4][128] (channel reciprocals per tile, ping-pong)
+constexpr int kOffRed = kOffCc + 4096;                // float [8 warps][4 tiles] partial maxima
 constexpr int kOffXs = kOffRed + 128;                 // float4 [256] partial statistics exchange
 constexpr int kOffMeta = kOffXs + 4096;               // 2 x GroupMeta
-constexpr int kOffBar = kOffMeta + 512;               // tma_bar, mma_bar
-constexpr int kOffTmem = kOffBar + 16;
+constexpr int kOffBar = kOffMeta + 512;               // tma, full, empty, meta[2] mbarriers
+constexpr int kOffTmem = kOffBar + 48;
 constexpr int kSmemUsed = kOffTmem + 16;
 constexpr int kSmemBytes = kSmemUsed + 1024;          // + alignment slack
 
@@ -114,7 +115,9 @@ __device__ __forceinline__ void mma_f16(uint32_t dtmem, uint64_t da, uint64_t db
       "l"(da), "l"(db), "r"(kIdesc), "r"(acc));
 }
 
-// 32 consecutive fp32 columns of this thread's TMEM lane
+// 32 consecutive fp32 columns of this thread's TMEM lane.  The wait takes
+// the loaded registers as operands, so no use of them can move above it,
+// and carries no memory clobber, so ordinary shared-memory loads can.
 __device__ __forceinline__ void tmem_ld32(uint32_t addr, float (&v)[32]) {
   uint32_t r[32];
   asm volatile(
@@ -125,9 +128,31 @@ __device__ __forceinline__ void tmem_ld32(uint32_t addr, float (&v)[32]) {
         "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
         "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(addr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]), "+r"(r[8]),
+        "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]),
+        "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]),
+        "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31]));
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// barrier of the two warps (w, w + 4) that share TMEM lane quadrant w
+__device__ __forceinline__ void pair_sync(int quadrant) {
+  asm volatile("bar.sync %0, 64;" ::"r"(1 + quadrant) : "memory");
+}
+// barrier of the 8 math warps (the producer warp never joins it)
+__device__ __forceinline__ void math_sync() { asm volatile("bar.sync 15, 256;" ::: "memory"); }
+// barrier of the 256 math threads that also returns whether any of them passed true
+__device__ __forceinline__ bool math_any(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 q, %1, 0;\n bar.red.or.pred p, 15, 256, q;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v))
+      : "memory");
+  return r != 0;
 }
 
 __device__ __forceinline__ float min3f(float a, float b, float c) {
@@ -142,19 +167,26 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
 }
 
 // Shifted sums of 32 values x_k * w_k - shift with packed f32x2 arithmetic
-// (two independent accumulator chains per statistic).
-__device__ __forceinline__ void shifted_sums(const float* x, const float* w, float shift, float2 (&s1)[2],
-                                             float2 (&s2)[2]) {
+// (four independent accumulator chains per statistic).
+__device__ __forceinline__ void shifted_sums(const float* x, const float* w, float shift, float2 (&s1)[4],
+                                             float2 (&s2)[4]) {
   const float2 nk = make_float2(-shift, -shift);
 #pragma unroll
-  for (int k = 0; k < 32; k += 4) {
-    const float4 ww = *reinterpret_cast<const float4*>(w + k);
-    const float2 d0 = __ffma2_rn(make_float2(x[k], x[k + 1]), make_float2(ww.x, ww.y), nk);
-    const float2 d1 = __ffma2_rn(make_float2(x[k + 2], x[k + 3]), make_float2(ww.z, ww.w), nk);
+  for (int k = 0; k < 32; k += 8) {
+    const float4 w0 = *reinterpret_cast<const float4*>(w + k);
+    const float4 w1 = *reinterpret_cast<const float4*>(w + k + 4);
+    const float2 d0 = __ffma2_rn(make_float2(x[k], x[k + 1]), make_float2(w0.x, w0.y), nk);
+    const float2 d1 = __ffma2_rn(make_float2(x[k + 2], x[k + 3]), make_float2(w0.z, w0.w), nk);
+    const float2 d2 = __ffma2_rn(make_float2(x[k + 4], x[k + 5]), make_float2(w1.x, w1.y), nk);
+    const float2 d3 = __ffma2_rn(make_float2(x[k + 6], x[k + 7]), make_float2(w1.z, w1.w), nk);
     s1[0] = __fadd2_rn(s1[0], d0);
     s1[1] = __fadd2_rn(s1[1], d1);
+    s1[2] = __fadd2_rn(s1[2], d2);
+    s1[3] = __fadd2_rn(s1[3], d3);
     s2[0] = __ffma2_rn(d0, d0, s2[0]);
     s2[1] = __ffma2_rn(d1, d1, s2[1]);
+    s2[2] = __ffma2_rn(d2, d2, s2[2]);
+    s2[3] = __ffma2_rn(d3, d3, s2[3]);
   }
 }
 
@@ -162,8 +194,9 @@ __device__ __forceinline__ void shifted_sums(const float* x, const float* w, flo
 struct Moments {
   float mean, m2;
 };
-__device__ __forceinline__ Moments moments(const float2 (&s1)[2], const float2 (&s2)[2], float shift, float n) {
-  const float a = (s1[0].x + s1[0].y) + (s1[1].x + s1[1].y), q = (s2[0].x + s2[0].y) + (s2[1].x + s2[1].y);
+__device__ __forceinline__ Moments moments(const float2 (&s1)[4], const float2 (&s2)[4], float shift, float n) {
+  const float a = ((s1[0].x + s1[0].y) + (s1[1].x + s1[1].y)) + ((s1[2].x + s1[2].y) + (s1[3].x + s1[3].y));
+  const float q = ((s2[0].x + s2[0].y) + (s2[1].x + s2[1].y)) + ((s2[2].x + s2[2].y) + (s2[3].x + s2[3].y));
   Moments m;
   m.mean = shift + a / n;
   m.m2 = fmaxf(q - a * (a / n), 0.f);
@@ -181,10 +214,13 @@ __device__ __forceinline__ float combined_std(Moments a, Moments b, float n) {
 // rows of D1, channel rows of D2); half hf = warp / 4 owns columns
 // 64hf..64hf+63 of those rows.  Row statistics that span both halves are
 // combined through shared memory (thread tid and its partner tid ^ 128).
+// The group: `valid` has bit t set for each present tile t; `store_blk` is,
+// for thread q < 8, the block of page q of the group; once the last TMEM
+// read is done, one lane per warp arrives on `empty_bar` (0: none).
 template <int T, int bits, bool is_v>
-__device__ void quantize_group_from_tmem(unsigned char* smem, uint32_t tbase, const GroupMeta& gm,
-                                         const PoolGeom g, int iters, float eps, unsigned char* stage,
-                                         uint8_t* pool, int num_heads, int head) {
+__device__ void quantize_group_from_tmem(unsigned char* smem, uint32_t tbase, int valid, int store_blk,
+                                         uint32_t empty_bar, const PoolGeom g, int iters, float eps,
+                                         unsigned char* stage, uint8_t* pool, int num_heads, int head) {
   constexpr int G = kRows / T;                 // tiles in the group
   constexpr int kPagesPerTile = T / kPageTokens;
   constexpr int kLocal = T <= 64 ? 64 / T : 1; // whole tiles inside my 64 token columns (T <= 64)
@@ -192,14 +228,17 @@ __device__ void quantize_group_from_tmem(unsigned char* smem, uint32_t tbase, co
   const int qd = warp & 3, hf = warp >> 2;
   const int row = 32 * qd + lane;             // token of D1 / channel of D2
   float* rr = reinterpret_cast<float*>(smem + kOffRr);
-  float* cc = reinterpret_cast<float*>(smem + kOffCc);  // [G][128]
+  // c_j per tile in two buffers: iteration `it` reads and updates buffer it&1
+  // and writes the renormalized values into the other one
+  float* cc_buf = reinterpret_cast<float*>(smem + kOffCc);  // [2][G][128]
+  float* cc = cc_buf;
   float* red = reinterpret_cast<float*>(smem + kOffRed);
   float4* xs = reinterpret_cast<float4*>(smem + kOffXs);
   const uint32_t lane_addr = tbase + (static_cast<uint32_t>(32 * qd) << 16);
   const uint32_t d1 = lane_addr + 64 * hf;        // channels 64hf.. of token `row`
   const uint32_t d2 = lane_addr + 128 + 64 * hf;  // tokens 64hf.. of channel `row`
   const int my_tile = row / T;                    // tile of token `row`
-  const bool tok_live = gm.valid[my_tile] != 0;
+  const bool tok_live = (valid >> my_tile) & 1;
   // tiles whose channel statistics this thread computes: T=32 -> 2hf, 2hf+1; T=64 -> hf; T=128 -> 0
   auto ch_tile = [&](int lt) { return T == 128 ? 0 : hf * kLocal + lt; };
 
@@ -211,64 +250,83 @@ __device__ void quantize_group_from_tmem(unsigned char* smem, uint32_t tbase, co
   }
   float Ri = 1.f;
   if (hf == 0) rr[row] = 1.f;
-  __syncthreads();
+  math_sync();
 
+  auto tile_exp = [&](int t) {  // exponent of the tile's max C over the warps that hold it
+    float m = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      const bool holds = T == 128 ? true : (t / kLocal == (w >> 2));
+      if (holds) m = fmaxf(m, red[w * 4 + t]);
+    }
+    int e;
+    frexpf(m, &e);
+    return e;
+  };
   for (int it = 0; it < iters; ++it) {
-    // ---- channel step: channel `row`, token columns 64hf..64hf+63
-    {
-      if constexpr (T <= 64) {
+    cc = cc_buf + (it & 1) * (4 * kRows);
+    float* cc_next = cc_buf + ((it + 1) & 1) * (4 * kRows);
+    // ---- channel step: channel `row`, token columns 64hf..64hf+63.  The new
+    // c_j are published with the per-warp maxima of C for the renormalization.
+    if constexpr (T <= 64) {
 #pragma unroll
-        for (int lt = 0; lt < kLocal; ++lt) {
-          const int t = ch_tile(lt);
-          if (!gm.valid[t]) continue;
-          float2 s1[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-          float2 s2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-          float shift = 0.f;
-#pragma unroll
-          for (int ch = 0; ch < T / 32; ++ch) {
-            float x[32];
-            tmem_ld32(d2 + lt * T + ch * 32, x);
-            if (ch == 0) shift = x[0] * rr[t * T];
-            shifted_sums(x, rr + t * T + ch * 32, shift, s1, s2);
-          }
-          const Moments mo = moments(s1, s2, shift, static_cast<float>(T));
-          const float c = cc[t * kRows + row];
-          const float sigma = fmaxf(c * sqrtf(mo.m2 / static_cast<float>(T)), eps);
-          Cj[lt] *= sigma;
-          cc[t * kRows + row] = fminf(c / sigma, FLT_MAX);  // a zero channel keeps a finite factor
-        }
-        __syncthreads();
-      } else {
-        float2 s1[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-        float2 s2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      for (int lt = 0; lt < kLocal; ++lt) {
+        const int t = ch_tile(lt);
+        if (!((valid >> t) & 1)) continue;
+        float2 s1[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        float2 s2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
         float shift = 0.f;
 #pragma unroll
-        for (int ch = 0; ch < 2; ++ch) {
+        for (int ch = 0; ch < T / 32; ++ch) {
           float x[32];
-          tmem_ld32(d2 + ch * 32, x);
-          if (ch == 0) shift = x[0] * rr[64 * hf];
-          shifted_sums(x, rr + 64 * hf + ch * 32, shift, s1, s2);
+          tmem_ld32(d2 + lt * T + ch * 32, x);
+          if (ch == 0) shift = x[0] * rr[t * T];
+          shifted_sums(x, rr + t * T + ch * 32, shift, s1, s2);
         }
-        const Moments mo = moments(s1, s2, shift, 64.f);
-        xs[tid] = make_float4(mo.mean, mo.m2, 0.f, 0.f);
-        __syncthreads();
-        const float4 o = xs[tid ^ 128];
-        const Moments other = {o.x, o.y};
-        const float sd = hf == 0 ? combined_std(mo, other, 64.f) : combined_std(other, mo, 64.f);
-        const float c = cc[row];
-        const float sigma = fmaxf(c * sd, eps);
-        Cj[0] *= sigma;
-        __syncthreads();
-        if (hf == 0) cc[row] = fminf(c / sigma, FLT_MAX);
-        __syncthreads();
+        const Moments mo = moments(s1, s2, shift, static_cast<float>(T));
+        const float c = cc[t * kRows + row];
+        const float sigma = fmaxf(c * sqrtf(mo.m2 / static_cast<float>(T)), eps);
+        Cj[lt] *= sigma;
+        cc[t * kRows + row] = fminf(c / sigma, FLT_MAX);  // a zero channel keeps a finite factor
       }
+    } else {
+      float2 s1[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      float2 s2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      float shift = 0.f;
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {
+        float x[32];
+        tmem_ld32(d2 + ch * 32, x);
+        if (ch == 0) shift = x[0] * rr[64 * hf];
+        shifted_sums(x, rr + 64 * hf + ch * 32, shift, s1, s2);
+      }
+      const Moments mo = moments(s1, s2, shift, 64.f);
+      xs[tid] = make_float4(mo.mean, mo.m2, 0.f, 0.f);
+      pair_sync(qd);
+      const float4 o = xs[tid ^ 128];
+      const Moments other = {o.x, o.y};
+      const float sd = hf == 0 ? combined_std(mo, other, 64.f) : combined_std(other, mo, 64.f);
+      const float c = cc[row];
+      const float sigma = fmaxf(c * sd, eps);
+      Cj[0] *= sigma;
+      pair_sync(qd);  // both halves have read cc[row]
+      if (hf == 0) cc[row] = fminf(c / sigma, FLT_MAX);
     }
-    // ---- token step: token `row`, channel columns 64hf..64hf+63
+#pragma unroll
+    for (int lt = 0; lt < kLocal; ++lt) {
+      const float m = warp_max(Cj[lt]);
+      if (lane == 0) red[warp * 4 + ch_tile(lt)] = m;
+    }
+    math_sync();
+    // ---- token step with this iteration's c (before the renormalization,
+    // which leaves Y = X' c r unchanged)
+    float r_new = 0.f;
     {
       Moments mo = {0.f, 0.f};
+      const float r = rr[row];  // read before the pair barrier: the owner rewrites it below
       if (tok_live) {
-        float2 s1[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-        float2 s2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        float2 s1[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        float2 s2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
         const float* cvec = cc + my_tile * kRows + 64 * hf;
         float shift = 0.f;
 #pragma unroll
@@ -281,55 +339,35 @@ __device__ void quantize_group_from_tmem(unsigned char* smem, uint32_t tbase, co
         mo = moments(s1, s2, shift, 64.f);
       }
       xs[tid] = make_float4(mo.mean, mo.m2, 0.f, 0.f);
-      __syncthreads();
-      float r_new = 0.f;
+      pair_sync(qd);
       if (tok_live) {
         const float4 o = xs[tid ^ 128];
         const Moments other = {o.x, o.y};
         const float sd = hf == 0 ? combined_std(mo, other, 64.f) : combined_std(other, mo, 64.f);
-        const float r = rr[row];
         const float rho = fmaxf(r * sd, eps);
         Ri *= rho;
         r_new = fminf(r / rho, FLT_MAX);  // a zero token keeps a finite factor
       }
-      __syncthreads();
-      if (tok_live && hf == 0) rr[row] = r_new;
     }
-    // ---- (C, R) -> (C / 2^k, R 2^k) per tile, max C in [1, 2)
-#pragma unroll
-    for (int lt = 0; lt < kLocal; ++lt) {
-      const float m = warp_max(Cj[lt]);
-      if (lane == 0) red[warp * 4 + ch_tile(lt)] = m;
-    }
-    __syncthreads();
-    auto tile_exp = [&](int t) {  // exponent of the tile's max C over the warps that hold it
-      float m = 0.f;
-#pragma unroll
-      for (int w = 0; w < 8; ++w) {
-        const int whf = w >> 2;
-        const bool holds = T == 128 ? true : (t / kLocal == whf);
-        if (holds) m = fmaxf(m, red[w * 4 + t]);
-      }
-      int e;
-      frexpf(m, &e);
-      return e;
-    };
+    // ---- (C, R) -> (C / 2^k, R 2^k) per tile, max C in [1, 2): every thread
+    // rescales what it owns; cc and rr are read again only after the barrier
 #pragma unroll
     for (int lt = 0; lt < kLocal; ++lt) {
       const int t = ch_tile(lt);
       const int e = tile_exp(t);
       Cj[lt] = ldexpf(Cj[lt], 1 - e);
-      if (T < 128 || hf == 0) cc[t * kRows + row] = fminf(ldexpf(cc[t * kRows + row], e - 1), FLT_MAX);
+      if (T < 128 || hf == 0) cc_next[t * kRows + row] = fminf(ldexpf(cc[t * kRows + row], e - 1), FLT_MAX);
     }
     {
       const int e = tile_exp(my_tile);
       Ri = ldexpf(Ri, e - 1);
-      if (hf == 0) rr[row] = fminf(ldexpf(rr[row], 1 - e), FLT_MAX);
+      if (tok_live && hf == 0) rr[row] = fminf(ldexpf(r_new, 1 - e), FLT_MAX);
     }
-    __syncthreads();
+    math_sync();
   }
 
   // ---- RTN on D1: token `row`, channels 64hf..64hf+63
+  cc = cc_buf + (iters & 1) * (4 * kRows);
   constexpr int qmax = (1 << bits) - 1;
   constexpr bool kGrouped = is_v && bits != 3;  // V in the decode lane order
   const int local = row % T, page_in_tile = local / kPageTokens, p = local % kPageTokens;
@@ -354,7 +392,7 @@ __device__ void quantize_group_from_tmem(unsigned char* smem, uint32_t tbase, co
     }
   }
   xs[tid] = make_float4(zu, mu, 0.f, 0.f);
-  __syncthreads();
+  pair_sync(qd);
   if (tok_live) {
     const float4 o = xs[tid ^ 128];
     zu = fminf(zu, o.x);
@@ -377,8 +415,17 @@ __device__ void quantize_group_from_tmem(unsigned char* smem, uint32_t tbase, co
       float x[32];
 #pragma unroll
       for (int c = 0; c < 64; ++c) {
-        if ((c & 31) == 0) tmem_ld32(d1 + c, x);  // pass 2: the codes
-        const float u = x[c & 31] * cvec[c];
+        if ((c & 31) == 0) {  // pass 2: u_j = x_j c_j for the next 32 channels, then the codes
+          tmem_ld32(d1 + c, x);
+#pragma unroll
+          for (int k = 0; k < 32; k += 4) {
+            const float4 cv = *reinterpret_cast<const float4*>(cvec + c + k);
+            const float2 u0 = __fmul2_rn(make_float2(x[k], x[k + 1]), make_float2(cv.x, cv.y));
+            const float2 u1 = __fmul2_rn(make_float2(x[k + 2], x[k + 3]), make_float2(cv.z, cv.w));
+            x[k] = u0.x; x[k + 1] = u0.y; x[k + 2] = u1.x; x[k + 3] = u1.y;
+          }
+        }
+        const float u = x[c & 31];
         const uint32_t qb = __float_as_uint(__fadd_rn(__fmaf_rn(u, a, b0), 12582912.0f));
         const int bit = c * bits;
         if constexpr (bits == 3) {
@@ -415,8 +462,17 @@ __device__ void quantize_group_from_tmem(unsigned char* smem, uint32_t tbase, co
       float x[32];
 #pragma unroll
       for (int c = 0; c < 64; ++c) {
-        if ((c & 31) == 0) tmem_ld32(d1 + c, x);  // pass 2: the codes
-        const float u = x[c & 31] * cvec[c];
+        if ((c & 31) == 0) {  // pass 2: u_j = x_j c_j for the next 32 channels, then the codes
+          tmem_ld32(d1 + c, x);
+#pragma unroll
+          for (int k = 0; k < 32; k += 4) {
+            const float4 cv = *reinterpret_cast<const float4*>(cvec + c + k);
+            const float2 u0 = __fmul2_rn(make_float2(x[k], x[k + 1]), make_float2(cv.x, cv.y));
+            const float2 u1 = __fmul2_rn(make_float2(x[k + 2], x[k + 3]), make_float2(cv.z, cv.w));
+            x[k] = u0.x; x[k + 1] = u0.y; x[k + 2] = u1.x; x[k + 3] = u1.y;
+          }
+        }
+        const float u = x[c & 31];
         const uint32_t qb = __float_as_uint(__fadd_rn(__fmaf_rn(u, a, b0), 12582912.0f));
         const int n = (64 * hf + c) >> 3, g8 = c & 7;
         const int m = n / h - hf * nm, e = n % h;
@@ -444,22 +500,27 @@ __device__ void quantize_group_from_tmem(unsigned char* smem, uint32_t tbase, co
       *reinterpret_cast<__half2*>(page + g.meta_off + 4 * p) =
           __halves2half2(__float2half_rn(s * Ri), __float2half_rn(z * Ri));
   }
+  // every TMEM read of this group is done: the producer may overwrite it
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncwarp();
+  if (empty_bar != 0 && lane == 0)
+    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(empty_bar) : "memory");
   // C slices: channel thread `row` writes C~ of its tiles into page k = row / cs of the tile
 #pragma unroll
   for (int lt = 0; lt < kLocal; ++lt) {
     const int t = ch_tile(lt);
-    if (!gm.valid[t] || (T == 128 && hf != 0)) continue;
+    if (!((valid >> t) & 1) || (T == 128 && hf != 0)) continue;
     const int pg = row / g.cs_channels;
     *reinterpret_cast<__half*>(stage + (t * kPagesPerTile + pg) * g.page_bytes + g.cslice_off +
                                2 * (row % g.cs_channels)) = __float2half_rn(Cj[lt]);
   }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  __syncthreads();
+  math_sync();
   // page stores: thread q < 8 stores page q of the group
   if (tid < 8) {
     const int t = tid / kPagesPerTile, k = tid % kPagesPerTile;
-    if (t < G && gm.valid[t]) {
-      const int blk = gm.pages[t][k];
+    if (t < G && ((valid >> t) & 1)) {
+      const int blk = store_blk;
       uint8_t* dst = pool + (static_cast<size_t>(blk) * num_heads + head) * static_cast<size_t>(g.page_bytes);
       asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
                    "r"(smem_u32(stage + tid * g.page_bytes)), "r"(g.page_bytes)
@@ -471,12 +532,16 @@ __device__ void quantize_group_from_tmem(unsigned char* smem, uint32_t tbase, co
 
 // the group function for this item's code width and K|V
 template <int T, int BK, int BV>
-__device__ __forceinline__ void quantize_group_dispatch(unsigned char* smem, uint32_t tbase, const GroupMeta& gm,
-                                                        bool is_v, const PoolGeom g, int iters, float eps,
-                                                        unsigned char* stage, uint8_t* pool, int num_heads,
+__device__ __forceinline__ void quantize_group_dispatch(unsigned char* smem, uint32_t tbase, int valid, int store_blk,
+                                                        uint32_t empty_bar, bool is_v, const PoolGeom g, int iters,
+                                                        float eps, unsigned char* stage, uint8_t* pool, int num_heads,
                                                         int head) {
-  if (is_v) quantize_group_from_tmem<T, BV, true>(smem, tbase, gm, g, iters, eps, stage, pool, num_heads, head);
-  else quantize_group_from_tmem<T, BK, false>(smem, tbase, gm, g, iters, eps, stage, pool, num_heads, head);
+  if (is_v)
+    quantize_group_from_tmem<T, BV, true>(smem, tbase, valid, store_blk, empty_bar, g, iters, eps, stage, pool,
+                                          num_heads, head);
+  else
+    quantize_group_from_tmem<T, BK, false>(smem, tbase, valid, store_blk, empty_bar, g, iters, eps, stage, pool,
+                                           num_heads, head);
 }
 
 __device__ void build_h(unsigned char* smem) {
@@ -506,7 +571,19 @@ __device__ void tmem_free(uint32_t tbase) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tbase), "r"(256));
 }
 
-// thread 0: the 16 MMAs of a group, completion on mma_bar
+// one thread: the 16 MMAs of a group (the caller commits)
+__device__ void issue_mmas_nocommit(unsigned char* smem, uint32_t tbase) {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t sx = smem_u32(smem + kOffX), sh = smem_u32(smem + kOffH);
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    const uint32_t koff = (s >> 2) * 16384 + (s & 3) * 32;
+    mma_f16(tbase, sw128_desc(sx + koff), sw128_desc(sh + koff), s > 0);          // D1 = X H
+    mma_f16(tbase + 128, sw128_desc(sh + koff), sw128_desc(sx + koff), s > 0);    // D2 = H X^T
+  }
+}
+
+// one thread: the 16 MMAs of a group, completion on mma_bar
 __device__ void issue_mmas(unsigned char* smem, uint32_t tbase, uint32_t mma_bar) {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t sx = smem_u32(smem + kOffX), sh = smem_u32(smem + kOffH);
@@ -525,6 +602,11 @@ struct QuantTcArgs {
   int num_items;  // groups x heads x 2
   int groups;
 };
+
+// true when this CTA's k-th item exists (the producer left its loop early)
+__device__ __forceinline__ bool item_left(const QuantTcArgs& qa, int k) {
+  return blockIdx.x + static_cast<long long>(k) * gridDim.x < qa.num_items;
+}
 
 // thread 0: validate the group's tiles, fill its metadata slot and issue the
 // TMA loads of its valid tiles; returns the number of valid tiles.
@@ -581,82 +663,101 @@ __device__ int prepare_group(const QuantTcArgs& qa, const CUtensorMap* tmk, cons
 
 template <int T, int BK, int BV>
 __global__ void __launch_bounds__(kQThreads, 2) quantize_tc_kernel(const __grid_constant__ CUtensorMap tmk,
-                                                                 const __grid_constant__ CUtensorMap tmv,
-                                                                 QuantTcArgs qa) {
+                                                    const __grid_constant__ CUtensorMap tmv, QuantTcArgs qa) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   unsigned char* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  constexpr int G = kRows / T;
+  constexpr int kPagesPerTile = T / kPageTokens;
   const QuantizeArgs& a = qa.a;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   GroupMeta* meta = reinterpret_cast<GroupMeta*>(smem + kOffMeta);
-  const uint32_t tma_bar = smem_u32(smem + kOffBar), mma_bar = smem_u32(smem + kOffBar + 8);
-  int* flag = reinterpret_cast<int*>(smem + kOffTmem + 4);
+  // tma: rows landed (producer only); full: the group's MMAs are done (TMEM
+  // holds it, rows buffer free); empty: the 8 math warps finished reading
+  // TMEM; meta[2]: a group's metadata slot is written
+  const uint32_t tma_bar = smem_u32(smem + kOffBar), full_bar = tma_bar + 8, empty_bar = tma_bar + 16;
+  const uint32_t meta_bar0 = tma_bar + 24;
 
   build_h(smem);
   if (tid == 0) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tma_bar));
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(mma_bar));
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(full_bar));
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 8;" ::"r"(empty_bar));
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(meta_bar0));
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(meta_bar0 + 8));
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    *flag = 0;
   }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   const uint32_t tbase = tmem_alloc(smem);  // includes a __syncthreads
 
-  uint32_t tma_phase = 0, mma_phase = 0;
-  int slot = 0;
-  int item = blockIdx.x;
-  if (tid == 0 && item < qa.num_items) prepare_group<T>(qa, &tmk, &tmv, item, &meta[0], smem, tma_bar);
-  __syncthreads();
-  int iter = 0;
-  for (; item < qa.num_items; item += gridDim.x, ++iter) {
-    GroupMeta& gm = meta[slot];
-    const int kv = item & 1, head = (item >> 1) % a.cfg.num_kv_heads;
-    const bool live = gm.nvalid > 0;
-    if (live) {
-      if (tid == 0) {
-        if (!mbar_wait(tma_bar, tma_phase)) {
-          report_error(a.dev_status, KVQ_ERR_DEVICE_TIMEOUT);
-          *flag = 1;
-        } else {
-          issue_mmas(smem, tbase, mma_bar);
+  if (warp == kMathThreads / 32) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t tma_phase = 0;
+      int k = 0;
+      bool tma_pending = false;
+      for (int item = blockIdx.x; item < qa.num_items; item += gridDim.x, ++k) {
+        const int slot = k & 1;
+        if (k > 0 && !mbar_wait(full_bar, (k - 1) & 1)) break;  // previous MMAs done: rows buffer free
+        const int nvalid = prepare_group<T>(qa, &tmk, &tmv, item, &meta[slot], smem, tma_bar);
+        asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(meta_bar0 + 8 * slot) : "memory");
+        if (nvalid > 0) {
+          tma_pending = true;
+          if (!mbar_wait(tma_bar, tma_phase)) break;
+          tma_pending = false;
+          tma_phase ^= 1u;
+        }
+        if (k > 0 && !mbar_wait(empty_bar, (k - 1) & 1)) break;  // math warps done with the previous TMEM
+        if (nvalid > 0) {
+          issue_mmas_nocommit(smem, tbase);
+          asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(full_bar)
+                       : "memory");
+        } else {  // nothing to compute: the previous MMAs were already waited for
+          asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(full_bar) : "memory");
         }
       }
-      tma_phase ^= 1u;
-      __syncthreads();
-      if (*flag) break;
-      if (!mbar_wait(mma_bar, mma_phase)) {
-        report_error(a.dev_status, KVQ_ERR_DEVICE_TIMEOUT);
-        *flag = 1;
+      if (item_left(qa, k)) report_error(a.dev_status, KVQ_ERR_DEVICE_TIMEOUT);
+      if (tma_pending) (void)mbar_wait(tma_bar, tma_phase);  // a load still in flight must land first
+      if (k > 0) (void)mbar_wait(full_bar, (k - 1) & 1);    // and the last MMAs must be done
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ math warps
+    int k = 0;
+    for (int item = blockIdx.x; item < qa.num_items; item += gridDim.x, ++k) {
+      const int slot = k & 1;
+      bool ok = mbar_wait(meta_bar0 + 8 * slot, (k >> 1) & 1);
+      const GroupMeta& gm = meta[slot];
+      int valid = 0, store_blk = 0;
+      if (ok) {
+        for (int t = 0; t < G; ++t) valid |= (gm.valid[t] ? 1 : 0) << t;
+        if (tid < 8 && tid / kPagesPerTile < G && ((valid >> (tid / kPagesPerTile)) & 1))
+          store_blk = gm.pages[tid / kPagesPerTile][tid % kPagesPerTile];
+        ok = mbar_wait(full_bar, k & 1);
       }
-      mma_phase ^= 1u;
+      if (math_any(!ok)) {  // one decision for all math threads
+        if (tid == 0) report_error(a.dev_status, KVQ_ERR_DEVICE_TIMEOUT);
+        break;
+      }
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      __syncthreads();
+      const int kv = item & 1, head = (item >> 1) % a.cfg.num_kv_heads;
+      if (valid != 0) {
+        // the staging buffer used two groups ago must have been read by its stores
+        if (tid < 8) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+        math_sync();
+        const PoolGeom g = kv ? a.gv : a.gk;
+        unsigned char* stage = smem + kOffStage + (k & 1) * kStageBytes;
+        quantize_group_dispatch<T, BK, BV>(smem, tbase, valid, store_blk, empty_bar, kv != 0, g, a.cfg.iters,
+                                           a.cfg.std_eps, stage, static_cast<uint8_t*>(kv ? a.v_pool : a.k_pool),
+                                           a.cfg.num_kv_heads, head);
+      } else {
+        if (tid < 8) asm volatile("cp.async.bulk.commit_group;" ::: "memory");  // keeps one group per item
+        __syncwarp();
+        if (lane == 0) asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(empty_bar) : "memory");
+      }
     }
-    const bool ok = *flag == 0;
-    // the rows buffer is free again: bring in the next group
-    if (tid == 0) {
-      const int next = item + gridDim.x;
-      if (next < qa.num_items && ok) prepare_group<T>(qa, &tmk, &tmv, next, &meta[slot ^ 1], smem, tma_bar);
-    }
-    if (live && ok) {
-      // the staging buffer used two groups ago must have been read by its stores
-      if (tid < 8) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-      __syncthreads();
-      const PoolGeom g = kv ? a.gv : a.gk;
-      unsigned char* stage = smem + kOffStage + (iter & 1) * kStageBytes;
-      quantize_group_dispatch<T, BK, BV>(smem, tbase, gm, kv != 0, g, a.cfg.iters, a.cfg.std_eps, stage,
-                                 static_cast<uint8_t*>(kv ? a.v_pool : a.k_pool), a.cfg.num_kv_heads, head);
-    }
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-    __syncthreads();
-    slot ^= 1;
-    if (*flag) break;
+    if (tid < 8) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
   }
-  if (*flag && tid == 0) {
-    // a wait gave up: let a load that may still be in flight land (bounded)
-    (void)mbar_wait(tma_bar, tma_phase);
-  }
-  if (tid < 8) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-  tmem_free(tbase);
+  tmem_free(tbase);  // includes a __syncthreads of all warps
 }
 
 // ---------------------------------------------------------------- append
@@ -665,7 +766,7 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_tc_kernel(const __grid_
 // and quantized by the same code path as kvq_quantize_tiles (bit-identical
 // pages); the remaining new tokens go to the fp16 tail.
 template <int T, int BK, int BV>
-__global__ void __launch_bounds__(kQThreads, 2) append_tc_kernel(AppendArgs a) {
+__global__ void __launch_bounds__(kMathThreads, 2) append_tc_kernel(AppendArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   unsigned char* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   constexpr int kPagesPerTile = T / kPageTokens;
@@ -688,7 +789,7 @@ __global__ void __launch_bounds__(kQThreads, 2) append_tc_kernel(AppendArgs a) {
 
   if (l0 / T < end / T) {  // at least one tile completes: tensor-core set-up
     build_h(smem);
-    for (int i = tid; i < kRows * kHeadDim / 8; i += kQThreads) {  // rows of the unused tiles: zeros
+    for (int i = tid; i < kRows * kHeadDim / 8; i += kMathThreads) {  // rows of the unused tiles: zeros
       const int r = i / 16, c = i % 16;
       if (r >= T) *reinterpret_cast<uint4*>(smem + kOffX + sw128_off(r, c * 8)) = make_uint4(0, 0, 0, 0);
     }
@@ -713,7 +814,7 @@ __global__ void __launch_bounds__(kQThreads, 2) append_tc_kernel(AppendArgs a) {
         }
       }
       // rows of the tile: 16-byte pieces into the swizzled layout
-      for (int i = tid; i < T * 16; i += kQThreads) {
+      for (int i = tid; i < T * 16; i += kMathThreads) {
         const int r = i / 16, c = i % 16;
         const int q = t * T + r;
         const __half* row = (q < l0) ? tail_base + static_cast<size_t>(q % T) * kHeadDim
@@ -744,8 +845,9 @@ __global__ void __launch_bounds__(kQThreads, 2) append_tc_kernel(AppendArgs a) {
       if (*flag == 1) break;
       if (tid < 8) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
       __syncthreads();
-      quantize_group_dispatch<T, BK, BV>(smem, tbase, *gm, kv != 0, g, a.cfg.iters, a.cfg.std_eps,
-                                 smem + kOffStage + (iter & 1) * kStageBytes, pool, nh, head);
+      const int store_blk = tid < kPagesPerTile ? gm->pages[0][tid] : 0;
+      quantize_group_dispatch<T, BK, BV>(smem, tbase, 1, store_blk, 0u, kv != 0, g, a.cfg.iters, a.cfg.std_eps,
+                                         smem + kOffStage + (iter & 1) * kStageBytes, pool, nh, head);
       asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
       __syncthreads();
     }
@@ -755,7 +857,7 @@ __global__ void __launch_bounds__(kQThreads, 2) append_tc_kernel(AppendArgs a) {
   // remaining tokens of the unfinished tile go to the tail (16-byte pieces)
   const int first = max(l0, (end / T) * T);
   const int count = end - first;
-  for (int idx = tid; idx < count * (kHeadDim / 8); idx += kQThreads) {
+  for (int idx = tid; idx < count * (kHeadDim / 8); idx += kMathThreads) {
     const int r = idx / (kHeadDim / 8), piece = idx % (kHeadDim / 8);
     const int q = first + r;
     const uint4 v = *reinterpret_cast<const uint4*>(
@@ -826,7 +928,7 @@ cudaError_t launch_append_tc(const AppendArgs& a, cudaStream_t s) {
   if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   if (e != cudaSuccess) return e;
   dim3 grid(a.num_seqs, a.cfg.num_kv_heads, 2);
-  kern<<<grid, kQThreads, kSmemBytes, s>>>(a);
+  kern<<<grid, kMathThreads, kSmemBytes, s>>>(a);
   return cudaGetLastError();
 }
 
