@@ -196,6 +196,35 @@ KVQ_API kvq_status kvq_paged_decode_attention(const kvq_config* cfg, const void*
                                       size_t workspace_bytes, int num_splits,
                                       int32_t* dev_status, void* stream);
 
+/* Size of the scratch array built into the library for
+ * kvq_paged_decode_attention_static_scratch (32 MiB per device). */
+#define KVQ_DECODE_STATIC_SCRATCH_BYTES ((size_t)32 << 20)
+
+/* kvq_paged_decode_attention without a caller workspace.  The method on the
+ * pages has no counterpart of this call: it exists for callers that cannot
+ * allocate device memory when they decode (a runtime that gave the whole
+ * device to its KV pool and weights at start-up, a serving loop that must not
+ * take cudaMalloc's implicit device synchronization, a C embedding with no
+ * device allocator).  It allocates and frees nothing.
+ *   Arguments, layouts and results: as kvq_paged_decode_attention, minus
+ *   workspace / workspace_bytes.  The workspace is a static device array of
+ *   KVQ_DECODE_STATIC_SCRATCH_BYTES in the library, one per device.
+ *   Size limit: if kvq_decode_workspace_bytes(cfg, num_seqs, num_splits)
+ *   exceeds KVQ_DECODE_STATIC_SCRATCH_BYTES the call returns
+ *   KVQ_ERR_WORKSPACE (detail in kvq_last_error) before touching the device;
+ *   use fewer sequences per call, a smaller num_splits, or the workspace entry.
+ *   Set-up: the first call on each device (that device current) looks up the
+ *   array's address with cudaGetSymbolAddress; make that first call before
+ *   any stream capture begins.  Device ordinals 0..63.
+ *   Concurrency: calls on the same device share the array; two calls that
+ *   overlap in time (different streams, or unordered host threads) race on it
+ *   and corrupt each other's results.  Order them (one stream, or events). */
+KVQ_API kvq_status kvq_paged_decode_attention_static_scratch(
+    const kvq_config* cfg, const void* q, void* out, const int32_t* seq_lens, int num_seqs,
+    const int32_t* block_tables, int max_blocks_per_seq, int num_blocks, const void* k_pool, const void* v_pool,
+    const void* k_tail, const void* v_tail, float softmax_scale, int num_splits, int32_t* dev_status,
+    void* stream);
+
 /* Inspection (tests, tools): read num_tiles tiles back out of a pool.
  *   tile_desc : device int32 [num_tiles][2] = {seq, tile_idx}; all heads.
  *   is_v      : 0 = K pool / bits_k, 1 = V pool / bits_v.

@@ -5,6 +5,7 @@
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
+#include <mutex>
 #include <string>
 
 #include "kvq_internal.h"
@@ -301,3 +302,78 @@ kvq_status kvq_unpack_tiles(const kvq_config* cfg, const int32_t* tile_desc, int
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------- decode, static scratch
+// kvq_paged_decode_attention_static_scratch runs the same decode as
+// kvq_paged_decode_attention, with its workspace taken from a fixed scratch
+// array compiled into the library instead of a caller-allocated buffer.  It is
+// for callers that cannot allocate device memory when they decode: a runtime
+// that hands the whole device to its KV pool and weights at start-up (a later
+// cudaMalloc fails or fragments that budget), a serving loop that must not take
+// cudaMalloc's implicit device-wide synchronization between steps, or a plain C
+// embedding that links only this library and has no device allocator of its
+// own.  This entry point allocates and frees nothing: it looks up the address
+// of the array once per device and passes it down.
+//
+// The array is one per device and shared by all callers of this entry point:
+// two of its calls that overlap on a device (different streams, or threads
+// without ordering between their streams) race on it and corrupt each other's
+// partial results.  Order them on one stream, or with events.
+//
+// Nothing in the scratch has to start at zero: the schedule kernel writes the
+// unit counts, prefixes and chunk sizes it and the merge later read, and every
+// partial record the merge reads is written by the tile kernel of the same
+// call first.  So no clearing is done.
+namespace {
+
+static __device__ __align__(256) unsigned char g_decode_scratch[KVQ_DECODE_STATIC_SCRATCH_BYTES];
+
+constexpr int kMaxScratchDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_ptr[kMaxScratchDevices] = {};
+
+// Device address of the current device's copy of the scratch; the first call
+// per device looks it up (cudaGetSymbolAddress, with that device current).
+kvq_status scratch_for_current_device(void** ptr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_status(e, "querying the current device");
+  if (dev < 0 || dev >= kMaxScratchDevices)
+    return fail(KVQ_ERR_UNSUPPORTED, "device %d: the static decode scratch covers devices 0..%d", dev,
+                kMaxScratchDevices - 1);
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e != cudaSuccess) return cuda_status(e, "looking up the static decode scratch");
+    if (p == nullptr) return fail(KVQ_ERR_CUDA, "the static decode scratch has no device address");
+    g_scratch_ptr[dev] = p;
+  }
+  *ptr = g_scratch_ptr[dev];
+  return KVQ_OK;
+}
+
+}  // namespace
+
+extern "C" kvq_status kvq_paged_decode_attention_static_scratch(
+    const kvq_config* cfg, const void* q, void* out, const int32_t* seq_lens, int num_seqs,
+    const int32_t* block_tables, int max_blocks_per_seq, int num_blocks, const void* k_pool, const void* v_pool,
+    const void* k_tail, const void* v_tail, float softmax_scale, int num_splits, int32_t* dev_status, void* stream) {
+  KVQ_TRY(check_config(cfg));
+  if (num_seqs < 0) return fail(KVQ_ERR_INVALID_ARG, "num_seqs must be >= 0 (got %d)", num_seqs);
+  if (num_splits < 0 || num_splits > 65535)
+    return fail(KVQ_ERR_INVALID_ARG, "num_splits must be 0..65535 (got %d)", num_splits);
+  int sms = 0;
+  if (num_splits == 0) KVQ_TRY(device_sm_count(&sms));
+  const size_t need = kvq::decode_workspace_bytes(*cfg, num_seqs, num_splits, sms);
+  if (need > KVQ_DECODE_STATIC_SCRATCH_BYTES)
+    return fail(KVQ_ERR_WORKSPACE,
+                "decode of %d sequences (num_splits %d) needs %zu bytes of scratch; the static scratch holds %zu: "
+                "pass fewer sequences or a smaller num_splits, or use kvq_paged_decode_attention with a workspace",
+                num_seqs, num_splits, need, static_cast<size_t>(KVQ_DECODE_STATIC_SCRATCH_BYTES));
+  void* scratch = nullptr;
+  KVQ_TRY(scratch_for_current_device(&scratch));
+  return kvq_paged_decode_attention(cfg, q, out, seq_lens, num_seqs, block_tables, max_blocks_per_seq, num_blocks,
+                                    k_pool, v_pool, k_tail, v_tail, softmax_scale, scratch,
+                                    KVQ_DECODE_STATIC_SCRATCH_BYTES, num_splits, dev_status, stream);
+}

@@ -28,8 +28,8 @@ KVQ_ERR_DEVICE_TIMEOUT = 6
 
 EXPORTED_SYMBOLS = (
     "kvq_get_layout", "kvq_decode_workspace_bytes", "kvq_quantize_tiles", "kvq_append_tokens",
-    "kvq_paged_decode_attention", "kvq_unpack_tiles", "kvq_status_string", "kvq_last_error",
-    "kvq_version",
+    "kvq_paged_decode_attention", "kvq_paged_decode_attention_static_scratch", "kvq_unpack_tiles",
+    "kvq_status_string", "kvq_last_error", "kvq_version",
 )
 
 
@@ -90,6 +90,8 @@ _SIGNATURES = {
     "kvq_append_tokens": [_cfgp, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp],
     "kvq_paged_decode_attention": [_cfgp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _vp, _vp, _vp, _vp, _f32, _vp,
                                    _sz, _i32, _vp, _vp],
+    "kvq_paged_decode_attention_static_scratch": [_cfgp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _vp, _vp, _vp,
+                                                  _vp, _f32, _i32, _vp, _vp],
     "kvq_unpack_tiles": [_cfgp, _vp, _i32, _vp, _i32, _i32, _i32, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
 }
 
@@ -218,6 +220,30 @@ def paged_decode_attention(cfg: Config, q, out, seq_lens, block_tables, k_pool, 
         _ptr(workspace, "workspace", torch.uint8), workspace.numel(), num_splits,
         _ptr(dev_status, "dev_status", torch.int32), _stream(stream))
     _check(st, "kvq_paged_decode_attention")
+
+
+# bytes of the library's static decode scratch (one per device)
+DECODE_STATIC_SCRATCH_BYTES = 32 << 20
+
+
+def paged_decode_attention_static_scratch(cfg: Config, q, out, seq_lens, block_tables, k_pool, v_pool, k_tail,
+                                          v_tail, softmax_scale: float | None = None, num_splits: int = 0,
+                                          num_blocks: int | None = None, dev_status=None, stream=None) -> None:
+    """``paged_decode_attention`` on the library's static per-device scratch
+    instead of a workspace: allocates nothing.  Calls that overlap on one
+    device race on that scratch; the first call per device should come before
+    any stream capture."""
+    if softmax_scale is None:
+        softmax_scale = cfg.head_dim ** -0.5
+    nb = k_pool.shape[0] if num_blocks is None else num_blocks
+    st = load_library().kvq_paged_decode_attention_static_scratch(
+        ctypes.byref(cfg.c()), _ptr(q, "q", torch.float16), _ptr(out, "out", torch.float16),
+        _ptr(seq_lens, "seq_lens", torch.int32), seq_lens.shape[0],
+        _ptr(block_tables, "block_tables", torch.int32), block_tables.shape[1], nb,
+        _ptr(k_pool, "k_pool", torch.uint8), _ptr(v_pool, "v_pool", torch.uint8),
+        _ptr(k_tail, "k_tail", torch.float16), _ptr(v_tail, "v_tail", torch.float16), float(softmax_scale),
+        num_splits, _ptr(dev_status, "dev_status", torch.int32), _stream(stream))
+    _check(st, "kvq_paged_decode_attention_static_scratch")
 
 
 def unpack_tiles(cfg: Config, tile_desc, block_tables, pool, is_v: bool, codes=None, meta=None, cvec=None,
