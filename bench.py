@@ -53,11 +53,18 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def source_digest() -> str:
+# sources a kernel's code depends on (a change to any of them voids its ncu traffic figure)
+KERNEL_SOURCES = {
+    "quantize_tc_kernel": ("kvq_quantize_tc.cu", "kvq_device.cuh", "kvq_internal.h"),
+    "decode_tiles_kernel": ("kvq_decode.cu", "kvq_device.cuh", "kvq_internal.h"),
+}
+
+
+def source_digest(kernel: str) -> str:
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "quantized_paged_kv_tile_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
@@ -73,7 +80,7 @@ def ncu_traffic(kernel: str, units_now: float):
             rec = json.load(f)[kernel]
     except (OSError, KeyError, ValueError):
         return None
-    if rec.get("source_digest") != source_digest():
+    if rec.get("source_digest") != source_digest(kernel):
         return None
     return rec["dram_bytes_per_launch"] * units_now / rec["units_per_launch"]
 
@@ -203,6 +210,19 @@ def cpu_sample_bytes(w, bm, n_pairs):
 
 
 # --------------------------------------------------------------------------- GPU arm
+
+def workload_config(w, world: int) -> dict:
+    """The `config` object of the JSON line (both arms)."""
+    lens0 = np.asarray(w.lens, dtype=np.int64)
+    lens1 = lens0 + w.append_tokens
+    rows_gb = float(lens0.sum()) * w.num_kv_heads * 128 * 2 * 2 / 1e9
+    return {"workload": f"{w.name}: {w.num_seqs} seqs x {int(lens0[0])} cached tokens + {w.append_tokens} appended, "
+                        f"{w.num_kv_heads} KV heads, {w.num_q_heads} query heads, d=128, T={w.tile_tokens}, P=16, "
+                        f"b_K={w.bits_k}, b_V={w.bits_v}, n={w.iters}, pages scattered by a seeded permutation",
+            "global_batch": w.num_seqs * world, "seq_len": int(lens1.max()),
+            "parallelism": f"replicas x{world} (no data-path collective)",
+            "l2": f"inputs larger than L2 (fp16 rows {rows_gb:.1f} GB per replica)"}
+
 
 def run_kvq(args, ranks):
     import torch
@@ -371,21 +391,15 @@ def run_kvq(args, ranks):
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": ranks.world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": f"{w.name}: {B} seqs x {int(lens0[0])} cached tokens + {w.append_tokens} appended, "
-                               f"{H} KV heads, {w.num_q_heads} query heads, d=128, T={T}, P=16, "
-                               f"b_K={w.bits_k}, b_V={w.bits_v}, n={w.iters}, pages scattered by a seeded "
-                               f"permutation",
-                   "global_batch": B * ranks.world, "seq_len": int(lens1.max()),
-                   "parallelism": f"replicas x{ranks.world} (no data-path collective)",
-                   "l2": "inputs larger than L2 (fp16 rows 3.2 GB, pages 0.9 GB per replica)"},
+        "config": workload_config(w, ranks.world),
         "decode": {"gbs": d_gbs, "ms": d_avg, "frac": d_gbs / peak, "tok_per_s": B / (d_avg * 1e-3),
                    "kv_tok_per_s": bm["kv_tokens"] / (d_avg * 1e-3), "bytes": bm["decode"],
                    "fp16_bytes_equiv": bm["kv_tokens"] * H * 512},
         "quantize": {"gbs": q_gbs, "ms": q_avg, "frac": q_gbs / peak, "bytes": bm["quantize"]},
         "append": {"ms": statistics.mean(a_ms), "bytes": bm["append"]},
-        "roofline": {"bound": "hbm", "kernel": "quantize_tiles_kernel", "achieved": q_gbs, "peak": peak,
+        "roofline": {"bound": "hbm", "kernel": "quantize_tc_kernel", "achieved": q_gbs, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": q_gbs / peak,
-                     "traffic": ncu_traffic("quantize_tiles_kernel", bm["quant_units"])},
+                     "traffic": ncu_traffic("quantize_tc_kernel", bm["quant_units"])},
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps, "clocks": clk,
     }
     return line
@@ -395,7 +409,8 @@ def run_kvq(args, ranks):
 
 def run_reference(args, ranks):
     from quantized_paged_kv_tile_b200 import synth
-    w = synth.workload(args.workload)
+    over = {"num_seqs": args.num_seqs} if args.num_seqs > 0 else {}
+    w = synth.workload(args.workload, **over)
     bm = byte_model(w, 0, 0)
     procs = max(1, min(os.cpu_count() or 1, 8))
     pairs = oracle_pairs(w, procs)
@@ -412,13 +427,11 @@ def run_reference(args, ranks):
     value = nbytes * len(times) / sum(times) / 1e9
     sample = (f"per step {len(pairs)} of {w.num_seqs * w.num_kv_heads} (sequence, KV head) pairs: fp64 quantize "
               f"of every K and V tile, dequantize, fp64 decode of the query group, {procs} processes")
-    lens1 = np.asarray(w.lens) + w.append_tokens
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": ranks.world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(times),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{w.name} (oracle sample)", "global_batch": w.num_seqs,
-                   "seq_len": int(lens1.max()), "parallelism": "host cores"},
+        "config": workload_config(w, ranks.world),
         "cpu_baseline": {"value": value, "unit": "GB/s", "cores": procs, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
