@@ -74,12 +74,15 @@ __device__ __forceinline__ long long gtime() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
+// a waiting thread may be suspended up to this long per try (it resumes when
+// the phase completes)
+constexpr uint32_t kSuspendHintNs = 20000;
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
       : "memory");
   return ok != 0;
 }
@@ -155,6 +158,33 @@ __device__ __forceinline__ bool math_any(bool v) {
   return r != 0;
 }
 
+// Scalar helpers for the per-row statistics (not per element).  The
+// approximate forms are within 2 ulp; a scale change that small moves a code
+// only for values within ~1e-7 of a rounding boundary.
+__device__ __forceinline__ float sqrt_fast(float x) {
+  float y;
+  asm("sqrt.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float div_fast(float a, float b) {  // full range, 2 ulp
+  float y;
+  asm("div.full.f32 %0, %1, %2;" : "=f"(y) : "f"(a), "f"(b));
+  return y;
+}
+// the exponent frexpf would return, for m >= 0
+__device__ __forceinline__ int frexp_exponent(float m) {
+  const uint32_t be = __float_as_uint(m) >> 23;
+  if (be - 1u < 254u) return static_cast<int>(be) - 126;  // normal
+  int e;
+  frexpf(m, &e);  // zero, subnormal, inf, nan
+  return e;
+}
+// ldexpf(x, k): one exact multiply when 2^k is a normal float
+__device__ __forceinline__ float scale_pow2(float x, int k) {
+  if (k >= -126 && k <= 127) return x * __uint_as_float(static_cast<uint32_t>(k + 127) << 23);
+  return ldexpf(x, k);
+}
+
 __device__ __forceinline__ float min3f(float a, float b, float c) {
   float d;
   asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -205,7 +235,7 @@ __device__ __forceinline__ Moments moments(const float2 (&s1)[4], const float2 (
 // two halves of n values each (always combined in the order (first, second))
 __device__ __forceinline__ float combined_std(Moments a, Moments b, float n) {
   const float dm = a.mean - b.mean;
-  return sqrtf((a.m2 + b.m2 + dm * dm * (0.5f * n)) / (2.f * n));
+  return sqrt_fast((a.m2 + b.m2 + dm * dm * (0.5f * n)) * (0.5f / n));
 }
 
 // Everything after the group's rows are in shared memory and the MMAs are
@@ -254,14 +284,14 @@ __device__ void quantize_group_from_tmem(unsigned char* smem, uint32_t tbase, in
 
   auto tile_exp = [&](int t) {  // exponent of the tile's max C over the warps that hold it
     float m = 0.f;
+    if constexpr (T == 128) {
 #pragma unroll
-    for (int w = 0; w < 8; ++w) {
-      const bool holds = T == 128 ? true : (t / kLocal == (w >> 2));
-      if (holds) m = fmaxf(m, red[w * 4 + t]);
+      for (int w = 0; w < 8; ++w) m = fmaxf(m, red[w * 4]);
+    } else {  // tile t lives in the token columns of half t / kLocal: warps 4h..4h+3
+      const float* rw = red + 16 * (t / kLocal) + t;
+      m = fmaxf(fmaxf(rw[0], rw[4]), fmaxf(rw[8], rw[12]));
     }
-    int e;
-    frexpf(m, &e);
-    return e;
+    return frexp_exponent(m);
   };
   for (int it = 0; it < iters; ++it) {
     cc = cc_buf + (it & 1) * (4 * kRows);
@@ -285,9 +315,9 @@ __device__ void quantize_group_from_tmem(unsigned char* smem, uint32_t tbase, in
         }
         const Moments mo = moments(s1, s2, shift, static_cast<float>(T));
         const float c = cc[t * kRows + row];
-        const float sigma = fmaxf(c * sqrtf(mo.m2 / static_cast<float>(T)), eps);
+        const float sigma = fmaxf(c * sqrt_fast(mo.m2 * (1.f / static_cast<float>(T))), eps);
         Cj[lt] *= sigma;
-        cc[t * kRows + row] = fminf(c / sigma, FLT_MAX);  // a zero channel keeps a finite factor
+        cc[t * kRows + row] = fminf(div_fast(c, sigma), FLT_MAX);  // a zero channel keeps a finite factor
       }
     } else {
       float2 s1[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
@@ -310,7 +340,7 @@ __device__ void quantize_group_from_tmem(unsigned char* smem, uint32_t tbase, in
       const float sigma = fmaxf(c * sd, eps);
       Cj[0] *= sigma;
       pair_sync(qd);  // both halves have read cc[row]
-      if (hf == 0) cc[row] = fminf(c / sigma, FLT_MAX);
+      if (hf == 0) cc[row] = fminf(div_fast(c, sigma), FLT_MAX);
     }
 #pragma unroll
     for (int lt = 0; lt < kLocal; ++lt) {
@@ -346,7 +376,7 @@ __device__ void quantize_group_from_tmem(unsigned char* smem, uint32_t tbase, in
         const float sd = hf == 0 ? combined_std(mo, other, 64.f) : combined_std(other, mo, 64.f);
         const float rho = fmaxf(r * sd, eps);
         Ri *= rho;
-        r_new = fminf(r / rho, FLT_MAX);  // a zero token keeps a finite factor
+        r_new = fminf(div_fast(r, rho), FLT_MAX);  // a zero token keeps a finite factor
       }
     }
     // ---- (C, R) -> (C / 2^k, R 2^k) per tile, max C in [1, 2): every thread
@@ -355,13 +385,13 @@ __device__ void quantize_group_from_tmem(unsigned char* smem, uint32_t tbase, in
     for (int lt = 0; lt < kLocal; ++lt) {
       const int t = ch_tile(lt);
       const int e = tile_exp(t);
-      Cj[lt] = ldexpf(Cj[lt], 1 - e);
-      if (T < 128 || hf == 0) cc_next[t * kRows + row] = fminf(ldexpf(cc[t * kRows + row], e - 1), FLT_MAX);
+      Cj[lt] = scale_pow2(Cj[lt], 1 - e);
+      if (T < 128 || hf == 0) cc_next[t * kRows + row] = fminf(scale_pow2(cc[t * kRows + row], e - 1), FLT_MAX);
     }
     {
       const int e = tile_exp(my_tile);
-      Ri = ldexpf(Ri, e - 1);
-      if (tok_live && hf == 0) rr[row] = fminf(ldexpf(r_new, 1 - e), FLT_MAX);
+      Ri = scale_pow2(Ri, e - 1);
+      if (tok_live && hf == 0) rr[row] = fminf(scale_pow2(r_new, 1 - e), FLT_MAX);
     }
     math_sync();
   }
@@ -399,8 +429,8 @@ __device__ void quantize_group_from_tmem(unsigned char* smem, uint32_t tbase, in
     mu = fmaxf(mu, o.y);
     const float r = rr[row];
     const float z = zu * r, mx = mu * r;
-    const float s = (mx - z) / static_cast<float>(qmax);
-    const float a = s > 0.f ? r / s : 0.f;  // s == 0: every code is 0
+    const float s = div_fast(mx - z, static_cast<float>(qmax));
+    const float a = s > 0.f ? div_fast(r, s) : 0.f;  // s == 0: every code is 0
     const float b0 = -zu * a;
     // q = t + 1.5 * 2^23 holds round_half_even(t) in its low mantissa bits,
     // so its bit pattern is 0x4B400000 + code.  Words are built by shift-adds
@@ -408,6 +438,8 @@ __device__ void quantize_group_from_tmem(unsigned char* smem, uint32_t tbase, in
     // (arithmetic mod 2^32); codes lie in [0, 2^b - 1] because min and max of
     // the row map to 0 and 2^b - 1 by construction.
     constexpr uint32_t kMagicBits = 0x4B400000u;
+    const float2 a2 = make_float2(a, a), b2 = make_float2(b0, b0);
+    const float2 magic2 = make_float2(12582912.0f, 12582912.0f);  // 1.5 * 2^23
     if constexpr (!kGrouped) {
       uint32_t words[2 * bits];  // channels 64hf..64hf+63: 2b words
 #pragma unroll
@@ -415,18 +447,19 @@ __device__ void quantize_group_from_tmem(unsigned char* smem, uint32_t tbase, in
       float x[32];
 #pragma unroll
       for (int c = 0; c < 64; ++c) {
-        if ((c & 31) == 0) {  // pass 2: u_j = x_j c_j for the next 32 channels, then the codes
+        if ((c & 31) == 0) {  // pass 2 for the next 32 channels: u_j = x_j c_j, then u_j a + b0 + magic
           tmem_ld32(d1 + c, x);
 #pragma unroll
           for (int k = 0; k < 32; k += 4) {
             const float4 cv = *reinterpret_cast<const float4*>(cvec + c + k);
             const float2 u0 = __fmul2_rn(make_float2(x[k], x[k + 1]), make_float2(cv.x, cv.y));
             const float2 u1 = __fmul2_rn(make_float2(x[k + 2], x[k + 3]), make_float2(cv.z, cv.w));
-            x[k] = u0.x; x[k + 1] = u0.y; x[k + 2] = u1.x; x[k + 3] = u1.y;
+            const float2 q0 = __fadd2_rn(__ffma2_rn(u0, a2, b2), magic2);
+            const float2 q1 = __fadd2_rn(__ffma2_rn(u1, a2, b2), magic2);
+            x[k] = q0.x; x[k + 1] = q0.y; x[k + 2] = q1.x; x[k + 3] = q1.y;
           }
         }
-        const float u = x[c & 31];
-        const uint32_t qb = __float_as_uint(__fadd_rn(__fmaf_rn(u, a, b0), 12582912.0f));
+        const uint32_t qb = __float_as_uint(x[c & 31]);
         const int bit = c * bits;
         if constexpr (bits == 3) {
           const uint32_t code = (qb - kMagicBits) & 7u;
@@ -462,20 +495,23 @@ __device__ void quantize_group_from_tmem(unsigned char* smem, uint32_t tbase, in
       float x[32];
 #pragma unroll
       for (int c = 0; c < 64; ++c) {
-        if ((c & 31) == 0) {  // pass 2: u_j = x_j c_j for the next 32 channels, then the codes
+        if ((c & 31) == 0) {  // pass 2 for the next 32 channels: u_j = x_j c_j, then u_j a + b0 + magic
           tmem_ld32(d1 + c, x);
 #pragma unroll
           for (int k = 0; k < 32; k += 4) {
             const float4 cv = *reinterpret_cast<const float4*>(cvec + c + k);
             const float2 u0 = __fmul2_rn(make_float2(x[k], x[k + 1]), make_float2(cv.x, cv.y));
             const float2 u1 = __fmul2_rn(make_float2(x[k + 2], x[k + 3]), make_float2(cv.z, cv.w));
-            x[k] = u0.x; x[k + 1] = u0.y; x[k + 2] = u1.x; x[k + 3] = u1.y;
+            const float2 q0 = __fadd2_rn(__ffma2_rn(u0, a2, b2), magic2);
+            const float2 q1 = __fadd2_rn(__ffma2_rn(u1, a2, b2), magic2);
+            x[k] = q0.x; x[k + 1] = q0.y; x[k + 2] = q1.x; x[k + 3] = q1.y;
           }
         }
-        const float u = x[c & 31];
-        const uint32_t qb = __float_as_uint(__fadd_rn(__fmaf_rn(u, a, b0), 12582912.0f));
-        const int n = (64 * hf + c) >> 3, g8 = c & 7;
-        const int m = n / h - hf * nm, e = n % h;
+        const uint32_t qb = __float_as_uint(x[c & 31]);
+        // n = 8 hf + c / 8 and 8 hf is a multiple of h, so m and e depend on c
+        // alone: compile-time register indices after unrolling
+        const int q8 = c >> 3, g8 = c & 7;
+        const int m = q8 / h, e = q8 % h;
         hw[g8 * nm + m] += qb << (bits * e);
       }
       uint32_t k0 = 0;
@@ -518,7 +554,7 @@ __device__ void quantize_group_from_tmem(unsigned char* smem, uint32_t tbase, in
   math_sync();
   // page stores: thread q < 8 stores page q of the group
   if (tid < 8) {
-    const int t = tid / kPagesPerTile, k = tid % kPagesPerTile;
+    const int t = tid / kPagesPerTile;
     if (t < G && ((valid >> t) & 1)) {
       const int blk = store_blk;
       uint8_t* dst = pool + (static_cast<size_t>(blk) * num_heads + head) * static_cast<size_t>(g.page_bytes);
