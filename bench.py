@@ -288,8 +288,9 @@ def run_kvq(args, ranks):
                            stream=stream)
         if ev is not None:
             ev[1].record(stream)
-        kvq.append_tokens(cfg, new_k, new_v, cu_new, before, max_new, bt, k_pool, v_pool, k_tail, v_tail,
-                          num_blocks=nblocks, dev_status=status, stream=stream)
+        if max_new > 0:  # no unfinished prefill rows and no new tokens: nothing to append
+            kvq.append_tokens(cfg, new_k, new_v, cu_new, before, max_new, bt, k_pool, v_pool, k_tail, v_tail,
+                              num_blocks=nblocks, dev_status=status, stream=stream)
         if ev is not None:
             ev[2].record(stream)
         kvq.paged_decode_attention(cfg, q, out, seq_lens, bt, k_pool, v_pool, k_tail, v_tail, ws,
@@ -386,7 +387,8 @@ def run_kvq(args, ranks):
                          f"tile, dequantize, fp64 decode of the query group; {secs:.1f} s wall on {procs} "
                          f"processes, same byte model"}
 
-    launches_per_step = 1 + 1 + 2
+    # quantize; append (when there are rows to append); decode = schedule + tiles + merge
+    launches_per_step = 1 + (1 if max_new > 0 else 0) + 3
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": ranks.world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True, "scaling": "weak",
