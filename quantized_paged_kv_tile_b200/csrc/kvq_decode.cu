@@ -370,54 +370,40 @@ __global__ void __launch_bounds__(kDecWarps * 32, T == 128 ? 2 : 3) decode_tiles
       const unsigned char* sK = stage_base + st * Geo::kStage;
       const unsigned char* sV = sK + NP * Geo::kPageK;
 
-      // -- q'' = q' * C~K in hi/lo fp16 pairs (A operand rows g and g+8) and sigma
-      uint32_t qa_hi[16], qa_lo[16];
+      // -- scores: D[16 rows][8 tokens] per (page, n-block); rows g / g+8 = head g hi / lo.
+      // The A fragments, q'' = q' * C~K in hi/lo fp16 pairs, are built per
+      // k-block from q' and the tile's C~K slice (not all held at once), and
+      // sigma = sum_j q''_j is accumulated on the way.  Pages go in chunks of
+      // up to 4 so that one chunk's code words and accumulators are live; the
+      // chunk's scores (log2 domain, tokens 8nb + 2t, 8nb + 2t + 1 of each page)
+      // are kept.
+      constexpr int kPc = NP < 4 ? NP : 4;
       float sig = 0.f;
-      {
-        float ck[32];
+      float sc[NP][2][2];
+      float mt = -INFINITY;
+      // C~K of channels 32t + c, c + 1 (c even) within the tile's page slices
+      auto ck_pair = [&](int c) {
+        const int ch = 32 * t + c;
+        const __half2 h = *reinterpret_cast<const __half2*>(sK + (ch / Geo::kCs) * Geo::kPageK + Geo::kCodesK + 64 +
+                                                            2 * (ch % Geo::kCs));
+        return __half22float2(h);
+      };
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const int c0 = 32 * t + 8 * v;  // channels c0..c0+7, within one page slice
-          const unsigned char* src = sK + (c0 / Geo::kCs) * Geo::kPageK + Geo::kCodesK + 64 + 2 * (c0 % Geo::kCs);
-          const uint4 raw = *reinterpret_cast<const uint4*>(src);
-          const __half2* hp = reinterpret_cast<const __half2*>(&raw);
+      for (int pc = 0; pc < NP; pc += kPc) {
+        float sd[kPc][2][4];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const float2 f = __half22float2(hp[k]);
-            ck[8 * v + 2 * k] = f.x;
-            ck[8 * v + 2 * k + 1] = f.y;
-          }
-        }
+        for (int pg = 0; pg < kPc; ++pg)
 #pragma unroll
-        for (int p = 0; p < 16; ++p) {
-          const int c0 = pair_ch0<BK>(p), c1 = c0 + pair_gap<BK>();
-          const float x0 = qs[c0] * ck[c0], x1 = qs[c1] * ck[c1];
-          sig += x0 + x1;
-          const __half2 hv = __floats2half2_rn(x0, x1);
-          const float2 hf = __half22float2(hv);
-          qa_hi[p] = h2_as_u32(hv);
-          qa_lo[p] = h2_as_u32(__floats2half2_rn(x0 - hf.x, x1 - hf.y));
-        }
-        sig += __shfl_xor_sync(kFull, sig, 1);
-        sig += __shfl_xor_sync(kFull, sig, 2);
-      }
-
-      // -- scores: D[16 rows][8 tokens] per (page, n-block); rows g / g+8 = head g hi / lo
-      float sd[NP][2][4];
+          for (int nb = 0; nb < 2; ++nb)
 #pragma unroll
-      for (int pg = 0; pg < NP; ++pg)
-#pragma unroll
-        for (int nb = 0; nb < 2; ++nb)
-#pragma unroll
-          for (int k = 0; k < 4; ++k) sd[pg][nb][k] = 0.f;
-      {
+            for (int k = 0; k < 4; ++k) sd[pg][nb][k] = 0.f;
         // lane (g, t) reads its 4*BK-byte chunk (channels 32t..32t+31) of tokens g and 8+g
-        uint32_t rec[NP][2][BK];
+        uint32_t rec[kPc][2][BK];
 #pragma unroll
-        for (int pg = 0; pg < NP; ++pg)
+        for (int pg = 0; pg < kPc; ++pg)
 #pragma unroll
           for (int nb = 0; nb < 2; ++nb) {
-            const unsigned char* src = sK + pg * Geo::kPageK + (8 * nb + g) * (16 * BK) + t * (4 * BK);
+            const unsigned char* src = sK + (pc + pg) * Geo::kPageK + (8 * nb + g) * (16 * BK) + t * (4 * BK);
             if constexpr (BK == 4) {
               const uint4 v = *reinterpret_cast<const uint4*>(src);
               rec[pg][nb][0] = v.x; rec[pg][nb][1] = v.y; rec[pg][nb][2] = v.z; rec[pg][nb][3] = v.w;
@@ -429,36 +415,45 @@ __global__ void __launch_bounds__(kDecWarps * 32, T == 128 ? 2 : 3) decode_tiles
         constexpr int kbPerWord = 8 / BK;  // k-blocks per word: 2 (b=4) or 4 (b=2)
 #pragma unroll
         for (int wd = 0; wd < BK; ++wd) {
-          uint32_t pr[NP][2][16 / BK];
+          uint32_t pr[kPc][2][16 / BK];
 #pragma unroll
-          for (int pg = 0; pg < NP; ++pg)
+          for (int pg = 0; pg < kPc; ++pg)
 #pragma unroll
             for (int nb = 0; nb < 2; ++nb) unpack_word<BK>(rec[pg][nb][wd], pr[pg][nb]);
 #pragma unroll
           for (int j = 0; j < kbPerWord; ++j) {
             const int kb = wd * kbPerWord + j;
-            const uint32_t afr[4] = {qa_hi[2 * kb], qa_lo[2 * kb], qa_hi[2 * kb + 1], qa_lo[2 * kb + 1]};
+            // pairs 2kb, 2kb+1: channels (c0, c1) and (c0+1, c1+1), c0 even
+            const int c0 = pair_ch0<BK>(2 * kb), c1 = c0 + pair_gap<BK>();
+            const float2 ka = ck_pair(c0), kc = ck_pair(c1);
+            const float x00 = qs[c0] * ka.x, x01 = qs[c0 + 1] * ka.y;
+            const float x10 = qs[c1] * kc.x, x11 = qs[c1 + 1] * kc.y;
+            if (pc == 0) sig += (x00 + x01) + (x10 + x11);
+            const __half2 h0 = __floats2half2_rn(x00, x10), h1 = __floats2half2_rn(x01, x11);
+            const float2 f0 = __half22float2(h0), f1 = __half22float2(h1);
+            const uint32_t afr[4] = {h2_as_u32(h0), h2_as_u32(__floats2half2_rn(x00 - f0.x, x10 - f0.y)),
+                                     h2_as_u32(h1), h2_as_u32(__floats2half2_rn(x01 - f1.x, x11 - f1.y))};
 #pragma unroll
-            for (int pg = 0; pg < NP; ++pg)
+            for (int pg = 0; pg < kPc; ++pg)
 #pragma unroll
               for (int nb = 0; nb < 2; ++nb) mma16816(sd[pg][nb], afr, pr[pg][nb][2 * j], pr[pg][nb][2 * j + 1]);
           }
         }
-      }
-
-      // -- scores in the log2 domain; tokens (8nb + 2t, 8nb + 2t + 1) of each page
-      float sc[NP][2][2];
-      float mt = -INFINITY;
+        if (pc == 0) {
+          sig += __shfl_xor_sync(kFull, sig, 1);
+          sig += __shfl_xor_sync(kFull, sig, 2);
+        }
 #pragma unroll
-      for (int pg = 0; pg < NP; ++pg) {
-        const unsigned char* meta = sK + pg * Geo::kPageK + Geo::kCodesK;
+        for (int pg = 0; pg < kPc; ++pg) {
+          const unsigned char* meta = sK + (pc + pg) * Geo::kPageK + Geo::kCodesK;
 #pragma unroll
-        for (int nb = 0; nb < 2; ++nb) {
-          const uint2 mm = *reinterpret_cast<const uint2*>(meta + 4 * (8 * nb + 2 * t));
-          const float2 m0 = __half22float2(u32_as_h2(mm.x)), m1 = __half22float2(u32_as_h2(mm.y));
-          sc[pg][nb][0] = m0.x * (sd[pg][nb][0] + sd[pg][nb][2]) + m0.y * sig;
-          sc[pg][nb][1] = m1.x * (sd[pg][nb][1] + sd[pg][nb][3]) + m1.y * sig;
-          mt = fmaxf(mt, fmaxf(sc[pg][nb][0], sc[pg][nb][1]));
+          for (int nb = 0; nb < 2; ++nb) {
+            const uint2 mm = *reinterpret_cast<const uint2*>(meta + 4 * (8 * nb + 2 * t));
+            const float2 m0 = __half22float2(u32_as_h2(mm.x)), m1 = __half22float2(u32_as_h2(mm.y));
+            sc[pc + pg][nb][0] = m0.x * (sd[pg][nb][0] + sd[pg][nb][2]) + m0.y * sig;
+            sc[pc + pg][nb][1] = m1.x * (sd[pg][nb][1] + sd[pg][nb][3]) + m1.y * sig;
+            mt = fmaxf(mt, fmaxf(sc[pc + pg][nb][0], sc[pc + pg][nb][1]));
+          }
         }
       }
       mt = fmaxf(mt, __shfl_xor_sync(kFull, mt, 1));
