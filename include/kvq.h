@@ -239,6 +239,15 @@ KVQ_API kvq_status kvq_unpack_tiles(const kvq_config* cfg, const int32_t* tile_d
                             const void* pool, int is_v, uint8_t* codes, void* meta, void* cvec,
                             float* out_rot, float* out_orig, int32_t* dev_status, void* stream);
 
+/* Self-test of device-side failure detection: launches, on `stream`, one
+ * single-thread kernel per kernel file that waits with that file's bounded
+ * mbarrier wait on a barrier nothing ever arrives at.  Each wait gives up
+ * after its limit (2 s) and records KVQ_ERR_DEVICE_TIMEOUT in *dev_status
+ * (device int32, required); nothing traps and the context stays usable.
+ * Takes about 4 s of device time.  Returns KVQ_ERR_INVALID_ARG for a NULL
+ * dev_status, KVQ_ERR_CUDA on a launch error. */
+KVQ_API kvq_status kvq_selftest_bounded_wait(int32_t* dev_status, void* stream);
+
 /* Static text for a status code. */
 KVQ_API const char* kvq_status_string(kvq_status s);
 /* Detail of the last error on the calling host thread ("" if none). */

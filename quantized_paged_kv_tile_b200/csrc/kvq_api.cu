@@ -301,6 +301,13 @@ kvq_status kvq_unpack_tiles(const kvq_config* cfg, const int32_t* tile_desc, int
   return cuda_status(kvq::launch_unpack_tiles(a, static_cast<cudaStream_t>(stream)), "kvq_unpack_tiles launch");
 }
 
+kvq_status kvq_selftest_bounded_wait(int32_t* dev_status, void* stream) {
+  if (dev_status == nullptr) return fail(KVQ_ERR_INVALID_ARG, "dev_status is NULL");
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  KVQ_TRY(cuda_status(kvq::launch_selftest_wait_quantize(dev_status, s), "quantize wait self-test launch"));
+  return cuda_status(kvq::launch_selftest_wait_decode(dev_status, s), "decode wait self-test launch");
+}
+
 }  // extern "C"
 
 // ------------------------------------------------------- decode, static scratch

@@ -550,6 +550,15 @@ __global__ void __launch_bounds__(kDecWarps * 32, T == 128 ? 2 : 3) decode_tiles
   }
 }
 
+// ------------------------------------------------------------------ self-test
+// The decode kernel's bounded wait on a barrier that nothing arrives at.
+__global__ void selftest_wait_decode_kernel(int32_t* dev_status) {
+  __shared__ __align__(8) uint64_t bar;
+  mbar_init(&bar, 1);
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  if (!mbar_wait_bounded(&bar, 0)) report_error(dev_status, KVQ_ERR_DEVICE_TIMEOUT);
+}
+
 // ------------------------------------------------------------------ merge
 constexpr int kMergeThreads = 256;
 
@@ -731,6 +740,11 @@ size_t decode_workspace_bytes(const kvq_config& cfg, int num_seqs, int num_split
                            ? static_cast<size_t>(num_seqs) * cfg.num_kv_heads * num_splits
                            : static_cast<size_t>(kUnitsPerSm) * num_sms + static_cast<size_t>(num_seqs) * cfg.num_kv_heads;
   return wl.part_off + units * cfg.group_size * kPartFloats * sizeof(float);
+}
+
+cudaError_t launch_selftest_wait_decode(int32_t* dev_status, cudaStream_t s) {
+  selftest_wait_decode_kernel<<<1, 1, 0, s>>>(dev_status);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_paged_decode(const DecodeArgs& a, cudaStream_t s) {

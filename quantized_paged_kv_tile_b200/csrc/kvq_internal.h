@@ -110,4 +110,10 @@ struct DecodeArgs {
 size_t decode_workspace_bytes(const kvq_config& cfg, int num_seqs, int num_splits, int num_sms);
 cudaError_t launch_paged_decode(const DecodeArgs& a, cudaStream_t s);
 
+// Self-tests of the bounded mbarrier waits (one per kernel file): a wait on
+// a barrier nothing arrives at gives up after its limit and records
+// KVQ_ERR_DEVICE_TIMEOUT in *dev_status.
+cudaError_t launch_selftest_wait_quantize(int32_t* dev_status, cudaStream_t s);
+cudaError_t launch_selftest_wait_decode(int32_t* dev_status, cudaStream_t s);
+
 }  // namespace kvq

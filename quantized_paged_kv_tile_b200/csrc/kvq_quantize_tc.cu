@@ -796,6 +796,17 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_tc_kernel(const __grid_
   tmem_free(tbase);  // includes a __syncthreads of all warps
 }
 
+// ---------------------------------------------------------------- self-test
+// One thread waits, with the kernels' bounded wait, on a barrier that nothing
+// arrives at; the wait gives up after its limit and the timeout is recorded.
+__global__ void selftest_wait_kernel(int32_t* dev_status) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = smem_u32(&bar);
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(b));
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  if (!mbar_wait(b, 0)) report_error(dev_status, KVQ_ERR_DEVICE_TIMEOUT);
+}
+
 // ---------------------------------------------------------------- append
 // One CTA per (sequence, KV head, K|V): every tile completed by the new
 // tokens is loaded (old tail rows + new rows) into the same swizzled layout
@@ -1002,6 +1013,11 @@ struct AppendLauncher {
 };
 
 }  // namespace
+
+cudaError_t launch_selftest_wait_quantize(int32_t* dev_status, cudaStream_t s) {
+  selftest_wait_kernel<<<1, 1, 0, s>>>(dev_status);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_quantize_tiles(const QuantizeArgs& a, cudaStream_t s) {
   if (a.num_tiles == 0) return cudaSuccess;

@@ -29,7 +29,7 @@ KVQ_ERR_DEVICE_TIMEOUT = 6
 EXPORTED_SYMBOLS = (
     "kvq_get_layout", "kvq_decode_workspace_bytes", "kvq_quantize_tiles", "kvq_append_tokens",
     "kvq_paged_decode_attention", "kvq_paged_decode_attention_static_scratch", "kvq_unpack_tiles",
-    "kvq_status_string", "kvq_last_error", "kvq_version",
+    "kvq_selftest_bounded_wait", "kvq_status_string", "kvq_last_error", "kvq_version",
 )
 
 
@@ -92,6 +92,7 @@ _SIGNATURES = {
                                    _sz, _i32, _vp, _vp],
     "kvq_paged_decode_attention_static_scratch": [_cfgp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _vp, _vp, _vp,
                                                   _vp, _f32, _i32, _vp, _vp],
+    "kvq_selftest_bounded_wait": [_vp, _vp],
     "kvq_unpack_tiles": [_cfgp, _vp, _i32, _vp, _i32, _i32, _i32, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
 }
 
@@ -244,6 +245,13 @@ def paged_decode_attention_static_scratch(cfg: Config, q, out, seq_lens, block_t
         _ptr(k_tail, "k_tail", torch.float16), _ptr(v_tail, "v_tail", torch.float16), float(softmax_scale),
         num_splits, _ptr(dev_status, "dev_status", torch.int32), _stream(stream))
     _check(st, "kvq_paged_decode_attention_static_scratch")
+
+
+def selftest_bounded_wait(dev_status, stream=None) -> None:
+    """Run the device-side bounded-wait self-test (about 4 s): afterwards
+    ``dev_status`` holds KVQ_ERR_DEVICE_TIMEOUT."""
+    st = load_library().kvq_selftest_bounded_wait(_ptr(dev_status, "dev_status", torch.int32), _stream(stream))
+    _check(st, "kvq_selftest_bounded_wait")
 
 
 def unpack_tiles(cfg: Config, tile_desc, block_tables, pool, is_v: bool, codes=None, meta=None, cvec=None,

@@ -155,3 +155,9 @@ def test_block_table_is_a_permutation():
     assert bt.shape == (6, 8193)
     assert np.array_equal(np.sort(bt.ravel()), np.arange(6 * 8193))
     assert not np.array_equal(bt.ravel(), np.arange(6 * 8193))
+
+
+def test_selftest_rejects_null_status(lib):
+    # fails on the host before any launch
+    assert lib.kvq_selftest_bounded_wait(None, None) == kvq.KVQ_ERR_INVALID_ARG
+    assert "dev_status" in lib.kvq_last_error().decode()
