@@ -47,6 +47,16 @@ oracle follows (and the CUDA path implements independently) are:
 5. Decode: out = softmax(q K^T / sqrt(d)) V in fp64 over the dequantized
    tiles followed by the raw fp16 rows of the unfinished last tile.
 
+Variant (not on the pages; a randomized rotation): with a nonzero 32-bit
+``seed`` the rotation is X' = X D_s H, D_s = diag(s) with s_j = -1 where the
+j-th output of SplitMix64 started at state ``seed`` has its top bit set and
++1 otherwise (SplitMix64 as published by Steele, Lea and Flood, "Fast
+splittable pseudorandom number generators", OOPSLA 2014: the state advances
+by the golden-ratio gamma 0x9E3779B97F4A7C15 and each output is the state
+passed through the finalizer z ^= z >> 30; z *= 0xBF58476D1CE4E5B9;
+z ^= z >> 27; z *= 0x94D049BB133111EB; z ^= z >> 31).  The inverse is
+X = X' H D_s.  Seed 0 is the plain rotation of 1.
+
 Precision.  Everything runs in fp64 unless a caller asks for float32: where a
 floating-point value decides an integer code, the parity tests run the
 quantizer in float32, the precision the GPU takes that decision in.
@@ -90,16 +100,42 @@ def sylvester_signs(d: int) -> np.ndarray:
     return np.rint(sylvester_hadamard(d) * math.sqrt(d))
 
 
-def rotate(x: np.ndarray, dtype=np.float64) -> np.ndarray:
-    """X' = X H for token rows X[..., d] (the rotation of step 1).
+_MASK64 = (1 << 64) - 1
 
-    Computed as (X times the +-1 matrix) / sqrt(d): for fp16 inputs the +-1
-    sums are exact in fp64, so a rotated channel that is zero in exact
-    arithmetic comes out exactly zero.
+
+def splitmix64_outputs(seed: int, n: int) -> list:
+    """The first n outputs of SplitMix64 started at state ``seed`` (the
+    generator's published definition, restated in the module docstring)."""
+    state = seed & _MASK64
+    out = []
+    for _ in range(n):
+        state = (state + 0x9E3779B97F4A7C15) & _MASK64
+        z = state
+        z = ((z ^ (z >> 30)) * 0xBF58476D1CE4E5B9) & _MASK64
+        z = ((z ^ (z >> 27)) * 0x94D049BB133111EB) & _MASK64
+        out.append(z ^ (z >> 31))
+    return out
+
+
+def rotation_signs(d: int, seed: int = 0) -> np.ndarray:
+    """Channel signs s of the randomized rotation (all +1 for seed 0)."""
+    if seed == 0:
+        return np.ones(d, dtype=np.float64)
+    return np.array([-1.0 if v >> 63 else 1.0 for v in splitmix64_outputs(seed, d)], dtype=np.float64)
+
+
+def rotate(x: np.ndarray, dtype=np.float64, seed: int = 0) -> np.ndarray:
+    """X' = X D_s H for token rows X[..., d] (the rotation of step 1; D_s = I
+    for seed 0).
+
+    Computed as (X times the signs times the +-1 matrix) / sqrt(d): for fp16
+    inputs the +-1 sums are exact in fp64, so a rotated channel that is zero
+    in exact arithmetic comes out exactly zero.
     """
     x = np.asarray(x).astype(dtype)
     d = x.shape[-1]
-    return (x @ sylvester_signs(d).astype(dtype)) / dtype(math.sqrt(d))
+    xs = x * rotation_signs(d, seed).astype(dtype)
+    return (xs @ sylvester_signs(d).astype(dtype)) / dtype(math.sqrt(d))
 
 
 # ---------------------------------------------------------------------------
@@ -168,7 +204,7 @@ def asymmetric_rtn(y: np.ndarray, bits: int):
 # ---------------------------------------------------------------------------
 
 def quantize_tile(x: np.ndarray, bits: int, iters: int, eps: float = EPS,
-                  dtype=np.float64, return_parts: bool = False):
+                  dtype=np.float64, return_parts: bool = False, seed: int = 0):
     """Quantize one T x d tile of raw fp16 K or V rows (steps 1-4 above).
 
     Returns a dict with ``codes`` (uint8 T x d), ``s_t`` / ``z_t`` (fp16 per
@@ -178,7 +214,7 @@ def quantize_tile(x: np.ndarray, bits: int, iters: int, eps: float = EPS,
     x = np.asarray(x)
     if x.ndim != 2:
         raise ValueError("a tile is T x d")
-    xr = rotate(x.astype(np.float16).astype(dtype), dtype)
+    xr = rotate(x.astype(np.float16).astype(dtype), dtype, seed)
     y, c, r = sinkhorn_normalize(xr, iters, eps)
     codes, s, z = asymmetric_rtn(y, bits)
     out = {
@@ -192,17 +228,18 @@ def quantize_tile(x: np.ndarray, bits: int, iters: int, eps: float = EPS,
     return out
 
 
-def dequantize_tile(codes, s_t, z_t, c_t):
+def dequantize_tile(codes, s_t, z_t, c_t, seed: int = 0):
     """Inverse of ``quantize_tile`` in fp64.
 
-    Returns (rotated-domain tile X^', original-domain tile X^ = X^' H).
+    Returns (rotated-domain tile X^', original-domain tile X^ = X^' H D_s).
     """
     codes = np.asarray(codes, dtype=np.float64)
     s = np.asarray(s_t, dtype=np.float64)
     z = np.asarray(z_t, dtype=np.float64)
     c = np.asarray(c_t, dtype=np.float64)
     xr_hat = (codes * s[:, None] + z[:, None]) * c[None, :]
-    return xr_hat, xr_hat @ sylvester_hadamard(codes.shape[1])
+    d = codes.shape[1]
+    return xr_hat, (xr_hat @ sylvester_hadamard(d)) * rotation_signs(d, seed)[None, :]
 
 
 def plain_rtn_baseline(x: np.ndarray, bits: int) -> np.ndarray:
@@ -359,11 +396,11 @@ def attention_fp64(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float | N
     return (w[:, None] * v).sum(axis=0) / w.sum()
 
 
-def sequence_kv_hat(tiles, tail_rows: np.ndarray) -> np.ndarray:
+def sequence_kv_hat(tiles, tail_rows: np.ndarray, seed: int = 0) -> np.ndarray:
     """Original-domain K^ (or V^) of one (sequence, KV head): the
     dequantized full tiles in order, then the raw fp16 rows of the unfinished
     tile.  ``tiles`` is a list of ``quantize_tile``-style dicts."""
-    parts = [dequantize_tile(t["codes"], t["s_t"], t["z_t"], t["c_t"])[1] for t in tiles]
+    parts = [dequantize_tile(t["codes"], t["s_t"], t["z_t"], t["c_t"], seed)[1] for t in tiles]
     parts.append(np.asarray(tail_rows, dtype=np.float16).astype(np.float64).reshape(-1, HEAD_DIM))
     return np.concatenate(parts, axis=0)
 
@@ -379,10 +416,10 @@ def decode_sequence(q_heads: np.ndarray, k_hat: list, v_hat: list, group: int,
 
 
 def quantize_sequence(rows: np.ndarray, tile_tokens: int, bits: int, iters: int,
-                      dtype=np.float64):
+                      dtype=np.float64, seed: int = 0):
     """Quantize every full tile of one (sequence, KV head): rows [L][d] fp16.
     Returns (list of tile dicts, raw tail rows)."""
     n_full = rows.shape[0] // tile_tokens
-    tiles = [quantize_tile(rows[t * tile_tokens:(t + 1) * tile_tokens], bits, iters, dtype=dtype)
+    tiles = [quantize_tile(rows[t * tile_tokens:(t + 1) * tile_tokens], bits, iters, dtype=dtype, seed=seed)
              for t in range(n_full)]
     return tiles, rows[n_full * tile_tokens:]

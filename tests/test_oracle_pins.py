@@ -388,3 +388,70 @@ def test_decode_gqa_mapping_and_tail():
         # KV head 1's values sit near 4, KV head 0's near 0
         assert abs(out[h].mean() - 4.0 * (h // g)) < 0.6
         np.testing.assert_array_equal(out[h], o.attention_fp64(qh[h], k_hat[h // g], v_hat[h // g]))
+
+
+# --------------------------------------------------------------------------- randomized rotation (variant)
+
+def test_splitmix64_matches_published_first_output():
+    # a wrong constant, shift or update order in the generator changes it
+    lines = [ln for ln in open(os.path.join(GOLDEN, "splitmix64_seed0.txt")) if not ln.startswith("#")]
+    want = int(lines[0].strip(), 16)
+    assert o.splitmix64_outputs(0, 1)[0] == want
+
+
+def test_rotation_signs_seed0_plain_and_seeded_balanced():
+    np.testing.assert_array_equal(o.rotation_signs(128, 0), np.ones(128))
+    for seed in (1, 12345, 0xDEADBEEF):
+        s = o.rotation_signs(128, seed)
+        assert set(np.unique(s)) == {-1.0, 1.0}
+        assert 0.3 < np.mean(s < 0) < 0.7  # a stuck sign bit would give 0 or 1
+    assert not np.array_equal(o.rotation_signs(128, 1), o.rotation_signs(128, 2))
+
+
+def test_randomized_rotation_is_orthogonal_and_inverted():
+    # X' = X D_s H keeps inner products between rows (Gram matrix), and the
+    # dequantization's inverse X' H D_s recovers X: a sign applied on the
+    # wrong side (H D_s instead of D_s H) breaks the inversion
+    rng = np.random.default_rng(21)
+    x = rng.standard_normal((16, 128))
+    seed = 777
+    xr = o.rotate(x, seed=seed)
+    np.testing.assert_allclose(xr @ xr.T, x @ x.T, rtol=1e-12, atol=1e-10)
+    back = (xr @ o.sylvester_hadamard(128)) * o.rotation_signs(128, seed)[None, :]
+    np.testing.assert_allclose(back, x, atol=1e-12)
+    wrong = (xr * o.rotation_signs(128, seed)[None, :]) @ o.sylvester_hadamard(128)
+    assert not np.allclose(wrong, x, atol=1e-3)
+    # a unit row e_k maps to s_k times row k of H
+    h = o.sylvester_hadamard(128)
+    s = o.rotation_signs(128, seed)
+    for k in (0, 5, 127):
+        e = np.zeros((1, 128))
+        e[0, k] = 1.0
+        np.testing.assert_allclose(o.rotate(e, seed=seed)[0], s[k] * h[k], atol=0)
+
+
+def test_randomized_rotation_dequantizes_and_decodes():
+    # dequantized tile within one step per element; decode over the seeded
+    # quantization equals brute-force attention on its original-domain rows
+    rng = np.random.default_rng(22)
+    seed, t = 4242, 32
+    x = outlier_tile(rng, t)
+    q = o.quantize_tile(x, 4, 4, return_parts=True, seed=seed)
+    xr_hat, x_hat = o.dequantize_tile(q["codes"], q["s_t"], q["z_t"], q["c_t"], seed)
+    step = (q["s"] * q["r"])[:, None] * q["c"][None, :]
+    fp16_slack = 2.0 ** -10 * (np.abs(q["xr"]) + step * 15)
+    assert np.all(np.abs(xr_hat - q["xr"]) <= step / 2 + 3 * fp16_slack)
+    err = np.linalg.norm(x_hat - x.astype(np.float64)) / np.linalg.norm(x.astype(np.float64))
+    assert err < 0.15
+    rows_k = rng.standard_normal((t + 5, 128)).astype(np.float16)
+    rows_v = rng.standard_normal((t + 5, 128)).astype(np.float16)
+    tk, tail_k = o.quantize_sequence(rows_k, t, 4, 2, seed=seed)
+    tv, tail_v = o.quantize_sequence(rows_v, t, 4, 2, seed=seed)
+    k_hat, v_hat = o.sequence_kv_hat(tk, tail_k, seed), o.sequence_kv_hat(tv, tail_v, seed)
+    qv = rng.standard_normal(128)
+    want = brute_attention(qv.tolist(), k_hat.tolist(), v_hat.tolist(), 1 / math.sqrt(128))
+    np.testing.assert_allclose(o.decode_sequence(qv[None], [k_hat], [v_hat], 1)[0], want, rtol=1e-11, atol=1e-13)
+    # the keys really are the seeded reconstruction: closer to the raw rows
+    # than the unseeded decoder's reading of the same codes
+    k_plain = o.sequence_kv_hat(tk, tail_k, 0)
+    assert np.linalg.norm(k_hat - rows_k) < 0.5 * np.linalg.norm(k_plain - rows_k)
