@@ -31,6 +31,14 @@
  *     (all codes 0 when s_i == 0).
  *     Stored: s~_i = fp16(s_i R_i), z~_i = fp16(z_i R_i), C~_j = fp16(C_j).
  *   Dequantization: X^'_ij = (code_ij s~_i + z~_i) C~_j and X^ = X^' H.
+ *   Randomized rotation (a variant, not on the pages): with rotation_seed
+ *   != 0 every H above becomes D_s H on the way in (Y = X D_s H, q' = H D_s q)
+ *   and H D_s on the way out (X^ = X^' H D_s, out = D_s H acc'), D_s =
+ *   diag(s) with s_j = -1 where the j-th output (j = 0..d-1) of SplitMix64
+ *   started at state rotation_seed has its top bit set, else +1.  SplitMix64
+ *   (Steele, Lea and Flood, OOPSLA 2014): state += 0x9E3779B97F4A7C15;
+ *   z = state; z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9;
+ *   z = (z ^ (z >> 27)) * 0x94D049BB133111EB; output z ^ (z >> 31).
  *   A sequence of L tokens holds floor(L/T) quantized tiles, tile t covering
  *   tokens [tT, (t+1)T); the last L mod T tokens stay raw fp16 in a tail
  *   buffer until their tile fills.
@@ -116,6 +124,8 @@ typedef struct {
   int bits_v;        /* b for V codes: 2, 3 or 4                         */
   int iters;         /* n: normalization iterations, 0..64               */
   float std_eps;     /* std clamp, > 0 (1e-6 in the method)              */
+  uint32_t rotation_seed; /* 0: the rotation H; else the randomized       */
+                          /* rotation D_s H (see Definitions)             */
 } kvq_config;
 
 typedef struct {

@@ -299,6 +299,10 @@ __global__ void __launch_bounds__(kDecWarps * 32, T == 128 ? 2 : 3) decode_tiles
 #pragma unroll
       for (int i = 0; i < 32; ++i) qs[i] = 0.f;
     }
+    if (a.cfg.rotation_seed != 0) {  // q' = H D_s q
+#pragma unroll
+      for (int i = 0; i < 32; ++i) qs[i] *= rotation_sign(a.cfg.rotation_seed, 32 * t + i);
+    }
 #pragma unroll
     for (int bit = 0; bit < 5; ++bit) {  // channel bits 0..4: in-register butterflies
       const int m = 1 << bit;
@@ -684,7 +688,8 @@ __global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(DecodeArgs 
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const int c = 4 * lane + k;
-        out[hh * kHeadDim + c] = __float2half_rn((v[k] / kSqrtHeadDim + sm.et[hh] * sm.tl[hh][c]) * sm.inv_l[hh]);
+        out[hh * kHeadDim + c] = __float2half_rn(
+            (v[k] / kSqrtHeadDim * rotation_sign(a.cfg.rotation_seed, c) + sm.et[hh] * sm.tl[hh][c]) * sm.inv_l[hh]);
       }
     }
     __syncthreads();

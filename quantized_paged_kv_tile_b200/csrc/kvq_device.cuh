@@ -81,6 +81,18 @@ __device__ __forceinline__ void fwht128_warp(float v[4], int lane) {
   }
 }
 
+// Sign s_j of channel j in the randomized rotation D_s H: -1 where the j-th
+// output of SplitMix64 (Steele, Lea and Flood, OOPSLA 2014) started at state
+// `seed` has its top bit set, else +1; seed 0 (the plain rotation): +1.
+__device__ __forceinline__ float rotation_sign(uint32_t seed, int j) {
+  if (seed == 0) return 1.f;
+  uint64_t z = static_cast<uint64_t>(seed) + static_cast<uint64_t>(j + 1) * 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  z ^= z >> 31;
+  return (z >> 63) ? -1.f : 1.f;
+}
+
 constexpr float kSqrtHeadDim = 11.313708498984761f;  // sqrt(128) rounded to fp32
 constexpr float kLog2e = 1.4426950408889634f;
 

@@ -580,11 +580,14 @@ __device__ __forceinline__ void quantize_group_dispatch(unsigned char* smem, uin
                                            num_heads, head);
 }
 
-__device__ void build_h(unsigned char* smem) {
+// The +-1 matrix M[r][k] = s_k (-1)^popcount(r & k) in the operand layout.
+// It is B of D1 = X M^T = X D_s H and A of D2 = M X^T = H D_s X^T (H is
+// symmetric), so one copy serves both layouts; s = 1 for the plain rotation.
+__device__ void build_h(unsigned char* smem, uint32_t seed) {
   for (int idx = threadIdx.x; idx < kRows * kHeadDim; idx += blockDim.x) {
     const int r = idx >> 7, k = idx & 127;
-    const __half v = __float2half_rn((__popc(r & k) & 1) ? -1.f : 1.f);
-    *reinterpret_cast<__half*>(smem + kOffH + sw128_off(r, k)) = v;
+    const float h = (__popc(r & k) & 1) ? -1.f : 1.f;
+    *reinterpret_cast<__half*>(smem + kOffH + sw128_off(r, k)) = __float2half_rn(h * rotation_sign(seed, k));
   }
 }
 
@@ -713,7 +716,7 @@ __global__ void __launch_bounds__(kQThreads, 2) quantize_tc_kernel(const __grid_
   const uint32_t tma_bar = smem_u32(smem + kOffBar), full_bar = tma_bar + 8, empty_bar = tma_bar + 16;
   const uint32_t meta_bar0 = tma_bar + 24;
 
-  build_h(smem);
+  build_h(smem, a.cfg.rotation_seed);
   if (tid == 0) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tma_bar));
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(full_bar));
@@ -835,7 +838,7 @@ __global__ void __launch_bounds__(kMathThreads, 2) append_tc_kernel(AppendArgs a
   int* flag = reinterpret_cast<int*>(smem + kOffTmem + 4);
 
   if (l0 / T < end / T) {  // at least one tile completes: tensor-core set-up
-    build_h(smem);
+    build_h(smem, a.cfg.rotation_seed);
     for (int i = tid; i < kRows * kHeadDim / 8; i += kMathThreads) {  // rows of the unused tiles: zeros
       const int r = i / 16, c = i % 16;
       if (r >= T) *reinterpret_cast<uint4*>(smem + kOffX + sw128_off(r, c * 8)) = make_uint4(0, 0, 0, 0);

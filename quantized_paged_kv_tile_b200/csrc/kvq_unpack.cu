@@ -68,7 +68,9 @@ __global__ void __launch_bounds__(kThreads) unpack_tiles_kernel(UnpackArgs a) {
     if (a.out_orig) {
       fwht128_warp(v, lane);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) a.out_orig[(th * T + i) * kHeadDim + 4 * lane + k] = v[k] / kSqrtHeadDim;
+      for (int k = 0; k < 4; ++k)  // X^ = X^' H D_s
+        a.out_orig[(th * T + i) * kHeadDim + 4 * lane + k] =
+            v[k] / kSqrtHeadDim * rotation_sign(a.cfg.rotation_seed, 4 * lane + k);
     }
   }
 }

@@ -42,7 +42,8 @@ class KvqError(RuntimeError):
 class _Config(ctypes.Structure):
     _fields_ = [("head_dim", ctypes.c_int), ("num_kv_heads", ctypes.c_int), ("group_size", ctypes.c_int),
                 ("tile_tokens", ctypes.c_int), ("page_tokens", ctypes.c_int), ("bits_k", ctypes.c_int),
-                ("bits_v", ctypes.c_int), ("iters", ctypes.c_int), ("std_eps", ctypes.c_float)]
+                ("bits_v", ctypes.c_int), ("iters", ctypes.c_int), ("std_eps", ctypes.c_float),
+                ("rotation_seed", ctypes.c_uint32)]
 
 
 class _Layout(ctypes.Structure):
@@ -66,10 +67,12 @@ class Config:
     head_dim: int = 128
     page_tokens: int = 16
     std_eps: float = 1e-6
+    rotation_seed: int = 0  # 0: the Hadamard rotation; else the randomized rotation D_s H
 
     def c(self) -> _Config:
         return _Config(self.head_dim, self.num_kv_heads, self.group_size, self.tile_tokens,
-                       self.page_tokens, self.bits_k, self.bits_v, self.iters, self.std_eps)
+                       self.page_tokens, self.bits_k, self.bits_v, self.iters, self.std_eps,
+                       self.rotation_seed & 0xFFFFFFFF)
 
     @property
     def num_q_heads(self) -> int:
