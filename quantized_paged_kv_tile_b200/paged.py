@@ -120,3 +120,60 @@ class PagedKVCache:
         """Stored bytes per (token, KV head) for K+V, pages only."""
         p = self.cfg.page_tokens
         return (self.layout["page_bytes_k"] + self.layout["page_bytes_v"]) / p
+
+
+class DecodeStepGraph:
+    """One serving step of a ``PagedKVCache`` -- append one token per sequence,
+    then decode -- captured once in a CUDA graph and replayed.
+
+    Stage the step's rows in ``new_k`` / ``new_v`` ([B][H_kv][d] fp16) and its
+    queries in ``q`` ([B][H_q][d] fp16), call ``replay()``, read ``out``.  The
+    sequence lengths advance on the device inside the graph (the append reads
+    them as the lengths before the step, then they grow by one); the host only
+    tracks them to refuse a step past the allocated pages.  The first decode
+    and append calls happen eagerly before capture.
+    """
+
+    def __init__(self, cache: PagedKVCache, num_splits: int | None = None):
+        self.cache = cache
+        cfg, b, dev = cache.cfg, cache.num_seqs, cache.device
+        self.num_splits = cache.num_splits if num_splits is None else num_splits
+        self.new_k = torch.zeros((b, cfg.num_kv_heads, cfg.head_dim), dtype=torch.float16, device=dev)
+        self.new_v = torch.zeros_like(self.new_k)
+        self.q = torch.zeros((b, cfg.num_q_heads, cfg.head_dim), dtype=torch.float16, device=dev)
+        self.out = torch.empty_like(self.q)
+        self._cu = torch.arange(b + 1, dtype=torch.int32, device=dev)
+        need = kvq.decode_workspace_bytes(cfg, b, self.num_splits)
+        if cache.workspace.numel() < need:
+            cache.workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        self.graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            # the decode once eagerly on the current contents (no state change)
+            self._decode()
+        torch.cuda.current_stream(dev).wait_stream(side)
+        torch.cuda.synchronize(dev)
+        with torch.cuda.graph(self.graph):
+            self._step()
+
+    def _decode(self) -> None:
+        c = self.cache
+        kvq.paged_decode_attention(c.cfg, self.q, self.out, c.seq_lens, c.block_tables, c.k_pool, c.v_pool,
+                                   c.k_tail, c.v_tail, c.workspace, num_splits=self.num_splits,
+                                   num_blocks=c.num_blocks, dev_status=c.dev_status)
+
+    def _step(self) -> None:
+        c = self.cache
+        kvq.append_tokens(c.cfg, self.new_k, self.new_v, self._cu, c.seq_lens, 1, c.block_tables, c.k_pool,
+                          c.v_pool, c.k_tail, c.v_tail, num_blocks=c.num_blocks, dev_status=c.dev_status)
+        c.seq_lens.add_(1)
+        self._decode()
+
+    def replay(self) -> torch.Tensor:
+        c = self.cache
+        if np.any(c.host_lens + 1 > c.blocks_per_seq * c.cfg.page_tokens):
+            raise ValueError("append past the allocated pages")
+        self.graph.replay()
+        c.host_lens = c.host_lens + 1
+        return self.out

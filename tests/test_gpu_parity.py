@@ -185,6 +185,27 @@ def test_decode_matches_oracle(over):
             assert err <= ATTN_REL_L2_MAX, (s, hq, err)
 
 
+DECODE_SWEEP = [(t, bk, bv, g) for t in (32, 64, 128) for bk in (2, 4) for bv in (2, 4) for g in (2, 8)]
+
+
+@pytest.mark.parametrize("t,bk,bv,g", DECODE_SWEEP)
+def test_decode_sweep_every_instantiation(t, bk, bv, g):
+    # every decode template (T, b_K, b_V) with a small and the largest group;
+    # 3 full tiles plus a ragged tail, split over 2 chunks
+    L = 3 * t + 7
+    w = synth.workload("tiny", num_seqs=1, lens=(L,), num_kv_heads=1, group_size=g, tile_tokens=t, bits_k=bk,
+                       bits_v=bv, iters=1)
+    cfg, cache, rk, rv = _prefilled(w, num_splits=2)
+    q = synth.queries(w, device="cuda")
+    out = cache.decode(q)
+    torch.cuda.synchronize()
+    assert cache.status() == 0
+    ref = oracle_decode_sequence(cfg, rk.cpu().numpy(), rv.cpu().numpy(), q.cpu().numpy()[0])
+    out_h = out.float().cpu().numpy()[0]
+    for hq in range(g):
+        assert rel_l2(out_h[hq], ref[hq]) <= ATTN_REL_L2_MAX, hq
+
+
 def test_decode_only_on_oracle_packed_pages():
     # isolate the read path: seeded random codes / metadata packed by the oracle
     rng = np.random.default_rng(99)
