@@ -404,7 +404,45 @@ def run_kvq(args, ranks):
                      "traffic": ncu_traffic("quantize_tc_kernel", bm["quant_units"])},
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps, "clocks": clk,
     }
+    if args.serving_steps > 0:
+        line["serving"] = serving_loop(w, cfg, rows_k, rows_v, args.serving_steps, dev)
     return line
+
+
+def serving_loop(w, cfg, rows_k, rows_v, steps, dev):
+    """The serving loop of the workload after its prefill: ``steps`` graph-
+    replayed steps of one appended token per sequence plus a decode, each
+    timed with CUDA events; tile-completion steps reported apart."""
+    import torch
+    from quantized_paged_kv_tile_b200 import synth
+    from quantized_paged_kv_tile_b200.paged import DecodeStepGraph, PagedKVCache
+    lens0 = np.asarray(w.lens, dtype=np.int64)
+    bps = int(math.ceil((lens0.max() + steps) / 16))
+    cache = PagedKVCache(cfg, w.num_seqs, bps * 16, device=dev, block_table=synth.block_table(w, bps))
+    cache.prefill(rows_k, rows_v, lens0)
+    graph = DecodeStepGraph(cache)
+    ms, done = [], []
+    for i in range(steps):
+        graph.new_k.copy_(synth.kv_rows(w, "k", w.num_seqs, device=dev, stream_id=1 + i))
+        graph.new_v.copy_(synth.kv_rows(w, "v", w.num_seqs, device=dev, stream_id=1 + i))
+        graph.q.copy_(synth.queries(w, device=dev, step=i))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        graph.replay()
+        e1.record()
+        ms.append((e0, e1))
+        done.append(bool(np.any((lens0 + i + 1) % w.tile_tokens == 0)))
+    torch.cuda.synchronize(dev)
+    if cache.status() != 0:
+        raise RuntimeError(f"device status {cache.status()} in the serving loop")
+    t = np.array([a.elapsed_time(b) for a, b in ms])
+    comp = t[np.array(done)]
+    plain = t[~np.array(done)]
+    return {"steps": steps, "graph": True, "mean_ms": float(t.mean()), "p50_ms": float(np.percentile(t, 50)),
+            "p99_ms": float(np.percentile(t, 99)), "completion_steps": int(comp.size),
+            "completion_step_ms": float(comp.mean()) if comp.size else None,
+            "other_step_ms": float(plain.mean()) if plain.size else None,
+            "decode_tok_per_s": w.num_seqs / (float(t.mean()) * 1e-3)}
 
 
 # --------------------------------------------------------------------------- reference arm
@@ -450,6 +488,8 @@ def main():
                     help="override the workload's sequence count (smaller inputs for profiler captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--serving-steps", type=int, default=0,
+                    help="after the measurement, time this many graph-replayed append+decode serving steps")
     args = ap.parse_args()
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
