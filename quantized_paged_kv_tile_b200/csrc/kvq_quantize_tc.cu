@@ -381,15 +381,23 @@ __device__ void quantize_group_from_tmem(unsigned char* smem, uint32_t tbase, in
     }
     // ---- (C, R) -> (C / 2^k, R 2^k) per tile, max C in [1, 2): every thread
     // rescales what it owns; cc and rr are read again only after the barrier
+    // (the exponent of the token's tile is reused when that tile is one of
+    // the channel tiles just handled: warp-uniform, T = 128 always)
+    int e_my = 0;
+    bool have_my = false;
 #pragma unroll
     for (int lt = 0; lt < kLocal; ++lt) {
       const int t = ch_tile(lt);
       const int e = tile_exp(t);
+      if (t == my_tile) {
+        e_my = e;
+        have_my = true;
+      }
       Cj[lt] = scale_pow2(Cj[lt], 1 - e);
       if (T < 128 || hf == 0) cc_next[t * kRows + row] = fminf(scale_pow2(cc[t * kRows + row], e - 1), FLT_MAX);
     }
     {
-      const int e = tile_exp(my_tile);
+      const int e = have_my ? e_my : tile_exp(my_tile);
       Ri = scale_pow2(Ri, e - 1);
       if (tok_live && hf == 0) rr[row] = fminf(scale_pow2(r_new, 1 - e), FLT_MAX);
     }
@@ -520,13 +528,16 @@ __device__ void quantize_group_from_tmem(unsigned char* smem, uint32_t tbase, in
       // word (lane L = 4*g8 + t, k = 2m + u) = low half from the even token of
       // the pair {2t + 8u, 2t + 8u + 1}, high half from the odd token
       const int t4 = (p & 7) >> 1, u = p >> 3, odd = p & 1;
+      // low halves of (mine, other) in token order: bytes 0,1 of the even
+      // token's value, then bytes 0,1 of the odd token's
+      const uint32_t order = odd ? 0x1054u : 0x5410u;
 #pragma unroll
       for (int idx = 0; idx < 8 * nm; ++idx) {
-        const uint32_t mine = (hw[idx] - k0) & 0xFFFFu;
+        const uint32_t mine = hw[idx] - k0;  // its low 16 bits hold the fields
         const uint32_t other = __shfl_xor_sync(kFull, mine, 1);
         const int g8 = idx / nm, m = hf * nm + idx % nm;
         if ((g8 & 1) == odd) {  // the pair's two tokens split the words
-          const uint32_t word = odd ? (other | (mine << 16)) : (mine | (other << 16));
+          const uint32_t word = __byte_perm(mine, other, order);
           const int L = 4 * g8 + t4, kk = 2 * m + u;
           *reinterpret_cast<uint32_t*>(page + ((kk >> 2) * 32 + L) * 16 + (kk & 3) * 4) = word;
         }
