@@ -225,8 +225,9 @@ struct Moments {
   float mean, m2;
 };
 __device__ __forceinline__ Moments moments(const float2 (&s1)[4], const float2 (&s2)[4], float shift, float n) {
-  const float a = ((s1[0].x + s1[0].y) + (s1[1].x + s1[1].y)) + ((s1[2].x + s1[2].y) + (s1[3].x + s1[3].y));
-  const float q = ((s2[0].x + s2[0].y) + (s2[1].x + s2[1].y)) + ((s2[2].x + s2[2].y) + (s2[3].x + s2[3].y));
+  const float2 a2 = __fadd2_rn(__fadd2_rn(s1[0], s1[1]), __fadd2_rn(s1[2], s1[3]));
+  const float2 q2 = __fadd2_rn(__fadd2_rn(s2[0], s2[1]), __fadd2_rn(s2[2], s2[3]));
+  const float a = a2.x + a2.y, q = q2.x + q2.y;
   Moments m;
   m.mean = shift + a / n;
   m.m2 = fmaxf(q - a * (a / n), 0.f);
@@ -344,7 +345,8 @@ __device__ void quantize_group_from_tmem(unsigned char* smem, uint32_t tbase, in
     }
 #pragma unroll
     for (int lt = 0; lt < kLocal; ++lt) {
-      const float m = warp_max(Cj[lt]);
+      // C_j > 0: the float order is the order of the bit patterns
+      const float m = __uint_as_float(__reduce_max_sync(kFull, __float_as_uint(Cj[lt])));
       if (lane == 0) red[warp * 4 + ch_tile(lt)] = m;
     }
     math_sync();

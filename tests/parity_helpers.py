@@ -141,3 +141,26 @@ def oracle_decode_sequence(cfg: kvq.Config, rows_k: np.ndarray, rows_v: np.ndarr
         k_hat.append(o.sequence_kv_hat(tk, tail_k))
         v_hat.append(o.sequence_kv_hat(tv, tail_v))
     return o.decode_sequence(q.astype(np.float64), k_hat, v_hat, cfg.group_size, scale)
+
+
+def gpu_pages_kv_hat(cfg: kvq.Config, cache, seq: int, head: int, length: int, is_v: bool) -> np.ndarray:
+    """Original-domain K^ (or V^) of (seq, head) over the first ``length``
+    tokens as the GPU stored them: its pages read back by the oracle's own
+    page reader, then the raw tail."""
+    t, p = cfg.tile_tokens, cfg.page_tokens
+    n_full, tau = length // t, length % t
+    bits = cfg.bits_v if is_v else cfg.bits_k
+    pool = cache.v_pool if is_v else cache.k_pool
+    ids = cache.block_tables[seq, :n_full * (t // p)].long()
+    host = pool.index_select(0, ids)[:, head:head + 1].cpu().numpy()
+    tiles = [o.read_tile_pages(host, range(i * (t // p), (i + 1) * (t // p)), 0, bits, t, is_v) for i in range(n_full)]
+    tail = (cache.v_tail if is_v else cache.k_tail)[seq, head, :tau].cpu().numpy()
+    return o.sequence_kv_hat(tiles, tail, cfg.rotation_seed)
+
+
+def decode_over_gpu_pages(cfg: kvq.Config, cache, seq: int, length: int, q_heads: np.ndarray) -> np.ndarray:
+    """fp64 attention of every query head of ``seq`` over the GPU's own pages
+    (isolates the read path from the write path)."""
+    k_hat = [gpu_pages_kv_hat(cfg, cache, seq, h, length, False) for h in range(cfg.num_kv_heads)]
+    v_hat = [gpu_pages_kv_hat(cfg, cache, seq, h, length, True) for h in range(cfg.num_kv_heads)]
+    return o.decode_sequence(np.asarray(q_heads, dtype=np.float64), k_hat, v_hat, cfg.group_size)
