@@ -283,7 +283,7 @@ def code_bit_position(channel: int, token: int, bits: int, is_v: bool,
     K (and V at 3 bits): a plain little-endian bitstream, token-major:
     field index token * d + channel.
 
-    V at 2 or 4 bits: grouped for the decode kernel's register layout.
+    V at 2, 4 or 8 bits: grouped for the decode kernel's register layout.
     n = channel // 8 and g = channel % 8; t = (token % 8) // 2,
     u = token // 8 and s = token % 2.  The page's 32 "lanes" are
     L = 4 g + t.  Each lane owns 2*bits little-endian 32-bit words holding
@@ -295,8 +295,8 @@ def code_bit_position(channel: int, token: int, bits: int, is_v: bool,
     """
     if not is_v or bits == 3:
         return (token * d + channel) * bits
-    if d != 128 or bits not in (2, 4):
-        raise ValueError("grouped V layout is defined for d=128, b in {2,4}")
+    if d != 128 or bits not in (2, 4, 8):
+        raise ValueError("grouped V layout is defined for d=128, b in {2,4,8}")
     n, g = divmod(channel, 8)
     t = (token % 8) // 2
     u = token // 8

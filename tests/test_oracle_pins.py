@@ -194,7 +194,7 @@ def test_token_permutation_equivariance():
 
 # --------------------------------------------------------------------------- RTN
 
-@pytest.mark.parametrize("bits", [2, 3, 4])
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
 def test_rtn_brute_force_and_bounds(bits):
     # brute force: each code is the nearest grid point c*s + z (fp64, no ties);
     # min row entry -> 0, max -> 2^b - 1, error <= s/2, codes in range.
@@ -237,7 +237,7 @@ def test_constant_row_gives_zero_scale():
 
 # --------------------------------------------------------------------------- tile quantizer
 
-@pytest.mark.parametrize("t,bits,iters", [(32, 2, 1), (64, 4, 4), (128, 3, 8), (64, 2, 0)])
+@pytest.mark.parametrize("t,bits,iters", [(32, 2, 1), (64, 4, 4), (128, 3, 8), (64, 2, 0), (64, 8, 4)])
 def test_dequantized_tile_within_half_step(t, bits, iters):
     # X^' - X' is bounded by (s/2) R_i C_j plus the fp16 rounding of the
     # metadata; a missing R or C factor in s~, z~ or C~ breaks it by orders of magnitude.
@@ -251,7 +251,7 @@ def test_dequantized_tile_within_half_step(t, bits, iters):
     # original domain: the inverse rotation is exact up to rounding
     np.testing.assert_allclose(x_hat, xr_hat @ o.sylvester_hadamard(128), rtol=0, atol=1e-12)
     err = np.linalg.norm(x_hat - x.astype(np.float64)) / np.linalg.norm(x.astype(np.float64))
-    assert err < {2: 0.7, 3: 0.3, 4: 0.15}[bits]
+    assert err < {2: 0.7, 3: 0.3, 4: 0.15, 8: 0.02}[bits]
 
 
 @pytest.mark.parametrize("t,bits,iters", [(t, b, n) for t in (32, 64, 128) for b in (2, 3, 4) for n in (1, 4, 8)])
@@ -285,7 +285,8 @@ def test_float32_mode_agrees_with_fp64():
 
 # --------------------------------------------------------------------------- format
 
-@pytest.mark.parametrize("bits,is_v", [(2, False), (3, False), (4, False), (2, True), (3, True), (4, True)])
+@pytest.mark.parametrize("bits,is_v", [(2, False), (3, False), (4, False), (8, False), (2, True), (3, True),
+                                       (4, True), (8, True)])
 def test_code_positions_are_a_bijection(bits, is_v):
     pos = sorted(o.code_bit_position(c, p, bits, is_v) for p in range(16) for c in range(128))
     assert pos == list(range(0, 16 * 128 * bits, bits))
@@ -298,6 +299,8 @@ def test_layout_sizes_hand_computed():
     assert o.page_layout(2, 128)["page_bytes"] == 608
     assert o.page_layout(3, 32)["page_bytes"] == 960
     assert o.page_layout(4, 64)["cslice_channels"] == 32
+    # b=8, T=64: 2048 + 64 + 32*2 = 2176
+    assert o.page_layout(8, 64)["page_bytes"] == 2176
 
 
 def test_code_positions_golden():
@@ -316,7 +319,7 @@ def test_code_positions_golden():
     assert n >= 8
 
 
-@pytest.mark.parametrize("bits,is_v", [(2, True), (4, True), (3, False), (4, False)])
+@pytest.mark.parametrize("bits,is_v", [(2, True), (4, True), (8, True), (3, False), (4, False), (8, False)])
 def test_pack_unpack_roundtrip(bits, is_v):
     rng = np.random.default_rng(bits + 10 * is_v)
     codes = rng.integers(0, 1 << bits, size=(16, 128)).astype(np.uint8)
