@@ -18,7 +18,8 @@
  * Definitions (the pages give the outline only; these are the concrete
  * readings the library implements):
  *   d = head_dim = 128, P = page_tokens = 16, T = tile_tokens in {32,64,128},
- *   b = bits in {2,3,4}, n = iters >= 0, eps = std_eps (1e-6).
+ *   b = bits in {2,3,4,8} (8 for K and V together), n = iters >= 0,
+ *   eps = std_eps (1e-6).
  *   H = orthonormal Sylvester Hadamard, H[j][k] = (-1)^popcount(j&k)/sqrt(d).
  *   For one tile X (T x d fp16, one sequence, one KV head, K or V):
  *     Y = X H;  C = 1_d;  R = 1_T;  repeat n times:
@@ -54,7 +55,7 @@
  *     uint8 pool[num_blocks][num_kv_heads][page_bytes]
  *   One page region (block, head) holds P tokens of one KV head:
  *     [codes | meta | C slice], each region starting on a 16-byte boundary.
- *   codes: P*d*b/8 bytes (1024 at b=4, 768 at b=3, 512 at b=2), a little-
+ *   codes: P*d*b/8 bytes (2048 at b=8, 1024 at b=4, 768 at b=3, 512 at b=2), a little-
  *     endian bitstream; a code occupies b bits at the bit offset below.
  *   meta:  P entries of {fp16 s~, fp16 z~} (64 bytes), token-major.
  *   C slice: page k of its tile (k = logical block index mod T/P) carries
@@ -62,7 +63,7 @@
  *   page_bytes = codes + 64 + 2*d*P/T  (1152 for T=64, b=4).
  *   Bit offset of the code of (channel c, token p of the page):
  *     K, and V at b=3:   (p*d + c) * b                (token-major)
- *     V at b in {2,4}:   the decode kernel's grouped order.  With
+ *     V at b in {2,4,8}: the decode kernel's grouped order.  With
  *       n = c/8, g = c%8, t = (p%8)/2, u = p/8, s = p%2, F = 32/b,
  *       h = F/2, k = 2*(n/h) + u, e = n%h, lane = 4*g + t:
  *       byte of word = ((k/4)*32 + lane)*16 + (k%4)*4,
@@ -120,8 +121,8 @@ typedef struct {
   int group_size;    /* g = query heads per KV head, 1..8                */
   int tile_tokens;   /* T: 32, 64 or 128                                 */
   int page_tokens;   /* P: must be 16                                    */
-  int bits_k;        /* b for K codes: 2, 3 or 4                         */
-  int bits_v;        /* b for V codes: 2, 3 or 4                         */
+  int bits_k;        /* b for K codes: 2, 3, 4 or 8 (8 with bits_v = 8) */
+  int bits_v;        /* b for V codes: 2, 3, 4 or 8 (8 with bits_k = 8) */
   int iters;         /* n: normalization iterations, 0..64               */
   float std_eps;     /* std clamp, > 0 (1e-6 in the method)              */
   uint32_t rotation_seed; /* 0: the rotation H; else the randomized       */
@@ -196,7 +197,8 @@ KVQ_API kvq_status kvq_append_tokens(const kvq_config* cfg, const void* new_k, c
  *   num_splits   : split-K factor over tiles per (sequence, KV head); 0 picks
  *                  one from the device size.  The output does not depend on it
  *                  beyond rounding.
- * Decode supports b in {2, 4} for K and V (KVQ_ERR_UNSUPPORTED for 3). */
+ * Decode supports b in {2, 4} for K and V, and 8 for both
+ * (KVQ_ERR_UNSUPPORTED for 3). */
 KVQ_API kvq_status kvq_paged_decode_attention(const kvq_config* cfg, const void* q, void* out,
                                       const int32_t* seq_lens, int num_seqs,
                                       const int32_t* block_tables, int max_blocks_per_seq,

@@ -48,7 +48,10 @@ kvq_status check_config(const kvq_config* c) {
   if (c->group_size < 1 || c->group_size > kvq::kMaxGroup)
     return fail(KVQ_ERR_UNSUPPORTED, "group_size must be 1..8 (got %d)", c->group_size);
   for (int b : {c->bits_k, c->bits_v})
-    if (b < 2 || b > 4) return fail(KVQ_ERR_UNSUPPORTED, "bits must be 2, 3 or 4 (got %d)", b);
+    if (b != 2 && b != 3 && b != 4 && b != 8)
+      return fail(KVQ_ERR_UNSUPPORTED, "bits must be 2, 3, 4 or 8 (got %d)", b);
+  if ((c->bits_k == 8) != (c->bits_v == 8))
+    return fail(KVQ_ERR_UNSUPPORTED, "8-bit codes are for K and V together (got %d / %d)", c->bits_k, c->bits_v);
   if (c->iters < 0 || c->iters > 64) return fail(KVQ_ERR_INVALID_ARG, "iters must be 0..64 (got %d)", c->iters);
   if (!(c->std_eps > 0.f) || !(c->std_eps < 1e30f))
     return fail(KVQ_ERR_INVALID_ARG, "std_eps must be a positive finite float");
@@ -218,7 +221,7 @@ kvq_status kvq_paged_decode_attention(const kvq_config* cfg, const void* q, void
                                       size_t workspace_bytes, int num_splits, int32_t* dev_status, void* stream) {
   KVQ_TRY(check_config(cfg));
   if (cfg->bits_k == 3 || cfg->bits_v == 3)
-    return fail(KVQ_ERR_UNSUPPORTED, "decode reads 2- or 4-bit codes only (3-bit pages are storage-only)");
+    return fail(KVQ_ERR_UNSUPPORTED, "decode reads 2-, 4- or 8-bit codes only (3-bit pages are storage-only)");
   if (num_seqs < 0 || num_splits < 0) return fail(KVQ_ERR_INVALID_ARG, "negative num_seqs or num_splits");
   if (num_seqs == 0) return ok();
   if (num_seqs > 65535) return fail(KVQ_ERR_INVALID_ARG, "num_seqs > 65535");

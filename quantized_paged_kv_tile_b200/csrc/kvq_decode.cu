@@ -39,7 +39,6 @@ namespace {
 // 132 floats = 528 bytes, so every record and its acc start 16-byte aligned.
 constexpr int kPartFloats = 4 + kHeadDim;
 constexpr int kPartAcc = 4;
-constexpr int kDecWarps = 4;               // warps per decode CTA
 constexpr int kUnitsPerSm = 32;            // work-unit budget of the automatic split
 constexpr long long kWaitLimitNs = 2000000000LL;  // bounded mbarrier waits: 2 s
 
@@ -122,7 +121,11 @@ __device__ __forceinline__ __half2 u32_as_h2(uint32_t u) { return *reinterpret_c
 template <int B>
 __device__ __forceinline__ void unpack_word(uint32_t w, uint32_t out[16 / B]) {
   const uint32_t magic = 0x64006400u;
-  if constexpr (B == 4) {
+  if constexpr (B == 8) {  // pair e (0..1) = (byte e, byte e+2)
+    const __half2 k1024 = __float2half2_rn(1024.f);
+    out[0] = h2_as_u32(__hsub2(u32_as_h2(lop3_and_or(w, 0x00FF00FFu, magic)), k1024));
+    out[1] = h2_as_u32(__hsub2(u32_as_h2(lop3_and_or(w >> 8, 0x00FF00FFu, magic)), k1024));
+  } else if constexpr (B == 4) {
     const uint32_t w8 = w >> 8;
     const __half2 k1024 = __float2half2_rn(1024.f);
     const __half2 s16 = __float2half2_rn(1.f / 16.f), o64 = __float2half2_rn(-64.f);
@@ -150,13 +153,14 @@ __device__ __forceinline__ void unpack_word(uint32_t w, uint32_t out[16 / B]) {
 // Channel pair p (0..15) of lane-quad t in the K register order:
 // b = 4: word p/4, nibbles (p%4, p%4+4) -> channels 32t + 8(p/4) + p%4 + {0, 4}
 // b = 2: word p/8, fields (p%8, p%8+8) -> channels 32t + 16(p/8) + p%8 + {0, 8}
+// b = 8: word p/2, bytes (p%2, p%2+2) -> channels 32t + 4(p/2) + p%2 + {0, 2}
 template <int B>
 __device__ __forceinline__ constexpr int pair_ch0(int p) {
-  return B == 4 ? 8 * (p / 4) + (p % 4) : 16 * (p / 8) + (p % 8);
+  return B == 8 ? 4 * (p / 2) + (p % 2) : (B == 4 ? 8 * (p / 4) + (p % 4) : 16 * (p / 8) + (p % 8));
 }
 template <int B>
 __device__ __forceinline__ constexpr int pair_gap() {
-  return B == 4 ? 4 : 8;
+  return B == 8 ? 2 : (B == 4 ? 4 : 8);
 }
 
 // ------------------------------------------------------------------ schedule
@@ -229,13 +233,17 @@ struct DecodeGeom {
   static constexpr int kPageK = kCodesK + 64 + kCsBytes;
   static constexpr int kPageV = kCodesV + 64 + kCsBytes;
   static constexpr int kStage = kPages * (kPageK + kPageV);    // one tile, K pages then V pages
-  static constexpr int kSmem = kDecWarps * (2 * kStage + 16);
+  // warps per CTA: 4, fewer when two stages per warp would not fit (8-bit codes)
+  static constexpr int kWarps = 4 * (2 * kStage + 16) <= 200 * 1024 ? 4 : (2 * (2 * kStage + 16) <= 200 * 1024 ? 2 : 1);
+  static constexpr int kSmem = kWarps * (2 * kStage + 16);
 };
 
 template <int T, int BK, int BV>
-__global__ void __launch_bounds__(kDecWarps * 32, T == 128 ? 2 : 3) decode_tiles_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 1 : (T == 128 ? 2 : 3))
+    decode_tiles_kernel(DecodeArgs a) {
   using Geo = DecodeGeom<T, BK, BV>;
   constexpr int NP = Geo::kPages;
+  constexpr int kDecWarps = Geo::kWarps;
   extern __shared__ __align__(128) unsigned char smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
@@ -381,7 +389,8 @@ __global__ void __launch_bounds__(kDecWarps * 32, T == 128 ? 2 : 3) decode_tiles
       // up to 4 so that one chunk's code words and accumulators are live; the
       // chunk's scores (log2 domain, tokens 8nb + 2t, 8nb + 2t + 1 of each page)
       // are kept.
-      constexpr int kPc = NP < 4 ? NP : 4;
+      constexpr int kPcMax = BK == 8 ? 2 : 4;
+      constexpr int kPc = NP < kPcMax ? NP : kPcMax;
       float sig = 0.f;
       float sc[NP][2][2];
       float mt = -INFINITY;
@@ -408,7 +417,12 @@ __global__ void __launch_bounds__(kDecWarps * 32, T == 128 ? 2 : 3) decode_tiles
 #pragma unroll
           for (int nb = 0; nb < 2; ++nb) {
             const unsigned char* src = sK + (pc + pg) * Geo::kPageK + (8 * nb + g) * (16 * BK) + t * (4 * BK);
-            if constexpr (BK == 4) {
+            if constexpr (BK == 8) {
+              const uint4 v0 = *reinterpret_cast<const uint4*>(src);
+              const uint4 v1 = *reinterpret_cast<const uint4*>(src + 16);
+              rec[pg][nb][0] = v0.x; rec[pg][nb][1] = v0.y; rec[pg][nb][2] = v0.z; rec[pg][nb][3] = v0.w;
+              rec[pg][nb][4] = v1.x; rec[pg][nb][5] = v1.y; rec[pg][nb][6] = v1.z; rec[pg][nb][7] = v1.w;
+            } else if constexpr (BK == 4) {
               const uint4 v = *reinterpret_cast<const uint4*>(src);
               rec[pg][nb][0] = v.x; rec[pg][nb][1] = v.y; rec[pg][nb][2] = v.z; rec[pg][nb][3] = v.w;
             } else {
@@ -709,9 +723,9 @@ cudaError_t launch_tiles_t(const DecodeArgs& a, cudaStream_t s, int grid) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Geo::kSmem);
   if (e != cudaSuccess) return e;
   int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kDecWarps * 32, Geo::kSmem);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, Geo::kWarps * 32, Geo::kSmem);
   if (e != cudaSuccess) return e;
-  kern<<<grid * std::max(per_sm, 1), kDecWarps * 32, Geo::kSmem, s>>>(a);
+  kern<<<grid * std::max(per_sm, 1), Geo::kWarps * 32, Geo::kSmem, s>>>(a);
   return cudaGetLastError();
 }
 
@@ -720,6 +734,7 @@ cudaError_t launch_tiles_bits(const DecodeArgs& a, cudaStream_t s, int grid) {
   if (a.cfg.bits_k == 4 && a.cfg.bits_v == 4) return launch_tiles_t<T, 4, 4>(a, s, grid);
   if (a.cfg.bits_k == 4 && a.cfg.bits_v == 2) return launch_tiles_t<T, 4, 2>(a, s, grid);
   if (a.cfg.bits_k == 2 && a.cfg.bits_v == 4) return launch_tiles_t<T, 2, 4>(a, s, grid);
+  if (a.cfg.bits_k == 8 && a.cfg.bits_v == 8) return launch_tiles_t<T, 8, 8>(a, s, grid);
   return launch_tiles_t<T, 2, 2>(a, s, grid);
 }
 

@@ -42,7 +42,7 @@ namespace {
 constexpr int kMathThreads = 256;       // 8 math warps: warps w and w+4 share TMEM lane quadrant w, split the columns
 constexpr int kQThreads = kMathThreads + 32;  // + 1 producer warp (metadata, TMA, MMA) in the quantize kernel
 constexpr int kRows = 128;                 // token rows per MMA group
-constexpr int kMaxPageBytes = 1024 + 64 + 128;
+constexpr int kMaxPageBytes = 2048 + 64 + 128;  // 8-bit codes, T = 32
 constexpr int kStageBytes = 8 * kMaxPageBytes;  // the group's 8 pages
 constexpr long long kWaitNs = 2000000000LL;
 
@@ -1010,6 +1010,7 @@ cudaError_t dispatch_bits(const Args& a, cudaStream_t s) {
     if (bk == 2 && bv == 3) return L<TT, 2, 3>::run(a, s);                    \
     if (bk == 3 && bv == 4) return L<TT, 3, 4>::run(a, s);                    \
     if (bk == 3 && bv == 2) return L<TT, 3, 2>::run(a, s);                    \
+    if (bk == 8 && bv == 8) return L<TT, 8, 8>::run(a, s);                    \
     return L<TT, 3, 3>::run(a, s);
     KVQ_BITS(32)
     KVQ_BITS(64)

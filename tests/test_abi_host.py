@@ -51,7 +51,7 @@ def test_version_and_status_strings(lib):
 
 
 @pytest.mark.parametrize("t", [32, 64, 128])
-@pytest.mark.parametrize("bk,bv", [(4, 4), (4, 2), (3, 2), (2, 3)])
+@pytest.mark.parametrize("bk,bv", [(4, 4), (4, 2), (3, 2), (2, 3), (8, 8)])
 def test_layout_matches_oracle(lib, t, bk, bv):
     cfg = kvq.Config(num_kv_heads=8, group_size=4, tile_tokens=t, bits_k=bk, bits_v=bv, iters=4)
     lay = kvq.get_layout(cfg)
@@ -65,7 +65,8 @@ def test_layout_matches_oracle(lib, t, bk, bv):
 
 @pytest.mark.parametrize("field,value,status", [
     ("head_dim", 64, kvq.KVQ_ERR_UNSUPPORTED), ("tile_tokens", 48, kvq.KVQ_ERR_UNSUPPORTED),
-    ("bits_k", 5, kvq.KVQ_ERR_UNSUPPORTED), ("group_size", 9, kvq.KVQ_ERR_UNSUPPORTED),
+    ("bits_k", 5, kvq.KVQ_ERR_UNSUPPORTED), ("bits_k", 8, kvq.KVQ_ERR_UNSUPPORTED),  # 8 only with bits_v = 8
+    ("group_size", 9, kvq.KVQ_ERR_UNSUPPORTED),
     ("iters", -1, kvq.KVQ_ERR_INVALID_ARG), ("std_eps", 0.0, kvq.KVQ_ERR_INVALID_ARG),
     ("page_tokens", 32, kvq.KVQ_ERR_UNSUPPORTED), ("num_kv_heads", 0, kvq.KVQ_ERR_INVALID_ARG),
 ])

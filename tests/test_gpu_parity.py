@@ -50,6 +50,9 @@ QUANT_CASES = [
     (128, 4, 2, 2, 3, (384, 130)),
     (128, 3, 4, 8, 1, (256,)),
     (64, 2, 2, 0, 2, (192,)),               # n = 0: plain RTN of the rotated tile
+    (64, 8, 8, 4, 2, (300, 70)),            # 8-bit codes
+    (128, 8, 8, 2, 1, (260,)),
+    (32, 8, 8, 1, 1, (100,)),
 ]
 
 
@@ -185,7 +188,8 @@ def test_decode_matches_oracle(over):
             assert err <= ATTN_REL_L2_MAX, (s, hq, err)
 
 
-DECODE_SWEEP = [(t, bk, bv, g) for t in (32, 64, 128) for bk in (2, 4) for bv in (2, 4) for g in (2, 8)]
+DECODE_SWEEP = ([(t, bk, bv, g) for t in (32, 64, 128) for bk in (2, 4) for bv in (2, 4) for g in (2, 8)]
+                + [(t, 8, 8, g) for t in (32, 64, 128) for g in (2, 8)])
 
 
 @pytest.mark.parametrize("t,bk,bv,g", DECODE_SWEEP)
