@@ -46,6 +46,9 @@ oracle follows (and the CUDA path implements independently) are:
    (H is symmetric and its own inverse).
 5. Decode: out = softmax(q K^T / sqrt(d)) V in fp64 over the dequantized
    tiles followed by the raw fp16 rows of the unfinished last tile.
+6. Chunked prefill: each of a chunk's n query tokens attends, as in 5, to
+   the cached context followed by the chunk's own raw fp16 rows up to and
+   including itself (causal).
 
 Variant (not on the pages; a randomized rotation): with a nonzero 32-bit
 ``seed`` the rotation is X' = X D_s H, D_s = diag(s) with s_j = -1 where the
@@ -412,6 +415,36 @@ def decode_sequence(q_heads: np.ndarray, k_hat: list, v_hat: list, group: int,
     out = np.zeros(q_heads.shape, dtype=np.float64)
     for h in range(q_heads.shape[0]):
         out[h] = attention_fp64(q_heads[h], k_hat[h // group], v_hat[h // group], scale)
+    return out
+
+
+def prefill_chunk_sequence(q_chunk: np.ndarray, k_hat: list, v_hat: list, k_new: np.ndarray,
+                           v_new: np.ndarray, group: int, scale: float | None = None) -> np.ndarray:
+    """Chunked prefill of one sequence over its cache  [AIT, TL;DR].
+
+    The attention backend reads the compressed pages in every phase, so a
+    chunk of n new tokens attends to the cached context as stored (the
+    dequantized tiles, then the raw tail: ``k_hat`` / ``v_hat``, lists
+    indexed by KV head of [L][d]) and to the chunk's own rows, which are not
+    in the cache yet and enter as the raw fp16 rows they are.  Chunk token i
+    sees the L context tokens and chunk tokens 0..i (causal); query head h
+    reads KV head h // group.
+
+    q_chunk [n][H_q][d]; k_new / v_new [n][H_kv][d].  Returns [n][H_q][d]
+    (fp64).  Appending the chunk to the cache afterwards is the write path's
+    business (tiles the chunk completes get quantized), not this function's.
+    """
+    q_chunk = np.asarray(q_chunk, dtype=np.float64)
+    k_new = np.asarray(k_new, dtype=np.float16).astype(np.float64)
+    v_new = np.asarray(v_new, dtype=np.float16).astype(np.float64)
+    n, hq = q_chunk.shape[:2]
+    out = np.zeros(q_chunk.shape, dtype=np.float64)
+    for i in range(n):
+        for h in range(hq):
+            kv = h // group
+            keys = np.concatenate([k_hat[kv], k_new[:i + 1, kv]], axis=0)
+            vals = np.concatenate([v_hat[kv], v_new[:i + 1, kv]], axis=0)
+            out[i, h] = attention_fp64(q_chunk[i, h], keys, vals, scale)
     return out
 
 

@@ -458,3 +458,119 @@ def test_randomized_rotation_dequantizes_and_decodes():
     # than the unseeded decoder's reading of the same codes
     k_plain = o.sequence_kv_hat(tk, tail_k, 0)
     assert np.linalg.norm(k_hat - rows_k) < 0.5 * np.linalg.norm(k_plain - rows_k)
+
+
+# --------------------------------------------------------------------------- chunked prefill
+
+def _ctx(rng, hkv, length, t=32):
+    """Context of ``length`` tokens per KV head as the cache holds it."""
+    k_hat, v_hat = [], []
+    for _ in range(hkv):
+        rk = rng.standard_normal((length, 128)).astype(np.float16)
+        rv = rng.standard_normal((length, 128)).astype(np.float16)
+        tk, tail_k = o.quantize_sequence(rk, t, 4, 2)
+        tv, tail_v = o.quantize_sequence(rv, t, 4, 2)
+        k_hat.append(o.sequence_kv_hat(tk, tail_k))
+        v_hat.append(o.sequence_kv_hat(tv, tail_v))
+    return k_hat, v_hat
+
+
+def test_prefill_causal_count_closed_form():
+    # all keys equal -> uniform weights over exactly the visible keys.  With
+    # context values 0 and new value j+1 at chunk position j, token i's
+    # output is (1 + ... + (i+1)) / (L + i + 1): an off-by-one in the mask or
+    # a dropped context shifts it
+    L, n, g = 7, 5, 2
+    u = np.full(128, 0.25)
+    k_hat = [np.tile(u, (L, 1))]
+    v_hat = [np.zeros((L, 128))]
+    k_new = np.tile(u, (n, 1, 1)).astype(np.float16)
+    v_new = np.zeros((n, 1, 128), dtype=np.float16)
+    v_new[:, 0, 0] = np.arange(1, n + 1)
+    q = np.random.default_rng(31).standard_normal((n, g, 128))
+    out = o.prefill_chunk_sequence(q, k_hat, v_hat, k_new, v_new, g)
+    for i in range(n):
+        want = (i + 1) * (i + 2) / 2 / (L + i + 1)
+        for h in range(g):
+            assert out[i, h, 0] == pytest.approx(want, rel=1e-13)
+            assert np.all(out[i, h, 1:] == 0)
+
+
+def test_prefill_two_key_softmax_closed_form():
+    # one context key, chunk of one token: weight of the new key is the
+    # logistic of the score difference times the scale
+    rng = np.random.default_rng(32)
+    q = rng.standard_normal((1, 1, 128))
+    k1, k2 = rng.standard_normal((1, 128)), rng.standard_normal((1, 1, 128)).astype(np.float16)
+    v1 = np.zeros((1, 128))
+    v2 = np.ones((1, 1, 128), dtype=np.float16)
+    for scale in (None, 0.05):
+        sc = 1 / math.sqrt(128) if scale is None else scale
+        a = float(q[0, 0] @ k1[0]) * sc
+        b = float(q[0, 0] @ k2[0, 0].astype(np.float64)) * sc
+        w2 = 1.0 / (1.0 + math.exp(a - b))
+        out = o.prefill_chunk_sequence(q, [k1], [v1], k2, v2, 1, scale)
+        np.testing.assert_allclose(out[0, 0], np.full(128, w2), rtol=1e-12)
+
+
+def test_prefill_gqa_mapping():
+    # query head h reads KV head h // g: values constant per KV head
+    rng = np.random.default_rng(33)
+    hkv, g, L, n = 3, 4, 40, 6
+    k_hat = [rng.standard_normal((L, 128)) for _ in range(hkv)]
+    v_hat = [np.full((L, 128), float(kv + 1)) for kv in range(hkv)]
+    k_new = rng.standard_normal((n, hkv, 128)).astype(np.float16)
+    v_new = np.broadcast_to(np.arange(1, hkv + 1, dtype=np.float16)[None, :, None], (n, hkv, 128)).copy()
+    out = o.prefill_chunk_sequence(rng.standard_normal((n, hkv * g, 128)), k_hat, v_hat, k_new, v_new, g)
+    for h in range(hkv * g):
+        np.testing.assert_allclose(out[:, h], float(h // g + 1), rtol=1e-13)
+
+
+def test_prefill_one_token_is_decode_over_appended_cache():
+    # a chunk of one token is a decode step over the context plus that row
+    rng = np.random.default_rng(34)
+    hkv, g = 2, 3
+    k_hat, v_hat = _ctx(rng, hkv, 75)
+    k_new = rng.standard_normal((1, hkv, 128)).astype(np.float16)
+    v_new = rng.standard_normal((1, hkv, 128)).astype(np.float16)
+    q = rng.standard_normal((1, hkv * g, 128))
+    out = o.prefill_chunk_sequence(q, k_hat, v_hat, k_new, v_new, g)
+    k_app = [np.concatenate([k_hat[h], k_new[:, h].astype(np.float64)]) for h in range(hkv)]
+    v_app = [np.concatenate([v_hat[h], v_new[:, h].astype(np.float64)]) for h in range(hkv)]
+    np.testing.assert_array_equal(out[0], o.decode_sequence(q[0], k_app, v_app, g))
+
+
+def test_prefill_later_rows_do_not_leak():
+    # changing chunk rows after position i leaves token i's output alone;
+    # changing row i itself moves it
+    rng = np.random.default_rng(35)
+    hkv, g, n = 1, 2, 6
+    k_hat, v_hat = _ctx(rng, hkv, 33)
+    k_new = rng.standard_normal((n, hkv, 128)).astype(np.float16)
+    v_new = rng.standard_normal((n, hkv, 128)).astype(np.float16)
+    q = rng.standard_normal((n, hkv * g, 128))
+    base = o.prefill_chunk_sequence(q, k_hat, v_hat, k_new, v_new, g)
+    for i in range(n - 1):
+        k2, v2 = k_new.copy(), v_new.copy()
+        k2[i + 1:] = rng.standard_normal(k2[i + 1:].shape)
+        v2[i + 1:] = rng.standard_normal(v2[i + 1:].shape)
+        out = o.prefill_chunk_sequence(q, k_hat, v_hat, k2, v2, g)
+        np.testing.assert_array_equal(out[:i + 1], base[:i + 1])
+        assert np.abs(out[i + 1] - base[i + 1]).max() > 1e-3
+        v3 = v_new.copy()
+        v3[i] += np.float16(1.0)
+        assert np.abs(o.prefill_chunk_sequence(q, k_hat, v_hat, k_new, v3, g)[i] - base[i]).max() > 1e-4
+
+
+def test_prefill_empty_context_is_causal_attention():
+    # no cached tokens: plain causal attention over the chunk (brute force)
+    rng = np.random.default_rng(36)
+    n = 4
+    k_new = rng.standard_normal((n, 1, 128)).astype(np.float16)
+    v_new = rng.standard_normal((n, 1, 128)).astype(np.float16)
+    q = rng.standard_normal((n, 1, 128))
+    out = o.prefill_chunk_sequence(q, [np.zeros((0, 128))], [np.zeros((0, 128))], k_new, v_new, 1)
+    for i in range(n):
+        want = brute_attention(q[i, 0].tolist(), k_new[:i + 1, 0].astype(np.float64).tolist(),
+                               v_new[:i + 1, 0].astype(np.float64).tolist(), 1 / math.sqrt(128))
+        np.testing.assert_allclose(out[i, 0], want, rtol=1e-12, atol=1e-14)
