@@ -208,6 +208,37 @@ KVQ_API kvq_status kvq_paged_decode_attention(const kvq_config* cfg, const void*
                                       size_t workspace_bytes, int num_splits,
                                       int32_t* dev_status, void* stream);
 
+/* Read path, chunked prefill: attention of a chunk of new tokens per sequence
+ * over the quantized cache and the chunk itself.  The method reads the
+ * compressed pages directly in every phase of attention (aitrends.kr article
+ * 74976, "TL;DR"; glossary "attention backend"); the chunk's own rows are not
+ * cached yet and enter as raw fp16.  Chunk token i of sequence s (query head
+ * j, reading KV head j / group_size) attends to the ctx_lens[s] cached tokens
+ * (full tiles from the pools, the last ctx_lens[s] mod T from the tails) and
+ * to chunk tokens 0..i: softmax(q.k * softmax_scale) V in fp32.
+ *   q, out       : device fp16 [cu_chunk[num_seqs]][num_kv_heads*group_size][d],
+ *                  the chunk tokens of all sequences packed; q not rotated.
+ *   k_new, v_new : device fp16 [cu_chunk[num_seqs]][num_kv_heads][d], the
+ *                  chunk's K and V rows.
+ *   cu_chunk     : device int32 [num_seqs+1], prefix sums of chunk lengths.
+ *   ctx_lens     : device int32 [num_seqs], tokens cached before the chunk.
+ *   max_chunk_tokens: host bound >= every chunk length (sizes the launch:
+ *                  one CTA per sequence, KV head and 128 query rows).
+ * No workspace: each CTA merges its context and chunk parts itself.
+ * The chunk is not appended: call kvq_append_tokens with the same rows and
+ * cu_chunk afterwards (tiles it completes are then quantized).  A chunk
+ * longer than max_chunk_tokens, or negative, is reported through dev_status
+ * (KVQ_ERR_DEVICE_BOUNDS) and only its first max_chunk_tokens tokens are
+ * written; pages outside the pool likewise (the tile is skipped).  b in
+ * {2, 4} for K and V, or 8 for both (KVQ_ERR_UNSUPPORTED for 3). */
+KVQ_API kvq_status kvq_paged_prefill_attention(const kvq_config* cfg, const void* q, void* out,
+                                       const void* k_new, const void* v_new, const int32_t* cu_chunk,
+                                       const int32_t* ctx_lens, int num_seqs, int max_chunk_tokens,
+                                       const int32_t* block_tables, int max_blocks_per_seq,
+                                       int num_blocks, const void* k_pool, const void* v_pool,
+                                       const void* k_tail, const void* v_tail, float softmax_scale,
+                                       int32_t* dev_status, void* stream);
+
 /* Size of the scratch array built into the library for
  * kvq_paged_decode_attention_static_scratch (32 MiB per device). */
 #define KVQ_DECODE_STATIC_SCRATCH_BYTES ((size_t)32 << 20)

@@ -266,6 +266,60 @@ kvq_status kvq_paged_decode_attention(const kvq_config* cfg, const void* q, void
                      "kvq_paged_decode_attention launch");
 }
 
+kvq_status kvq_paged_prefill_attention(const kvq_config* cfg, const void* q, void* out, const void* k_new,
+                                       const void* v_new, const int32_t* cu_chunk, const int32_t* ctx_lens,
+                                       int num_seqs, int max_chunk_tokens, const int32_t* block_tables,
+                                       int max_blocks_per_seq, int num_blocks, const void* k_pool,
+                                       const void* v_pool, const void* k_tail, const void* v_tail,
+                                       float softmax_scale, int32_t* dev_status, void* stream) {
+  KVQ_TRY(check_config(cfg));
+  if (cfg->bits_k == 3 || cfg->bits_v == 3)
+    return fail(KVQ_ERR_UNSUPPORTED, "prefill attention reads 2-, 4- or 8-bit codes only (3-bit pages are storage-only)");
+  if (num_seqs < 0 || max_chunk_tokens < 0) return fail(KVQ_ERR_INVALID_ARG, "negative num_seqs or max_chunk_tokens");
+  if (num_seqs == 0 || max_chunk_tokens == 0) return ok();
+  if (num_seqs > 65535) return fail(KVQ_ERR_INVALID_ARG, "num_seqs > 65535");
+  if (max_chunk_tokens > (1 << 20)) return fail(KVQ_ERR_INVALID_ARG, "max_chunk_tokens > 2^20");
+  const long long units = static_cast<long long>(num_seqs) * cfg->num_kv_heads * kvq::prefill_row_tiles(*cfg, max_chunk_tokens);
+  if (units > 0x7fffffffLL)
+    return fail(KVQ_ERR_INVALID_ARG, "num_seqs x max_chunk_tokens too large for one launch");
+  if (!(softmax_scale > 0.f) || !(softmax_scale < 1e30f))
+    return fail(KVQ_ERR_INVALID_ARG, "softmax_scale must be a positive finite float");
+  KVQ_TRY(check_ptr(q, "q"));
+  KVQ_TRY(check_ptr(out, "out"));
+  KVQ_TRY(check_ptr(k_new, "k_new"));
+  KVQ_TRY(check_ptr(v_new, "v_new"));
+  KVQ_TRY(check_ptr(cu_chunk, "cu_chunk"));
+  KVQ_TRY(check_ptr(ctx_lens, "ctx_lens"));
+  KVQ_TRY(check_tables(block_tables, max_blocks_per_seq, num_blocks));
+  KVQ_TRY(check_ptr(k_pool, "k_pool"));
+  KVQ_TRY(check_ptr(v_pool, "v_pool"));
+  KVQ_TRY(check_ptr(k_tail, "k_tail"));
+  KVQ_TRY(check_ptr(v_tail, "v_tail"));
+  KVQ_TRY(check_ptr(dev_status, "dev_status", true));
+  kvq::PrefillArgs a{};
+  a.cfg = *cfg;
+  a.q = q;
+  a.out = out;
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.cu_chunk = cu_chunk;
+  a.ctx_lens = ctx_lens;
+  a.num_seqs = num_seqs;
+  a.max_chunk = max_chunk_tokens;
+  a.row_tiles = kvq::prefill_row_tiles(*cfg, max_chunk_tokens);
+  a.block_tables = block_tables;
+  a.max_blocks_per_seq = max_blocks_per_seq;
+  a.num_blocks = num_blocks;
+  a.k_pool = k_pool;
+  a.v_pool = v_pool;
+  a.k_tail = k_tail;
+  a.v_tail = v_tail;
+  a.softmax_scale = softmax_scale;
+  a.dev_status = dev_status;
+  return cuda_status(kvq::launch_paged_prefill(a, static_cast<cudaStream_t>(stream)),
+                     "kvq_paged_prefill_attention launch");
+}
+
 kvq_status kvq_unpack_tiles(const kvq_config* cfg, const int32_t* tile_desc, int num_tiles,
                             const int32_t* block_tables, int num_seqs, int max_blocks_per_seq, int num_blocks,
                             const void* pool,

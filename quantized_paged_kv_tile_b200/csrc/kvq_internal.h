@@ -110,6 +110,30 @@ struct DecodeArgs {
 size_t decode_workspace_bytes(const kvq_config& cfg, int num_seqs, int num_splits, int num_sms);
 cudaError_t launch_paged_decode(const DecodeArgs& a, cudaStream_t s);
 
+struct PrefillArgs {
+  kvq_config cfg;
+  const void* q;             // [cu_chunk[B]][H_kv*g][d] fp16
+  void* out;                 // same shape
+  const void* k_new;         // [cu_chunk[B]][H_kv][d] fp16
+  const void* v_new;
+  const int32_t* cu_chunk;   // [B+1]
+  const int32_t* ctx_lens;   // [B]
+  int num_seqs;
+  int max_chunk;             // host bound on chunk lengths
+  int row_tiles;             // 128-row query tiles per (sequence, KV head)
+  const int32_t* block_tables;
+  int max_blocks_per_seq;
+  int num_blocks;
+  const void* k_pool;
+  const void* v_pool;
+  const void* k_tail;
+  const void* v_tail;
+  float softmax_scale;
+  int32_t* dev_status;
+};
+int prefill_row_tiles(const kvq_config& cfg, int max_chunk);
+cudaError_t launch_paged_prefill(const PrefillArgs& a, cudaStream_t s);
+
 // Self-tests of the bounded mbarrier waits (one per kernel file): a wait on
 // a barrier nothing arrives at gives up after its limit and records
 // KVQ_ERR_DEVICE_TIMEOUT in *dev_status.

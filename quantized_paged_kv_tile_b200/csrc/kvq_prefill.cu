@@ -1,0 +1,891 @@
+// Read path, chunked prefill: a chunk of n new tokens per sequence attends to
+// the quantized cache (pages read directly, never re-materialised as fp16;
+// aitrends.kr article 74976, "TL;DR" and glossary "attention backend") and,
+// causally, to its own raw fp16 rows.
+//
+// One kernel, one CTA (8 warps) per (sequence, KV head, 128 query rows).  The
+// query rows of a (sequence, KV head) are the chunk tokens x the g query heads
+// of that KV head, token-major: row i*g + j is chunk token i, head j.  Warp w
+// owns TMEM lanes 32 (w % 4) .. +31 (one query row per thread) and column half
+// w / 4.  Every contraction runs on the tcgen05 tensor cores (fp16 operands in
+// shared memory, 128-byte swizzle, K-major; fp32 accumulators in TMEM; one
+// thread issues, a commit to an mbarrier signals completion):
+//
+// A. Context tiles, rotated domain.  q' = q D_s H (one MMA against H, scaled
+//    into the log2 domain) and per tile of the context, exactly as the decode
+//    kernel's algebra:
+//      score_i = s~K_i (q'' . codeK_i) + z~K_i sum_j q''_j,   q'' = q' * C~K_t
+//      acc'_j += C~V_tj (sum_i p_i s~V_i codeV_ij + sum_i p_i z~V_i)
+//    QK: D_S[128][80] = q''_hi . B_K^T + q''_lo . B_K^T, B_K = the block's 64
+//    tokens of K codes as exact fp16 integers, a row of ones (column 64 of D_S
+//    is then sum_j q''_j) and zero rows.  PV: D_O[128][128] = P_hi . B_V^T +
+//    P_lo . B_V^T, P = p * s~V, B_V = V codes channel-major.  The hi / lo
+//    halves keep q'' and P fp32-accurate on fp16 operands; the codes are
+//    exact.  C~V scales D_O's columns per tile, so D_O is folded into register
+//    accumulators block by block.  Tiles are staged whole (K and V pages) by
+//    cp.async.bulk, double-buffered.
+// B. Raw keys, original domain: the fp16 tail of the cache, then the chunk's
+//    own rows, causal (chunk token i sees tail + chunk rows 0..i).  QK: q
+//    (fp16, exact) . K_raw^T; PV: P_hi / P_lo . V_raw^T (V transposed into
+//    shared memory).  Separate running max / sum / accumulator.
+// C. The two parts are merged by their log-sum-exp weights; the rotated part
+//    is taken back with one MMA against H (hi / lo halves of acc'), then the
+//    channel signs and 1/sqrt(d); fp16 output.
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+
+#include "kvq_device.cuh"
+
+namespace kvq {
+
+namespace {
+
+constexpr int kPfThreads = 256;
+constexpr int kRows = 128;                  // query rows per CTA (TMEM lanes)
+constexpr int kBlk = 64;                    // context tokens per MMA block
+constexpr int kNS = kBlk + 16;              // score columns: tokens, sum(q''), zero rows
+constexpr long long kWaitNs = 2000000000LL; // bounded waits: 2 s
+
+// shared memory map (offsets from a 1024-byte aligned base)
+constexpr int kOffAqHi = 0;                        // q''_hi: 128 x 128 fp16, two 16 KB channel atoms
+constexpr int kOffAqLo = 32768;                    // q''_lo
+constexpr int kOffBk = 65536;                      // B_K: 80 x 128 fp16, two 10 KB channel atoms
+constexpr int kBkAtom = kNS * 128;                 // 10240
+constexpr int kOffBv = kOffBk + 2 * kBkAtom;       // B_V: 128 channels x 64 tokens fp16 (16 KB)
+constexpr int kOffPHi = kOffBv + 16384;            // P_hi: 128 rows x 64 tokens fp16
+constexpr int kOffPLo = kOffPHi + 16384;           // P_lo
+constexpr int kOffRed = kOffPLo + 16384;           // float red[3][2][128]: row max, sum p, sum p z~V
+constexpr int kOffF = kOffRed + 3 * 2 * kRows * 4; // float tile scalars: C~K[128], C~V[128], s~K, z~K, s~V, z~V [128]
+constexpr int kOffBar = kOffF + 6 * 128 * 4;       // mbarriers: stage 0, stage 1, mma
+constexpr int kOffMisc = kOffBar + 64;             // TMEM slot, flags
+constexpr int kOffStage = kOffMisc + 64;
+// the set-up rotation borrows B_K .. B_V for H (128 x 128 fp16, 32 KB); the
+// final one borrows B_V .. P
+static_assert(kOffBk + 32768 <= kOffPHi, "H fits in front of P");
+static_assert(kOffBv + 32768 <= kOffRed, "H fits over B_V and P");
+static_assert(kOffBv % 1024 == 0 && kOffPHi % 1024 == 0 && kOffPLo % 1024 == 0, "atoms 1024-aligned");
+
+template <int T, int BK, int BV>
+struct PfGeom {
+  static constexpr int kPages = T / kPageTokens;
+  static constexpr int kCodesK = kPageTokens * kHeadDim * BK / 8;
+  static constexpr int kCodesV = kPageTokens * kHeadDim * BV / 8;
+  static constexpr int kCs = kHeadDim * kPageTokens / T;  // channels of C per page
+  static constexpr int kCsBytes = (2 * kCs + 15) / 16 * 16;
+  static constexpr int kPageK = kCodesK + 64 + kCsBytes;
+  static constexpr int kPageV = kCodesV + 64 + kCsBytes;
+  static constexpr int kStage = kPages * (kPageK + kPageV);
+  static constexpr int kValid = T < kBlk ? T : kBlk;  // tokens per block
+  static constexpr int kBlocks = T < kBlk ? 1 : T / kBlk;
+  static constexpr int kSmem = kOffStage + 2 * kStage + 1024;  // + alignment slack
+};
+
+// ------------------------------------------------------------------ PTX helpers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ long long gtime() {
+  long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  if (mbar_try(bar, parity)) return true;
+  const long long t0 = gtime();
+  while (!mbar_try(bar, parity))
+    if (gtime() - t0 > kWaitNs) return false;
+  return true;
+}
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;  // (a & b) | c
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+__device__ __forceinline__ __half2 u32_as_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+
+// A 32-bit word of b-bit codes -> h = 16/b fp16 pairs of exact small
+// integers, pair e = (field e, field e + h).
+// The fields land in fp16 mantissas under the exponent of 1024 (0x6400) and
+// are rebased by one subtraction or fused multiply-add.
+template <int B>
+__device__ __forceinline__ void unpack_pairs(uint32_t w, uint32_t out[16 / B]) {
+  const uint32_t magic = 0x64006400u;
+  const __half2 k1024 = __float2half2_rn(1024.f);
+  if constexpr (B == 8) {  // pair e (0..1) = (byte e, byte e+2)
+    out[0] = h2_as_u32(__hsub2(u32_as_h2(lop3_and_or(w, 0x00FF00FFu, magic)), k1024));
+    out[1] = h2_as_u32(__hsub2(u32_as_h2(lop3_and_or(w >> 8, 0x00FF00FFu, magic)), k1024));
+  } else if constexpr (B == 4) {  // pair e (0..3) = (nibble e, nibble e+4)
+    const uint32_t w8 = w >> 8;
+    const __half2 s16 = __float2half2_rn(1.f / 16.f), o64 = __float2half2_rn(-64.f);
+    out[0] = h2_as_u32(__hsub2(u32_as_h2(lop3_and_or(w, 0x000F000Fu, magic)), k1024));
+    out[1] = h2_as_u32(__hfma2(u32_as_h2(lop3_and_or(w, 0x00F000F0u, magic)), s16, o64));
+    out[2] = h2_as_u32(__hsub2(u32_as_h2(lop3_and_or(w8, 0x000F000Fu, magic)), k1024));
+    out[3] = h2_as_u32(__hfma2(u32_as_h2(lop3_and_or(w8, 0x00F000F0u, magic)), s16, o64));
+  } else {  // pair e (0..7) = (field e, field e+8)
+    const uint32_t w8 = w >> 8;
+    const __half2 s4 = __float2half2_rn(0.25f), o256 = __float2half2_rn(-256.f);
+    const __half2 s16 = __float2half2_rn(1.f / 16.f), o64 = __float2half2_rn(-64.f);
+    const __half2 s64 = __float2half2_rn(1.f / 64.f), o16 = __float2half2_rn(-16.f);
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const uint32_t x = half ? w8 : w;
+      out[4 * half + 0] = h2_as_u32(__hsub2(u32_as_h2(lop3_and_or(x, 0x00030003u, magic)), k1024));
+      out[4 * half + 1] = h2_as_u32(__hfma2(u32_as_h2(lop3_and_or(x, 0x000C000Cu, magic)), s4, o256));
+      out[4 * half + 2] = h2_as_u32(__hfma2(u32_as_h2(lop3_and_or(x, 0x00300030u, magic)), s16, o64));
+      out[4 * half + 3] = h2_as_u32(__hfma2(u32_as_h2(lop3_and_or(x, 0x00C000C0u, magic)), s64, o16));
+    }
+  }
+}
+
+// Order of the channels along the QK contraction: the K codes of a 32-bit
+// word (W = 32/b channels, fields in channel order) unpack into pairs
+// (field e, field e + W/2), so MMA position 2e + s of the word's group holds
+// channel e + s W/2.  q'' is written in the same order (the dot product does
+// not care which order, only that both operands share it).
+template <int B>
+__device__ __forceinline__ constexpr int qk_channel(int kpos) {
+  constexpr int W = 32 / B;
+  const int p = kpos % W;
+  return kpos - p + (p >> 1) + (p & 1) * (W / 2);
+}
+
+// Byte offset of (row r, position k) in a K-major fp16 operand of `rows` rows
+// stored as 64-element atoms of 128-byte rows with the 128-byte swizzle.
+__device__ __forceinline__ uint32_t sw_off(int r, int k, int rows) {
+  return (k >> 6) * rows * 128 + r * 128 + ((((k & 63) >> 3) ^ (r & 7)) << 4) + (k & 7) * 2;
+}
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t d = static_cast<uint64_t>((saddr >> 4) & 0x3FFF);  // start address
+  d |= static_cast<uint64_t>(1) << 16;                          // leading offset (unused with this swizzle)
+  d |= static_cast<uint64_t>(1024 >> 4) << 32;                  // 8-row groups 1024 B apart
+  d |= static_cast<uint64_t>(1) << 46;                          // descriptor version
+  d |= static_cast<uint64_t>(2) << 61;                          // 128-byte swizzle
+  return d;
+}
+// kind::f16 instruction descriptor: fp32 accumulate, fp16 A and B, both K-major, M = 128
+__host__ __device__ constexpr uint32_t idesc_m128(uint32_t n) { return (1u << 4) | ((n >> 3) << 17) | ((128u >> 4) << 24); }
+
+__device__ __forceinline__ void mma_f16(uint32_t dtmem, uint64_t da, uint64_t db, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
+          dtmem),
+      "l"(da), "l"(db), "r"(idesc), "r"(acc));
+}
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's TMEM lane
+__device__ __forceinline__ void tmem_ld32(uint32_t addr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%"
+      "19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(addr));
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]), "+r"(r[8]),
+        "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]),
+        "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]),
+        "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31]));
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+// 32 consecutive fp32 columns of this thread's TMEM lane from registers
+__device__ __forceinline__ void tmem_st32(uint32_t addr, const float (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
+      "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(addr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
+      "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+      "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+      "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+      "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+      "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+      "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ float tmem_ld1(uint32_t addr) {
+  uint32_t r;
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(addr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" : "+r"(r));
+  return __uint_as_float(r);
+}
+__device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ uint4 hi_lo_pack(const float (&x)[8], uint4& lo) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const __half2 hv = __floats2half2_rn(x[2 * k], x[2 * k + 1]);
+    const float2 hf = __half22float2(hv);
+    h[k] = h2_as_u32(hv);
+    l[k] = h2_as_u32(__floats2half2_rn(x[2 * k] - hf.x, x[2 * k + 1] - hf.y));
+  }
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
+  return make_uint4(h[0], h[1], h[2], h[3]);
+}
+
+// ------------------------------------------------------------------ kernel
+// H (Sylvester, +-1) times the channel signs s_k as a K-major operand at
+// `off`: element (r, k) = (-1)^popcount(r & k) s_k, or without signs.
+__device__ void build_h(unsigned char* smem, int off, uint32_t seed) {
+  for (int i = threadIdx.x; i < kHeadDim * 16; i += kPfThreads) {
+    const int r = i >> 4, pc = i & 15;
+    uint32_t w[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int c = 8 * pc + 2 * k;
+      const float x0 = ((__popc(r & c) & 1) ? -1.f : 1.f) * rotation_sign(seed, c);
+      const float x1 = ((__popc(r & (c + 1)) & 1) ? -1.f : 1.f) * rotation_sign(seed, c + 1);
+      w[k] = h2_as_u32(__floats2half2_rn(x0, x1));
+    }
+    *reinterpret_cast<uint4*>(smem + off + sw_off(r, 8 * pc, kHeadDim)) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// query rows (raw fp16) of this CTA into the q''_hi area; rows past the chunk: zeros
+__device__ void load_q_rows(unsigned char* smem, const PrefillArgs& a, int c0, int h, int rt, int rows_valid) {
+  const int G = a.cfg.group_size, hqn = a.cfg.num_kv_heads * G;
+  for (int i = threadIdx.x; i < kRows * 16; i += kPfThreads) {
+    const int r = i >> 4, pc = i & 15;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (r < rows_valid) {
+      const int gr = rt * kRows + r;
+      v = *reinterpret_cast<const uint4*>(static_cast<const __half*>(a.q) +
+                                          (static_cast<size_t>(c0 + gr / G) * hqn + h * G + gr % G) * kHeadDim +
+                                          8 * pc);
+    }
+    *reinterpret_cast<uint4*>(smem + kOffAqHi + sw_off(r, 8 * pc, kRows)) = v;
+  }
+}
+
+// one thread: D (+)= A . B^T over K = 16 * ksteps, A in `npass` hi / lo areas
+// (the second `a_lo` apart), atoms of A 16 KB apart, of B `b_atom` apart
+__device__ __forceinline__ void issue_mma(uint32_t d, uint32_t a0, uint32_t a_lo, int npass, uint32_t b0,
+                                          uint32_t b_atom, int ksteps, uint32_t idesc, uint32_t bar) {
+  fence_after();
+  for (int hl = 0; hl < npass; ++hl) {
+    const uint32_t sa = a0 + hl * a_lo;
+    for (int s = 0; s < ksteps; ++s) {
+      const uint32_t ka = (s >> 2) * 16384 + (s & 3) * 32, kb = (s >> 2) * b_atom + (s & 3) * 32;
+      mma_f16(d, sw128_desc(sa + ka), sw128_desc(b0 + kb), idesc, (hl | s) != 0);
+    }
+  }
+  mma_commit(bar);
+}
+
+__device__ __forceinline__ float f4_at(const float4& v, int k) {
+  return k == 0 ? v.x : (k == 1 ? v.y : (k == 2 ? v.z : v.w));
+}
+
+template <int T, int BK, int BV>
+__global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs a) {
+  using Geo = PfGeom<T, BK, BV>;
+  constexpr int NP = Geo::kPages;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  unsigned char* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int quad = warp & 3, eta = warp >> 2;  // TMEM lane quadrant, column half
+  const int row = 32 * quad + lane;            // this thread's query row (TMEM lane)
+  const int G = a.cfg.group_size, nh = a.cfg.num_kv_heads;
+  const int R = a.row_tiles;
+  const int rt = blockIdx.x % R, bh = blockIdx.x / R;
+  const int h = bh % nh, b = bh / nh;
+  const int c0 = a.cu_chunk[b];
+  const int n = a.cu_chunk[b + 1] - c0;
+  if ((n < 0 || n > a.max_chunk) && tid == 0 && rt == 0 && h == 0) report_error(a.dev_status, KVQ_ERR_DEVICE_BOUNDS);
+  const int nc = max(0, min(n, a.max_chunk));  // chunk tokens served
+  const int rows_valid = min(nc * G - rt * kRows, kRows);
+  if (rows_valid <= 0) return;
+  const int L = max(a.ctx_lens[b], 0);
+  const int F = L / T, tau = L - F * T;
+  // chunk token of this thread's row (rows past the chunk take the last one)
+  const int i_row = (rt * kRows + min(row, rows_valid - 1)) / G;
+  const int i_max = (rt * kRows + rows_valid - 1) / G;
+
+  const uint32_t s_base = smem_u32(smem);
+  const uint32_t bar_stage0 = s_base + kOffBar, bar_mma = s_base + kOffBar + 16;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
+  int* stage_bad = reinterpret_cast<int*>(smem + kOffMisc + 8);  // [2]
+  float* red = reinterpret_cast<float*>(smem + kOffRed);          // [3][2][128]
+  float* ckf = reinterpret_cast<float*>(smem + kOffF);            // C~K of the tile
+  float* cvf = ckf + 128;                                         // C~V
+  float* skf = ckf + 256;                                         // s~K, z~K, s~V, z~V per token
+  float* zkf = ckf + 384;
+  float* svf = ckf + 512;
+  float* zvf = ckf + 640;
+  const uint8_t* kpool = static_cast<const uint8_t*>(a.k_pool);
+  const uint8_t* vpool = static_cast<const uint8_t*>(a.v_pool);
+
+  if (tid == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_stage0));
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_stage0 + 8));
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_mma));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tslot)), "r"(512));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+
+  // warp 0 stages tile `tile` (all K pages, then all V pages) into stage st;
+  // bit st of `issued` (warp 0's copy) marks copies not yet waited for
+  uint32_t issued = 0u;
+  auto issue = [&](int tile, int st) {
+    const int lb = tile * NP + lane;
+    int blk = -1;
+    if (lane < NP)
+      blk = lb < a.max_blocks_per_seq ? a.block_tables[static_cast<size_t>(b) * a.max_blocks_per_seq + lb] : -1;
+    const bool bad = lane < NP && (blk < 0 || blk >= a.num_blocks);
+    if (__any_sync(kFull, bad)) {
+      if (lane == 0) {
+        report_error(a.dev_status, KVQ_ERR_DEVICE_BOUNDS);
+        stage_bad[st] = 1;
+      }
+      return;
+    }
+    if (lane == 0) {
+      stage_bad[st] = 0;
+      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar_stage0 + 8 * st),
+                   "r"(NP * (Geo::kPageK + Geo::kPageV))
+                   : "memory");
+    }
+    __syncwarp();
+    if (lane < NP) {
+      const uint32_t dst = s_base + kOffStage + st * Geo::kStage;
+      const size_t reg = static_cast<size_t>(blk) * nh + h;
+      bulk_g2s(dst + lane * Geo::kPageK, kpool + reg * Geo::kPageK, Geo::kPageK, bar_stage0 + 8 * st);
+      bulk_g2s(dst + NP * Geo::kPageK + lane * Geo::kPageV, vpool + reg * Geo::kPageV, Geo::kPageV,
+               bar_stage0 + 8 * st);
+    }
+    issued |= 1u << st;
+  };
+  __syncthreads();  // barriers initialised
+  if (warp == 0 && F > 0) issue(0, 0);
+
+  const uint32_t t_lane = static_cast<uint32_t>(32 * quad) << 16;
+  uint32_t tbase = 0, mma_phase = 0;
+  bool ok = true;
+  float acc[64];  // rotated-domain accumulator of the context
+#pragma unroll
+  for (int i = 0; i < 64; ++i) acc[i] = 0.f;
+  float m_ctx = -INFINITY, l_ctx = 0.f;
+
+  // ---- set-up: q rows and H D_s; q' = q D_s H on the tensor cores
+  load_q_rows(smem, a, c0, h, rt, rows_valid);
+  build_h(smem, kOffBk, a.cfg.rotation_seed);
+  fence_async_smem();
+  fence_before();
+  __syncthreads();
+  fence_after();
+  tbase = *tslot;
+  // TMEM columns: D_S 0..79, D_O 128..255, 256..383 q' (context part), then
+  // the parked context accumulator (raw part)
+  const uint32_t d_s = tbase, d_o = tbase + 128, d_park = tbase + 256;
+  if (F > 0) {
+    if (tid == 0)
+      issue_mma(d_o, s_base + kOffAqHi, 0, 1, s_base + kOffBk, 16384, 8, idesc_m128(kHeadDim), bar_mma);
+    ok = mbar_wait(bar_mma, mma_phase);
+    mma_phase ^= 1u;
+    fence_after();
+    const float qscale = a.softmax_scale * kLog2e / kSqrtHeadDim;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      float x[32];
+      tmem_ld32(d_o + t_lane + 64 * eta + 32 * half, x);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) x[i] *= qscale;
+      tmem_st32(d_park + t_lane + 64 * eta + 32 * half, x);
+    }
+    fence_before();
+  }
+  __syncthreads();
+  // B_K, B_V, P start zeroed (padding rows / tokens stay zero); B_K row 64 = ones
+  for (int i = tid; i < (kOffRed - kOffBk) / 16; i += kPfThreads)
+    *reinterpret_cast<uint4*>(smem + kOffBk + 16 * i) = make_uint4(0, 0, 0, 0);
+  __syncthreads();
+  if (tid < 16)
+    *reinterpret_cast<uint4*>(smem + kOffBk + sw_off(kBlk, 8 * tid, kNS)) =
+        make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u);
+  if (__syncthreads_or(!ok)) {
+    if (tid == 0) report_error(a.dev_status, KVQ_ERR_DEVICE_TIMEOUT);
+    ok = false;
+  }
+
+  // ================================================================ A. context tiles
+  uint32_t st_phase = 0u;  // bit s: parity to wait for on stage s
+  for (int t = 0; t < F && ok; ++t) {
+    const int st = t & 1;
+    if (warp == 0 && t + 1 < F) issue(t + 1, st ^ 1);
+    if (stage_bad[st]) {  // pages outside the pool: tile skipped (reported)
+      __syncthreads();
+      continue;
+    }
+    const bool got = mbar_wait(bar_stage0 + 8 * st, (st_phase >> st) & 1u);
+    st_phase ^= 1u << st;
+    if (got) issued &= ~(1u << st);
+    if (__syncthreads_or(!got)) {
+      if (tid == 0) report_error(a.dev_status, KVQ_ERR_DEVICE_TIMEOUT);
+      ok = false;
+      break;
+    }
+    const unsigned char* sK = smem + kOffStage + st * Geo::kStage;
+    const unsigned char* sV = sK + NP * Geo::kPageK;
+    // tile scalars as floats: C~ per channel, (s~, z~) per token
+    if (tid < kHeadDim) {
+      const int c = tid, pg = c / Geo::kCs, o = 2 * (c % Geo::kCs);
+      ckf[c] = __half2float(*reinterpret_cast<const __half*>(sK + pg * Geo::kPageK + Geo::kCodesK + 64 + o));
+      cvf[c] = __half2float(*reinterpret_cast<const __half*>(sV + pg * Geo::kPageV + Geo::kCodesV + 64 + o));
+    } else if (tid - kHeadDim < T) {
+      const int tok = tid - kHeadDim, pg = tok / kPageTokens, o = 4 * (tok % kPageTokens);
+      const float2 k2 = __half22float2(*reinterpret_cast<const __half2*>(sK + pg * Geo::kPageK + Geo::kCodesK + o));
+      const float2 v2 = __half22float2(*reinterpret_cast<const __half2*>(sV + pg * Geo::kPageV + Geo::kCodesV + o));
+      skf[tok] = k2.x;
+      zkf[tok] = k2.y;
+      svf[tok] = v2.x;
+      zvf[tok] = v2.y;
+    }
+    __syncthreads();
+
+    // -- q'' = q' * C~K in hi / lo halves, in the QK channel order; pieces
+    // 4 half .. 4 half + 3 use channels 32 half .. 32 half + 31 of this
+    // thread's 64 (a word's channel group never straddles 32)
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      float qv[32];
+      tmem_ld32(d_park + t_lane + 64 * eta + 32 * half, qv);
+#pragma unroll
+      for (int pq = 0; pq < 4; ++pq) {
+        const int pc = 4 * half + pq;
+        constexpr int kSecond = BK == 2 ? 8 : 4;  // the piece's channels: two aligned groups of 4
+        const int first = qk_channel<BK>(8 * pc);
+        const float4 g0 = *reinterpret_cast<const float4*>(ckf + 64 * eta + first);
+        const float4 g1 = *reinterpret_cast<const float4*>(ckf + 64 * eta + first + kSecond);
+        float x[8];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          const int cl = qk_channel<BK>(8 * pc + m);
+          const float cval = cl < first + 4 ? f4_at(g0, cl - first) : f4_at(g1, cl - first - kSecond);
+          x[m] = qv[cl - 32 * half] * cval;
+        }
+        uint4 lo;
+        const uint4 hi = hi_lo_pack(x, lo);
+        const int kpos = 64 * eta + 8 * pc;
+        *reinterpret_cast<uint4*>(smem + kOffAqHi + sw_off(row, kpos, kRows)) = hi;
+        *reinterpret_cast<uint4*>(smem + kOffAqLo + sw_off(row, kpos, kRows)) = lo;
+      }
+    }
+
+    for (int kb = 0; kb < Geo::kBlocks && ok; ++kb) {
+      const int pg0 = kb * (kBlk / kPageTokens);  // first page of the block
+      // -- B_K: token rows, 16-byte pieces of 8 MMA positions
+      for (int i = tid; i < Geo::kValid * 16; i += kPfThreads) {
+        const int tok = i >> 4, pc = i & 15;
+        const unsigned char* rec = sK + (pg0 + tok / kPageTokens) * Geo::kPageK + (tok % kPageTokens) * (16 * BK);
+        uint32_t pr[4];
+        if constexpr (BK == 4) {
+          unpack_pairs<4>(*reinterpret_cast<const uint32_t*>(rec + 4 * pc), pr);
+        } else if constexpr (BK == 2) {
+          uint32_t all[8];
+          unpack_pairs<2>(*reinterpret_cast<const uint32_t*>(rec + 4 * (pc >> 1)), all);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) pr[k] = (pc & 1) ? all[4 + k] : all[k];
+        } else {
+          const uint2 w = *reinterpret_cast<const uint2*>(rec + 8 * pc);
+          unpack_pairs<8>(w.x, pr);
+          unpack_pairs<8>(w.y, pr + 2);
+        }
+        *reinterpret_cast<uint4*>(smem + kOffBk + sw_off(tok, 8 * pc, kNS)) = make_uint4(pr[0], pr[1], pr[2], pr[3]);
+      }
+      // -- B_V: channel rows, token pairs.  Lane L = 4 g + t of a page owns
+      // words k (16-byte row k / 4); word k holds channels 8 (h (k / 2) + e) + g
+      // for tokens 2t + 8 (k % 2) and the next, h = 16 / b pairs per word.
+      constexpr int kRowsPerLane = BV / 2;  // 16-byte rows per lane (2 b words / 4)
+      constexpr int kVUnits = (Geo::kValid / kPageTokens) * 32 * kRowsPerLane;
+      for (int i = tid; i < kVUnits; i += kPfThreads) {
+        const int pgl = i / (32 * kRowsPerLane), rem = i % (32 * kRowsPerLane);
+        const int j = rem / 32, ln = rem % 32;
+        const uint4 v4 = *reinterpret_cast<const uint4*>(sV + (pg0 + pgl) * Geo::kPageV + (j * 32 + ln) * 16);
+        const uint32_t wv[4] = {v4.x, v4.y, v4.z, v4.w};
+        const int g8 = ln >> 2, tt = ln & 3;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int k = 4 * j + q;
+          constexpr int hV = 16 / BV;
+          uint32_t pr[hV];
+          unpack_pairs<BV>(wv[q], pr);
+          const int kpos = kPageTokens * pgl + 2 * tt + 8 * (k & 1);
+#pragma unroll
+          for (int e = 0; e < hV; ++e) {
+            const int c = 8 * (hV * (k >> 1) + e) + g8;
+            *reinterpret_cast<uint32_t*>(smem + kOffBv + sw_off(c, kpos, kHeadDim)) = pr[e];
+          }
+        }
+      }
+      fence_async_smem();
+      __syncthreads();
+      if (tid == 0)
+        issue_mma(d_s, s_base + kOffAqHi, kOffAqLo - kOffAqHi, 2, s_base + kOffBk, kBkAtom, 8, idesc_m128(kNS),
+                  bar_mma);
+      const bool got_s = mbar_wait(bar_mma, mma_phase);
+      mma_phase ^= 1u;
+      fence_after();
+      // -- scores of this thread's 32 tokens (log2 domain), block max
+      const bool live = 32 * eta < Geo::kValid;  // warp-uniform
+      const int tok0 = kBlk * kb + 32 * eta;     // first token (within the tile) of this thread
+      float sc[32];
+      float mloc = -INFINITY;
+      if (live) {
+        tmem_ld32(d_s + t_lane + 32 * eta, sc);
+        const float sig = tmem_ld1(d_s + t_lane + kBlk);
+#pragma unroll
+        for (int j4 = 0; j4 < 8; ++j4) {
+          const float4 s4 = *reinterpret_cast<const float4*>(skf + tok0 + 4 * j4);
+          const float4 z4 = *reinterpret_cast<const float4*>(zkf + tok0 + 4 * j4);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            float& v = sc[4 * j4 + k];
+            v = f4_at(s4, k) * v + f4_at(z4, k) * sig;
+            mloc = fmaxf(mloc, v);
+          }
+        }
+      }
+      red[(0 * 2 + eta) * kRows + row] = mloc;
+      if (__syncthreads_or(!got_s)) {
+        if (tid == 0) report_error(a.dev_status, KVQ_ERR_DEVICE_TIMEOUT);
+        ok = false;
+        break;
+      }
+      const float m_new = fmaxf(m_ctx, fmaxf(red[row], red[kRows + row]));
+      const float alpha = exp2f(m_ctx - m_new);
+      // -- P = p * s~V (hi / lo), sums of p and p z~V
+      float lsum = 0.f, wsum = 0.f;
+      if (live) {
+#pragma unroll
+        for (int pc = 0; pc < 4; ++pc) {
+          float x[8];
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            const float4 s4 = *reinterpret_cast<const float4*>(svf + tok0 + 8 * pc + 4 * hf);
+            const float4 z4 = *reinterpret_cast<const float4*>(zvf + tok0 + 8 * pc + 4 * hf);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const float p = exp2f(sc[8 * pc + 4 * hf + k] - m_new);
+              lsum += p;
+              wsum += p * f4_at(z4, k);
+              x[4 * hf + k] = p * f4_at(s4, k);
+            }
+          }
+          uint4 lo;
+          const uint4 hi = hi_lo_pack(x, lo);
+          const int kpos = 32 * eta + 8 * pc;
+          *reinterpret_cast<uint4*>(smem + kOffPHi + sw_off(row, kpos, kRows)) = hi;
+          *reinterpret_cast<uint4*>(smem + kOffPLo + sw_off(row, kpos, kRows)) = lo;
+        }
+      }
+      red[(1 * 2 + eta) * kRows + row] = lsum;
+      red[(2 * 2 + eta) * kRows + row] = wsum;
+      fence_async_smem();
+      fence_before();
+      __syncthreads();
+      if (tid == 0)
+        issue_mma(d_o, s_base + kOffPHi, kOffPLo - kOffPHi, 2, s_base + kOffBv, 16384, 4, idesc_m128(kHeadDim),
+                  bar_mma);
+      l_ctx = l_ctx * alpha + red[2 * kRows + row] + red[3 * kRows + row];
+      const float wtot = red[4 * kRows + row] + red[5 * kRows + row];
+      m_ctx = m_new;
+      const bool got_o = mbar_wait(bar_mma, mma_phase);
+      mma_phase ^= 1u;
+      fence_after();
+      // -- fold D_O into the accumulators: acc'_c = alpha acc'_c + C~V_c (D_c + sum p z~V)
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        float x[32];
+        tmem_ld32(d_o + t_lane + 64 * eta + 32 * half, x);
+#pragma unroll
+        for (int i4 = 0; i4 < 8; ++i4) {
+          const float4 c4 = *reinterpret_cast<const float4*>(cvf + 64 * eta + 32 * half + 4 * i4);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            float& A = acc[32 * half + 4 * i4 + k];
+            A = alpha * A + f4_at(c4, k) * (x[4 * i4 + k] + wtot);
+          }
+        }
+      }
+      fence_before();
+      if (__syncthreads_or(!got_o)) {
+        if (tid == 0) report_error(a.dev_status, KVQ_ERR_DEVICE_TIMEOUT);
+        ok = false;
+      }
+    }
+  }
+
+  // ================================================================ B. raw keys
+  // keys j: the tail (j < tau), then chunk rows j - tau; row i sees j <= tau + i.
+  // The context accumulator waits in TMEM meanwhile.
+  if (F > 0) {
+    float x[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) x[i] = acc[i];
+    tmem_st32(d_park + t_lane + 64 * eta, x);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) x[i] = acc[32 + i];
+    tmem_st32(d_park + t_lane + 64 * eta + 32, x);
+  }
+  float m_raw = -INFINITY, l_raw = 0.f;
+  float racc[64];  // the raw-part accumulator (original domain)
+#pragma unroll
+  for (int i = 0; i < 64; ++i) racc[i] = 0.f;
+  const int nkeys = tau + i_max + 1;
+  if (ok) load_q_rows(smem, a, c0, h, rt, rows_valid);
+  const float rscale = a.softmax_scale * kLog2e;
+  const __half* kt = static_cast<const __half*>(a.k_tail) + (static_cast<size_t>(b) * nh + h) * T * kHeadDim;
+  const __half* vt = static_cast<const __half*>(a.v_tail) + (static_cast<size_t>(b) * nh + h) * T * kHeadDim;
+  const __half* kn = static_cast<const __half*>(a.k_new) + (static_cast<size_t>(c0) * nh + h) * kHeadDim;
+  const __half* vn = static_cast<const __half*>(a.v_new) + (static_cast<size_t>(c0) * nh + h) * kHeadDim;
+  const size_t new_stride = static_cast<size_t>(nh) * kHeadDim;
+  auto key_row = [&](int j, bool val) -> const __half* {
+    if (j < tau) return (val ? vt : kt) + static_cast<size_t>(j) * kHeadDim;
+    return (val ? vn : kn) + static_cast<size_t>(j - tau) * new_stride;
+  };
+  for (int j0 = 0; j0 < nkeys && ok; j0 += kBlk) {
+    // -- K rows into B_K (keys past the end: zeros), V rows transposed into B_V
+    for (int i = tid; i < kBlk * 16; i += kPfThreads) {
+      const int r = i >> 4, pc = i & 15;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (j0 + r < nkeys) v = *reinterpret_cast<const uint4*>(key_row(j0 + r, false) + 8 * pc);
+      *reinterpret_cast<uint4*>(smem + kOffBk + sw_off(r, 8 * pc, kNS)) = v;
+    }
+    for (int i = tid; i < (kBlk / 2) * 16; i += kPfThreads) {
+      const int r2 = i >> 4, pc = i & 15;  // keys 2 r2, 2 r2 + 1; channels 8 pc ..
+      uint4 v0 = make_uint4(0, 0, 0, 0), v1 = make_uint4(0, 0, 0, 0);
+      if (j0 + 2 * r2 < nkeys) v0 = *reinterpret_cast<const uint4*>(key_row(j0 + 2 * r2, true) + 8 * pc);
+      if (j0 + 2 * r2 + 1 < nkeys) v1 = *reinterpret_cast<const uint4*>(key_row(j0 + 2 * r2 + 1, true) + 8 * pc);
+      const uint32_t a4[4] = {v0.x, v0.y, v0.z, v0.w}, b4[4] = {v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        // channels 8 pc + 2k (low halves) and 8 pc + 2k + 1 (high halves)
+        *reinterpret_cast<uint32_t*>(smem + kOffBv + sw_off(8 * pc + 2 * k, 2 * r2, kHeadDim)) =
+            __byte_perm(a4[k], b4[k], 0x5410);
+        *reinterpret_cast<uint32_t*>(smem + kOffBv + sw_off(8 * pc + 2 * k + 1, 2 * r2, kHeadDim)) =
+            __byte_perm(a4[k], b4[k], 0x7632);
+      }
+    }
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0)
+      issue_mma(d_s, s_base + kOffAqHi, 0, 1, s_base + kOffBk, kBkAtom, 8, idesc_m128(kBlk), bar_mma);
+    const bool got_s = mbar_wait(bar_mma, mma_phase);
+    mma_phase ^= 1u;
+    fence_after();
+    float sc[32];
+    float mloc = -INFINITY;
+    const int jt = j0 + 32 * eta;  // first key of this thread
+    const bool live = jt < nkeys;  // warp-uniform
+    if (live) {
+      tmem_ld32(d_s + t_lane + 32 * eta, sc);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        sc[j] = (jt + j <= tau + i_row) ? sc[j] * rscale : -INFINITY;
+        mloc = fmaxf(mloc, sc[j]);
+      }
+    }
+    red[eta * kRows + row] = mloc;
+    if (__syncthreads_or(!got_s)) {
+      if (tid == 0) report_error(a.dev_status, KVQ_ERR_DEVICE_TIMEOUT);
+      ok = false;
+      break;
+    }
+    const float m_new = fmaxf(m_raw, fmaxf(red[row], red[kRows + row]));
+    const float alpha = exp2f(m_raw - m_new);
+    float lsum = 0.f;
+    if (live) {
+#pragma unroll
+      for (int pc = 0; pc < 4; ++pc) {
+        float x[8];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          const float p = exp2f(sc[8 * pc + m] - m_new);
+          lsum += p;
+          x[m] = p;
+        }
+        uint4 lo;
+        const uint4 hi = hi_lo_pack(x, lo);
+        const int kpos = 32 * eta + 8 * pc;
+        *reinterpret_cast<uint4*>(smem + kOffPHi + sw_off(row, kpos, kRows)) = hi;
+        *reinterpret_cast<uint4*>(smem + kOffPLo + sw_off(row, kpos, kRows)) = lo;
+      }
+    } else {  // keys past the end: P stays zero for them
+#pragma unroll
+      for (int pc = 0; pc < 4; ++pc) {
+        const int kpos = 32 * eta + 8 * pc;
+        *reinterpret_cast<uint4*>(smem + kOffPHi + sw_off(row, kpos, kRows)) = make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(smem + kOffPLo + sw_off(row, kpos, kRows)) = make_uint4(0, 0, 0, 0);
+      }
+    }
+    red[(2 + eta) * kRows + row] = lsum;
+    fence_async_smem();
+    fence_before();
+    __syncthreads();
+    if (tid == 0)
+      issue_mma(d_o, s_base + kOffPHi, kOffPLo - kOffPHi, 2, s_base + kOffBv, 16384, 4, idesc_m128(kHeadDim),
+                bar_mma);
+    l_raw = l_raw * alpha + red[2 * kRows + row] + red[3 * kRows + row];
+    m_raw = m_new;
+    const bool got_o = mbar_wait(bar_mma, mma_phase);
+    mma_phase ^= 1u;
+    fence_after();
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      float x[32];
+      tmem_ld32(d_o + t_lane + 64 * eta + 32 * half, x);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) racc[32 * half + i] = alpha * racc[32 * half + i] + x[i];
+    }
+    fence_before();
+    if (__syncthreads_or(!got_o)) {
+      if (tid == 0) report_error(a.dev_status, KVQ_ERR_DEVICE_TIMEOUT);
+      ok = false;
+    }
+  }
+
+  // ================================================================ C. merge, inverse rotation, output
+  const float m_all = fmaxf(m_ctx, m_raw);
+  const float w_ctx = l_ctx > 0.f ? exp2f(m_ctx - m_all) : 0.f;
+  const float w_raw = l_raw > 0.f ? exp2f(m_raw - m_all) : 0.f;
+  const float inv_l = 1.f / (l_ctx * w_ctx + l_raw * w_raw);
+  bool have_rot = F > 0 && ok;  // block-uniform
+  if (have_rot) {
+    // acc' (times its weight) in hi / lo halves as the A operand, H (no signs) as B
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      float y[32];
+      tmem_ld32(d_park + t_lane + 64 * eta + 32 * half, y);
+#pragma unroll
+      for (int pc = 0; pc < 4; ++pc) {
+        float x[8];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) x[m] = y[8 * pc + m] * w_ctx;
+        uint4 lo;
+        const uint4 hi = hi_lo_pack(x, lo);
+        const int kpos = 64 * eta + 32 * half + 8 * pc;
+        *reinterpret_cast<uint4*>(smem + kOffAqHi + sw_off(row, kpos, kRows)) = hi;
+        *reinterpret_cast<uint4*>(smem + kOffAqLo + sw_off(row, kpos, kRows)) = lo;
+      }
+    }
+    build_h(smem, kOffBv, 0u);
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0)
+      issue_mma(d_o, s_base + kOffAqHi, kOffAqLo - kOffAqHi, 2, s_base + kOffBv, 16384, 8, idesc_m128(kHeadDim),
+                bar_mma);
+    const bool got = mbar_wait(bar_mma, mma_phase);
+    mma_phase ^= 1u;
+    fence_after();
+    if (__syncthreads_or(!got)) {
+      if (tid == 0) report_error(a.dev_status, KVQ_ERR_DEVICE_TIMEOUT);
+      ok = have_rot = false;
+    }
+  }
+  {
+    const int gr = rt * kRows + min(row, rows_valid - 1);
+    __half* o = static_cast<__half*>(a.out) + (static_cast<size_t>(c0 + gr / G) * nh * G + h * G + gr % G) * kHeadDim +
+                64 * eta;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      float x[32];
+      if (have_rot) {
+        tmem_ld32(d_o + t_lane + 64 * eta + 32 * half, x);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) x[i] = 0.f;
+      }
+#pragma unroll
+      for (int pc = 0; pc < 4; ++pc) {
+        uint32_t w[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int i = 8 * pc + 2 * k, c = 64 * eta + 32 * half + i;
+          const float r0 = x[i] * (rotation_sign(a.cfg.rotation_seed, c) / kSqrtHeadDim);
+          const float r1 = x[i + 1] * (rotation_sign(a.cfg.rotation_seed, c + 1) / kSqrtHeadDim);
+          w[k] = h2_as_u32(__floats2half2_rn((r0 + racc[32 * half + i] * w_raw) * inv_l,
+                                             (r1 + racc[32 * half + i + 1] * w_raw) * inv_l));
+        }
+        if (row < rows_valid) *reinterpret_cast<uint4*>(o + 32 * half + 8 * pc) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+  }
+  if (!ok && warp == 0) {  // let copies in flight land before the shared memory is released
+    for (int s = 0; s < 2; ++s)
+      if (issued & (1u << s)) (void)mbar_wait(bar_stage0 + 8 * s, (st_phase >> s) & 1u);
+  }
+  fence_before();
+  __syncthreads();
+  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tbase), "r"(512));
+}
+
+template <int T, int BK, int BV>
+cudaError_t launch_t(const PrefillArgs& a, cudaStream_t s, long long units) {
+  using Geo = PfGeom<T, BK, BV>;
+  auto kern = prefill_attn_kernel<T, BK, BV>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Geo::kSmem);
+  if (e != cudaSuccess) return e;
+  kern<<<static_cast<unsigned>(units), kPfThreads, Geo::kSmem, s>>>(a);
+  return cudaGetLastError();
+}
+
+template <int T>
+cudaError_t launch_bits(const PrefillArgs& a, cudaStream_t s, long long units) {
+  if (a.cfg.bits_k == 4 && a.cfg.bits_v == 4) return launch_t<T, 4, 4>(a, s, units);
+  if (a.cfg.bits_k == 4 && a.cfg.bits_v == 2) return launch_t<T, 4, 2>(a, s, units);
+  if (a.cfg.bits_k == 2 && a.cfg.bits_v == 4) return launch_t<T, 2, 4>(a, s, units);
+  if (a.cfg.bits_k == 8 && a.cfg.bits_v == 8) return launch_t<T, 8, 8>(a, s, units);
+  return launch_t<T, 2, 2>(a, s, units);
+}
+
+}  // namespace
+
+int prefill_row_tiles(const kvq_config& cfg, int max_chunk) {
+  return static_cast<int>((static_cast<long long>(max_chunk) * cfg.group_size + kRows - 1) / kRows);
+}
+
+cudaError_t launch_paged_prefill(const PrefillArgs& a, cudaStream_t s) {
+  const long long units = static_cast<long long>(a.num_seqs) * a.cfg.num_kv_heads * a.row_tiles;
+  if (units == 0) return cudaSuccess;
+  switch (a.cfg.tile_tokens) {
+    case 32: return launch_bits<32>(a, s, units);
+    case 64: return launch_bits<64>(a, s, units);
+    default: return launch_bits<128>(a, s, units);
+  }
+}
+
+}  // namespace kvq

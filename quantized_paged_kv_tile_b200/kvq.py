@@ -30,6 +30,7 @@ EXPORTED_SYMBOLS = (
     "kvq_get_layout", "kvq_decode_workspace_bytes", "kvq_quantize_tiles", "kvq_append_tokens",
     "kvq_paged_decode_attention", "kvq_paged_decode_attention_static_scratch", "kvq_unpack_tiles",
     "kvq_selftest_bounded_wait", "kvq_status_string", "kvq_last_error", "kvq_version",
+    "kvq_paged_prefill_attention",
 )
 
 
@@ -96,6 +97,8 @@ _SIGNATURES = {
     "kvq_paged_decode_attention_static_scratch": [_cfgp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _vp, _vp, _vp,
                                                   _vp, _f32, _i32, _vp, _vp],
     "kvq_selftest_bounded_wait": [_vp, _vp],
+    "kvq_paged_prefill_attention": [_cfgp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _i32, _i32, _vp, _vp,
+                                    _vp, _vp, _f32, _vp, _vp],
     "kvq_unpack_tiles": [_cfgp, _vp, _i32, _vp, _i32, _i32, _i32, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
 }
 
@@ -224,6 +227,27 @@ def paged_decode_attention(cfg: Config, q, out, seq_lens, block_tables, k_pool, 
         _ptr(workspace, "workspace", torch.uint8), workspace.numel(), num_splits,
         _ptr(dev_status, "dev_status", torch.int32), _stream(stream))
     _check(st, "kvq_paged_decode_attention")
+
+
+def paged_prefill_attention(cfg: Config, q, out, k_new, v_new, cu_chunk, ctx_lens, max_chunk_tokens: int,
+                            block_tables, k_pool, v_pool, k_tail, v_tail,
+                            softmax_scale: float | None = None, num_blocks: int | None = None, dev_status=None,
+                            stream=None) -> None:
+    """Read path, chunked prefill: chunk rows (q, out fp16 [N][H_q][d];
+    k_new, v_new fp16 [N][H_kv][d], N = cu_chunk[-1]) attend to the cached
+    context of their sequence and causally to their own chunk."""
+    if softmax_scale is None:
+        softmax_scale = cfg.head_dim ** -0.5
+    nb = k_pool.shape[0] if num_blocks is None else num_blocks
+    st = load_library().kvq_paged_prefill_attention(
+        ctypes.byref(cfg.c()), _ptr(q, "q", torch.float16), _ptr(out, "out", torch.float16),
+        _ptr(k_new, "k_new", torch.float16), _ptr(v_new, "v_new", torch.float16),
+        _ptr(cu_chunk, "cu_chunk", torch.int32), _ptr(ctx_lens, "ctx_lens", torch.int32), ctx_lens.shape[0],
+        int(max_chunk_tokens), _ptr(block_tables, "block_tables", torch.int32), block_tables.shape[1], nb,
+        _ptr(k_pool, "k_pool", torch.uint8), _ptr(v_pool, "v_pool", torch.uint8),
+        _ptr(k_tail, "k_tail", torch.float16), _ptr(v_tail, "v_tail", torch.float16), float(softmax_scale),
+        _ptr(dev_status, "dev_status", torch.int32), _stream(stream))
+    _check(st, "kvq_paged_prefill_attention")
 
 
 # bytes of the library's static decode scratch (one per device)

@@ -7,6 +7,8 @@ turns user-level operations into the three library calls:
                     kvq_append_tokens for the unfinished last tile
   append(rows)   -> kvq_append_tokens (quantizes tiles as they fill)
   decode(q)      -> kvq_paged_decode_attention
+  prefill_chunk(q, rows) -> kvq_paged_prefill_attention over the cache and
+                    the chunk, then kvq_append_tokens of the chunk
 All arithmetic runs in the library's kernels; this module only sizes and
 indexes buffers (PyTorch provides the memory and the stream).
 """
@@ -110,6 +112,30 @@ class PagedKVCache:
         kvq.paged_decode_attention(self.cfg, q, out, self.seq_lens, self.block_tables, self.k_pool, self.v_pool,
                                    self.k_tail, self.v_tail, ws, num_splits=splits, num_blocks=self.num_blocks,
                                    dev_status=self.dev_status, stream=stream)
+        return out
+
+    def prefill_chunk(self, q: torch.Tensor, new_k: torch.Tensor, new_v: torch.Tensor, counts,
+                      out: torch.Tensor | None = None, append: bool = True, stream=None) -> torch.Tensor:
+        """Chunked prefill: packed chunk rows (``counts`` tokens per sequence;
+        q fp16 [N][H_q][d], new_k / new_v fp16 [N][H_kv][d]) attend to the
+        cached context and causally to their own chunk; then (``append``) the
+        chunk joins the cache.  Returns out fp16 [N][H_q][d]."""
+        counts = np.asarray(counts, dtype=np.int64)
+        if counts.shape != (self.num_seqs,) or np.any(counts < 0):
+            raise ValueError("counts: one non-negative chunk length per sequence")
+        if append and np.any(self.host_lens + counts > self.blocks_per_seq * self.cfg.page_tokens):
+            raise ValueError("append past the allocated pages")
+        if out is None:
+            out = torch.empty_like(q)
+        max_chunk = int(counts.max()) if counts.size else 0
+        cu = torch.from_numpy(np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)).to(self.device)
+        kvq.paged_prefill_attention(self.cfg, q, out, new_k, new_v, cu, self.seq_lens, max_chunk, self.block_tables,
+                                    self.k_pool, self.v_pool, self.k_tail, self.v_tail, num_blocks=self.num_blocks,
+                                    dev_status=self.dev_status, stream=stream)
+        if append and max_chunk > 0:
+            self._append(new_k, new_v, self.host_lens, counts, stream)
+            self.host_lens = self.host_lens + counts
+            self.seq_lens.copy_(torch.from_numpy(self.host_lens.astype(np.int32)))
         return out
 
     def status(self) -> int:

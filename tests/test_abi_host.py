@@ -104,6 +104,25 @@ def test_argument_errors_launch_nothing(lib):
                                   None) == kvq.KVQ_OK
 
 
+def test_prefill_argument_errors_launch_nothing(lib):
+    cfg = kvq.Config(num_kv_heads=2, group_size=4, tile_tokens=64, bits_k=4, bits_v=4, iters=4)
+    c = cfg.c()
+    def call(conf, num_seqs=3, max_chunk=40, q=16, scale=0.1, tables=16):
+        return lib.kvq_paged_prefill_attention(ctypes.byref(conf), q, 16, 16, 16, 16, 16, num_seqs, max_chunk,
+                                               tables, 4, 8, 16, 16, 16, 16, scale, None, None)
+    c3 = kvq.Config(num_kv_heads=2, group_size=4, tile_tokens=64, bits_k=4, bits_v=3, iters=4).c()
+    assert call(c3) == kvq.KVQ_ERR_UNSUPPORTED
+    assert call(c, num_seqs=-1) == kvq.KVQ_ERR_INVALID_ARG
+    assert call(c, max_chunk=-2) == kvq.KVQ_ERR_INVALID_ARG
+    assert call(c, q=None) == kvq.KVQ_ERR_INVALID_ARG
+    assert call(c, q=24) == kvq.KVQ_ERR_INVALID_ARG            # misaligned
+    assert call(c, scale=0.0) == kvq.KVQ_ERR_INVALID_ARG
+    assert call(c, tables=None) == kvq.KVQ_ERR_INVALID_ARG
+    assert call(c, num_seqs=70000) == kvq.KVQ_ERR_INVALID_ARG
+    assert call(c, num_seqs=0) == kvq.KVQ_OK                   # nothing to do
+    assert call(c, max_chunk=0) == kvq.KVQ_OK
+
+
 def test_binding_rejects_cpu_tensors(lib):
     cfg = kvq.Config(num_kv_heads=1, group_size=1, tile_tokens=64, bits_k=4, bits_v=4, iters=1)
     x = torch.zeros((64, 1, 128), dtype=torch.float16)
