@@ -54,18 +54,19 @@ constexpr int kOffAqHi = 0;                        // q''_hi: 128 x 128 fp16, tw
 constexpr int kOffAqLo = 32768;                    // q''_lo
 constexpr int kOffBk = 65536;                      // B_K: 80 x 128 fp16, two 10 KB channel atoms
 constexpr int kBkAtom = kNS * 128;                 // 10240
-constexpr int kOffBv = kOffBk + 2 * kBkAtom;       // B_V: 128 channels x 64 tokens fp16 (16 KB)
-constexpr int kOffPHi = kOffBv + 16384;            // P_hi: 128 rows x 64 tokens fp16
+constexpr int kOffBv = kOffBk + 2 * kBkAtom;       // B_V: 2 buffers of 128 channels x 64 tokens fp16 (16 KB)
+constexpr int kOffPHi = kOffBv + 2 * 16384;        // P_hi: 128 rows x 64 tokens fp16
 constexpr int kOffPLo = kOffPHi + 16384;           // P_lo
 constexpr int kOffRed = kOffPLo + 16384;           // float red[3][2][128]: row max, sum p, sum p z~V
-constexpr int kOffF = kOffRed + 3 * 2 * kRows * 4; // float tile scalars: C~K[128], C~V[128], s~K, z~K, s~V, z~V [128]
-constexpr int kOffBar = kOffF + 6 * 128 * 4;       // mbarriers: stage 0, stage 1, mma
+constexpr int kOffF = kOffRed + 3 * 2 * kRows * 4; // 2 x float tile scalars: C~K[128], C~V[128], s~K, z~K, s~V, z~V [128]
+constexpr int kFBuf = 6 * 128;                     // floats per scalar buffer
+constexpr int kOffBar = kOffF + 2 * kFBuf * 4;     // mbarriers: stage 0, stage 1, mma, qk, pv
 constexpr int kOffMisc = kOffBar + 64;             // TMEM slot, flags
 constexpr int kOffStage = kOffMisc + 64;
 // the set-up rotation borrows B_K .. B_V for H (128 x 128 fp16, 32 KB); the
-// final one borrows B_V .. P
+// final one borrows the two B_V buffers
 static_assert(kOffBk + 32768 <= kOffPHi, "H fits in front of P");
-static_assert(kOffBv + 32768 <= kOffRed, "H fits over B_V and P");
+static_assert(kOffBv + 32768 <= kOffPHi, "H fits over the B_V buffers");
 static_assert(kOffBv % 1024 == 0 && kOffPHi % 1024 == 0 && kOffPLo % 1024 == 0, "atoms 1024-aligned");
 
 template <int T, int BK, int BV>
@@ -81,6 +82,7 @@ struct PfGeom {
   static constexpr int kValid = T < kBlk ? T : kBlk;  // tokens per block
   static constexpr int kBlocks = T < kBlk ? 1 : T / kBlk;
   static constexpr int kSmem = kOffStage + 2 * kStage + 1024;  // + alignment slack
+  static_assert(kSmem <= 232448, "shared memory per block");
 };
 
 // ------------------------------------------------------------------ PTX helpers
@@ -189,6 +191,13 @@ __device__ __forceinline__ void mma_f16(uint32_t dtmem, uint64_t da, uint64_t db
           dtmem),
       "l"(da), "l"(db), "r"(idesc), "r"(acc));
 }
+// A from TMEM (one row per lane, fp16 pairs per 32-bit column), B from shared memory
+__device__ __forceinline__ void mma_f16_ta(uint32_t dtmem, uint32_t atmem, uint64_t db, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(
+          dtmem),
+      "r"(atmem), "l"(db), "r"(idesc), "r"(acc));
+}
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
@@ -231,6 +240,15 @@ __device__ __forceinline__ void tmem_st32(uint32_t addr, const float (&v)[32]) {
       : "memory");
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
+// 16 consecutive 32-bit columns of this thread's TMEM lane from registers
+__device__ __forceinline__ void tmem_st16(uint32_t addr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          addr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
 __device__ __forceinline__ float tmem_ld1(uint32_t addr) {
   uint32_t r;
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(addr));
@@ -241,17 +259,25 @@ __device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::aft
 __device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
+// fp32 pair -> fp16 hi + fp16 lo with hi + lo = v to about 2^-22 relative
+__device__ __forceinline__ uint32_t hi_lo2(float2 v, uint32_t& lo) {
+  const __half2 hv = __float22half2_rn(v);
+  const float2 hf = __half22float2(hv);
+  lo = h2_as_u32(__float22half2_rn(__fadd2_rn(v, make_float2(-hf.x, -hf.y))));
+  return h2_as_u32(hv);
+}
 __device__ __forceinline__ uint4 hi_lo_pack(const float (&x)[8], uint4& lo) {
   uint32_t h[4], l[4];
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const __half2 hv = __floats2half2_rn(x[2 * k], x[2 * k + 1]);
-    const float2 hf = __half22float2(hv);
-    h[k] = h2_as_u32(hv);
-    l[k] = h2_as_u32(__floats2half2_rn(x[2 * k] - hf.x, x[2 * k + 1] - hf.y));
-  }
+  for (int k = 0; k < 4; ++k) h[k] = hi_lo2(make_float2(x[2 * k], x[2 * k + 1]), l[k]);
   lo = make_uint4(l[0], l[1], l[2], l[3]);
   return make_uint4(h[0], h[1], h[2], h[3]);
+}
+// 2^x for x <= 0 (the hardware approximation; -inf gives 0)
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // ------------------------------------------------------------------ kernel
@@ -303,6 +329,19 @@ __device__ __forceinline__ void issue_mma(uint32_t d, uint32_t a0, uint32_t a_lo
   mma_commit(bar);
 }
 
+// one thread: D = q''_hi . B_K^T + q''_lo . B_K^T with q'' in TMEM (hi at
+// column a_hi, lo 64 columns on; 8 columns per 16-element K step)
+__device__ __forceinline__ void issue_qk_ta(uint32_t d, uint32_t a_hi, uint32_t b0, uint32_t bar) {
+  fence_after();
+#pragma unroll
+  for (int hl = 0; hl < 2; ++hl)
+#pragma unroll
+    for (int s = 0; s < 8; ++s)
+      mma_f16_ta(d, a_hi + 64 * hl + 8 * s, sw128_desc(b0 + (s >> 2) * kBkAtom + (s & 3) * 32), idesc_m128(kNS),
+                 (hl | s) != 0);
+  mma_commit(bar);
+}
+
 __device__ __forceinline__ float f4_at(const float4& v, int k) {
   return k == 0 ? v.x : (k == 1 ? v.y : (k == 2 ? v.z : v.w));
 }
@@ -334,15 +373,12 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
 
   const uint32_t s_base = smem_u32(smem);
   const uint32_t bar_stage0 = s_base + kOffBar, bar_mma = s_base + kOffBar + 16;
+  const uint32_t bar_qk = s_base + kOffBar + 24, bar_pv = s_base + kOffBar + 32;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   int* stage_bad = reinterpret_cast<int*>(smem + kOffMisc + 8);  // [2]
   float* red = reinterpret_cast<float*>(smem + kOffRed);          // [3][2][128]
-  float* ckf = reinterpret_cast<float*>(smem + kOffF);            // C~K of the tile
-  float* cvf = ckf + 128;                                         // C~V
-  float* skf = ckf + 256;                                         // s~K, z~K, s~V, z~V per token
-  float* zkf = ckf + 384;
-  float* svf = ckf + 512;
-  float* zvf = ckf + 640;
+  float* fbase = reinterpret_cast<float*>(smem + kOffF);          // tile scalars, buffer = tile parity
+  int* tile_bad = reinterpret_cast<int*>(smem + kOffMisc + 16);   // [2], by tile parity
   const uint8_t* kpool = static_cast<const uint8_t*>(a.k_pool);
   const uint8_t* vpool = static_cast<const uint8_t*>(a.v_pool);
 
@@ -350,6 +386,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_stage0));
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_stage0 + 8));
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_mma));
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_qk));
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_pv));
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) {
@@ -409,8 +447,9 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
   fence_after();
   tbase = *tslot;
   // TMEM columns: D_S 0..79, D_O 128..255, 256..383 q' (context part), then
-  // the parked context accumulator (raw part)
-  const uint32_t d_s = tbase, d_o = tbase + 128, d_park = tbase + 256;
+  // the parked context accumulator (raw part); 384..447 / 448..511 q''_hi /
+  // q''_lo as the QK MMA's A operand (row = lane, 2 fp16 per column)
+  const uint32_t d_s = tbase, d_o = tbase + 128, d_park = tbase + 256, a_q = tbase + 384;
   if (F > 0) {
     if (tid == 0)
       issue_mma(d_o, s_base + kOffAqHi, 0, 1, s_base + kOffBk, 16384, 8, idesc_m128(kHeadDim), bar_mma);
@@ -442,54 +481,72 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
   }
 
   // ================================================================ A. context tiles
-  uint32_t st_phase = 0u;  // bit s: parity to wait for on stage s
-  for (int t = 0; t < F && ok; ++t) {
+  // Software pipeline over the context's 64-token blocks gb = 0 .. NB-1: the
+  // operands of block gb+1 are built while PV(gb) runs on the tensor cores,
+  // and block gb's accumulator update overlaps QK(gb+1).
+  const int NB = F * Geo::kBlocks;
+  uint32_t st_phase = 0u, qk_phase = 0u, pv_phase = 0u;  // st_phase bit s: stage s
+
+  // tile t, shared memory only: wait for its pages (skipped when outside the
+  // pool: the tile's blocks then run with zero scalars and masked scores),
+  // stage the tile scalars as floats; starts the copies of tile t+1.
+  // Block-uniform; false on a timeout.
+  auto prep_scalars = [&](int t) -> bool {
     const int st = t & 1;
     if (warp == 0 && t + 1 < F) issue(t + 1, st ^ 1);
-    if (stage_bad[st]) {  // pages outside the pool: tile skipped (reported)
-      __syncthreads();
-      continue;
+    const bool bad = stage_bad[st] != 0;
+    bool got = true;
+    if (!bad) {
+      got = mbar_wait(bar_stage0 + 8 * st, (st_phase >> st) & 1u);
+      st_phase ^= 1u << st;
+      if (got) issued &= ~(1u << st);
     }
-    const bool got = mbar_wait(bar_stage0 + 8 * st, (st_phase >> st) & 1u);
-    st_phase ^= 1u << st;
-    if (got) issued &= ~(1u << st);
     if (__syncthreads_or(!got)) {
       if (tid == 0) report_error(a.dev_status, KVQ_ERR_DEVICE_TIMEOUT);
-      ok = false;
-      break;
+      return false;
     }
     const unsigned char* sK = smem + kOffStage + st * Geo::kStage;
     const unsigned char* sV = sK + NP * Geo::kPageK;
-    // tile scalars as floats: C~ per channel, (s~, z~) per token
+    float* f = fbase + st * kFBuf;
     if (tid < kHeadDim) {
       const int c = tid, pg = c / Geo::kCs, o = 2 * (c % Geo::kCs);
-      ckf[c] = __half2float(*reinterpret_cast<const __half*>(sK + pg * Geo::kPageK + Geo::kCodesK + 64 + o));
-      cvf[c] = __half2float(*reinterpret_cast<const __half*>(sV + pg * Geo::kPageV + Geo::kCodesV + 64 + o));
+      f[c] = bad ? 0.f : __half2float(*reinterpret_cast<const __half*>(sK + pg * Geo::kPageK + Geo::kCodesK + 64 + o));
+      f[128 + c] =
+          bad ? 0.f : __half2float(*reinterpret_cast<const __half*>(sV + pg * Geo::kPageV + Geo::kCodesV + 64 + o));
     } else if (tid - kHeadDim < T) {
       const int tok = tid - kHeadDim, pg = tok / kPageTokens, o = 4 * (tok % kPageTokens);
-      const float2 k2 = __half22float2(*reinterpret_cast<const __half2*>(sK + pg * Geo::kPageK + Geo::kCodesK + o));
-      const float2 v2 = __half22float2(*reinterpret_cast<const __half2*>(sV + pg * Geo::kPageV + Geo::kCodesV + o));
-      skf[tok] = k2.x;
-      zkf[tok] = k2.y;
-      svf[tok] = v2.x;
-      zvf[tok] = v2.y;
+      float2 k2 = make_float2(0.f, 0.f), v2 = make_float2(0.f, 0.f);
+      if (!bad) {
+        k2 = __half22float2(*reinterpret_cast<const __half2*>(sK + pg * Geo::kPageK + Geo::kCodesK + o));
+        v2 = __half22float2(*reinterpret_cast<const __half2*>(sV + pg * Geo::kPageV + Geo::kCodesV + o));
+      }
+      f[256 + tok] = k2.x;
+      f[384 + tok] = k2.y;
+      f[512 + tok] = v2.x;
+      f[640 + tok] = v2.y;
     }
-    __syncthreads();
-
-    // -- q'' = q' * C~K in hi / lo halves, in the QK channel order; pieces
-    // 4 half .. 4 half + 3 use channels 32 half .. 32 half + 31 of this
-    // thread's 64 (a word's channel group never straddles 32)
+    if (tid == 0) tile_bad[st] = bad;
+    return true;
+  };
+  // tile t's q'' = q' * C~K (hi / lo) into TMEM in the QK channel order; the
+  // scalars of tile t must be visible (a barrier after prep_scalars)
+  auto build_qpp = [&](int t) {
+    const float* f = fbase + (t & 1) * kFBuf;
+    // q'' pieces 4 half .. 4 half + 3 use channels 32 half .. 32 half + 31 of
+    // this thread's 64 (a word's channel group never straddles 32); MMA
+    // positions 64 eta + 32 half .. +31 go to 16 TMEM columns each for hi, lo
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
       float qv[32];
       tmem_ld32(d_park + t_lane + 64 * eta + 32 * half, qv);
+      uint32_t whi[16], wlo[16];
 #pragma unroll
       for (int pq = 0; pq < 4; ++pq) {
         const int pc = 4 * half + pq;
         constexpr int kSecond = BK == 2 ? 8 : 4;  // the piece's channels: two aligned groups of 4
         const int first = qk_channel<BK>(8 * pc);
-        const float4 g0 = *reinterpret_cast<const float4*>(ckf + 64 * eta + first);
-        const float4 g1 = *reinterpret_cast<const float4*>(ckf + 64 * eta + first + kSecond);
+        const float4 g0 = *reinterpret_cast<const float4*>(f + 64 * eta + first);
+        const float4 g1 = *reinterpret_cast<const float4*>(f + 64 * eta + first + kSecond);
         float x[8];
 #pragma unroll
         for (int m = 0; m < 8; ++m) {
@@ -499,154 +556,213 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
         }
         uint4 lo;
         const uint4 hi = hi_lo_pack(x, lo);
-        const int kpos = 64 * eta + 8 * pc;
-        *reinterpret_cast<uint4*>(smem + kOffAqHi + sw_off(row, kpos, kRows)) = hi;
-        *reinterpret_cast<uint4*>(smem + kOffAqLo + sw_off(row, kpos, kRows)) = lo;
+        whi[4 * pq] = hi.x;
+        whi[4 * pq + 1] = hi.y;
+        whi[4 * pq + 2] = hi.z;
+        whi[4 * pq + 3] = hi.w;
+        wlo[4 * pq] = lo.x;
+        wlo[4 * pq + 1] = lo.y;
+        wlo[4 * pq + 2] = lo.z;
+        wlo[4 * pq + 3] = lo.w;
       }
+      tmem_st16(a_q + t_lane + 32 * eta + 16 * half, whi);
+      tmem_st16(a_q + 64 + t_lane + 32 * eta + 16 * half, wlo);
     }
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+  };
 
-    for (int kb = 0; kb < Geo::kBlocks && ok; ++kb) {
-      const int pg0 = kb * (kBlk / kPageTokens);  // first page of the block
-      // -- B_K: token rows, 16-byte pieces of 8 MMA positions
-      for (int i = tid; i < Geo::kValid * 16; i += kPfThreads) {
-        const int tok = i >> 4, pc = i & 15;
-        const unsigned char* rec = sK + (pg0 + tok / kPageTokens) * Geo::kPageK + (tok % kPageTokens) * (16 * BK);
-        uint32_t pr[4];
-        if constexpr (BK == 4) {
-          unpack_pairs<4>(*reinterpret_cast<const uint32_t*>(rec + 4 * pc), pr);
-        } else if constexpr (BK == 2) {
-          uint32_t all[8];
-          unpack_pairs<2>(*reinterpret_cast<const uint32_t*>(rec + 4 * (pc >> 1)), all);
+  // block gb's codes: K into B_K (token rows), V into B_V buffer gb & 1
+  // (channel rows, token pairs; lane L = 4 g + t of a page owns words k in
+  // 16-byte rows k / 4, word k holding channels 8 (h (k / 2) + e) + g for
+  // tokens 2t + 8 (k % 2) and the next, h = 16 / b pairs per word)
+  auto unpack_block = [&](int gb) {
+    const int t = gb / Geo::kBlocks, kb = gb % Geo::kBlocks;
+    const unsigned char* sK = smem + kOffStage + (t & 1) * Geo::kStage;
+    const unsigned char* sV = sK + NP * Geo::kPageK;
+    const int pg0 = kb * (kBlk / kPageTokens);
+    for (int i = tid; i < Geo::kValid * 16; i += kPfThreads) {
+      const int tok = i >> 4, pc = i & 15;
+      const unsigned char* rec = sK + (pg0 + tok / kPageTokens) * Geo::kPageK + (tok % kPageTokens) * (16 * BK);
+      uint32_t pr[4];
+      if constexpr (BK == 4) {
+        unpack_pairs<4>(*reinterpret_cast<const uint32_t*>(rec + 4 * pc), pr);
+      } else if constexpr (BK == 2) {
+        uint32_t all[8];
+        unpack_pairs<2>(*reinterpret_cast<const uint32_t*>(rec + 4 * (pc >> 1)), all);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) pr[k] = (pc & 1) ? all[4 + k] : all[k];
-        } else {
-          const uint2 w = *reinterpret_cast<const uint2*>(rec + 8 * pc);
-          unpack_pairs<8>(w.x, pr);
-          unpack_pairs<8>(w.y, pr + 2);
+        for (int k = 0; k < 4; ++k) pr[k] = (pc & 1) ? all[4 + k] : all[k];
+      } else {
+        const uint2 w = *reinterpret_cast<const uint2*>(rec + 8 * pc);
+        unpack_pairs<8>(w.x, pr);
+        unpack_pairs<8>(w.y, pr + 2);
+      }
+      *reinterpret_cast<uint4*>(smem + kOffBk + sw_off(tok, 8 * pc, kNS)) = make_uint4(pr[0], pr[1], pr[2], pr[3]);
+    }
+    unsigned char* bv = smem + kOffBv + (gb & 1) * 16384;
+    constexpr int kRowsPerLane = BV / 2;  // 16-byte rows per lane (2 b words / 4)
+    constexpr int kVUnits = (Geo::kValid / kPageTokens) * 32 * kRowsPerLane;
+    for (int i = tid; i < kVUnits; i += kPfThreads) {
+      const int pgl = i / (32 * kRowsPerLane), rem = i % (32 * kRowsPerLane);
+      const int j = rem / 32, ln = rem % 32;
+      const uint4 v4 = *reinterpret_cast<const uint4*>(sV + (pg0 + pgl) * Geo::kPageV + (j * 32 + ln) * 16);
+      const uint32_t wv[4] = {v4.x, v4.y, v4.z, v4.w};
+      const int g8 = ln >> 2, tt = ln & 3;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int k = 4 * j + q;
+        constexpr int hV = 16 / BV;
+        uint32_t pr[hV];
+        unpack_pairs<BV>(wv[q], pr);
+        const int kpos = kPageTokens * pgl + 2 * tt + 8 * (k & 1);
+#pragma unroll
+        for (int e = 0; e < hV; ++e) {
+          const int c = 8 * (hV * (k >> 1) + e) + g8;
+          *reinterpret_cast<uint32_t*>(bv + sw_off(c, kpos, kHeadDim)) = pr[e];
         }
-        *reinterpret_cast<uint4*>(smem + kOffBk + sw_off(tok, 8 * pc, kNS)) = make_uint4(pr[0], pr[1], pr[2], pr[3]);
-      }
-      // -- B_V: channel rows, token pairs.  Lane L = 4 g + t of a page owns
-      // words k (16-byte row k / 4); word k holds channels 8 (h (k / 2) + e) + g
-      // for tokens 2t + 8 (k % 2) and the next, h = 16 / b pairs per word.
-      constexpr int kRowsPerLane = BV / 2;  // 16-byte rows per lane (2 b words / 4)
-      constexpr int kVUnits = (Geo::kValid / kPageTokens) * 32 * kRowsPerLane;
-      for (int i = tid; i < kVUnits; i += kPfThreads) {
-        const int pgl = i / (32 * kRowsPerLane), rem = i % (32 * kRowsPerLane);
-        const int j = rem / 32, ln = rem % 32;
-        const uint4 v4 = *reinterpret_cast<const uint4*>(sV + (pg0 + pgl) * Geo::kPageV + (j * 32 + ln) * 16);
-        const uint32_t wv[4] = {v4.x, v4.y, v4.z, v4.w};
-        const int g8 = ln >> 2, tt = ln & 3;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int k = 4 * j + q;
-          constexpr int hV = 16 / BV;
-          uint32_t pr[hV];
-          unpack_pairs<BV>(wv[q], pr);
-          const int kpos = kPageTokens * pgl + 2 * tt + 8 * (k & 1);
-#pragma unroll
-          for (int e = 0; e < hV; ++e) {
-            const int c = 8 * (hV * (k >> 1) + e) + g8;
-            *reinterpret_cast<uint32_t*>(smem + kOffBv + sw_off(c, kpos, kHeadDim)) = pr[e];
-          }
-        }
-      }
-      fence_async_smem();
-      __syncthreads();
-      if (tid == 0)
-        issue_mma(d_s, s_base + kOffAqHi, kOffAqLo - kOffAqHi, 2, s_base + kOffBk, kBkAtom, 8, idesc_m128(kNS),
-                  bar_mma);
-      const bool got_s = mbar_wait(bar_mma, mma_phase);
-      mma_phase ^= 1u;
-      fence_after();
-      // -- scores of this thread's 32 tokens (log2 domain), block max
-      const bool live = 32 * eta < Geo::kValid;  // warp-uniform
-      const int tok0 = kBlk * kb + 32 * eta;     // first token (within the tile) of this thread
-      float sc[32];
-      float mloc = -INFINITY;
-      if (live) {
-        tmem_ld32(d_s + t_lane + 32 * eta, sc);
-        const float sig = tmem_ld1(d_s + t_lane + kBlk);
-#pragma unroll
-        for (int j4 = 0; j4 < 8; ++j4) {
-          const float4 s4 = *reinterpret_cast<const float4*>(skf + tok0 + 4 * j4);
-          const float4 z4 = *reinterpret_cast<const float4*>(zkf + tok0 + 4 * j4);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            float& v = sc[4 * j4 + k];
-            v = f4_at(s4, k) * v + f4_at(z4, k) * sig;
-            mloc = fmaxf(mloc, v);
-          }
-        }
-      }
-      red[(0 * 2 + eta) * kRows + row] = mloc;
-      if (__syncthreads_or(!got_s)) {
-        if (tid == 0) report_error(a.dev_status, KVQ_ERR_DEVICE_TIMEOUT);
-        ok = false;
-        break;
-      }
-      const float m_new = fmaxf(m_ctx, fmaxf(red[row], red[kRows + row]));
-      const float alpha = exp2f(m_ctx - m_new);
-      // -- P = p * s~V (hi / lo), sums of p and p z~V
-      float lsum = 0.f, wsum = 0.f;
-      if (live) {
-#pragma unroll
-        for (int pc = 0; pc < 4; ++pc) {
-          float x[8];
-#pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {
-            const float4 s4 = *reinterpret_cast<const float4*>(svf + tok0 + 8 * pc + 4 * hf);
-            const float4 z4 = *reinterpret_cast<const float4*>(zvf + tok0 + 8 * pc + 4 * hf);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const float p = exp2f(sc[8 * pc + 4 * hf + k] - m_new);
-              lsum += p;
-              wsum += p * f4_at(z4, k);
-              x[4 * hf + k] = p * f4_at(s4, k);
-            }
-          }
-          uint4 lo;
-          const uint4 hi = hi_lo_pack(x, lo);
-          const int kpos = 32 * eta + 8 * pc;
-          *reinterpret_cast<uint4*>(smem + kOffPHi + sw_off(row, kpos, kRows)) = hi;
-          *reinterpret_cast<uint4*>(smem + kOffPLo + sw_off(row, kpos, kRows)) = lo;
-        }
-      }
-      red[(1 * 2 + eta) * kRows + row] = lsum;
-      red[(2 * 2 + eta) * kRows + row] = wsum;
-      fence_async_smem();
-      fence_before();
-      __syncthreads();
-      if (tid == 0)
-        issue_mma(d_o, s_base + kOffPHi, kOffPLo - kOffPHi, 2, s_base + kOffBv, 16384, 4, idesc_m128(kHeadDim),
-                  bar_mma);
-      l_ctx = l_ctx * alpha + red[2 * kRows + row] + red[3 * kRows + row];
-      const float wtot = red[4 * kRows + row] + red[5 * kRows + row];
-      m_ctx = m_new;
-      const bool got_o = mbar_wait(bar_mma, mma_phase);
-      mma_phase ^= 1u;
-      fence_after();
-      // -- fold D_O into the accumulators: acc'_c = alpha acc'_c + C~V_c (D_c + sum p z~V)
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        float x[32];
-        tmem_ld32(d_o + t_lane + 64 * eta + 32 * half, x);
-#pragma unroll
-        for (int i4 = 0; i4 < 8; ++i4) {
-          const float4 c4 = *reinterpret_cast<const float4*>(cvf + 64 * eta + 32 * half + 4 * i4);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            float& A = acc[32 * half + 4 * i4 + k];
-            A = alpha * A + f4_at(c4, k) * (x[4 * i4 + k] + wtot);
-          }
-        }
-      }
-      fence_before();
-      if (__syncthreads_or(!got_o)) {
-        if (tid == 0) report_error(a.dev_status, KVQ_ERR_DEVICE_TIMEOUT);
-        ok = false;
       }
     }
+  };
+
+  if (NB > 0 && ok) {
+    ok = prep_scalars(0);
+    if (ok) {
+      unpack_block(0);
+      __syncthreads();  // scalars of tile 0 visible
+      build_qpp(0);
+      fence_async_smem();
+      fence_before();
+      __syncthreads();
+      if (tid == 0) issue_qk_ta(d_s, a_q, s_base + kOffBk, bar_qk);
+    }
+  }
+  for (int gb = 0; gb < NB && ok; ++gb) {
+    const int t = gb / Geo::kBlocks, kb = gb % Geo::kBlocks;
+    const float* f = fbase + (t & 1) * kFBuf;
+    // -- scores of block gb (log2 domain) once QK(gb) is done, block max
+    const bool got_s = mbar_wait(bar_qk, qk_phase);
+    qk_phase ^= 1u;
+    fence_after();
+    const bool live = 32 * eta < Geo::kValid;  // warp-uniform
+    const bool masked = tile_bad[t & 1] != 0;  // block-uniform
+    const int tok0 = kBlk * kb + 32 * eta;     // first token (within the tile) of this thread
+    float sc[32];
+    float mloc = -INFINITY;
+    if (live) {
+      tmem_ld32(d_s + t_lane + 32 * eta, sc);
+      const float sig = tmem_ld1(d_s + t_lane + kBlk);
+      const float2 sig2 = make_float2(sig, sig);
+#pragma unroll
+      for (int j4 = 0; j4 < 8; ++j4) {
+        const float4 s4 = *reinterpret_cast<const float4*>(f + 256 + tok0 + 4 * j4);
+        const float4 z4 = *reinterpret_cast<const float4*>(f + 384 + tok0 + 4 * j4);
+        const float2 v0 = __ffma2_rn(make_float2(s4.x, s4.y), make_float2(sc[4 * j4], sc[4 * j4 + 1]),
+                                     __fmul2_rn(make_float2(z4.x, z4.y), sig2));
+        const float2 v1 = __ffma2_rn(make_float2(s4.z, s4.w), make_float2(sc[4 * j4 + 2], sc[4 * j4 + 3]),
+                                     __fmul2_rn(make_float2(z4.z, z4.w), sig2));
+        sc[4 * j4] = v0.x;
+        sc[4 * j4 + 1] = v0.y;
+        sc[4 * j4 + 2] = v1.x;
+        sc[4 * j4 + 3] = v1.y;
+        mloc = fmaxf(mloc, fmaxf(fmaxf(v0.x, v0.y), fmaxf(v1.x, v1.y)));
+      }
+      if (masked) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) sc[j] = -INFINITY;
+        mloc = -INFINITY;
+      }
+    }
+    red[eta * kRows + row] = mloc;
+    if (__syncthreads_or(!got_s)) {
+      if (tid == 0) report_error(a.dev_status, KVQ_ERR_DEVICE_TIMEOUT);
+      ok = false;
+      break;
+    }
+    const float m_new = fmaxf(m_ctx, fmaxf(red[row], red[kRows + row]));
+    const bool none = m_new == -INFINITY;  // nothing seen yet (masked blocks only)
+    const float alpha = none ? 1.f : ex2(m_ctx - m_new);
+    const float m_use = none ? 0.f : m_new;  // p = 2^(-inf) = 0 either way
+    // -- P = p * s~V (hi / lo), sums of p and p z~V (PV(gb-1) is done: its P is free)
+    float2 lsum2 = make_float2(0.f, 0.f), wsum2 = make_float2(0.f, 0.f);
+    if (live) {
+      const float2 mneg = make_float2(-m_use, -m_use);
+#pragma unroll
+      for (int pc = 0; pc < 4; ++pc) {
+        uint32_t h[4], l[4];
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const float4 s4 = *reinterpret_cast<const float4*>(f + 512 + tok0 + 8 * pc + 4 * hf);
+          const float4 z4 = *reinterpret_cast<const float4*>(f + 640 + tok0 + 8 * pc + 4 * hf);
+#pragma unroll
+          for (int k2 = 0; k2 < 2; ++k2) {
+            const int j = 8 * pc + 4 * hf + 2 * k2;
+            const float2 e = __fadd2_rn(make_float2(sc[j], sc[j + 1]), mneg);
+            const float2 p2 = make_float2(ex2(e.x), ex2(e.y));
+            const float2 sv = k2 ? make_float2(s4.z, s4.w) : make_float2(s4.x, s4.y);
+            const float2 zv = k2 ? make_float2(z4.z, z4.w) : make_float2(z4.x, z4.y);
+            lsum2 = __fadd2_rn(lsum2, p2);
+            wsum2 = __ffma2_rn(p2, zv, wsum2);
+            h[2 * hf + k2] = hi_lo2(__fmul2_rn(p2, sv), l[2 * hf + k2]);
+          }
+        }
+        const int kpos = 32 * eta + 8 * pc;
+        *reinterpret_cast<uint4*>(smem + kOffPHi + sw_off(row, kpos, kRows)) = make_uint4(h[0], h[1], h[2], h[3]);
+        *reinterpret_cast<uint4*>(smem + kOffPLo + sw_off(row, kpos, kRows)) = make_uint4(l[0], l[1], l[2], l[3]);
+      }
+    }
+    red[(1 * 2 + eta) * kRows + row] = lsum2.x + lsum2.y;
+    red[(2 * 2 + eta) * kRows + row] = wsum2.x + wsum2.y;
+    fence_async_smem();
+    fence_before();
+    __syncthreads();
+    if (tid == 0)
+      issue_mma(d_o, s_base + kOffPHi, kOffPLo - kOffPHi, 2, s_base + kOffBv + (gb & 1) * 16384, 16384, 4,
+                idesc_m128(kHeadDim), bar_pv);
+    l_ctx = l_ctx * alpha + red[2 * kRows + row] + red[3 * kRows + row];
+    const float wtot = red[4 * kRows + row] + red[5 * kRows + row];
+    m_ctx = m_new;
+    // -- while PV(gb) runs (shared memory only): block gb+1's codes and, on a
+    // tile change, the next tile's scalars
+    const bool more = gb + 1 < NB;
+    const bool new_tile = more && (gb + 1) % Geo::kBlocks == 0;
+    if (new_tile) ok = prep_scalars((gb + 1) / Geo::kBlocks);
+    if (more && ok) unpack_block(gb + 1);
+    // -- fold D_O into the accumulators: acc'_c = alpha acc'_c + C~V_c (D_c + sum p z~V)
+    const bool got_o = mbar_wait(bar_pv, pv_phase);
+    pv_phase ^= 1u;
+    fence_after();
+    const float2 alpha2 = make_float2(alpha, alpha), w2 = make_float2(wtot, wtot);
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      float x[32];
+      tmem_ld32(d_o + t_lane + 64 * eta + 32 * half, x);
+#pragma unroll
+      for (int i4 = 0; i4 < 8; ++i4) {
+        const float4 c4 = *reinterpret_cast<const float4*>(f + 128 + 64 * eta + 32 * half + 4 * i4);
+#pragma unroll
+        for (int k2 = 0; k2 < 2; ++k2) {
+          const int i = 32 * half + 4 * i4 + 2 * k2;
+          const float2 cv = k2 ? make_float2(c4.z, c4.w) : make_float2(c4.x, c4.y);
+          const float2 r = __ffma2_rn(alpha2, make_float2(acc[i], acc[i + 1]),
+                                      __fmul2_rn(cv, __fadd2_rn(make_float2(x[4 * i4 + 2 * k2], x[4 * i4 + 2 * k2 + 1]), w2)));
+          acc[i] = r.x;
+          acc[i + 1] = r.y;
+        }
+      }
+    }
+    // -- no MMA in flight: the next tile's q'' into TMEM, then QK(gb+1)
+    if (new_tile && ok) {
+      fence_before();
+      __syncthreads();  // next tile's scalars visible; D_O reads done
+      fence_after();
+      build_qpp((gb + 1) / Geo::kBlocks);
+    }
+    fence_async_smem();
+    fence_before();
+    if (__syncthreads_or(!got_o)) {
+      if (tid == 0) report_error(a.dev_status, KVQ_ERR_DEVICE_TIMEOUT);
+      ok = false;
+    }
+    if (more && ok && tid == 0) issue_qk_ta(d_s, a_q, s_base + kOffBk, bar_qk);
   }
 
   // ================================================================ B. raw keys
@@ -726,7 +842,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
       break;
     }
     const float m_new = fmaxf(m_raw, fmaxf(red[row], red[kRows + row]));
-    const float alpha = exp2f(m_raw - m_new);
+    const float alpha = ex2(m_raw - m_new);
     float lsum = 0.f;
     if (live) {
 #pragma unroll
@@ -734,7 +850,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
         float x[8];
 #pragma unroll
         for (int m = 0; m < 8; ++m) {
-          const float p = exp2f(sc[8 * pc + m] - m_new);
+          const float p = ex2(sc[8 * pc + m] - m_new);
           lsum += p;
           x[m] = p;
         }

@@ -169,3 +169,27 @@ def test_prefill_chunk_longer_than_bound_is_reported():
     for r in range(21):
         for hq in range(w.num_q_heads):
             assert rel_l2(oh[r, hq], fh[r, hq]) <= 1e-6
+
+
+def test_prefill_tile_outside_pool_is_skipped_and_reported():
+    # one tile of sequence 0 points outside the pool: reported, and the
+    # output is attention over the context without that tile's tokens
+    ctx, chunk = (640, 300), (24, 40)
+    w, cache, q, k_new, v_new = _setup(64, 4, 4, 4, ctx, chunk)
+    cfg = cache.cfg
+    k_hat = [gpu_pages_kv_hat(cfg, cache, 0, h, ctx[0], False) for h in range(cfg.num_kv_heads)]
+    v_hat = [gpu_pages_kv_hat(cfg, cache, 0, h, ctx[0], True) for h in range(cfg.num_kv_heads)]
+    bad_tile, t, per = 3, cfg.tile_tokens, cfg.tile_tokens // cfg.page_tokens
+    cache.block_tables[0, bad_tile * per + 1] = cache.num_blocks + 7
+    out = cache.prefill_chunk(q, k_new, v_new, chunk, append=False)
+    torch.cuda.synchronize()
+    assert cache.status() == kvq.KVQ_ERR_DEVICE_BOUNDS
+    keep = np.r_[0:bad_tile * t, (bad_tile + 1) * t:ctx[0]]
+    k_cut = [k[keep] for k in k_hat]
+    v_cut = [v[keep] for v in v_hat]
+    qh, kh, vh, oh = (x.float().cpu().numpy() for x in (q, k_new, v_new, out))
+    ref = o.prefill_chunk_sequence(qh[:24], k_cut, v_cut, kh[:24], vh[:24], cfg.group_size)
+    for i in range(24):
+        for hq in range(cfg.num_q_heads):
+            assert rel_l2(oh[i, hq], ref[i, hq]) <= ATTN_REL_L2_MAX
+    assert np.all(np.isfinite(oh))
