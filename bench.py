@@ -9,6 +9,12 @@ d=128, T=64, 4-bit K and V, n=4):
   2. kvq_append_tokens    the step's new token per sequence (fp16 tail)
   3. kvq_paged_decode_attention  one decode query per sequence over the
                           packed pages plus the tail (split-K + merge)
+With ``--prefill-chunk N`` the line also carries a ``prefill`` object: one
+kvq_paged_prefill_attention call per sequence batch, N new tokens per
+sequence attending to the whole cache built by the step (quantized tiles
+plus tail) and causally to themselves, timed with CUDA events, with its
+tensor-core roofline (algorithmic FLOPs: 4 d per query row and visible key).
+
 ``value`` is the step's algorithmic bytes (what the method must move: fp16
 rows read and packed pages written by 1, tail rows by 2, packed pages,
 tables, tail, q and out by 3) per second over the timed steps; the
@@ -43,6 +49,26 @@ FALLBACK_HBM_GBS = 6650.0
 
 
 # --------------------------------------------------------------------------- helpers
+
+def tensor_peak():
+    """Dense fp16/bf16 tensor-core TFLOP/s (fp16 runs at the bf16 rate)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 1590.0, "fallback"
+
+
+def prefill_flops(ctx_lens, chunk, num_q_heads, d=128):
+    """Algorithmic FLOPs of one chunked-prefill call: QK and PV, 2 d each,
+    per (query row, visible key); chunk token i of a sequence sees its
+    context plus chunk tokens 0..i."""
+    keys = 0.0
+    for L in ctx_lens:
+        keys += chunk * float(L) + chunk * (chunk + 1) / 2.0
+    return 4.0 * d * num_q_heads * keys
+
 
 def hbm_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -406,7 +432,54 @@ def run_kvq(args, ranks):
     }
     if args.serving_steps > 0:
         line["serving"] = serving_loop(w, cfg, rows_k, rows_v, args.serving_steps, dev)
+    if args.prefill_chunk > 0:
+        line["prefill"] = prefill_leg(w, cfg, args, dev, stream, seq_lens, bt, nblocks, k_pool, v_pool, k_tail,
+                                      v_tail, status, lens1)
+        line["gpu_launches_prefill"] = args.steps
     return line
+
+
+def prefill_leg(w, cfg, args, dev, stream, seq_lens, bt, nblocks, k_pool, v_pool, k_tail, v_tail, status, lens1):
+    """Chunked prefill over the step's cache: every sequence gets
+    ``--prefill-chunk`` new tokens attending to its cached tokens and
+    causally to themselves (one library call, inputs resident in HBM)."""
+    import torch
+    from quantized_paged_kv_tile_b200 import kvq, synth
+    n = args.prefill_chunk
+    B = w.num_seqs
+    k_new = synth.kv_rows(w, "k", B * n, device=dev, stream_id=7)
+    v_new = synth.kv_rows(w, "v", B * n, device=dev, stream_id=7)
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed * 1000 + 9)
+    q = torch.randn((B * n, w.num_q_heads, 128), generator=g, device=dev).to(torch.float16)
+    out = torch.empty_like(q)
+    cu = torch.arange(0, B * n + 1, n, dtype=torch.int32, device=dev)
+
+    def call():
+        kvq.paged_prefill_attention(cfg, q, out, k_new, v_new, cu, seq_lens, n, bt, k_pool, v_pool, k_tail, v_tail,
+                                    num_blocks=nblocks, dev_status=status, stream=stream)
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for e0, e1 in evs:
+        e0.record(stream)
+        call()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} after the prefill calls")
+    ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    flops = prefill_flops(lens1, n, w.num_q_heads)
+    peak, kind = tensor_peak()
+    tflops = flops / (ms * 1e-3) / 1e12
+    return {"chunk_tokens": n, "ms": ms, "chunk_tok_per_s": B * n / (ms * 1e-3), "flops": flops,
+            "context": f"{B} seqs x {int(lens1[0])} cached tokens (quantized tiles + fp16 tail)",
+            "roofline": {"bound": "tensor", "kernel": "prefill_attn_kernel", "achieved": tflops, "peak": peak,
+                         "peak_kind": kind, "unit": "TFLOP/s", "frac": tflops / peak, "traffic": None,
+                         "note": "algorithmic FLOPs; the kernel runs each product on hi and lo fp16 halves, "
+                                 "so its tensor-core work is twice this"}}
 
 
 def serving_loop(w, cfg, rows_k, rows_v, steps, dev):
@@ -488,6 +561,8 @@ def main():
                     help="override the workload's sequence count (smaller inputs for profiler captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--prefill-chunk", type=int, default=0,
+                    help="also time chunked-prefill attention of this many new tokens per sequence over the cache")
     ap.add_argument("--serving-steps", type=int, default=0,
                     help="after the measurement, time this many graph-replayed append+decode serving steps")
     args = ap.parse_args()

@@ -259,11 +259,17 @@ __device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::aft
 __device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-// fp32 pair -> fp16 hi + fp16 lo with hi + lo = v to about 2^-22 relative
+// fp32 pair -> fp16 hi and fp16 lo with v = hi + lo * 2^-11 to about 2^-22
+// relative.  The residual is carried scaled by 2^11 (|lo| <= |hi|) so that it
+// stays a normal fp16 number whenever hi is: an unscaled residual of a value
+// below 0.125 would be subnormal.  Products with hi and with lo accumulate in
+// separate fp32 accumulators, combined as D_hi + D_lo * 2^-11.
+constexpr float kLoScale = 2048.f, kLoInv = 1.f / 2048.f;
 __device__ __forceinline__ uint32_t hi_lo2(float2 v, uint32_t& lo) {
   const __half2 hv = __float22half2_rn(v);
   const float2 hf = __half22float2(hv);
-  lo = h2_as_u32(__float22half2_rn(__fadd2_rn(v, make_float2(-hf.x, -hf.y))));
+  const float2 r = __fadd2_rn(v, make_float2(-hf.x, -hf.y));
+  lo = h2_as_u32(__float22half2_rn(__fmul2_rn(r, make_float2(kLoScale, kLoScale))));
   return h2_as_u32(hv);
 }
 __device__ __forceinline__ uint4 hi_lo_pack(const float (&x)[8], uint4& lo) {
@@ -314,31 +320,32 @@ __device__ void load_q_rows(unsigned char* smem, const PrefillArgs& a, int c0, i
   }
 }
 
-// one thread: D (+)= A . B^T over K = 16 * ksteps, A in `npass` hi / lo areas
-// (the second `a_lo` apart), atoms of A 16 KB apart, of B `b_atom` apart
-__device__ __forceinline__ void issue_mma(uint32_t d, uint32_t a0, uint32_t a_lo, int npass, uint32_t b0,
-                                          uint32_t b_atom, int ksteps, uint32_t idesc, uint32_t bar) {
+// one thread: D_hi = A_hi . B^T (and D_lo = A_lo . B^T when npass = 2, A_lo
+// `a_lo` bytes after A_hi) over K = 16 * ksteps; atoms of A 16 KB apart, of B
+// `b_atom` apart
+__device__ __forceinline__ void issue_mma(uint32_t d_hi, uint32_t d_lo, uint32_t a0, uint32_t a_lo, int npass,
+                                          uint32_t b0, uint32_t b_atom, int ksteps, uint32_t idesc, uint32_t bar) {
   fence_after();
   for (int hl = 0; hl < npass; ++hl) {
     const uint32_t sa = a0 + hl * a_lo;
     for (int s = 0; s < ksteps; ++s) {
       const uint32_t ka = (s >> 2) * 16384 + (s & 3) * 32, kb = (s >> 2) * b_atom + (s & 3) * 32;
-      mma_f16(d, sw128_desc(sa + ka), sw128_desc(b0 + kb), idesc, (hl | s) != 0);
+      mma_f16(hl ? d_lo : d_hi, sw128_desc(sa + ka), sw128_desc(b0 + kb), idesc, s != 0);
     }
   }
   mma_commit(bar);
 }
 
-// one thread: D = q''_hi . B_K^T + q''_lo . B_K^T with q'' in TMEM (hi at
-// column a_hi, lo 64 columns on; 8 columns per 16-element K step)
-__device__ __forceinline__ void issue_qk_ta(uint32_t d, uint32_t a_hi, uint32_t b0, uint32_t bar) {
+// one thread: D_hi = q''_hi . B_K^T and D_lo = q''_lo . B_K^T with q'' in
+// TMEM (hi at column a_hi, lo 64 columns on; 8 columns per 16-element K step)
+__device__ __forceinline__ void issue_qk_ta(uint32_t d_hi, uint32_t d_lo, uint32_t a_hi, uint32_t b0, uint32_t bar) {
   fence_after();
 #pragma unroll
   for (int hl = 0; hl < 2; ++hl)
 #pragma unroll
     for (int s = 0; s < 8; ++s)
-      mma_f16_ta(d, a_hi + 64 * hl + 8 * s, sw128_desc(b0 + (s >> 2) * kBkAtom + (s & 3) * 32), idesc_m128(kNS),
-                 (hl | s) != 0);
+      mma_f16_ta(hl ? d_lo : d_hi, a_hi + 64 * hl + 8 * s, sw128_desc(b0 + (s >> 2) * kBkAtom + (s & 3) * 32),
+                 idesc_m128(kNS), s != 0);
   mma_commit(bar);
 }
 
@@ -448,11 +455,13 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
   tbase = *tslot;
   // TMEM columns: D_S 0..79, D_O 128..255, 256..383 q' (context part), then
   // the parked context accumulator (raw part); 384..447 / 448..511 q''_hi /
-  // q''_lo as the QK MMA's A operand (row = lane, 2 fp16 per column)
+  // q''_lo as the QK MMA's A operand (row = lane, 2 fp16 per column).  The lo
+  // products of QK go to 128..207 (D_O is free then), those of PV to 0..127
+  // (D_S is free then).
   const uint32_t d_s = tbase, d_o = tbase + 128, d_park = tbase + 256, a_q = tbase + 384;
   if (F > 0) {
     if (tid == 0)
-      issue_mma(d_o, s_base + kOffAqHi, 0, 1, s_base + kOffBk, 16384, 8, idesc_m128(kHeadDim), bar_mma);
+      issue_mma(d_o, d_o, s_base + kOffAqHi, 0, 1, s_base + kOffBk, 16384, 8, idesc_m128(kHeadDim), bar_mma);
     ok = mbar_wait(bar_mma, mma_phase);
     mma_phase ^= 1u;
     fence_after();
@@ -632,7 +641,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
       fence_async_smem();
       fence_before();
       __syncthreads();
-      if (tid == 0) issue_qk_ta(d_s, a_q, s_base + kOffBk, bar_qk);
+      if (tid == 0) issue_qk_ta(d_s, d_o, a_q, s_base + kOffBk, bar_qk);
     }
   }
   for (int gb = 0; gb < NB && ok; ++gb) {
@@ -648,8 +657,19 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
     float sc[32];
     float mloc = -INFINITY;
     if (live) {
-      tmem_ld32(d_s + t_lane + 32 * eta, sc);
-      const float sig = tmem_ld1(d_s + t_lane + kBlk);
+      {
+        float lo[32];
+        tmem_ld32(d_s + t_lane + 32 * eta, sc);
+        tmem_ld32(d_o + t_lane + 32 * eta, lo);
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          const float2 v = __ffma2_rn(make_float2(lo[j], lo[j + 1]), make_float2(kLoInv, kLoInv),
+                                      make_float2(sc[j], sc[j + 1]));
+          sc[j] = v.x;
+          sc[j + 1] = v.y;
+        }
+      }
+      const float sig = tmem_ld1(d_s + t_lane + kBlk) + tmem_ld1(d_o + t_lane + kBlk) * kLoInv;
       const float2 sig2 = make_float2(sig, sig);
 #pragma unroll
       for (int j4 = 0; j4 < 8; ++j4) {
@@ -715,7 +735,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
     fence_before();
     __syncthreads();
     if (tid == 0)
-      issue_mma(d_o, s_base + kOffPHi, kOffPLo - kOffPHi, 2, s_base + kOffBv + (gb & 1) * 16384, 16384, 4,
+      issue_mma(d_o, d_s, s_base + kOffPHi, kOffPLo - kOffPHi, 2, s_base + kOffBv + (gb & 1) * 16384, 16384, 4,
                 idesc_m128(kHeadDim), bar_pv);
     l_ctx = l_ctx * alpha + red[2 * kRows + row] + red[3 * kRows + row];
     const float wtot = red[4 * kRows + row] + red[5 * kRows + row];
@@ -734,7 +754,18 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
       float x[32];
-      tmem_ld32(d_o + t_lane + 64 * eta + 32 * half, x);
+      {
+        float lo[32];
+        tmem_ld32(d_o + t_lane + 64 * eta + 32 * half, x);
+        tmem_ld32(d_s + t_lane + 64 * eta + 32 * half, lo);
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const float2 v = __ffma2_rn(make_float2(lo[i], lo[i + 1]), make_float2(kLoInv, kLoInv),
+                                      make_float2(x[i], x[i + 1]));
+          x[i] = v.x;
+          x[i + 1] = v.y;
+        }
+      }
 #pragma unroll
       for (int i4 = 0; i4 < 8; ++i4) {
         const float4 c4 = *reinterpret_cast<const float4*>(f + 128 + 64 * eta + 32 * half + 4 * i4);
@@ -762,7 +793,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
       if (tid == 0) report_error(a.dev_status, KVQ_ERR_DEVICE_TIMEOUT);
       ok = false;
     }
-    if (more && ok && tid == 0) issue_qk_ta(d_s, a_q, s_base + kOffBk, bar_qk);
+    if (more && ok && tid == 0) issue_qk_ta(d_s, d_o, a_q, s_base + kOffBk, bar_qk);
   }
 
   // ================================================================ B. raw keys
@@ -819,7 +850,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
     fence_async_smem();
     __syncthreads();
     if (tid == 0)
-      issue_mma(d_s, s_base + kOffAqHi, 0, 1, s_base + kOffBk, kBkAtom, 8, idesc_m128(kBlk), bar_mma);
+      issue_mma(d_s, d_s, s_base + kOffAqHi, 0, 1, s_base + kOffBk, kBkAtom, 8, idesc_m128(kBlk), bar_mma);
     const bool got_s = mbar_wait(bar_mma, mma_phase);
     mma_phase ^= 1u;
     fence_after();
@@ -873,7 +904,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
     fence_before();
     __syncthreads();
     if (tid == 0)
-      issue_mma(d_o, s_base + kOffPHi, kOffPLo - kOffPHi, 2, s_base + kOffBv, 16384, 4, idesc_m128(kHeadDim),
+      issue_mma(d_o, d_s, s_base + kOffPHi, kOffPLo - kOffPHi, 2, s_base + kOffBv, 16384, 4, idesc_m128(kHeadDim),
                 bar_mma);
     l_raw = l_raw * alpha + red[2 * kRows + row] + red[3 * kRows + row];
     m_raw = m_new;
@@ -882,10 +913,11 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
     fence_after();
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
-      float x[32];
+      float x[32], lo[32];
       tmem_ld32(d_o + t_lane + 64 * eta + 32 * half, x);
+      tmem_ld32(d_s + t_lane + 64 * eta + 32 * half, lo);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) racc[32 * half + i] = alpha * racc[32 * half + i] + x[i];
+      for (int i = 0; i < 32; ++i) racc[32 * half + i] = alpha * racc[32 * half + i] + (x[i] + lo[i] * kLoInv);
     }
     fence_before();
     if (__syncthreads_or(!got_o)) {
@@ -910,7 +942,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
       for (int pc = 0; pc < 4; ++pc) {
         float x[8];
 #pragma unroll
-        for (int m = 0; m < 8; ++m) x[m] = y[8 * pc + m] * w_ctx;
+        for (int m = 0; m < 8; ++m) x[m] = y[8 * pc + m] * (w_ctx * inv_l);  // bounded by max |V|
         uint4 lo;
         const uint4 hi = hi_lo_pack(x, lo);
         const int kpos = 64 * eta + 32 * half + 8 * pc;
@@ -922,7 +954,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
     fence_async_smem();
     __syncthreads();
     if (tid == 0)
-      issue_mma(d_o, s_base + kOffAqHi, kOffAqLo - kOffAqHi, 2, s_base + kOffBv, 16384, 8, idesc_m128(kHeadDim),
+      issue_mma(d_o, d_s, s_base + kOffAqHi, kOffAqLo - kOffAqHi, 2, s_base + kOffBv, 16384, 8, idesc_m128(kHeadDim),
                 bar_mma);
     const bool got = mbar_wait(bar_mma, mma_phase);
     mma_phase ^= 1u;
@@ -940,7 +972,11 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
     for (int half = 0; half < 2; ++half) {
       float x[32];
       if (have_rot) {
+        float lo[32];
         tmem_ld32(d_o + t_lane + 64 * eta + 32 * half, x);
+        tmem_ld32(d_s + t_lane + 64 * eta + 32 * half, lo);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) x[i] += lo[i] * kLoInv;
       } else {
 #pragma unroll
         for (int i = 0; i < 32; ++i) x[i] = 0.f;
@@ -953,8 +989,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
           const int i = 8 * pc + 2 * k, c = 64 * eta + 32 * half + i;
           const float r0 = x[i] * (rotation_sign(a.cfg.rotation_seed, c) / kSqrtHeadDim);
           const float r1 = x[i + 1] * (rotation_sign(a.cfg.rotation_seed, c + 1) / kSqrtHeadDim);
-          w[k] = h2_as_u32(__floats2half2_rn((r0 + racc[32 * half + i] * w_raw) * inv_l,
-                                             (r1 + racc[32 * half + i + 1] * w_raw) * inv_l));
+          w[k] = h2_as_u32(__floats2half2_rn(r0 + racc[32 * half + i] * (w_raw * inv_l),
+                                             r1 + racc[32 * half + i + 1] * (w_raw * inv_l)));
         }
         if (row < rows_valid) *reinterpret_cast<uint4*>(o + 32 * half + 8 * pc) = make_uint4(w[0], w[1], w[2], w[3]);
       }

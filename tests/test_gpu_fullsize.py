@@ -372,3 +372,52 @@ def test_mixed_batch_full_size():
                           q_h[s, head * g:(head + 1) * g])
     for j in range(g):
         assert rel_l2(out_h[s, head * g + j], ref[j]) <= ATTN_REL_L2_MAX
+
+
+def test_qwen3_4b_chunked_prefill_full_size():
+    """Chunked prefill in the launch configuration bench.py --prefill-chunk 512
+    times: the Qwen3-4B-shaped cache (6 x 131073 tokens: 2048 quantized tiles
+    and one tail token per (sequence, KV head)), 512 new tokens per sequence
+    in one kvq_paged_prefill_attention call; sampled outputs against the
+    oracle over the GPU's own pages and the raw chunk rows."""
+    w = synth.workload("qwen3_4b")
+    cfg, cache = make_cache(w, extra_tokens=512)
+    total = int(sum(w.lens))
+    rk = synth.kv_rows(w, "k", total, device="cuda")
+    rv = synth.kv_rows(w, "v", total, device="cuda")
+    cache.prefill(rk, rv, w.lens)
+    del rk, rv
+    cache.append(synth.kv_rows(w, "k", w.num_seqs, device="cuda", stream_id=1),
+                 synth.kv_rows(w, "v", w.num_seqs, device="cuda", stream_id=1))
+    n = 512
+    k_new = synth.kv_rows(w, "k", w.num_seqs * n, device="cuda", stream_id=7)
+    v_new = synth.kv_rows(w, "v", w.num_seqs * n, device="cuda", stream_id=7)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(w.seed * 1000 + 9)
+    q = torch.randn((w.num_seqs * n, w.num_q_heads, 128), generator=g, device="cuda").to(torch.float16)
+    out = cache.prefill_chunk(q, k_new, v_new, [n] * w.num_seqs, append=False)
+    torch.cuda.synchronize()
+    assert cache.status() == 0
+    oh, qh = out.float().cpu().numpy(), q.float().cpu().numpy()
+    kh, vh = k_new.cpu().numpy(), v_new.cpu().numpy()
+    assert np.all(np.isfinite(oh))
+    length = w.lens[0] + 1
+    t = cfg.tile_tokens
+    gsz = w.group_size
+    for seq, head in [(0, 0), (4, 6)]:
+        hat = []
+        for is_v in (False, True):
+            tiles = _gpu_tiles(cache, cfg, seq, range(length // t), head, is_v)
+            tail = (cache.v_tail if is_v else cache.k_tail)[seq, head, :length % t].cpu().numpy()
+            hat.append(o.sequence_kv_hat(tiles, tail))
+        base = seq * n
+        for i in (0, 1, 127, 128, 511):
+            # chunk token i: rows 0..i-1 of the chunk join the context as raw rows
+            k_ctx = [np.concatenate([hat[0], kh[base:base + i, head].astype(np.float64)])]
+            v_ctx = [np.concatenate([hat[1], vh[base:base + i, head].astype(np.float64)])]
+            ref = o.prefill_chunk_sequence(qh[base + i:base + i + 1, head * gsz:(head + 1) * gsz], k_ctx, v_ctx,
+                                           kh[base + i:base + i + 1, head:head + 1],
+                                           vh[base + i:base + i + 1, head:head + 1], gsz)
+            for j in range(gsz):
+                err = rel_l2(oh[base + i, head * gsz + j], ref[0, j])
+                assert err <= ATTN_REL_L2_MAX, ("prefill", seq, head, i, j, err)
