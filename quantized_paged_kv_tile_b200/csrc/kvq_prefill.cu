@@ -498,8 +498,9 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
 
   // tile t, shared memory only: wait for its pages (skipped when outside the
   // pool: the tile's blocks then run with zero scalars and masked scores),
-  // stage the tile scalars as floats; starts the copies of tile t+1.
-  // Block-uniform; false on a timeout.
+  // stage the tile scalars as floats; starts the copies of tile t+1.  Has no
+  // barrier of its own: returns this thread's wait result, which the caller
+  // folds into its next barrier (that barrier also publishes the scalars).
   auto prep_scalars = [&](int t) -> bool {
     const int st = t & 1;
     if (warp == 0 && t + 1 < F) issue(t + 1, st ^ 1);
@@ -509,10 +510,6 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
       got = mbar_wait(bar_stage0 + 8 * st, (st_phase >> st) & 1u);
       st_phase ^= 1u << st;
       if (got) issued &= ~(1u << st);
-    }
-    if (__syncthreads_or(!got)) {
-      if (tid == 0) report_error(a.dev_status, KVQ_ERR_DEVICE_TIMEOUT);
-      return false;
     }
     const unsigned char* sK = smem + kOffStage + st * Geo::kStage;
     const unsigned char* sV = sK + NP * Geo::kPageK;
@@ -535,7 +532,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
       f[640 + tok] = v2.y;
     }
     if (tid == 0) tile_bad[st] = bad;
-    return true;
+    return got;
   };
   // tile t's q'' = q' * C~K (hi / lo) into TMEM in the QK channel order; the
   // scalars of tile t must be visible (a barrier after prep_scalars)
@@ -633,10 +630,13 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
   };
 
   if (NB > 0 && ok) {
-    ok = prep_scalars(0);
+    const bool got0 = prep_scalars(0);
+    unpack_block(0);
+    if (__syncthreads_or(!got0)) {  // scalars of tile 0 visible
+      if (tid == 0) report_error(a.dev_status, KVQ_ERR_DEVICE_TIMEOUT);
+      ok = false;
+    }
     if (ok) {
-      unpack_block(0);
-      __syncthreads();  // scalars of tile 0 visible
       build_qpp(0);
       fence_async_smem();
       fence_before();
@@ -744,8 +744,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
     // tile change, the next tile's scalars
     const bool more = gb + 1 < NB;
     const bool new_tile = more && (gb + 1) % Geo::kBlocks == 0;
-    if (new_tile) ok = prep_scalars((gb + 1) / Geo::kBlocks);
-    if (more && ok) unpack_block(gb + 1);
+    const bool got_t = new_tile ? prep_scalars((gb + 1) / Geo::kBlocks) : true;
+    if (more) unpack_block(gb + 1);  // (garbage after a timed-out wait; dropped below)
     // -- fold D_O into the accumulators: acc'_c = alpha acc'_c + C~V_c (D_c + sum p z~V)
     const bool got_o = mbar_wait(bar_pv, pv_phase);
     pv_phase ^= 1u;
@@ -781,11 +781,14 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
       }
     }
     // -- no MMA in flight: the next tile's q'' into TMEM, then QK(gb+1)
-    if (new_tile && ok) {
+    if (new_tile) {
       fence_before();
-      __syncthreads();  // next tile's scalars visible; D_O reads done
+      if (__syncthreads_or(!got_t)) {  // next tile's scalars visible; D_O reads done
+        if (tid == 0) report_error(a.dev_status, KVQ_ERR_DEVICE_TIMEOUT);
+        ok = false;
+      }
       fence_after();
-      build_qpp((gb + 1) / Geo::kBlocks);
+      if (ok) build_qpp((gb + 1) / Geo::kBlocks);
     }
     fence_async_smem();
     fence_before();
