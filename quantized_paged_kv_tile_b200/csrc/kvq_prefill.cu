@@ -7,30 +7,35 @@
 // query rows of a (sequence, KV head) are the chunk tokens x the g query heads
 // of that KV head, token-major: row i*g + j is chunk token i, head j.  Warp w
 // owns TMEM lanes 32 (w % 4) .. +31 (one query row per thread) and column half
-// w / 4.  Every contraction runs on the tcgen05 tensor cores (fp16 operands in
-// shared memory, 128-byte swizzle, K-major; fp32 accumulators in TMEM; one
-// thread issues, a commit to an mbarrier signals completion):
+// w / 4 (32 of a block's 64 tokens in the softmax, 64 of the 128 channels in
+// the accumulators).  Every contraction runs on the tcgen05 tensor cores (fp16
+// operands, K-major with the 128-byte swizzle in shared memory or row-per-lane
+// in TMEM; fp32 accumulators in TMEM; one thread issues, a commit to an
+// mbarrier signals completion).  fp32 operands enter as hi + lo * 2^-11 fp16
+// pairs whose two products accumulate separately (see hi_lo2).
 //
 // A. Context tiles, rotated domain.  q' = q D_s H (one MMA against H, scaled
-//    into the log2 domain) and per tile of the context, exactly as the decode
-//    kernel's algebra:
+//    into the log2 domain, kept in TMEM) and per tile of the context, the
+//    decode kernel's algebra:
 //      score_i = s~K_i (q'' . codeK_i) + z~K_i sum_j q''_j,   q'' = q' * C~K_t
 //      acc'_j += C~V_tj (sum_i p_i s~V_i codeV_ij + sum_i p_i z~V_i)
-//    QK: D_S[128][80] = q''_hi . B_K^T + q''_lo . B_K^T, B_K = the block's 64
-//    tokens of K codes as exact fp16 integers, a row of ones (column 64 of D_S
-//    is then sum_j q''_j) and zero rows.  PV: D_O[128][128] = P_hi . B_V^T +
-//    P_lo . B_V^T, P = p * s~V, B_V = V codes channel-major.  The hi / lo
-//    halves keep q'' and P fp32-accurate on fp16 operands; the codes are
-//    exact.  C~V scales D_O's columns per tile, so D_O is folded into register
-//    accumulators block by block.  Tiles are staged whole (K and V pages) by
-//    cp.async.bulk, double-buffered.
+//    QK (per 64-token block): D_S[128][80] = q''_hi . B_K^T and its lo twin,
+//    with q'' built per tile into TMEM as the A operand and B_K = the block's
+//    K codes as exact fp16 integers, a row of ones (column 64 is then
+//    sum_j q''_j) and zero rows.  PV: D_O[128][128] = P_hi . B_V^T and its lo
+//    twin, P = p * s~V, B_V = V codes channel-major (exact).  C~V scales D_O's
+//    columns per tile, so D_O is folded into register accumulators block by
+//    block.  Tiles are staged whole (K and V pages) by cp.async.bulk, double-
+//    buffered; PV runs while the next block's codes are unpacked, and no TMEM
+//    load overlaps an MMA that writes TMEM.
 // B. Raw keys, original domain: the fp16 tail of the cache, then the chunk's
 //    own rows, causal (chunk token i sees tail + chunk rows 0..i).  QK: q
 //    (fp16, exact) . K_raw^T; PV: P_hi / P_lo . V_raw^T (V transposed into
-//    shared memory).  Separate running max / sum / accumulator.
+//    shared memory).  Separate running max / sum / accumulator; the context
+//    accumulator waits in TMEM meanwhile.
 // C. The two parts are merged by their log-sum-exp weights; the rotated part
-//    is taken back with one MMA against H (hi / lo halves of acc'), then the
-//    channel signs and 1/sqrt(d); fp16 output.
+//    (already divided by the softmax sum) is taken back with one MMA against H,
+//    then the channel signs and 1/sqrt(d); fp16 output.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -490,9 +495,11 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
   }
 
   // ================================================================ A. context tiles
-  // Software pipeline over the context's 64-token blocks gb = 0 .. NB-1: the
-  // operands of block gb+1 are built while PV(gb) runs on the tensor cores,
-  // and block gb's accumulator update overlaps QK(gb+1).
+  // Loop over the context's 64-token blocks gb = 0 .. NB-1.  Block gb+1's
+  // codes (and, on a tile change, the next tile's scalars) are unpacked in
+  // shared memory while PV(gb) runs; the TMEM reads of the accumulator fold
+  // and the next tile's q'' build wait until no MMA is in flight (an MMA
+  // writing TMEM slows concurrent tcgen05.ld), then QK(gb+1) is issued.
   const int NB = F * Geo::kBlocks;
   uint32_t st_phase = 0u, qk_phase = 0u, pv_phase = 0u;  // st_phase bit s: stage s
 
