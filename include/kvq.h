@@ -287,7 +287,8 @@ KVQ_API kvq_status kvq_unpack_tiles(const kvq_config* cfg, const int32_t* tile_d
  * mbarrier wait on a barrier nothing ever arrives at.  Each wait gives up
  * after its limit (2 s) and records KVQ_ERR_DEVICE_TIMEOUT in *dev_status
  * (device int32, required); nothing traps and the context stays usable.
- * Takes about 4 s of device time.  Returns KVQ_ERR_INVALID_ARG for a NULL
+ * Three such waits (quantize, decode, prefill kernels): about 6 s of device
+ * time.  Returns KVQ_ERR_INVALID_ARG for a NULL
  * dev_status, KVQ_ERR_CUDA on a launch error. */
 KVQ_API kvq_status kvq_selftest_bounded_wait(int32_t* dev_status, void* stream);
 

@@ -362,7 +362,8 @@ kvq_status kvq_selftest_bounded_wait(int32_t* dev_status, void* stream) {
   if (dev_status == nullptr) return fail(KVQ_ERR_INVALID_ARG, "dev_status is NULL");
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   KVQ_TRY(cuda_status(kvq::launch_selftest_wait_quantize(dev_status, s), "quantize wait self-test launch"));
-  return cuda_status(kvq::launch_selftest_wait_decode(dev_status, s), "decode wait self-test launch");
+  KVQ_TRY(cuda_status(kvq::launch_selftest_wait_decode(dev_status, s), "decode wait self-test launch"));
+  return cuda_status(kvq::launch_selftest_wait_prefill(dev_status, s), "prefill wait self-test launch");
 }
 
 }  // extern "C"

@@ -139,5 +139,6 @@ cudaError_t launch_paged_prefill(const PrefillArgs& a, cudaStream_t s);
 // KVQ_ERR_DEVICE_TIMEOUT in *dev_status.
 cudaError_t launch_selftest_wait_quantize(int32_t* dev_status, cudaStream_t s);
 cudaError_t launch_selftest_wait_decode(int32_t* dev_status, cudaStream_t s);
+cudaError_t launch_selftest_wait_prefill(int32_t* dev_status, cudaStream_t s);
 
 }  // namespace kvq

@@ -1015,6 +1015,17 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
   if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tbase), "r"(512));
 }
 
+// ---------------------------------------------------------------- self-test
+// One thread waits, with this kernel's bounded wait, on a barrier that nothing
+// arrives at; the wait gives up after its limit and the timeout is recorded.
+__global__ void selftest_wait_prefill_kernel(int32_t* dev_status) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = smem_u32(&bar);
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(b));
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  if (!mbar_wait(b, 0)) report_error(dev_status, KVQ_ERR_DEVICE_TIMEOUT);
+}
+
 template <int T, int BK, int BV>
 cudaError_t launch_t(const PrefillArgs& a, cudaStream_t s, long long units) {
   using Geo = PfGeom<T, BK, BV>;
@@ -1038,6 +1049,11 @@ cudaError_t launch_bits(const PrefillArgs& a, cudaStream_t s, long long units) {
 
 int prefill_row_tiles(const kvq_config& cfg, int max_chunk) {
   return static_cast<int>((static_cast<long long>(max_chunk) * cfg.group_size + kRows - 1) / kRows);
+}
+
+cudaError_t launch_selftest_wait_prefill(int32_t* dev_status, cudaStream_t s) {
+  selftest_wait_prefill_kernel<<<1, 1, 0, s>>>(dev_status);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_paged_prefill(const PrefillArgs& a, cudaStream_t s) {

@@ -275,7 +275,7 @@ def paged_decode_attention_static_scratch(cfg: Config, q, out, seq_lens, block_t
 
 
 def selftest_bounded_wait(dev_status, stream=None) -> None:
-    """Run the device-side bounded-wait self-test (about 4 s): afterwards
+    """Run the device-side bounded-wait self-test (about 6 s): afterwards
     ``dev_status`` holds KVQ_ERR_DEVICE_TIMEOUT."""
     st = load_library().kvq_selftest_bounded_wait(_ptr(dev_status, "dev_status", torch.int32), _stream(stream))
     _check(st, "kvq_selftest_bounded_wait")

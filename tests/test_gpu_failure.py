@@ -26,8 +26,8 @@ def test_bounded_wait_times_out_and_reports():
     torch.cuda.synchronize()
     elapsed = time.monotonic() - t0
     assert int(status.item()) == kvq.KVQ_ERR_DEVICE_TIMEOUT
-    assert 3.5 < elapsed < 30.0  # two waits of the kernels' 2 s limit
-    # the context keeps working: a normal prefill + decode afterwards
+    assert 5.5 < elapsed < 40.0  # three waits (quantize, decode, prefill) of the kernels' 2 s limit
+    # the context keeps working: a normal prefill + decode + chunked prefill afterwards
     w = synth.workload("tiny", lens=(200,))
     cfg, cache = make_cache(w)
     rk = synth.kv_rows(w, "k", 200, device="cuda")
@@ -41,4 +41,14 @@ def test_bounded_wait_times_out_and_reports():
     out_h = out.float().cpu().numpy()[0]
     for h in range(w.num_q_heads):
         assert rel_l2(out_h[h], ref[h]) <= ATTN_REL_L2_MAX
+    # a one-token chunk (raw) over the same cache equals that decode with the token appended first
+    ck = synth.kv_rows(w, "k", 1, device="cuda", stream_id=4)
+    cv = synth.kv_rows(w, "v", 1, device="cuda", stream_id=4)
+    pout = cache.prefill_chunk(q, ck, cv, [1], append=True)
+    dout = cache.decode(q)
+    torch.cuda.synchronize()
+    assert cache.status() == 0
+    p_h, d_h = pout.float().cpu().numpy()[0], dout.float().cpu().numpy()[0]
+    for h in range(w.num_q_heads):
+        assert rel_l2(p_h[h], d_h[h]) <= ATTN_REL_L2_MAX
 
