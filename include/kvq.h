@@ -224,6 +224,17 @@ KVQ_API kvq_status kvq_paged_decode_attention(const kvq_config* cfg, const void*
  *   ctx_lens     : device int32 [num_seqs], tokens cached before the chunk.
  *   max_chunk_tokens: host bound >= every chunk length (sizes the launch:
  *                  one CTA per sequence, KV head and 128 query rows).
+ *   block_tables, k_pool, v_pool, k_tail, v_tail, num_blocks: the cache, as
+ *                  for kvq_paged_decode_attention.
+ *   softmax_scale: scale of q.k (1/sqrt(d) in the method).
+ *   dev_status   : device int32, may be NULL; first device-detected error.
+ *   stream       : cudaStream_t (NULL = legacy default stream); the call is
+ *                  asynchronous on it.
+ * All buffers are caller-owned device memory, 16-byte aligned; the library
+ * keeps no pointer after the call.  Host-side checks (config, NULL or
+ * misaligned pointers, num_seqs outside 0..65535, max_chunk_tokens outside
+ * 0..2^20, a non-positive or non-finite scale) return KVQ_ERR_INVALID_ARG /
+ * KVQ_ERR_UNSUPPORTED before any launch.
  * No workspace: each CTA merges its context and chunk parts itself.
  * The chunk is not appended: call kvq_append_tokens with the same rows and
  * cu_chunk afterwards (tiles it completes are then quantized).  A chunk
