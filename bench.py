@@ -435,7 +435,7 @@ def run_kvq(args, ranks):
     if args.prefill_chunk > 0:
         line["prefill"] = prefill_leg(w, cfg, args, dev, stream, seq_lens, bt, nblocks, k_pool, v_pool, k_tail,
                                       v_tail, status, lens1)
-        line["gpu_launches_prefill"] = args.steps
+        line["gpu_launches_prefill"] = args.steps * line["prefill"]["launches_per_call"]
     return line
 
 
@@ -455,9 +455,14 @@ def prefill_leg(w, cfg, args, dev, stream, seq_lens, bt, nblocks, k_pool, v_pool
     out = torch.empty_like(q)
     cu = torch.arange(0, B * n + 1, n, dtype=torch.int32, device=dev)
 
+    splits = kvq.prefill_splits(cfg, B, n, int(lens1.max()), torch.cuda.get_device_properties(dev).multi_processor_count)
+    need = kvq.prefill_workspace_bytes(cfg, B, n, splits)
+    ws = torch.empty(need, dtype=torch.uint8, device=dev) if need > 0 else None
+
     def call():
         kvq.paged_prefill_attention(cfg, q, out, k_new, v_new, cu, seq_lens, n, bt, k_pool, v_pool, k_tail, v_tail,
-                                    num_blocks=nblocks, dev_status=status, stream=stream)
+                                    num_splits=splits, workspace=ws, num_blocks=nblocks, dev_status=status,
+                                    stream=stream)
 
     for _ in range(args.warmup):
         call()
@@ -475,6 +480,7 @@ def prefill_leg(w, cfg, args, dev, stream, seq_lens, bt, nblocks, k_pool, v_pool
     peak, kind = tensor_peak()
     tflops = flops / (ms * 1e-3) / 1e12
     return {"chunk_tokens": n, "ms": ms, "chunk_tok_per_s": B * n / (ms * 1e-3), "flops": flops,
+            "context_splits": splits, "launches_per_call": 1 if splits == 1 else 2,
             "context": f"{B} seqs x {int(lens1[0])} cached tokens (quantized tiles + fp16 tail)",
             "roofline": {"bound": "tensor", "kernel": "prefill_attn_kernel", "achieved": tflops, "peak": peak,
                          "peak_kind": kind, "unit": "TFLOP/s", "frac": tflops / peak, "traffic": None,

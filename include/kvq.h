@@ -208,6 +208,11 @@ KVQ_API kvq_status kvq_paged_decode_attention(const kvq_config* cfg, const void*
                                       size_t workspace_bytes, int num_splits,
                                       int32_t* dev_status, void* stream);
 
+/* Bytes of device workspace kvq_paged_prefill_attention needs with num_splits
+ * context splits (0 for num_splits = 1).  cfg, bytes: host pointers. */
+KVQ_API kvq_status kvq_prefill_workspace_bytes(const kvq_config* cfg, int num_seqs, int max_chunk_tokens,
+                                               int num_splits, size_t* bytes);
+
 /* Read path, chunked prefill: attention of a chunk of new tokens per sequence
  * over the quantized cache and the chunk itself.  The method reads the
  * compressed pages directly in every phase of attention (aitrends.kr article
@@ -223,7 +228,19 @@ KVQ_API kvq_status kvq_paged_decode_attention(const kvq_config* cfg, const void*
  *   cu_chunk     : device int32 [num_seqs+1], prefix sums of chunk lengths.
  *   ctx_lens     : device int32 [num_seqs], tokens cached before the chunk.
  *   max_chunk_tokens: host bound >= every chunk length (sizes the launch:
- *                  one CTA per sequence, KV head and 128 query rows).
+ *                  one CTA per sequence, KV head and 128 query rows, times
+ *                  num_splits).
+ *   num_splits   : 1..64.  1: one launch, each CTA runs its whole context.
+ *                  S > 1: the context tiles of each (sequence, KV head, row
+ *                  tile) are split over S CTAs that write partial softmax
+ *                  states to the workspace, then a second launch merges them
+ *                  (log-sum-exp) and adds the tail and the chunk rows; the
+ *                  result does not depend on S beyond rounding.  More CTAs
+ *                  fill the device when (sequences x KV heads x row tiles) is
+ *                  small or leaves a partial last wave.
+ *   workspace    : device, >= kvq_prefill_workspace_bytes(cfg, num_seqs,
+ *                  max_chunk_tokens, num_splits) bytes (may be NULL when that
+ *                  is 0); contents on entry are ignored.
  *   block_tables, k_pool, v_pool, k_tail, v_tail, num_blocks: the cache, as
  *                  for kvq_paged_decode_attention.
  *   softmax_scale: scale of q.k (1/sqrt(d) in the method).
@@ -233,9 +250,9 @@ KVQ_API kvq_status kvq_paged_decode_attention(const kvq_config* cfg, const void*
  * All buffers are caller-owned device memory, 16-byte aligned; the library
  * keeps no pointer after the call.  Host-side checks (config, NULL or
  * misaligned pointers, num_seqs outside 0..65535, max_chunk_tokens outside
- * 0..2^20, a non-positive or non-finite scale) return KVQ_ERR_INVALID_ARG /
- * KVQ_ERR_UNSUPPORTED before any launch.
- * No workspace: each CTA merges its context and chunk parts itself.
+ * 0..2^20, num_splits outside 1..64, a non-positive or non-finite scale)
+ * return KVQ_ERR_INVALID_ARG / KVQ_ERR_UNSUPPORTED, a short workspace
+ * KVQ_ERR_WORKSPACE, before any launch.
  * The chunk is not appended: call kvq_append_tokens with the same rows and
  * cu_chunk afterwards (tiles it completes are then quantized).  A chunk
  * longer than max_chunk_tokens, or negative, is reported through dev_status
@@ -248,6 +265,7 @@ KVQ_API kvq_status kvq_paged_prefill_attention(const kvq_config* cfg, const void
                                        const int32_t* block_tables, int max_blocks_per_seq,
                                        int num_blocks, const void* k_pool, const void* v_pool,
                                        const void* k_tail, const void* v_tail, float softmax_scale,
+                                       int num_splits, void* workspace, size_t workspace_bytes,
                                        int32_t* dev_status, void* stream);
 
 /* Size of the scratch array built into the library for

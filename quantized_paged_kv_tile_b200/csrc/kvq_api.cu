@@ -266,22 +266,34 @@ kvq_status kvq_paged_decode_attention(const kvq_config* cfg, const void* q, void
                      "kvq_paged_decode_attention launch");
 }
 
+kvq_status kvq_prefill_workspace_bytes(const kvq_config* cfg, int num_seqs, int max_chunk_tokens, int num_splits,
+                                       size_t* bytes) {
+  KVQ_TRY(check_config(cfg));
+  if (bytes == nullptr) return fail(KVQ_ERR_INVALID_ARG, "bytes is NULL");
+  if (num_seqs < 0 || max_chunk_tokens < 0) return fail(KVQ_ERR_INVALID_ARG, "negative num_seqs or max_chunk_tokens");
+  if (num_splits < 1 || num_splits > 64) return fail(KVQ_ERR_INVALID_ARG, "num_splits must be 1..64");
+  *bytes = kvq::prefill_workspace_bytes(*cfg, num_seqs, max_chunk_tokens, num_splits);
+  return ok();
+}
+
 kvq_status kvq_paged_prefill_attention(const kvq_config* cfg, const void* q, void* out, const void* k_new,
                                        const void* v_new, const int32_t* cu_chunk, const int32_t* ctx_lens,
                                        int num_seqs, int max_chunk_tokens, const int32_t* block_tables,
                                        int max_blocks_per_seq, int num_blocks, const void* k_pool,
                                        const void* v_pool, const void* k_tail, const void* v_tail,
-                                       float softmax_scale, int32_t* dev_status, void* stream) {
+                                       float softmax_scale, int num_splits, void* workspace,
+                                       size_t workspace_bytes, int32_t* dev_status, void* stream) {
   KVQ_TRY(check_config(cfg));
   if (cfg->bits_k == 3 || cfg->bits_v == 3)
     return fail(KVQ_ERR_UNSUPPORTED, "prefill attention reads 2-, 4- or 8-bit codes only (3-bit pages are storage-only)");
+  if (num_splits < 1 || num_splits > 64) return fail(KVQ_ERR_INVALID_ARG, "num_splits must be 1..64");
   if (num_seqs < 0 || max_chunk_tokens < 0) return fail(KVQ_ERR_INVALID_ARG, "negative num_seqs or max_chunk_tokens");
   if (num_seqs == 0 || max_chunk_tokens == 0) return ok();
   if (num_seqs > 65535) return fail(KVQ_ERR_INVALID_ARG, "num_seqs > 65535");
   if (max_chunk_tokens > (1 << 20)) return fail(KVQ_ERR_INVALID_ARG, "max_chunk_tokens > 2^20");
   const long long units = static_cast<long long>(num_seqs) * cfg->num_kv_heads * kvq::prefill_row_tiles(*cfg, max_chunk_tokens);
-  if (units > 0x7fffffffLL)
-    return fail(KVQ_ERR_INVALID_ARG, "num_seqs x max_chunk_tokens too large for one launch");
+  if (units * num_splits > 0x7fffffffLL)
+    return fail(KVQ_ERR_INVALID_ARG, "num_seqs x max_chunk_tokens x num_splits too large for one launch");
   if (!(softmax_scale > 0.f) || !(softmax_scale < 1e30f))
     return fail(KVQ_ERR_INVALID_ARG, "softmax_scale must be a positive finite float");
   KVQ_TRY(check_ptr(q, "q"));
@@ -295,6 +307,10 @@ kvq_status kvq_paged_prefill_attention(const kvq_config* cfg, const void* q, voi
   KVQ_TRY(check_ptr(v_pool, "v_pool"));
   KVQ_TRY(check_ptr(k_tail, "k_tail"));
   KVQ_TRY(check_ptr(v_tail, "v_tail"));
+  const size_t need = kvq::prefill_workspace_bytes(*cfg, num_seqs, max_chunk_tokens, num_splits);
+  KVQ_TRY(check_ptr(workspace, "workspace", need == 0));
+  if (workspace_bytes < need)
+    return fail(KVQ_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, need);
   KVQ_TRY(check_ptr(dev_status, "dev_status", true));
   kvq::PrefillArgs a{};
   a.cfg = *cfg;
@@ -315,6 +331,8 @@ kvq_status kvq_paged_prefill_attention(const kvq_config* cfg, const void* q, voi
   a.k_tail = k_tail;
   a.v_tail = v_tail;
   a.softmax_scale = softmax_scale;
+  a.num_splits = num_splits;
+  a.partials = static_cast<float*>(workspace);
   a.dev_status = dev_status;
   return cuda_status(kvq::launch_paged_prefill(a, static_cast<cudaStream_t>(stream)),
                      "kvq_paged_prefill_attention launch");

@@ -129,9 +129,13 @@ struct PrefillArgs {
   const void* k_tail;
   const void* v_tail;
   float softmax_scale;
+  int num_splits;            // context splits per (sequence, KV head, row tile); 1: one fused launch
+  int mode;                  // 0 fused; 1 split partials (grid units x splits); 2 combine (grid units)
+  float* partials;           // workspace for splits > 1: [units][splits][128][4 + d] floats
   int32_t* dev_status;
 };
 int prefill_row_tiles(const kvq_config& cfg, int max_chunk);
+size_t prefill_workspace_bytes(const kvq_config& cfg, int num_seqs, int max_chunk, int num_splits);
 cudaError_t launch_paged_prefill(const PrefillArgs& a, cudaStream_t s);
 
 // Self-tests of the bounded mbarrier waits (one per kernel file): a wait on

@@ -369,7 +369,10 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
   const int row = 32 * quad + lane;            // this thread's query row (TMEM lane)
   const int G = a.cfg.group_size, nh = a.cfg.num_kv_heads;
   const int R = a.row_tiles;
-  const int rt = blockIdx.x % R, bh = blockIdx.x / R;
+  // mode 1: CTA = (unit, split of the context tiles); modes 0 and 2: CTA = unit
+  const int S = a.mode == 1 ? a.num_splits : 1;
+  const int unit = blockIdx.x / S, split = blockIdx.x % S;
+  const int rt = unit % R, bh = unit / R;
   const int h = bh % nh, b = bh / nh;
   const int c0 = a.cu_chunk[b];
   const int n = a.cu_chunk[b + 1] - c0;
@@ -379,6 +382,11 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
   if (rows_valid <= 0) return;
   const int L = max(a.ctx_lens[b], 0);
   const int F = L / T, tau = L - F * T;
+  // the context tiles this CTA runs through: all (mode 0), its split's share
+  // (mode 1), none (mode 2: it combines the splits' partials instead)
+  const int t_lo = a.mode == 1 ? static_cast<int>(static_cast<long long>(F) * split / S) : 0;
+  const int t_hi = a.mode == 1 ? static_cast<int>(static_cast<long long>(F) * (split + 1) / S) : (a.mode == 0 ? F : 0);
+  const int Fr = t_hi - t_lo;
   // chunk token of this thread's row (rows past the chunk take the last one)
   const int i_row = (rt * kRows + min(row, rows_valid - 1)) / G;
   const int i_max = (rt * kRows + rows_valid - 1) / G;
@@ -440,7 +448,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
     issued |= 1u << st;
   };
   __syncthreads();  // barriers initialised
-  if (warp == 0 && F > 0) issue(0, 0);
+  if (warp == 0 && Fr > 0) issue(t_lo, 0);
 
   const uint32_t t_lane = static_cast<uint32_t>(32 * quad) << 16;
   uint32_t tbase = 0, mma_phase = 0;
@@ -464,7 +472,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
   // products of QK go to 128..207 (D_O is free then), those of PV to 0..127
   // (D_S is free then).
   const uint32_t d_s = tbase, d_o = tbase + 128, d_park = tbase + 256, a_q = tbase + 384;
-  if (F > 0) {
+  if (Fr > 0) {
     if (tid == 0)
       issue_mma(d_o, d_o, s_base + kOffAqHi, 0, 1, s_base + kOffBk, 16384, 8, idesc_m128(kHeadDim), bar_mma);
     ok = mbar_wait(bar_mma, mma_phase);
@@ -500,7 +508,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
   // shared memory while PV(gb) runs; the TMEM reads of the accumulator fold
   // and the next tile's q'' build wait until no MMA is in flight (an MMA
   // writing TMEM slows concurrent tcgen05.ld), then QK(gb+1) is issued.
-  const int NB = F * Geo::kBlocks;
+  const int NB = Fr * Geo::kBlocks;  // tile indices below are relative to t_lo
   uint32_t st_phase = 0u, qk_phase = 0u, pv_phase = 0u;  // st_phase bit s: stage s
 
   // tile t, shared memory only: wait for its pages (skipped when outside the
@@ -510,7 +518,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
   // folds into its next barrier (that barrier also publishes the scalars).
   auto prep_scalars = [&](int t) -> bool {
     const int st = t & 1;
-    if (warp == 0 && t + 1 < F) issue(t + 1, st ^ 1);
+    if (warp == 0 && t + 1 < Fr) issue(t_lo + t + 1, st ^ 1);
     const bool bad = stage_bad[st] != 0;
     bool got = true;
     if (!bad) {
@@ -806,6 +814,47 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
     if (more && ok && tid == 0) issue_qk_ta(d_s, d_o, a_q, s_base + kOffBk, bar_qk);
   }
 
+  if (a.mode == 1) {  // split partial: (m, l, acc') of this row over the split's tiles
+    if (row < rows_valid) {
+      float* part = a.partials + (static_cast<size_t>(blockIdx.x) * kRows + row) * (4 + kHeadDim);
+      if (eta == 0) *reinterpret_cast<float2*>(part) = make_float2(m_ctx, l_ctx);
+#pragma unroll
+      for (int i = 0; i < 64; i += 4)
+        *reinterpret_cast<float4*>(part + 4 + 64 * eta + i) = make_float4(acc[i], acc[i + 1], acc[i + 2], acc[i + 3]);
+    }
+    if (!ok && warp == 0) {  // let copies in flight land before the shared memory is released
+      for (int s = 0; s < 2; ++s)
+        if (issued & (1u << s)) (void)mbar_wait(bar_stage0 + 8 * s, (st_phase >> s) & 1u);
+    }
+    fence_before();
+    __syncthreads();
+    if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tbase), "r"(512));
+    return;
+  }
+  if (a.mode == 2 && F > 0 && row < rows_valid) {  // combine the splits' partials (log-sum-exp)
+    const float* part0 = a.partials + (static_cast<size_t>(unit) * a.num_splits * kRows + row) * (4 + kHeadDim);
+    const size_t sstride = static_cast<size_t>(kRows) * (4 + kHeadDim);
+    for (int sp = 0; sp < a.num_splits; ++sp) {
+      const float2 ml = *reinterpret_cast<const float2*>(part0 + sp * sstride);
+      if (ml.y > 0.f) m_ctx = fmaxf(m_ctx, ml.x);
+    }
+    for (int sp = 0; sp < a.num_splits; ++sp) {
+      const float* pp = part0 + sp * sstride;
+      const float2 ml = *reinterpret_cast<const float2*>(pp);
+      if (!(ml.y > 0.f)) continue;
+      const float wgt = ex2(ml.x - m_ctx);
+      l_ctx += wgt * ml.y;
+#pragma unroll
+      for (int i = 0; i < 64; i += 4) {
+        const float4 v = *reinterpret_cast<const float4*>(pp + 4 + 64 * eta + i);
+        acc[i] += wgt * v.x;
+        acc[i + 1] += wgt * v.y;
+        acc[i + 2] += wgt * v.z;
+        acc[i + 3] += wgt * v.w;
+      }
+    }
+  }
+
   // ================================================================ B. raw keys
   // keys j: the tail (j < tau), then chunk rows j - tau; row i sees j <= tau + i.
   // The context accumulator waits in TMEM meanwhile.
@@ -1056,13 +1105,34 @@ cudaError_t launch_selftest_wait_prefill(int32_t* dev_status, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+size_t prefill_workspace_bytes(const kvq_config& cfg, int num_seqs, int max_chunk, int num_splits) {
+  if (num_splits <= 1) return 0;
+  const size_t units = static_cast<size_t>(num_seqs) * cfg.num_kv_heads * prefill_row_tiles(cfg, max_chunk);
+  return units * num_splits * kRows * (4 + kHeadDim) * sizeof(float);
+}
+
+template <int T>
+cudaError_t launch_modes(const PrefillArgs& a, cudaStream_t s, long long units) {
+  if (a.num_splits <= 1) {
+    PrefillArgs f = a;
+    f.mode = 0;
+    return launch_bits<T>(f, s, units);
+  }
+  PrefillArgs p = a;
+  p.mode = 1;
+  cudaError_t e = launch_bits<T>(p, s, units * a.num_splits);
+  if (e != cudaSuccess) return e;
+  p.mode = 2;
+  return launch_bits<T>(p, s, units);
+}
+
 cudaError_t launch_paged_prefill(const PrefillArgs& a, cudaStream_t s) {
   const long long units = static_cast<long long>(a.num_seqs) * a.cfg.num_kv_heads * a.row_tiles;
   if (units == 0) return cudaSuccess;
   switch (a.cfg.tile_tokens) {
-    case 32: return launch_bits<32>(a, s, units);
-    case 64: return launch_bits<64>(a, s, units);
-    default: return launch_bits<128>(a, s, units);
+    case 32: return launch_modes<32>(a, s, units);
+    case 64: return launch_modes<64>(a, s, units);
+    default: return launch_modes<128>(a, s, units);
   }
 }
 

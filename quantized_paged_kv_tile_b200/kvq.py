@@ -30,7 +30,7 @@ EXPORTED_SYMBOLS = (
     "kvq_get_layout", "kvq_decode_workspace_bytes", "kvq_quantize_tiles", "kvq_append_tokens",
     "kvq_paged_decode_attention", "kvq_paged_decode_attention_static_scratch", "kvq_unpack_tiles",
     "kvq_selftest_bounded_wait", "kvq_status_string", "kvq_last_error", "kvq_version",
-    "kvq_paged_prefill_attention",
+    "kvq_prefill_workspace_bytes", "kvq_paged_prefill_attention",
 )
 
 
@@ -97,8 +97,9 @@ _SIGNATURES = {
     "kvq_paged_decode_attention_static_scratch": [_cfgp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _vp, _vp, _vp,
                                                   _vp, _f32, _i32, _vp, _vp],
     "kvq_selftest_bounded_wait": [_vp, _vp],
+    "kvq_prefill_workspace_bytes": [_cfgp, _i32, _i32, _i32, ctypes.POINTER(_sz)],
     "kvq_paged_prefill_attention": [_cfgp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _i32, _i32, _vp, _vp,
-                                    _vp, _vp, _f32, _vp, _vp],
+                                    _vp, _vp, _f32, _i32, _vp, _sz, _vp, _vp],
     "kvq_unpack_tiles": [_cfgp, _vp, _i32, _vp, _i32, _i32, _i32, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
 }
 
@@ -229,13 +230,44 @@ def paged_decode_attention(cfg: Config, q, out, seq_lens, block_tables, k_pool, 
     _check(st, "kvq_paged_decode_attention")
 
 
+def prefill_workspace_bytes(cfg: Config, num_seqs: int, max_chunk_tokens: int, num_splits: int) -> int:
+    out = _sz(0)
+    _check(load_library().kvq_prefill_workspace_bytes(ctypes.byref(cfg.c()), num_seqs, max_chunk_tokens, num_splits,
+                                                      ctypes.byref(out)), "kvq_prefill_workspace_bytes")
+    return out.value
+
+
+def prefill_splits(cfg: Config, num_seqs: int, max_chunk_tokens: int, max_context_tokens: int,
+                   num_sms: int) -> int:
+    """A context split count for kvq_paged_prefill_attention: the smallest S
+    (each split keeping at least 16 tiles) whose CTA count fills its last wave
+    to 95%, else the best fill found."""
+    units = num_seqs * cfg.num_kv_heads * -(-max_chunk_tokens * cfg.group_size // 128)
+    if units == 0:
+        return 1
+    tiles = max_context_tokens // cfg.tile_tokens
+    best, best_fill = 1, 0.0
+    for s in range(1, 17):
+        if s > 1 and tiles // s < 16:
+            break
+        n = units * s
+        fill = n / (-(-n // num_sms) * num_sms)
+        if fill >= 0.95:
+            return s
+        if fill > best_fill + 1e-9:
+            best, best_fill = s, fill
+    return best
+
+
 def paged_prefill_attention(cfg: Config, q, out, k_new, v_new, cu_chunk, ctx_lens, max_chunk_tokens: int,
-                            block_tables, k_pool, v_pool, k_tail, v_tail,
+                            block_tables, k_pool, v_pool, k_tail, v_tail, num_splits: int = 1, workspace=None,
                             softmax_scale: float | None = None, num_blocks: int | None = None, dev_status=None,
                             stream=None) -> None:
     """Read path, chunked prefill: chunk rows (q, out fp16 [N][H_q][d];
     k_new, v_new fp16 [N][H_kv][d], N = cu_chunk[-1]) attend to the cached
-    context of their sequence and causally to their own chunk."""
+    context of their sequence and causally to their own chunk.  With
+    ``num_splits`` > 1, ``workspace`` is a uint8 CUDA tensor of at least
+    ``prefill_workspace_bytes`` bytes."""
     if softmax_scale is None:
         softmax_scale = cfg.head_dim ** -0.5
     nb = k_pool.shape[0] if num_blocks is None else num_blocks
@@ -246,6 +278,7 @@ def paged_prefill_attention(cfg: Config, q, out, k_new, v_new, cu_chunk, ctx_len
         int(max_chunk_tokens), _ptr(block_tables, "block_tables", torch.int32), block_tables.shape[1], nb,
         _ptr(k_pool, "k_pool", torch.uint8), _ptr(v_pool, "v_pool", torch.uint8),
         _ptr(k_tail, "k_tail", torch.float16), _ptr(v_tail, "v_tail", torch.float16), float(softmax_scale),
+        int(num_splits), _ptr(workspace, "workspace", torch.uint8), 0 if workspace is None else workspace.numel(),
         _ptr(dev_status, "dev_status", torch.int32), _stream(stream))
     _check(st, "kvq_paged_prefill_attention")
 

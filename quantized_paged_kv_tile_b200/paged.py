@@ -115,11 +115,14 @@ class PagedKVCache:
         return out
 
     def prefill_chunk(self, q: torch.Tensor, new_k: torch.Tensor, new_v: torch.Tensor, counts,
-                      out: torch.Tensor | None = None, append: bool = True, stream=None) -> torch.Tensor:
+                      out: torch.Tensor | None = None, append: bool = True, num_splits: int | None = None,
+                      stream=None) -> torch.Tensor:
         """Chunked prefill: packed chunk rows (``counts`` tokens per sequence;
         q fp16 [N][H_q][d], new_k / new_v fp16 [N][H_kv][d]) attend to the
         cached context and causally to their own chunk; then (``append``) the
-        chunk joins the cache.  Returns out fp16 [N][H_q][d]."""
+        chunk joins the cache.  ``num_splits`` (default: chosen from the
+        context lengths and the SM count) splits long contexts over more
+        CTAs.  Returns out fp16 [N][H_q][d]."""
         counts = np.asarray(counts, dtype=np.int64)
         if counts.shape != (self.num_seqs,) or np.any(counts < 0):
             raise ValueError("counts: one non-negative chunk length per sequence")
@@ -129,9 +132,21 @@ class PagedKVCache:
             out = torch.empty_like(q)
         max_chunk = int(counts.max()) if counts.size else 0
         cu = torch.from_numpy(np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)).to(self.device)
+        if num_splits is None:
+            num_splits = 1
+            if self.device.type == "cuda":  # (anything else is refused by the binding below)
+                sms = torch.cuda.get_device_properties(self.device).multi_processor_count
+                num_splits = kvq.prefill_splits(self.cfg, self.num_seqs, max_chunk, int(self.host_lens.max()), sms)
+        need = kvq.prefill_workspace_bytes(self.cfg, self.num_seqs, max_chunk, num_splits)
+        ws = None
+        if need > 0:
+            if getattr(self, "prefill_workspace", None) is None or self.prefill_workspace.numel() < need:
+                self.prefill_workspace = torch.empty(need, dtype=torch.uint8, device=self.device)
+            ws = self.prefill_workspace
         kvq.paged_prefill_attention(self.cfg, q, out, new_k, new_v, cu, self.seq_lens, max_chunk, self.block_tables,
-                                    self.k_pool, self.v_pool, self.k_tail, self.v_tail, num_blocks=self.num_blocks,
-                                    dev_status=self.dev_status, stream=stream)
+                                    self.k_pool, self.v_pool, self.k_tail, self.v_tail, num_splits=num_splits,
+                                    workspace=ws, num_blocks=self.num_blocks, dev_status=self.dev_status,
+                                    stream=stream)
         if append and max_chunk > 0:
             self._append(new_k, new_v, self.host_lens, counts, stream)
             self.host_lens = self.host_lens + counts

@@ -107,9 +107,10 @@ def test_argument_errors_launch_nothing(lib):
 def test_prefill_argument_errors_launch_nothing(lib):
     cfg = kvq.Config(num_kv_heads=2, group_size=4, tile_tokens=64, bits_k=4, bits_v=4, iters=4)
     c = cfg.c()
-    def call(conf, num_seqs=3, max_chunk=40, q=16, scale=0.1, tables=16):
+    def call(conf, num_seqs=3, max_chunk=40, q=16, scale=0.1, tables=16, splits=1, ws=None, ws_bytes=0):
         return lib.kvq_paged_prefill_attention(ctypes.byref(conf), q, 16, 16, 16, 16, 16, num_seqs, max_chunk,
-                                               tables, 4, 8, 16, 16, 16, 16, scale, None, None)
+                                               tables, 4, 8, 16, 16, 16, 16, scale, splits, ws, ws_bytes, None,
+                                               None)
     c3 = kvq.Config(num_kv_heads=2, group_size=4, tile_tokens=64, bits_k=4, bits_v=3, iters=4).c()
     assert call(c3) == kvq.KVQ_ERR_UNSUPPORTED
     assert call(c, num_seqs=-1) == kvq.KVQ_ERR_INVALID_ARG
@@ -117,6 +118,15 @@ def test_prefill_argument_errors_launch_nothing(lib):
     assert call(c, q=None) == kvq.KVQ_ERR_INVALID_ARG
     assert call(c, q=24) == kvq.KVQ_ERR_INVALID_ARG            # misaligned
     assert call(c, scale=0.0) == kvq.KVQ_ERR_INVALID_ARG
+    assert call(c, splits=0) == kvq.KVQ_ERR_INVALID_ARG
+    assert call(c, splits=65) == kvq.KVQ_ERR_INVALID_ARG
+    # one 528-byte partial record per (sequence, KV head, 128-row tile, split, row)
+    assert kvq.prefill_workspace_bytes(cfg, 3, 40, 1) == 0
+    need = kvq.prefill_workspace_bytes(cfg, 3, 40, 3)
+    assert need == 3 * 2 * 2 * 3 * 128 * 132 * 4                # 40 tokens x g 4 = 160 rows -> 2 row tiles
+    assert call(c, splits=3) == kvq.KVQ_ERR_INVALID_ARG        # workspace NULL
+    assert call(c, splits=3, ws=16, ws_bytes=need - 1) == kvq.KVQ_ERR_WORKSPACE
+    assert str(need) in lib.kvq_last_error().decode()
     assert call(c, tables=None) == kvq.KVQ_ERR_INVALID_ARG
     assert call(c, num_seqs=70000) == kvq.KVQ_ERR_INVALID_ARG
     assert call(c, num_seqs=0) == kvq.KVQ_OK                   # nothing to do
@@ -181,3 +191,19 @@ def test_selftest_rejects_null_status(lib):
     # fails on the host before any launch
     assert lib.kvq_selftest_bounded_wait(None, None) == kvq.KVQ_ERR_INVALID_ARG
     assert "dev_status" in lib.kvq_last_error().decode()
+
+
+def test_prefill_split_heuristic():
+    cfg = kvq.Config(num_kv_heads=8, group_size=4, tile_tokens=64, bits_k=4, bits_v=4, iters=4)
+    # one sequence, 512-token chunk: 128 units on 148 SMs -> a split count that fills whole waves
+    s = kvq.prefill_splits(cfg, 1, 512, 131073, 148)
+    n = 128 * s
+    assert n / (-(-n // 148) * 148) >= 0.95 and 2048 // s >= 16
+    # six sequences: 768 units (5.19 waves) -> more CTAs
+    s6 = kvq.prefill_splits(cfg, 6, 512, 131073, 148)
+    n6 = 768 * s6
+    assert s6 > 1 and n6 / (-(-n6 // 148) * 148) >= 0.95
+    # short contexts are not split (each split keeps >= 16 tiles)
+    assert kvq.prefill_splits(cfg, 1, 512, 1500, 148) == 1
+    # no chunk tokens: nothing to split
+    assert kvq.prefill_splits(cfg, 4, 0, 131073, 148) == 1

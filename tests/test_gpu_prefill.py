@@ -96,6 +96,23 @@ def test_prefill_attention_matches_oracle(t, bk, bv, g, ctx, chunk):
     _check_against_oracle(w, cache, ctx, chunk, q, k_new, v_new, out)
 
 
+@pytest.mark.parametrize("splits", [2, 3, 7])
+@pytest.mark.parametrize("t,bk,bv,g,ctx,chunk", [CASES[0], CASES[1], CASES[2], CASES[4]])
+def test_prefill_attention_context_splits(t, bk, bv, g, ctx, chunk, splits):
+    # the context tiles split over several CTAs (some splits empty when a
+    # context has fewer tiles than splits), merged by a second launch
+    w, cache, q, k_new, v_new = _setup(t, bk, bv, g, ctx, chunk)
+    out = cache.prefill_chunk(q, k_new, v_new, chunk, append=False, num_splits=splits)
+    one = cache.prefill_chunk(q, k_new, v_new, chunk, append=False, num_splits=1)
+    torch.cuda.synchronize()
+    assert cache.status() == 0
+    _check_against_oracle(w, cache, ctx, chunk, q, k_new, v_new, out)
+    # split and unsplit agree to fp32 rounding before the fp16 output; two
+    # fp16 roundings of such values differ by at most one ulp, <= 2^-10 relative
+    oh, uh = out.float().cpu().numpy(), one.float().cpu().numpy()
+    assert max(rel_l2(oh[i, j], uh[i, j]) for i in range(oh.shape[0]) for j in range(oh.shape[1])) <= 2.0 ** -10
+
+
 def test_prefill_attention_randomized_rotation():
     ctx, chunk = (513, 200), (64, 31)
     w, cache, q, k_new, v_new = _setup(64, 4, 4, 4, ctx, chunk, rotation_seed=1234567)
@@ -181,7 +198,7 @@ def test_prefill_tile_outside_pool_is_skipped_and_reported():
     v_hat = [gpu_pages_kv_hat(cfg, cache, 0, h, ctx[0], True) for h in range(cfg.num_kv_heads)]
     bad_tile, t, per = 3, cfg.tile_tokens, cfg.tile_tokens // cfg.page_tokens
     cache.block_tables[0, bad_tile * per + 1] = cache.num_blocks + 7
-    out = cache.prefill_chunk(q, k_new, v_new, chunk, append=False)
+    out = cache.prefill_chunk(q, k_new, v_new, chunk, append=False, num_splits=2)
     torch.cuda.synchronize()
     assert cache.status() == kvq.KVQ_ERR_DEVICE_BOUNDS
     keep = np.r_[0:bad_tile * t, (bad_tile + 1) * t:ctx[0]]
