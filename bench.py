@@ -439,6 +439,31 @@ def run_kvq(args, ranks):
     return line
 
 
+def prefill_cpu_sample(w, chunk: int, ctx_tokens: int = 16384, tokens: int = 64):
+    """The oracle on a bounded sample of the chunked-prefill workload: one
+    (sequence, KV head) with a ``ctx_tokens`` context quantized by the oracle
+    (not timed), then, timed, the read path as the oracle states it: the
+    context dequantized and fp64 attention of the first ``tokens`` chunk
+    tokens x g query heads over it and causally over the chunk rows.
+    Returns (algorithmic FLOPs, seconds); one BLAS thread."""
+    from threadpoolctl import threadpool_limits
+    sys.path.insert(0, ROOT)
+    from oracle import kvq_oracle as o
+    from quantized_paged_kv_tile_b200 import synth
+    tokens = min(tokens, chunk)
+    with threadpool_limits(1):
+        rk = synth.kv_rows_one_head(w, "k", ctx_tokens + tokens, 0, stream_id=0)
+        rv = synth.kv_rows_one_head(w, "v", ctx_tokens + tokens, 0, stream_id=0)
+        tk, tail_k = o.quantize_sequence(rk[:ctx_tokens], w.tile_tokens, w.bits_k, w.iters)
+        tv, tail_v = o.quantize_sequence(rv[:ctx_tokens], w.tile_tokens, w.bits_v, w.iters)
+        q = np.random.default_rng(17).standard_normal((tokens, w.group_size, 128))
+        t0 = time.perf_counter()
+        kh, vh = o.sequence_kv_hat(tk, tail_k), o.sequence_kv_hat(tv, tail_v)
+        o.prefill_chunk_sequence(q, [kh], [vh], rk[ctx_tokens:, None], rv[ctx_tokens:, None], w.group_size)
+        secs = time.perf_counter() - t0
+    return prefill_flops([ctx_tokens], tokens, w.group_size), secs
+
+
 def prefill_leg(w, cfg, args, dev, stream, seq_lens, bt, nblocks, k_pool, v_pool, k_tail, v_tail, status, lens1):
     """Chunked prefill over the step's cache: every sequence gets
     ``--prefill-chunk`` new tokens attending to its cached tokens and
@@ -479,8 +504,15 @@ def prefill_leg(w, cfg, args, dev, stream, seq_lens, bt, nblocks, k_pool, v_pool
     flops = prefill_flops(lens1, n, w.num_q_heads)
     peak, kind = tensor_peak()
     tflops = flops / (ms * 1e-3) / 1e12
+    cpu = None
+    if not args.no_cpu_baseline:
+        sflops, secs = prefill_cpu_sample(w, n)
+        cpu = {"value": sflops / secs / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+               "sample": f"1 (sequence, KV head), a 16384-token context quantized by the oracle (untimed), then "
+                         f"dequantized and fp64 causal prefill attention of {min(64, n)} chunk tokens x "
+                         f"{w.group_size} query heads: {secs:.2f} s on one thread"}
     return {"chunk_tokens": n, "ms": ms, "chunk_tok_per_s": B * n / (ms * 1e-3), "flops": flops,
-            "context_splits": splits, "launches_per_call": 1 if splits == 1 else 2,
+            "context_splits": splits, "launches_per_call": 1 if splits == 1 else 2, "cpu_baseline": cpu,
             "context": f"{B} seqs x {int(lens1[0])} cached tokens (quantized tiles + fp16 tail)",
             "roofline": {"bound": "tensor", "kernel": "prefill_attn_kernel", "achieved": tflops, "peak": peak,
                          "peak_kind": kind, "unit": "TFLOP/s", "frac": tflops / peak, "traffic": None,

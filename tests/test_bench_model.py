@@ -24,3 +24,11 @@ def test_tensor_peak_reads_measured_file():
         assert kind == "measured" and peak == float(json.load(open(path))["bf16_tflops"])
     else:
         assert kind == "fallback"
+
+
+def test_prefill_cpu_sample_runs_the_oracle():
+    import bench
+    from quantized_paged_kv_tile_b200 import synth
+    w = synth.workload("qwen3_4b")
+    flops, secs = bench.prefill_cpu_sample(w, 512, ctx_tokens=128, tokens=4)
+    assert flops == bench.prefill_flops([128], 4, w.group_size) and secs > 0
