@@ -505,7 +505,7 @@ def prefill_leg(w, cfg, args, dev, stream, seq_lens, bt, nblocks, k_pool, v_pool
     peak, kind = tensor_peak()
     tflops = flops / (ms * 1e-3) / 1e12
     cpu = None
-    if not args.no_cpu_baseline:
+    if not args.no_cpu_baseline and os.environ.get("RANK", "0") == "0" and os.environ.get("WORLD_SIZE", "1") == "1":
         sflops, secs = prefill_cpu_sample(w, n)
         cpu = {"value": sflops / secs / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
                "sample": f"1 (sequence, KV head), a 16384-token context quantized by the oracle (untimed), then "
