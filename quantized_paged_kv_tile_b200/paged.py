@@ -50,6 +50,7 @@ class PagedKVCache:
         self.num_splits = num_splits
         self.workspace = torch.empty(kvq.decode_workspace_bytes(cfg, num_seqs, num_splits), dtype=torch.uint8,
                                      device=self.device)
+        self.prefill_workspace = None  # grown on demand by prefill_chunk when it splits contexts
         self.dev_status = torch.zeros(1, dtype=torch.int32, device=self.device)
 
     # ------------------------------------------------------------------ write
@@ -140,7 +141,7 @@ class PagedKVCache:
         need = kvq.prefill_workspace_bytes(self.cfg, self.num_seqs, max_chunk, num_splits)
         ws = None
         if need > 0:
-            if getattr(self, "prefill_workspace", None) is None or self.prefill_workspace.numel() < need:
+            if self.prefill_workspace is None or self.prefill_workspace.numel() < need:
                 self.prefill_workspace = torch.empty(need, dtype=torch.uint8, device=self.device)
             ws = self.prefill_workspace
         kvq.paged_prefill_attention(self.cfg, q, out, new_k, new_v, cu, self.seq_lens, max_chunk, self.block_tables,
