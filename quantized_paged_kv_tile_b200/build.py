@@ -45,17 +45,34 @@ def nvcc_path() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile csrc/*.cu into libkvq.so (sm_100a) unless it is up to date."""
-    if not force and not _stale():
-        return LIB_PATH
-    tmp = LIB_PATH + ".tmp"
-    cmd = [nvcc_path(), *NVCC_FLAGS, "-o", tmp, *sources()]
+def _run(cmd, verbose):
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         raise RuntimeError(f"nvcc failed ({res.returncode}):\n{res.stdout}\n{res.stderr}")
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile csrc/*.cu into libkvq.so (sm_100a) unless it is up to date.
+
+    Each translation unit compiles in its own nvcc process (they share no
+    device code), in parallel, then one nvcc call links the shared library."""
+    if not force and not _stale():
+        return LIB_PATH
+    import concurrent.futures
+    import tempfile
+    nvcc = nvcc_path()
+    compile_flags = [f for f in NVCC_FLAGS if f != "-shared"]
+    with tempfile.TemporaryDirectory(prefix="kvq_build_") as tmpdir:
+        objs = [os.path.join(tmpdir, os.path.basename(src) + ".o") for src in sources()]
+        jobs = [[nvcc, *compile_flags, "-c", "-o", obj, src] for src, obj in zip(sources(), objs)]
+        workers = max(1, min(len(jobs), os.cpu_count() or 1))
+        with concurrent.futures.ThreadPoolExecutor(workers) as pool:
+            for fut in [pool.submit(_run, cmd, verbose) for cmd in jobs]:
+                fut.result()
+        tmp = LIB_PATH + ".tmp"
+        _run([nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp, *objs], verbose)
     os.replace(tmp, LIB_PATH)
     return LIB_PATH
 
