@@ -574,3 +574,30 @@ def test_prefill_empty_context_is_causal_attention():
         want = brute_attention(q[i, 0].tolist(), k_new[:i + 1, 0].astype(np.float64).tolist(),
                                v_new[:i + 1, 0].astype(np.float64).tolist(), 1 / math.sqrt(128))
         np.testing.assert_allclose(out[i, 0], want, rtol=1e-12, atol=1e-14)
+
+
+def test_lse_merge_of_parts_is_attention_over_all_keys():
+    # the merge both split paths rely on: per part (max m, sum l, unnormalized
+    # accumulator a) in the log2 domain, merged with weights 2^(m_s - max m),
+    # reproduces attention over all keys; empty parts contribute nothing
+    rng = np.random.default_rng(37)
+    L = 300
+    q = rng.standard_normal(128)
+    k = rng.standard_normal((L, 128)) * 3
+    v = rng.standard_normal((L, 128))
+    want = o.attention_fp64(q, k, v)
+    scale = math.log2(math.e) / math.sqrt(128)
+    for cuts in ([0, 100, 100, 217, 300], [0, 1, 299, 300], [0, 300]):
+        parts = []
+        for a, b in zip(cuts[:-1], cuts[1:]):
+            if a == b:
+                parts.append((-math.inf, 0.0, np.zeros(128)))
+                continue
+            s = (k[a:b] @ q) * scale
+            m = s.max()
+            p = np.exp2(s - m)
+            parts.append((m, p.sum(), p @ v[a:b]))
+        mm = max(m for m, l, _ in parts if l > 0)
+        l_tot = sum(l * 2.0 ** (m - mm) for m, l, _ in parts if l > 0)
+        acc = sum(a * 2.0 ** (m - mm) for m, l, a in parts if l > 0)
+        np.testing.assert_allclose(acc / l_tot, want, rtol=1e-11, atol=1e-13)
