@@ -27,7 +27,9 @@ Sources (web pages, cited by title and section):
   logical -> physical mapping.
 
 The pages fix the method only in outline.  The concrete definitions this
-oracle follows (and the CUDA path implements independently) are:
+oracle follows (and the CUDA path implements independently, at d = 128; the
+format functions below also define d = 64 and 256, for which the library
+has no kernels yet) are:
 
 1. Rotation: X' = X H with H the orthonormal Sylvester Hadamard matrix,
    H[j, k] = (-1)^popcount(j & k) / sqrt(d), natural order, no random signs.
@@ -76,7 +78,8 @@ import math
 import numpy as np
 
 EPS = 1e-6          # std clamp of the normalization (both steps)
-HEAD_DIM = 128      # d: the one head size of the format
+HEAD_DIM = 128      # d: the head size the library implements (the format below also defines d = 64, 256)
+HEAD_DIMS = (64, 128, 256)
 PAGE_TOKENS = 16    # P: tokens per page (block)
 
 
@@ -289,17 +292,19 @@ def code_bit_position(channel: int, token: int, bits: int, is_v: bool,
     V at 2, 4 or 8 bits: grouped for the decode kernel's register layout.
     n = channel // 8 and g = channel % 8; t = (token % 8) // 2,
     u = token // 8 and s = token % 2.  The page's 32 "lanes" are
-    L = 4 g + t.  Each lane owns 2*bits little-endian 32-bit words holding
-    the codes of its 16 channels (n = 0..15) for the token pairs
-    {2t, 2t+1} (u = 0) and {2t+8, 2t+9} (u = 1).  With F = 32 / bits
-    fields per word and h = F / 2 pairs per word, the code lives in word
-    k = 2 (n // h) + u at field e + h s, e = n % h.  Lane L's word k is at
-    byte ((k // 4) * 32 + L) * 16 + (k % 4) * 4.
+    L = 4 g + t.  Each lane owns W = d*bits/64 little-endian 32-bit words
+    (2*bits at d = 128) holding the codes of its d/8 channels (n = 0..d/8-1)
+    for the token pairs {2t, 2t+1} (u = 0) and {2t+8, 2t+9} (u = 1).  With
+    F = 32 / bits fields per word and h = F / 2 pairs per word, the code
+    lives in word k = 2 (n // h) + u at field e + h s, e = n % h.  Lane L's
+    words sit in rows of R = min(4, W) words: word k is at byte
+    ((k // R) * 32 + L) * 4R + (k % R) * 4 (R = 4 for every b at d >= 128;
+    R = 2 only at d = 64, b = 2).
     """
     if not is_v or bits == 3:
         return (token * d + channel) * bits
-    if d != 128 or bits not in (2, 4, 8):
-        raise ValueError("grouped V layout is defined for d=128, b in {2,4,8}")
+    if d not in HEAD_DIMS or bits not in (2, 4, 8):
+        raise ValueError("grouped V layout is defined for d in {64, 128, 256}, b in {2, 4, 8}")
     n, g = divmod(channel, 8)
     t = (token % 8) // 2
     u = token // 8
@@ -309,7 +314,8 @@ def code_bit_position(channel: int, token: int, bits: int, is_v: bool,
     k = 2 * (n // h) + u
     e = n % h
     lane = 4 * g + t
-    word_byte = ((k // 4) * 32 + lane) * 16 + (k % 4) * 4
+    row = min(4, d * bits // 64)  # words per lane row
+    word_byte = ((k // row) * 32 + lane) * (4 * row) + (k % row) * 4
     return word_byte * 8 + bits * (e + h * s)
 
 
@@ -350,14 +356,15 @@ def write_tile_pages(pool: np.ndarray, block_ids, head: int, tile: dict,
     """Store one quantized tile into its T/P pages of a pool shaped
     [num_blocks][H_kv][page_bytes] (uint8).  ``block_ids`` are the physical
     blocks of the tile's pages in order."""
-    lay = page_layout(bits, tile_tokens)
+    d = tile["codes"].shape[1]
+    lay = page_layout(bits, tile_tokens, d)
     p = PAGE_TOKENS
     cs = lay["cslice_channels"]
     for k, blk in enumerate(block_ids):
         region = pool[blk, head]
         region[:] = 0
         toks = slice(k * p, (k + 1) * p)
-        region[:p * HEAD_DIM * bits // 8] = pack_page_codes(tile["codes"][toks], bits, is_v)
+        region[:p * d * bits // 8] = pack_page_codes(tile["codes"][toks], bits, is_v)
         meta = np.stack([tile["s_t"][toks], tile["z_t"][toks]], axis=1).astype(np.float16)
         region[lay["meta_off"]:lay["meta_off"] + 4 * p] = meta.reshape(-1).view(np.uint8)
         cvals = tile["c_t"][k * cs:(k + 1) * cs].astype(np.float16)
@@ -365,15 +372,15 @@ def write_tile_pages(pool: np.ndarray, block_ids, head: int, tile: dict,
 
 
 def read_tile_pages(pool: np.ndarray, block_ids, head: int, bits: int,
-                    tile_tokens: int, is_v: bool) -> dict:
+                    tile_tokens: int, is_v: bool, d: int = HEAD_DIM) -> dict:
     """Inverse of ``write_tile_pages`` (used on pages the oracle packed)."""
-    lay = page_layout(bits, tile_tokens)
+    lay = page_layout(bits, tile_tokens, d)
     p = PAGE_TOKENS
     cs = lay["cslice_channels"]
     codes, s_t, z_t, c_t = [], [], [], []
     for blk in block_ids:
         region = np.asarray(pool[blk, head], dtype=np.uint8)
-        codes.append(unpack_page_codes(region[:p * HEAD_DIM * bits // 8], bits, is_v))
+        codes.append(unpack_page_codes(region[:p * d * bits // 8], bits, is_v, d=d))
         meta = region[lay["meta_off"]:lay["meta_off"] + 4 * p].copy().view(np.float16).reshape(p, 2)
         s_t.append(meta[:, 0])
         z_t.append(meta[:, 1])
@@ -404,7 +411,8 @@ def sequence_kv_hat(tiles, tail_rows: np.ndarray, seed: int = 0) -> np.ndarray:
     dequantized full tiles in order, then the raw fp16 rows of the unfinished
     tile.  ``tiles`` is a list of ``quantize_tile``-style dicts."""
     parts = [dequantize_tile(t["codes"], t["s_t"], t["z_t"], t["c_t"], seed)[1] for t in tiles]
-    parts.append(np.asarray(tail_rows, dtype=np.float16).astype(np.float64).reshape(-1, HEAD_DIM))
+    d = tiles[0]["codes"].shape[1] if tiles else np.asarray(tail_rows).shape[-1]
+    parts.append(np.asarray(tail_rows, dtype=np.float16).astype(np.float64).reshape(-1, d))
     return np.concatenate(parts, axis=0)
 
 

@@ -27,7 +27,7 @@ def outlier_tile(rng, t, d=128, n_out=4, mult=20.0):
 
 # --------------------------------------------------------------------------- Hadamard
 
-@pytest.mark.parametrize("d", [2, 4, 8, 16, 32, 64, 128])
+@pytest.mark.parametrize("d", [2, 4, 8, 16, 32, 64, 128, 256])
 def test_hadamard_equals_scipy(d):
     # wrong recursion / order / sign -> differs from the library matrix
     h = o.sylvester_hadamard(d)
@@ -601,3 +601,95 @@ def test_lse_merge_of_parts_is_attention_over_all_keys():
         l_tot = sum(l * 2.0 ** (m - mm) for m, l, _ in parts if l > 0)
         acc = sum(a * 2.0 ** (m - mm) for m, l, a in parts if l > 0)
         np.testing.assert_allclose(acc / l_tot, want, rtol=1e-11, atol=1e-13)
+
+
+
+# --------------------------------------------------------------------------- head sizes 64 and 256 (format)
+
+@pytest.mark.parametrize("d", [64, 256])
+@pytest.mark.parametrize("bits,is_v", [(2, False), (3, False), (4, False), (8, False), (2, True), (3, True),
+                                       (4, True), (8, True)])
+def test_code_positions_are_a_bijection_at_other_head_sizes(d, bits, is_v):
+    # every (channel, token) of a page gets its own field inside p*d*b bits
+    pos = [o.code_bit_position(ch, tok, bits, is_v, d) for tok in range(16) for ch in range(d)]
+    assert len(set(pos)) == len(pos)
+    assert min(pos) >= 0 and max(pos) + bits <= 16 * d * bits
+    assert all(p % bits == 0 for p in pos)
+
+
+def test_grouped_v_positions_golden_other_head_sizes():
+    # hand-derived from the layout rule (n = c // 8, g = c % 8, t = (tok % 8) // 2,
+    # u = tok // 8, s = tok % 2, h = 16 / b, k = 2 (n // h) + u, e = n % h,
+    # lane 4 g + t, rows of min(4, d b / 64) words):
+    # d = 64, b = 2, channel 9, token 3: n 1, g 1, t 1, u 0, s 1; h 8, k 0, e 1,
+    #   lane 5, row width 2 -> byte 5 * 8 = 40, bit 320 + 2 (1 + 8) = 338
+    assert o.code_bit_position(9, 3, 2, True, 64) == 338
+    # d = 64, b = 2, channel 63, token 15: n 7, g 7, t 3, u 1, s 1; k 1, e 7, lane 31
+    #   -> byte 31 * 8 + 4 = 252, bit 2016 + 2 (7 + 8) = 2046 (the page's last field)
+    assert o.code_bit_position(63, 15, 2, True, 64) == 2046
+    # d = 256, b = 4, channel 200, token 9: n 25, g 0, t 0, u 1, s 1; h 4, k 13, e 1,
+    #   lane 0, rows of 4 -> byte (3 * 32) * 16 + 4 = 1540, bit 12320 + 4 (1 + 4) = 12340
+    assert o.code_bit_position(200, 9, 4, True, 256) == 12340
+    # d = 128 keeps its layout: rows of 4 words for every b
+    assert o.code_bit_position(9, 3, 2, True, 128) == (5 * 16) * 8 + 2 * (1 + 8)
+
+
+@pytest.mark.parametrize("d", [64, 256])
+@pytest.mark.parametrize("bits,is_v", [(2, True), (4, True), (8, True), (3, False), (4, False)])
+def test_pack_unpack_roundtrip_other_head_sizes(d, bits, is_v):
+    rng = np.random.default_rng(50 + d + bits)
+    codes = rng.integers(0, 1 << bits, size=(16, d)).astype(np.uint8)
+    region = o.pack_page_codes(codes, bits, is_v)
+    assert region.size == 16 * d * bits // 8
+    np.testing.assert_array_equal(o.unpack_page_codes(region, bits, is_v, d=d), codes)
+
+
+@pytest.mark.parametrize("d,t,bits", [(64, 64, 4), (256, 64, 2), (256, 128, 4), (64, 32, 8)])
+def test_layout_and_tile_pages_roundtrip_other_head_sizes(d, t, bits):
+    lay = o.page_layout(bits, t, d)
+    # codes p d b / 8 | 64 B of metadata | d p / T channels of C, each padded to 16 B
+    assert lay["codes"] == -(-16 * d * bits // 8 // 16) * 16
+    assert lay["cslice_channels"] == d * 16 // t
+    assert lay["page_bytes"] == lay["codes"] + 64 + -(-2 * (d * 16 // t) // 16) * 16
+    rng = np.random.default_rng(60 + d + t + bits)
+    for is_v in (False, True):
+        tile = o.quantize_tile(outlier_tile(rng, t, d=d), bits, 2)
+        pool = np.zeros((t // 16 + 3, 1, lay["page_bytes"]), dtype=np.uint8)
+        blocks = list(rng.permutation(pool.shape[0])[: t // 16])
+        o.write_tile_pages(pool, blocks, 0, tile, bits, t, is_v)
+        back = o.read_tile_pages(pool, blocks, 0, bits, t, is_v, d=d)
+        for k in ("codes", "s_t", "z_t", "c_t"):
+            np.testing.assert_array_equal(np.asarray(back[k]).view(np.uint8), np.asarray(tile[k]).view(np.uint8))
+
+
+@pytest.mark.parametrize("d", [64, 256])
+def test_dequantized_tile_within_half_step_other_head_sizes(d):
+    rng = np.random.default_rng(70 + d)
+    x = outlier_tile(rng, 64, d=d)
+    q = o.quantize_tile(x, 4, 4, return_parts=True)
+    xr_hat, x_hat = o.dequantize_tile(q["codes"], q["s_t"], q["z_t"], q["c_t"])
+    half = (q["s"] * q["r"])[:, None] * q["c"][None, :] / 2
+    fp16_slack = 2.0 ** -10 * (np.abs(q["xr"]) + (q["s"] * q["r"])[:, None] * q["c"][None, :] * 15)
+    assert np.all(np.abs(xr_hat - q["xr"]) <= half + 3 * fp16_slack)
+    np.testing.assert_allclose(x_hat, xr_hat @ o.sylvester_hadamard(d), rtol=0, atol=1e-12)
+    err = np.linalg.norm(x_hat - x.astype(np.float64)) / np.linalg.norm(x.astype(np.float64))
+    assert err < 0.15
+
+
+def test_prefill_causal_closed_form_at_d64():
+    # the attention functions take d from the rows (scale 1/sqrt(64)): same
+    # uniform-weight closed form as at d = 128
+    L, n = 5, 3
+    u = np.full(64, 0.5)
+    v_new = np.zeros((n, 1, 64), dtype=np.float16)
+    v_new[:, 0, 0] = np.arange(1, n + 1)
+    out = o.prefill_chunk_sequence(np.ones((n, 1, 64)), [np.tile(u, (L, 1))], [np.zeros((L, 64))],
+                                   np.tile(u, (n, 1, 1)).astype(np.float16), v_new, 1)
+    for i in range(n):
+        assert out[i, 0, 0] == pytest.approx((i + 1) * (i + 2) / 2 / (L + i + 1), rel=1e-13)
+    # and the one-key logistic weight uses 1/sqrt(64)
+    q = np.random.default_rng(38).standard_normal((1, 1, 64))
+    k1, k2 = np.random.default_rng(39).standard_normal((1, 64)), np.zeros((1, 1, 64), dtype=np.float16)
+    w2 = 1.0 / (1.0 + math.exp(float(q[0, 0] @ k1[0]) / 8.0))
+    got = o.prefill_chunk_sequence(q, [k1], [np.zeros((1, 64))], k2, np.ones((1, 1, 64), dtype=np.float16), 1)
+    np.testing.assert_allclose(got[0, 0], np.full(64, w2), rtol=1e-12)
