@@ -78,8 +78,14 @@
  *  - Every pointer argument marked "device" is a device pointer of the
  *    current CUDA device; every such pointer must be 16-byte aligned.
  *  - The caller owns every buffer (pools, tails, tables, workspace, status
- *    word).  The library allocates no device memory and keeps no state
- *    beyond a thread-local error message.
+ *    word).  No call allocates device memory.  State kept by the library:
+ *    a thread-local error message, and for
+ *    kvq_paged_decode_attention_static_scratch a static device array of
+ *    KVQ_DECODE_STATIC_SCRATCH_BYTES (32 MiB) that is part of the library's
+ *    device code, so every device that loads the library's module (at its
+ *    first kernel launch, or at start-up with CUDA_MODULE_LOADING=EAGER)
+ *    holds those 32 MiB until the process exits, whether or not that entry
+ *    point is ever called; plus that array's address per device.
  *  - Every call is asynchronous on `stream` (0 = legacy default stream) and
  *    never synchronizes.  Arguments are validated on the host first; an
  *    invalid call returns an error and launches nothing.
@@ -286,8 +292,13 @@ KVQ_API kvq_status kvq_paged_prefill_attention(const kvq_config* cfg, const void
  *   KVQ_ERR_WORKSPACE (detail in kvq_last_error) before touching the device;
  *   use fewer sequences per call, a smaller num_splits, or the workspace entry.
  *   Set-up: the first call on each device (that device current) looks up the
- *   array's address with cudaGetSymbolAddress; make that first call before
- *   any stream capture begins.  Device ordinals 0..63.
+ *   array's address with cudaGetSymbolAddress and keeps it; make that first
+ *   call before any stream capture begins.  Device ordinals 0..63.  The kept
+ *   address belongs to the device's current context: after cudaDeviceReset
+ *   (or any destruction of the primary context) the array may move, so do not
+ *   call this entry point again in that process after a reset.
+ *   Memory: the array is reserved on every device that loads the library's
+ *   module, whether or not this entry point is called.
  *   Concurrency: calls on the same device share the array; two calls that
  *   overlap in time (different streams, or unordered host threads) race on it
  *   and corrupt each other's results.  Order them (one stream, or events). */

@@ -99,11 +99,6 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
-__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t d;  // (a & b) | c
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
-}
 __device__ __forceinline__ void mma16816(float d[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
   asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
@@ -111,45 +106,6 @@ __device__ __forceinline__ void mma16816(float d[4], const uint32_t a[4], uint32
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
-__device__ __forceinline__ uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
-__device__ __forceinline__ __half2 u32_as_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
-
-// A 32-bit word of b-bit codes -> fp16 pairs holding exact small integers.
-// b = 4: pair e (0..3) = (nibble e, nibble e+4);  b = 2: pair e (0..7) =
-// (field e, field e+8).  The fields land in fp16 mantissas under the
-// exponent of 1024 (0x6400) and are rebased with one fused multiply-add.
-template <int B>
-__device__ __forceinline__ void unpack_word(uint32_t w, uint32_t out[16 / B]) {
-  const uint32_t magic = 0x64006400u;
-  if constexpr (B == 8) {  // pair e (0..1) = (byte e, byte e+2)
-    const __half2 k1024 = __float2half2_rn(1024.f);
-    out[0] = h2_as_u32(__hsub2(u32_as_h2(lop3_and_or(w, 0x00FF00FFu, magic)), k1024));
-    out[1] = h2_as_u32(__hsub2(u32_as_h2(lop3_and_or(w >> 8, 0x00FF00FFu, magic)), k1024));
-  } else if constexpr (B == 4) {
-    const uint32_t w8 = w >> 8;
-    const __half2 k1024 = __float2half2_rn(1024.f);
-    const __half2 s16 = __float2half2_rn(1.f / 16.f), o64 = __float2half2_rn(-64.f);
-    out[0] = h2_as_u32(__hsub2(u32_as_h2(lop3_and_or(w, 0x000F000Fu, magic)), k1024));
-    out[1] = h2_as_u32(__hfma2(u32_as_h2(lop3_and_or(w, 0x00F000F0u, magic)), s16, o64));
-    out[2] = h2_as_u32(__hsub2(u32_as_h2(lop3_and_or(w8, 0x000F000Fu, magic)), k1024));
-    out[3] = h2_as_u32(__hfma2(u32_as_h2(lop3_and_or(w8, 0x00F000F0u, magic)), s16, o64));
-  } else {
-    const uint32_t w8 = w >> 8;
-    const __half2 k1024 = __float2half2_rn(1024.f);
-    const __half2 s4 = __float2half2_rn(0.25f), o256 = __float2half2_rn(-256.f);
-    const __half2 s16 = __float2half2_rn(1.f / 16.f), o64 = __float2half2_rn(-64.f);
-    const __half2 s64 = __float2half2_rn(1.f / 64.f), o16 = __float2half2_rn(-16.f);
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const uint32_t x = half ? w8 : w;
-      out[4 * half + 0] = h2_as_u32(__hsub2(u32_as_h2(lop3_and_or(x, 0x00030003u, magic)), k1024));
-      out[4 * half + 1] = h2_as_u32(__hfma2(u32_as_h2(lop3_and_or(x, 0x000C000Cu, magic)), s4, o256));
-      out[4 * half + 2] = h2_as_u32(__hfma2(u32_as_h2(lop3_and_or(x, 0x00300030u, magic)), s16, o64));
-      out[4 * half + 3] = h2_as_u32(__hfma2(u32_as_h2(lop3_and_or(x, 0x00C000C0u, magic)), s64, o16));
-    }
-  }
-}
-
 // Channel pair p (0..15) of lane-quad t in the K register order:
 // b = 4: word p/4, nibbles (p%4, p%4+4) -> channels 32t + 8(p/4) + p%4 + {0, 4}
 // b = 2: word p/8, fields (p%8, p%8+8) -> channels 32t + 16(p/8) + p%8 + {0, 8}
@@ -437,7 +393,7 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
 #pragma unroll
           for (int pg = 0; pg < kPc; ++pg)
 #pragma unroll
-            for (int nb = 0; nb < 2; ++nb) unpack_word<BK>(rec[pg][nb][wd], pr[pg][nb]);
+            for (int nb = 0; nb < 2; ++nb) unpack_pairs<BK>(rec[pg][nb][wd], pr[pg][nb]);
 #pragma unroll
           for (int j = 0; j < kbPerWord; ++j) {
             const int kb = wd * kbPerWord + j;
@@ -525,8 +481,8 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
           const uint4 row = *reinterpret_cast<const uint4*>(sV + pg * Geo::kPageV + (((2 * q) >> 2) * 32 + lane) * 16);
           const uint32_t w0 = (q & 1) ? row.z : row.x, w1 = (q & 1) ? row.w : row.y;
           uint32_t p0[kPairsV], p1[kPairsV];
-          unpack_word<BV>(w0, p0);
-          unpack_word<BV>(w1, p1);
+          unpack_pairs<BV>(w0, p0);
+          unpack_pairs<BV>(w1, p1);
 #pragma unroll
           for (int e = 0; e < kPairsV; ++e) mma16816(dv[e], afr, p0[e], p1[e]);
         }

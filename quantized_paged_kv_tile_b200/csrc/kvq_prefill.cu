@@ -120,48 +120,6 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
                "l"(src), "r"(bytes), "r"(bar)
                : "memory");
 }
-__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t d;  // (a & b) | c
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
-}
-__device__ __forceinline__ uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
-__device__ __forceinline__ __half2 u32_as_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
-
-// A 32-bit word of b-bit codes -> h = 16/b fp16 pairs of exact small
-// integers, pair e = (field e, field e + h).
-// The fields land in fp16 mantissas under the exponent of 1024 (0x6400) and
-// are rebased by one subtraction or fused multiply-add.
-template <int B>
-__device__ __forceinline__ void unpack_pairs(uint32_t w, uint32_t out[16 / B]) {
-  const uint32_t magic = 0x64006400u;
-  const __half2 k1024 = __float2half2_rn(1024.f);
-  if constexpr (B == 8) {  // pair e (0..1) = (byte e, byte e+2)
-    out[0] = h2_as_u32(__hsub2(u32_as_h2(lop3_and_or(w, 0x00FF00FFu, magic)), k1024));
-    out[1] = h2_as_u32(__hsub2(u32_as_h2(lop3_and_or(w >> 8, 0x00FF00FFu, magic)), k1024));
-  } else if constexpr (B == 4) {  // pair e (0..3) = (nibble e, nibble e+4)
-    const uint32_t w8 = w >> 8;
-    const __half2 s16 = __float2half2_rn(1.f / 16.f), o64 = __float2half2_rn(-64.f);
-    out[0] = h2_as_u32(__hsub2(u32_as_h2(lop3_and_or(w, 0x000F000Fu, magic)), k1024));
-    out[1] = h2_as_u32(__hfma2(u32_as_h2(lop3_and_or(w, 0x00F000F0u, magic)), s16, o64));
-    out[2] = h2_as_u32(__hsub2(u32_as_h2(lop3_and_or(w8, 0x000F000Fu, magic)), k1024));
-    out[3] = h2_as_u32(__hfma2(u32_as_h2(lop3_and_or(w8, 0x00F000F0u, magic)), s16, o64));
-  } else {  // pair e (0..7) = (field e, field e+8)
-    const uint32_t w8 = w >> 8;
-    const __half2 s4 = __float2half2_rn(0.25f), o256 = __float2half2_rn(-256.f);
-    const __half2 s16 = __float2half2_rn(1.f / 16.f), o64 = __float2half2_rn(-64.f);
-    const __half2 s64 = __float2half2_rn(1.f / 64.f), o16 = __float2half2_rn(-16.f);
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const uint32_t x = half ? w8 : w;
-      out[4 * half + 0] = h2_as_u32(__hsub2(u32_as_h2(lop3_and_or(x, 0x00030003u, magic)), k1024));
-      out[4 * half + 1] = h2_as_u32(__hfma2(u32_as_h2(lop3_and_or(x, 0x000C000Cu, magic)), s4, o256));
-      out[4 * half + 2] = h2_as_u32(__hfma2(u32_as_h2(lop3_and_or(x, 0x00300030u, magic)), s16, o64));
-      out[4 * half + 3] = h2_as_u32(__hfma2(u32_as_h2(lop3_and_or(x, 0x00C000C0u, magic)), s64, o16));
-    }
-  }
-}
-
 // Order of the channels along the QK contraction: the K codes of a 32-bit
 // word (W = 32/b channels, fields in channel order) unpack into pairs
 // (field e, field e + W/2), so MMA position 2e + s of the word's group holds

@@ -6,8 +6,10 @@
 // per fixed-size token tile, Hadamard rotation along the channels, then
 // Sinkhorn-like alternating variance normalization, then asymmetric RTN.
 //
-// One CTA (4 warps) works on a group of 128 token rows = 128/T tiles of one
-// (KV head, K|V) at a time:
+// A persistent CTA of 8 math warps and 1 producer warp works on a group of
+// 128 token rows = 128/T tiles of one (KV head, K|V) at a time; the producer
+// warp loads and rotates the next group while the math warps finish the
+// current one:
 //   load    TMA (cp.async.bulk.tensor, 128-byte swizzle) brings the fp16
 //           rows into shared memory; the next group's load is issued as soon
 //           as the current group's MMAs have read the buffer

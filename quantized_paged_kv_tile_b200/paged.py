@@ -17,10 +17,32 @@ from __future__ import annotations
 
 import math
 
+import contextlib
+
 import numpy as np
 import torch
 
 from . import kvq
+
+
+@contextlib.contextmanager
+def _on_stream(stream):
+    """Run the enclosed calls on ``stream`` (a torch.cuda.Stream, or None for
+    the current stream): temporaries made inside are allocated and copied on
+    it, so the caching allocator never hands their memory to other work while
+    the stream's kernels still read it."""
+    if stream is None:
+        yield
+    else:
+        with torch.cuda.stream(stream):
+            yield
+
+
+def _in_use(buf):
+    """Mark a long-lived buffer as used by the current stream (it may have
+    been allocated on another), so that freeing it later waits for this use."""
+    if buf is not None and buf.is_cuda:
+        buf.record_stream(torch.cuda.current_stream(buf.device))
 
 
 class PagedKVCache:
@@ -67,26 +89,28 @@ class PagedKVCache:
         lens = np.asarray(lens, dtype=np.int64)
         if np.any(self.host_lens):
             raise RuntimeError("prefill expects an empty cache")
-        desc = torch.from_numpy(self.prefill_tile_desc(lens)).to(self.device)
-        kvq.quantize_tiles(self.cfg, rows_k, rows_v, desc, self.block_tables, self.k_pool, self.v_pool,
-                           num_blocks=self.num_blocks, dev_status=self.dev_status, stream=stream)
-        t = self.cfg.tile_tokens
-        full = (lens // t) * t
-        rest = lens - full
-        if rest.any():
-            starts = np.concatenate([[0], np.cumsum(lens)[:-1]])
-            idx = np.concatenate([np.arange(starts[s] + full[s], starts[s] + lens[s]) for s in range(len(lens))])
-            idx_t = torch.from_numpy(idx).to(self.device)
-            self._append(rows_k.index_select(0, idx_t), rows_v.index_select(0, idx_t), full, rest, stream)
-        self.host_lens = lens.copy()
-        self.seq_lens.copy_(torch.from_numpy(lens.astype(np.int32)))
+        with _on_stream(stream):
+            desc = torch.from_numpy(self.prefill_tile_desc(lens)).to(self.device)
+            kvq.quantize_tiles(self.cfg, rows_k, rows_v, desc, self.block_tables, self.k_pool, self.v_pool,
+                               num_blocks=self.num_blocks, dev_status=self.dev_status)
+            t = self.cfg.tile_tokens
+            full = (lens // t) * t
+            rest = lens - full
+            if rest.any():
+                starts = np.concatenate([[0], np.cumsum(lens)[:-1]])
+                idx = np.concatenate([np.arange(starts[s] + full[s], starts[s] + lens[s]) for s in range(len(lens))])
+                idx_t = torch.from_numpy(idx).to(self.device)
+                self._append(rows_k.index_select(0, idx_t), rows_v.index_select(0, idx_t), full, rest)
+            self.host_lens = lens.copy()
+            self.seq_lens.copy_(torch.from_numpy(lens.astype(np.int32)))
 
-    def _append(self, new_k, new_v, before, counts, stream=None) -> None:
+    def _append(self, new_k, new_v, before, counts) -> None:
+        # runs on the current stream (callers enter _on_stream first)
         cu = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
         kvq.append_tokens(self.cfg, new_k, new_v, torch.from_numpy(cu).to(self.device),
                           torch.from_numpy(np.asarray(before, dtype=np.int32)).to(self.device),
                           int(np.max(counts)), self.block_tables, self.k_pool, self.v_pool, self.k_tail,
-                          self.v_tail, num_blocks=self.num_blocks, dev_status=self.dev_status, stream=stream)
+                          self.v_tail, num_blocks=self.num_blocks, dev_status=self.dev_status)
 
     def append(self, new_k: torch.Tensor, new_v: torch.Tensor, counts=None, stream=None) -> None:
         """Append packed rows (``counts`` per sequence, default one each)."""
@@ -95,24 +119,28 @@ class PagedKVCache:
         counts = np.asarray(counts, dtype=np.int64)
         if np.any(self.host_lens + counts > self.blocks_per_seq * self.cfg.page_tokens):
             raise ValueError("append past the allocated pages")
-        self._append(new_k, new_v, self.host_lens, counts, stream)
-        self.host_lens = self.host_lens + counts
-        self.seq_lens.copy_(torch.from_numpy(self.host_lens.astype(np.int32)))
+        with _on_stream(stream):
+            self._append(new_k, new_v, self.host_lens, counts)
+            self.host_lens = self.host_lens + counts
+            self.seq_lens.copy_(torch.from_numpy(self.host_lens.astype(np.int32)))
 
     # ------------------------------------------------------------------- read
     def decode(self, q: torch.Tensor, out: torch.Tensor | None = None, num_splits: int | None = None,
                stream=None) -> torch.Tensor:
         """One decode step: q fp16 [B][H_q][d] -> out fp16 [B][H_q][d]."""
-        if out is None:
-            out = torch.empty_like(q)
         splits = self.num_splits if num_splits is None else num_splits
-        ws = self.workspace
-        need = kvq.decode_workspace_bytes(self.cfg, self.num_seqs, splits)
-        if ws.numel() < need:
-            ws = torch.empty(need, dtype=torch.uint8, device=self.device)
-        kvq.paged_decode_attention(self.cfg, q, out, self.seq_lens, self.block_tables, self.k_pool, self.v_pool,
-                                   self.k_tail, self.v_tail, ws, num_splits=splits, num_blocks=self.num_blocks,
-                                   dev_status=self.dev_status, stream=stream)
+        with _on_stream(stream):
+            if out is None:
+                out = torch.empty_like(q)
+            ws = self.workspace
+            need = kvq.decode_workspace_bytes(self.cfg, self.num_seqs, splits)
+            if ws.numel() < need:
+                ws = torch.empty(need, dtype=torch.uint8, device=self.device)  # freed after this call's work
+            else:
+                _in_use(ws)
+            kvq.paged_decode_attention(self.cfg, q, out, self.seq_lens, self.block_tables, self.k_pool,
+                                       self.v_pool, self.k_tail, self.v_tail, ws, num_splits=splits,
+                                       num_blocks=self.num_blocks, dev_status=self.dev_status)
         return out
 
     def prefill_chunk(self, q: torch.Tensor, new_k: torch.Tensor, new_v: torch.Tensor, counts,
@@ -129,29 +157,33 @@ class PagedKVCache:
             raise ValueError("counts: one non-negative chunk length per sequence")
         if append and np.any(self.host_lens + counts > self.blocks_per_seq * self.cfg.page_tokens):
             raise ValueError("append past the allocated pages")
-        if out is None:
-            out = torch.empty_like(q)
         max_chunk = int(counts.max()) if counts.size else 0
-        cu = torch.from_numpy(np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)).to(self.device)
         if num_splits is None:
             num_splits = 1
             if self.device.type == "cuda":  # (anything else is refused by the binding below)
                 sms = torch.cuda.get_device_properties(self.device).multi_processor_count
                 num_splits = kvq.prefill_splits(self.cfg, self.num_seqs, max_chunk, int(self.host_lens.max()), sms)
         need = kvq.prefill_workspace_bytes(self.cfg, self.num_seqs, max_chunk, num_splits)
-        ws = None
-        if need > 0:
-            if self.prefill_workspace is None or self.prefill_workspace.numel() < need:
-                self.prefill_workspace = torch.empty(need, dtype=torch.uint8, device=self.device)
-            ws = self.prefill_workspace
-        kvq.paged_prefill_attention(self.cfg, q, out, new_k, new_v, cu, self.seq_lens, max_chunk, self.block_tables,
-                                    self.k_pool, self.v_pool, self.k_tail, self.v_tail, num_splits=num_splits,
-                                    workspace=ws, num_blocks=self.num_blocks, dev_status=self.dev_status,
-                                    stream=stream)
-        if append and max_chunk > 0:
-            self._append(new_k, new_v, self.host_lens, counts, stream)
-            self.host_lens = self.host_lens + counts
-            self.seq_lens.copy_(torch.from_numpy(self.host_lens.astype(np.int32)))
+        with _on_stream(stream):
+            if out is None:
+                out = torch.empty_like(q)
+            cu = torch.from_numpy(np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)).to(self.device)
+            ws = None
+            if need > 0:
+                if self.prefill_workspace is None or self.prefill_workspace.numel() < need:
+                    # the old buffer (if any) may still be read by earlier work on
+                    # another stream: it was marked in use there when it was used
+                    self.prefill_workspace = torch.empty(need, dtype=torch.uint8, device=self.device)
+                ws = self.prefill_workspace
+                _in_use(ws)
+            kvq.paged_prefill_attention(self.cfg, q, out, new_k, new_v, cu, self.seq_lens, max_chunk,
+                                        self.block_tables, self.k_pool, self.v_pool, self.k_tail, self.v_tail,
+                                        num_splits=num_splits, workspace=ws, num_blocks=self.num_blocks,
+                                        dev_status=self.dev_status)
+            if append and max_chunk > 0:
+                self._append(new_k, new_v, self.host_lens, counts)
+                self.host_lens = self.host_lens + counts
+                self.seq_lens.copy_(torch.from_numpy(self.host_lens.astype(np.int32)))
         return out
 
     def status(self) -> int:

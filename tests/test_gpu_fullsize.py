@@ -110,11 +110,12 @@ def _check_tiles(cache, cfg, rows_k, rows_v, samples, stats_k, stats_v):
     for s, ti, r0 in samples:
         for h in range(cfg.num_kv_heads):
             for rows, bits, is_v, st in ((rows_k, cfg.bits_k, False, stats_k), (rows_v, cfg.bits_v, True, stats_v)):
-                ref = o.quantize_tile(rows[r0:r0 + t, h], bits, cfg.iters, dtype=np.float32)
+                tile = rows[r0:r0 + t, h]
+                ref = o.quantize_tile(tile, bits, cfg.iters, dtype=np.float32)
                 g = _gpu_tiles(cache, cfg, s, [ti], h, is_v)[0]
                 g_rot, _ = o.dequantize_tile(g["codes"], g["s_t"], g["z_t"], g["c_t"])
                 meta = np.stack([g["s_t"], g["z_t"]], axis=1)
-                st.add(g["codes"], meta, g["c_t"], g_rot.astype(np.float32), ref)
+                st.add(g["codes"], meta, g["c_t"], g_rot.astype(np.float32), ref, src=(tile, bits, cfg.iters, 0))
 
 
 def _decode_only_ref(cache, cfg, seq: int, head: int, length: int, q_heads: np.ndarray) -> np.ndarray:
@@ -185,13 +186,14 @@ def test_qwen3_4b_full_size():
     length = w.lens[0] + 1
     for seq, head in [(0, 0), (3, 5), (5, 7)]:
         _check_decode(out_h, q_h, cfg, cache, seq, head, length, "qwen3_4b")
-    # end to end for one (sequence, KV head): every one of its 2 x 2048 tiles
-    # within the quantize bar, and the decode over those pages within 1e-3.
-    # The output against attention over the oracle's own quantization is
-    # recorded, not held to 1e-3: over 131073 tokens one allowed difference
-    # (a code off by 1, or 1 fp16 ulp of metadata) on a dominant token can
-    # move it by more (measured: 1.3e-3 on one query head from 14 code and
-    # ~0.02% metadata differences in 33.5 M codes).
+    # End to end for one (sequence, KV head), held as a composition: every one
+    # of its 2 x 2048 tiles within the quantize bar with every code and
+    # metadata difference a rounding tie (checked against the fp64 oracle),
+    # and the decode over those pages within 1e-3.  The output against
+    # attention over the oracle's own quantization is printed, not held to
+    # 1e-3: over 131073 tokens one allowed tie (a code off by 1, or 1 fp16 ulp
+    # of metadata) on a dominant token can move it by more (measured: 1.3e-3
+    # on one query head from 14 code and ~0.02% metadata differences).
     seq, head = 2, 3
     rows_k = np.concatenate([rk_h[starts[seq]:starts[seq] + w.lens[seq], head], new_k[seq:seq + 1, head].cpu().numpy()])
     rows_v = np.concatenate([rv_h[starts[seq]:starts[seq] + w.lens[seq], head], new_v[seq:seq + 1, head].cpu().numpy()])
@@ -202,10 +204,14 @@ def test_qwen3_4b_full_size():
         ref_tiles, tail = o.quantize_sequence(rows, cfg.tile_tokens, bits, cfg.iters, dtype=np.float32)
         gpu_tiles = _gpu_tiles(cache, cfg, seq, range(len(ref_tiles)), head, is_v)
         st = TileStats()
-        for r, gt in zip(ref_tiles, gpu_tiles):
+        t = cfg.tile_tokens
+        for k, (r, gt) in enumerate(zip(ref_tiles, gpu_tiles)):
             g_rot, _ = o.dequantize_tile(gt["codes"], gt["s_t"], gt["z_t"], gt["c_t"])
-            st.add(gt["codes"], np.stack([gt["s_t"], gt["z_t"]], axis=1), gt["c_t"], g_rot.astype(np.float32), r)
+            st.add(gt["codes"], np.stack([gt["s_t"], gt["z_t"]], axis=1), gt["c_t"], g_rot.astype(np.float32), r,
+                   src=(rows[k * t:(k + 1) * t], bits, cfg.iters, 0))
         st.check()
+        print(f"qwen3_4b seq {seq} head {head} {name}: {st.tiles} tiles, {st.code_diffs} code and "
+              f"{st.meta_diffs} metadata differences, all rounding ties")
         hats[name] = (o.sequence_kv_hat(gpu_tiles, tail), o.sequence_kv_hat(ref_tiles, tail))
     for j in range(g):
         on_gpu_pages = o.attention_fp64(qs[j], hats["k"][0], hats["v"][0])

@@ -53,7 +53,8 @@ def test_seeded_quantize_matches_oracle(t, bk, bv, n):
             for h in range(2):
                 x = rows[starts[s] + i * t:starts[s] + (i + 1) * t, h]
                 ref = o.quantize_tile(x, bits, n, dtype=np.float32, seed=SEED)
-                st.add(g["codes"][j, h], g["meta"][j, h], g["cvec"][j, h], g["rot"][j, h], ref)
+                st.add(g["codes"][j, h], g["meta"][j, h], g["cvec"][j, h], g["rot"][j, h], ref,
+                       src=(x, bits, n, SEED))
                 # the GPU's original-domain read-back applies H D_s
                 _, ref_orig = o.dequantize_tile(g["codes"][j, h], g["meta"][j, h][:, 0], g["meta"][j, h][:, 1],
                                                 g["cvec"][j, h], SEED)

@@ -229,6 +229,58 @@ def test_rtn_golden_rows():
         assert codes[0].tolist() == want, (bits, vals)
 
 
+def test_plain_rtn_baseline_golden_rows():
+    # hand-derived rows, tests/golden/plain_rtn_worked_examples.txt: the
+    # fp16 rounding of the scale moves the reconstruction (a baseline that
+    # skipped it, used 2^(b+1) - 1 levels or scaled its input would not match)
+    path = os.path.join(GOLDEN, "plain_rtn_worked_examples.txt")
+    rows = 0
+    with open(path) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            bits, vals, codes, s16, z16, recon = line.split("|")
+            x = np.array([[float(v) for v in vals.split()]], dtype=np.float16)
+            want = np.array([float(v) for v in recon.split()])
+            got = o.plain_rtn_baseline(x, int(bits))
+            np.testing.assert_array_equal(got[0], want)
+            c, s, z = o.asymmetric_rtn(x.astype(np.float64), int(bits))
+            assert c[0].tolist() == [int(v) for v in codes.split()]
+            assert float(np.float16(s[0])) == float(s16) and float(np.float16(z[0])) == float(z16)
+            rows += 1
+    assert rows == 3
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+def test_plain_rtn_baseline_brute_force(bits):
+    # every code is the nearest point of the exact grid z + c s (brute force
+    # over c), the reconstruction uses the fp16-rounded s and z, the row min
+    # comes back exactly, and the error stays within s/2 plus the fp16
+    # rounding of s times the code
+    rng = np.random.default_rng(60 + bits)
+    x = (rng.standard_normal((32, 128)) * rng.uniform(0.05, 40, size=(32, 1))
+         + rng.uniform(-5, 5, size=(32, 1))).astype(np.float16)
+    xd = x.astype(np.float64)
+    qmax = (1 << bits) - 1
+    z = xd.min(axis=1)
+    s = (xd.max(axis=1) - z) / qmax
+    grid = np.arange(qmax + 1)[None, None, :] * s[:, None, None] + z[:, None, None]
+    dist = np.abs(xd[:, :, None] - grid)
+    near = dist <= dist.min(axis=2, keepdims=True) * (1 + 1e-12) + 1e-300
+    # an exact tie between two grid points goes to the even code (half to even)
+    code = np.where(near.sum(axis=2) > 1, np.argmax(near & (np.arange(qmax + 1) % 2 == 0), axis=2),
+                    dist.argmin(axis=2))
+    s16 = s.astype(np.float16).astype(np.float64)
+    z16 = z.astype(np.float16).astype(np.float64)
+    got = o.plain_rtn_baseline(x, bits)
+    np.testing.assert_array_equal(got, code * s16[:, None] + z16[:, None])
+    np.testing.assert_array_equal(got[np.arange(32), xd.argmin(axis=1)], z)
+    bound = s[:, None] / 2 + code * np.abs(s16 - s)[:, None]
+    assert np.all(np.abs(got - xd) <= bound * (1 + 1e-12))
+    assert not np.array_equal(s16, s)  # the fp16 rounding of s is exercised
+
+
 def test_constant_row_gives_zero_scale():
     y = np.full((2, 128), 0.75)
     codes, s, z = o.asymmetric_rtn(y, 4)

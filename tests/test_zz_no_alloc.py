@@ -12,7 +12,7 @@ import numpy as np
 import pytest
 import torch
 
-from parity_helpers import ATTN_REL_L2_MAX, make_cache, rel_l2
+from parity_helpers import make_cache
 from quantized_paged_kv_tile_b200 import build, kvq, synth
 
 
@@ -73,9 +73,7 @@ def test_static_scratch_matches_workspace_entry(over, splits):
                                                   num_blocks=cache.num_blocks, dev_status=cache.dev_status)
     torch.cuda.synchronize()
     assert cache.status() == 0
+    # the same kernels with the same split count on the same inputs: the
+    # outputs are bit-identical to the workspace entry point's, on both calls
     for out in outs:
-        out_h = out.float().cpu().numpy()
-        for s in range(w.num_seqs):
-            for hq in range(w.num_q_heads):
-                err = rel_l2(out_h[s, hq], ref_h[s, hq])
-                assert err <= ATTN_REL_L2_MAX, (s, hq, err)
+        assert torch.equal(out, ref)
