@@ -45,6 +45,7 @@ import numpy as np
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 METRIC = "paged decode attn GB/s & tok/s over quantized KV (% HBM peak); quantize GB/s"
+DECODE_LAUNCHES = 2  # kvq_paged_decode_attention: schedule, tiles (the merge runs inside the tiles kernel)
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -250,6 +251,174 @@ def workload_config(w, world: int) -> dict:
             "l2": f"inputs larger than L2 (fp16 rows {rows_gb:.1f} GB per replica)"}
 
 
+class StepSetup:
+    """Device buffers of one workload's step: every full tile of the batch
+    quantized (kvq_quantize_tiles), the unfinished prefill rows and the new
+    tokens appended (kvq_append_tokens), one decode query per sequence
+    (kvq_paged_decode_attention)."""
+
+    def __init__(self, w, dev):
+        import torch
+        from quantized_paged_kv_tile_b200 import kvq, synth
+        self.w = w
+        self.dev = dev
+        cfg = kvq.Config(num_kv_heads=w.num_kv_heads, group_size=w.group_size, tile_tokens=w.tile_tokens,
+                         bits_k=w.bits_k, bits_v=w.bits_v, iters=w.iters)
+        self.cfg = cfg
+        lay = kvq.get_layout(cfg)
+        self.lay = lay
+        B, H, T = w.num_seqs, w.num_kv_heads, w.tile_tokens
+        lens0 = np.asarray(w.lens, dtype=np.int64)
+        lens1 = lens0 + w.append_tokens
+        self.lens0, self.lens1 = lens0, lens1
+        bps = int(math.ceil(lens1.max() / 16))
+        bt_np = synth.block_table(w, bps)
+        self.nblocks = int(bt_np.max()) + 1
+        self.bt = torch.from_numpy(bt_np).to(dev)
+        total0 = int(lens0.sum())
+        self.rows_k = synth.kv_rows(w, "k", total0, device=dev)
+        self.rows_v = synth.kv_rows(w, "v", total0, device=dev)
+        starts = np.concatenate([[0], np.cumsum(lens0)[:-1]])
+        full0 = (lens0 // T) * T
+        desc_np = np.asarray([(starts[s] + i * T, s, i) for s in range(B) for i in range(lens0[s] // T)],
+                             dtype=np.int32).reshape(-1, 3)
+        self.desc = torch.from_numpy(desc_np).to(dev)
+        # the step's appended rows, contiguous per sequence: the unfinished
+        # prefill rows, then the new tokens
+        rest = [self.rows_k[starts[s] + full0[s]:starts[s] + lens0[s]] for s in range(B)]
+        rest_v = [self.rows_v[starts[s] + full0[s]:starts[s] + lens0[s]] for s in range(B)]
+        nk = synth.kv_rows(w, "k", B * w.append_tokens, device=dev, stream_id=1)
+        nv = synth.kv_rows(w, "v", B * w.append_tokens, device=dev, stream_id=1)
+        a = w.append_tokens
+        self.new_k = torch.cat([t for s in range(B) for t in (rest[s], nk[s * a:(s + 1) * a])]).contiguous()
+        self.new_v = torch.cat([t for s in range(B) for t in (rest_v[s], nv[s * a:(s + 1) * a])]).contiguous()
+        counts = lens1 - full0
+        self.cu_new = torch.from_numpy(np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)).to(dev)
+        self.before = torch.from_numpy(full0.astype(np.int32)).to(dev)
+        self.seq_lens = torch.from_numpy(lens1.astype(np.int32)).to(dev)
+        self.k_pool = torch.zeros((self.nblocks, H, lay["page_bytes_k"]), dtype=torch.uint8, device=dev)
+        self.v_pool = torch.zeros((self.nblocks, H, lay["page_bytes_v"]), dtype=torch.uint8, device=dev)
+        self.k_tail = torch.zeros((B, H, T, 128), dtype=torch.float16, device=dev)
+        self.v_tail = torch.zeros_like(self.k_tail)
+        self.q = synth.queries(w, device=dev)
+        self.out = torch.empty_like(self.q)
+        self.ws = torch.empty(kvq.decode_workspace_bytes(cfg, B, 0), dtype=torch.uint8, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.max_new = int(counts.max())
+        self.bm = byte_model(w, lay["page_bytes_k"], lay["page_bytes_v"])
+        # quantize; append (when there are rows to append); decode = schedule + tiles + merge
+        self.launches = (1 if len(desc_np) else 0) + (1 if self.max_new > 0 else 0) + DECODE_LAUNCHES
+
+    def quantize(self, stream):
+        from quantized_paged_kv_tile_b200 import kvq
+        kvq.quantize_tiles(self.cfg, self.rows_k, self.rows_v, self.desc, self.bt, self.k_pool, self.v_pool,
+                           num_blocks=self.nblocks, dev_status=self.status, stream=stream)
+
+    def append(self, stream):
+        from quantized_paged_kv_tile_b200 import kvq
+        if self.max_new > 0:  # no unfinished prefill rows and no new tokens: nothing to append
+            kvq.append_tokens(self.cfg, self.new_k, self.new_v, self.cu_new, self.before, self.max_new, self.bt,
+                              self.k_pool, self.v_pool, self.k_tail, self.v_tail, num_blocks=self.nblocks,
+                              dev_status=self.status, stream=stream)
+
+    def decode(self, stream):
+        from quantized_paged_kv_tile_b200 import kvq
+        kvq.paged_decode_attention(self.cfg, self.q, self.out, self.seq_lens, self.bt, self.k_pool, self.v_pool,
+                                   self.k_tail, self.v_tail, self.ws, num_blocks=self.nblocks,
+                                   dev_status=self.status, stream=stream)
+
+    def step(self, stream, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        self.quantize(stream)
+        if ev is not None:
+            ev[1].record(stream)
+        self.append(stream)
+        if ev is not None:
+            ev[2].record(stream)
+        self.decode(stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    def check_status(self, where):
+        if int(self.status.item()) != 0:
+            raise RuntimeError(f"device status {int(self.status.item())} {where}")
+
+
+def time_steps(S, stream, steps, warmup):
+    """Warm-up, then `steps` timed steps with CUDA events around each call;
+    returns per-call millisecond lists and the total."""
+    import torch
+    for _ in range(warmup):
+        S.step(stream)
+    torch.cuda.synchronize(S.dev)
+    S.check_status("after warm-up")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(steps):
+        S.step(stream, evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize(S.dev)
+    S.check_status("after the timed steps")
+    return {"q": [e[0].elapsed_time(e[1]) for e in evs], "a": [e[1].elapsed_time(e[2]) for e in evs],
+            "d": [e[2].elapsed_time(e[3]) for e in evs], "total": t0.elapsed_time(t1)}
+
+
+def call_objects(S, t, peak):
+    """The per-call `decode`, `quantize`, `append` objects of a timed step."""
+    w, bm = S.w, S.bm
+    q_avg, d_avg = statistics.mean(t["q"]), statistics.mean(t["d"])
+    d_gbs = bm["decode"] / (d_avg * 1e-3) / 1e9
+    dec = {"gbs": d_gbs, "ms": d_avg, "frac": d_gbs / peak, "tok_per_s": w.num_seqs / (d_avg * 1e-3),
+           "kv_tok_per_s": bm["kv_tokens"] / (d_avg * 1e-3), "bytes": bm["decode"],
+           "fp16_bytes_equiv": bm["kv_tokens"] * w.num_kv_heads * 512}
+    qu = None
+    if bm["quantize"] > 0:
+        q_gbs = bm["quantize"] / (q_avg * 1e-3) / 1e9
+        qu = {"gbs": q_gbs, "ms": q_avg, "frac": q_gbs / peak, "bytes": bm["quantize"]}
+    return dec, qu, {"ms": statistics.mean(t["a"]), "bytes": bm["append"]}
+
+
+def oracle_baseline(wname, w, bm, procs, pairs=None, overrides=None):
+    """The oracle (fp64, spawned processes, one BLAS thread each) on a
+    bounded sample of (sequence, KV head) pairs of the workload, same byte
+    model; with one process it is the single-core figure."""
+    pairs = pairs if pairs is not None else oracle_pairs(w, procs)
+    pool = OraclePool(procs)
+    try:
+        secs = pool.time(wname, overrides or {}, pairs)
+    finally:
+        pool.close()
+    per_pair = pair_bytes(w, bm)
+    nbytes = float(sum(per_pair[s] for s, _ in pairs))
+    return {"value": nbytes / secs / 1e9, "unit": "GB/s", "cores": procs, "kind": "oracle",
+            "sample": f"{len(pairs)} of {w.num_seqs * w.num_kv_heads} (sequence, KV head) pairs: fp64 quantize "
+                      f"of every K and V tile, dequantize, fp64 decode of the query group; {secs:.1f} s wall on "
+                      f"{procs} process{'es' if procs > 1 else ''}, same byte model"}
+
+
+def pair_bytes(w, bm):
+    """Algorithmic step bytes of one (sequence, KV head) pair, per sequence."""
+    d, t, p = 128, w.tile_tokens, 16
+    per_tok_head = d * (w.bits_k + w.bits_v) / 8 + 8 + 4 * d / t
+    lens0 = np.asarray(w.lens, dtype=np.int64)
+    lens1 = lens0 + w.append_tokens
+    full0, full1 = (lens0 // t) * t, (lens1 // t) * t
+    quant = full0 * (2 * d * 2 + per_tok_head)
+    append = (lens0 - full0 + w.append_tokens) * d * 2 * 2 * 2
+    decode = full1 * per_tok_head + full1 / p * 4 / w.num_kv_heads + (lens1 - full1) * d * 2 * 2 + \
+        w.group_size * d * 2 * 2
+    return quant + append + decode
+
+
+def small_pairs(w, n):
+    """n (sequence, KV head) pairs over the shortest sequences (a bounded
+    oracle sample of a workload with long sequences)."""
+    order = np.argsort(np.asarray(w.lens))
+    return [(int(order[i % len(order)]), (i // len(order) + i) % w.num_kv_heads) for i in range(n)]
+
+
 def run_kvq(args, ranks):
     import torch
     from quantized_paged_kv_tile_b200 import build, kvq, synth
@@ -260,76 +429,15 @@ def run_kvq(args, ranks):
     torch.cuda.set_device(dev)
     over = {"num_seqs": args.num_seqs} if args.num_seqs > 0 else {}
     w = synth.workload(args.workload, replica=ranks.rank, **over)
-    cfg = kvq.Config(num_kv_heads=w.num_kv_heads, group_size=w.group_size, tile_tokens=w.tile_tokens,
-                     bits_k=w.bits_k, bits_v=w.bits_v, iters=w.iters)
-    lay = kvq.get_layout(cfg)
-    B, H, T = w.num_seqs, w.num_kv_heads, w.tile_tokens
-    lens0 = np.asarray(w.lens, dtype=np.int64)
-    lens1 = lens0 + w.append_tokens
-    bps = int(math.ceil(lens1.max() / 16))
-    bt_np = synth.block_table(w, bps)
-    nblocks = int(bt_np.max()) + 1
-    bt = torch.from_numpy(bt_np).to(dev)
-    total0 = int(lens0.sum())
-    rows_k = synth.kv_rows(w, "k", total0, device=dev)
-    rows_v = synth.kv_rows(w, "v", total0, device=dev)
-    starts = np.concatenate([[0], np.cumsum(lens0)[:-1]])
-    full0 = (lens0 // T) * T
-    desc_np = np.asarray([(starts[s] + i * T, s, i) for s in range(B) for i in range(lens0[s] // T)],
-                         dtype=np.int32).reshape(-1, 3)
-    desc = torch.from_numpy(desc_np).to(dev)
-    # the step's appended rows: the unfinished prefill rows plus the new tokens
-    new_k = torch.cat([rows_k[starts[s] + full0[s]:starts[s] + lens0[s]] for s in range(B)] +
-                      [synth.kv_rows(w, "k", B * w.append_tokens, device=dev, stream_id=1)])
-    new_v = torch.cat([rows_v[starts[s] + full0[s]:starts[s] + lens0[s]] for s in range(B)] +
-                      [synth.kv_rows(w, "v", B * w.append_tokens, device=dev, stream_id=1)])
-    counts = lens1 - full0
-    # reorder so each sequence's rows are contiguous: rest rows then new rows
-    order = []
-    rest_start = np.concatenate([[0], np.cumsum(lens0 - full0)[:-1]])
-    new_base = int((lens0 - full0).sum())
-    for s in range(B):
-        order += list(range(rest_start[s], rest_start[s] + lens0[s] - full0[s]))
-        order += list(range(new_base + s * w.append_tokens, new_base + (s + 1) * w.append_tokens))
-    order_t = torch.tensor(order, dtype=torch.long, device=dev)
-    new_k, new_v = new_k.index_select(0, order_t).contiguous(), new_v.index_select(0, order_t).contiguous()
-    cu_new = torch.from_numpy(np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)).to(dev)
-    before = torch.from_numpy(full0.astype(np.int32)).to(dev)
-    seq_lens = torch.from_numpy(lens1.astype(np.int32)).to(dev)
-    k_pool = torch.zeros((nblocks, H, lay["page_bytes_k"]), dtype=torch.uint8, device=dev)
-    v_pool = torch.zeros((nblocks, H, lay["page_bytes_v"]), dtype=torch.uint8, device=dev)
-    k_tail = torch.zeros((B, H, T, 128), dtype=torch.float16, device=dev)
-    v_tail = torch.zeros_like(k_tail)
-    q = synth.queries(w, device=dev)
-    out = torch.empty_like(q)
-    ws = torch.empty(kvq.decode_workspace_bytes(cfg, B, 0), dtype=torch.uint8, device=dev)
-    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    S = StepSetup(w, dev)
+    cfg, B, H = S.cfg, w.num_seqs, w.num_kv_heads
     stream = torch.cuda.current_stream(dev)
-    max_new = int(counts.max())
-
-    def step(ev=None):
-        if ev is not None:
-            ev[0].record(stream)
-        kvq.quantize_tiles(cfg, rows_k, rows_v, desc, bt, k_pool, v_pool, num_blocks=nblocks, dev_status=status,
-                           stream=stream)
-        if ev is not None:
-            ev[1].record(stream)
-        if max_new > 0:  # no unfinished prefill rows and no new tokens: nothing to append
-            kvq.append_tokens(cfg, new_k, new_v, cu_new, before, max_new, bt, k_pool, v_pool, k_tail, v_tail,
-                              num_blocks=nblocks, dev_status=status, stream=stream)
-        if ev is not None:
-            ev[2].record(stream)
-        kvq.paged_decode_attention(cfg, q, out, seq_lens, bt, k_pool, v_pool, k_tail, v_tail, ws,
-                                   num_blocks=nblocks, dev_status=status, stream=stream)
-        if ev is not None:
-            ev[3].record(stream)
+    peak, peak_kind = hbm_peak()
 
     for _ in range(args.warmup):
-        step()
+        S.step(stream)
     torch.cuda.synchronize(dev)
-    if int(status.item()) != 0:
-        raise RuntimeError(f"device status {int(status.item())} after warm-up")
-
+    S.check_status("after warm-up")
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     visible = [x for x in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if x.strip()]
     clocks = ClockSampler(visible[ranks.local_rank] if len(visible) > ranks.local_rank else ranks.local_rank)
@@ -340,103 +448,220 @@ def run_kvq(args, ranks):
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
     for i in range(args.steps):
-        step(evs[i])
+        S.step(stream, evs[i])
     t_end.record(stream)
     torch.cuda.synchronize(dev)
     ranks.barrier()
     clk = clocks.stop()
     elapsed_ms = t_start.elapsed_time(t_end)
     max_ms = ranks.max(elapsed_ms)
-    q_ms = [e[0].elapsed_time(e[1]) for e in evs]
-    a_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    d_ms = [e[2].elapsed_time(e[3]) for e in evs]
-
-    bm = byte_model(w, lay["page_bytes_k"], lay["page_bytes_v"])
+    t = {"q": [e[0].elapsed_time(e[1]) for e in evs], "a": [e[1].elapsed_time(e[2]) for e in evs],
+         "d": [e[2].elapsed_time(e[3]) for e in evs]}
+    S.check_status("after the timed steps")
+    bm = S.bm
     step_bytes = bm["quantize"] + bm["append"] + bm["decode"]
     all_bytes = ranks.sum(step_bytes) * args.steps
     value = all_bytes / (max_ms * 1e-3) / 1e9
-    peak, peak_kind = hbm_peak()
-    q_avg, d_avg = statistics.mean(q_ms), statistics.mean(d_ms)
-    q_gbs = bm["quantize"] / (q_avg * 1e-3) / 1e9
-    d_gbs = bm["decode"] / (d_avg * 1e-3) / 1e9
+    dec, qu, app = call_objects(S, t, peak)
+    dec["roofline"] = {"bound": "hbm", "kernel": "decode (schedule + tiles + merge)", "achieved": dec["gbs"],
+                       "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": dec["frac"],
+                       "traffic": None}
 
-    # end to end through the public calls with host buffers: H2D of the step's
-    # inputs (fp16 rows, new rows, q) from pinned memory, the three calls,
-    # D2H of the output
-    e2e = None
+    # end to end through the public calls with host buffers.  (1) the whole
+    # step: H2D of its inputs (fp16 rows, new rows, q) from pinned memory,
+    # the three calls, D2H of the output.  (2) the steady decode step of a
+    # serving loop: H2D of the new token rows and q, append + decode, D2H of
+    # the output.
+    e2e = e2e_decode = None
     if not args.no_e2e:
-        host = {name: t.cpu().pin_memory() for name, t in
-                dict(rows_k=rows_k, rows_v=rows_v, new_k=new_k, new_v=new_v, q=q).items()}
-        out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        host = {name: x.cpu().pin_memory() for name, x in
+                dict(rows_k=S.rows_k, rows_v=S.rows_v, new_k=S.new_k, new_v=S.new_v, q=S.q).items()}
+        out_host = torch.empty(S.out.shape, dtype=S.out.dtype, pin_memory=True)
         d2h = out_host.numel() * out_host.element_size()
-        e2e_steps = max(1, min(args.steps, 3))
 
-        def e2e_step():
-            rows_k.copy_(host["rows_k"], non_blocking=True)
-            rows_v.copy_(host["rows_v"], non_blocking=True)
-            new_k.copy_(host["new_k"], non_blocking=True)
-            new_v.copy_(host["new_v"], non_blocking=True)
-            q.copy_(host["q"], non_blocking=True)
-            step()
-            out_host.copy_(out, non_blocking=True)
+        def e2e_run(names, body, n):
+            def one():
+                for nm in names:
+                    getattr(S, nm).copy_(host[nm], non_blocking=True)
+                body()
+                out_host.copy_(S.out, non_blocking=True)
+            one()
+            torch.cuda.synchronize(dev)
+            ranks.barrier()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(n):
+                one()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            ranks.barrier()
+            return ranks.max(e0.elapsed_time(e1)), sum(host[nm].numel() * host[nm].element_size() for nm in names)
 
-        e2e_step()
-        torch.cuda.synchronize(dev)
-        ranks.barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(e2e_steps):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        ranks.barrier()
-        e_ms = ranks.max(e0.elapsed_time(e1))
-        e2e = {"value": ranks.sum(step_bytes) * e2e_steps / (e_ms * 1e-3) / 1e9, "unit": "GB/s",
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": e2e_steps,
-               "ms_per_step": e_ms / e2e_steps}
-    if int(status.item()) != 0:
-        raise RuntimeError(f"device status {int(status.item())} after the timed steps")
+        n = max(1, min(args.steps, 3))
+        e_ms, h2d = e2e_run(("rows_k", "rows_v", "new_k", "new_v", "q"), lambda: S.step(stream), n)
+        e2e = {"value": ranks.sum(step_bytes) * n / (e_ms * 1e-3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": n, "ms_per_step": e_ms / n}
+        n = max(3, args.steps)
+        e_ms, h2d = e2e_run(("new_k", "new_v", "q"), lambda: (S.append(stream), S.decode(stream)), n)
+        dbytes = ranks.sum(bm["append"] + bm["decode"])
+        e2e_decode = {"value": dbytes * n / (e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                      "tok_per_s": ranks.sum(B) * n / (e_ms * 1e-3), "h2d_bytes_per_step": int(h2d),
+                      "d2h_bytes_per_step": int(d2h), "steps": n, "ms_per_step": e_ms / n,
+                      "what": "steady serving step: new token rows and q from pinned host memory, append + "
+                              "decode, output back to the host"}
+        S.check_status("after the end-to-end steps")
 
+    solo = ranks.rank == 0 and ranks.world == 1
     cpu = None
-    if ranks.rank == 0 and ranks.world == 1 and not args.no_cpu_baseline:
+    if solo and not args.no_cpu_baseline:
         procs = max(1, min(os.cpu_count() or 1, 8))
-        pairs = oracle_pairs(w, procs)
-        pool = OraclePool(procs)
-        try:
-            secs = pool.time(args.workload, {}, pairs)
-        finally:
-            pool.close()
-        cpu = {"value": cpu_sample_bytes(w, bm, len(pairs)) / secs / 1e9, "unit": "GB/s", "cores": procs,
-               "kind": "oracle",
-               "sample": f"{len(pairs)} of {B * H} (sequence, KV head) pairs: fp64 quantize of every K and V "
-                         f"tile, dequantize, fp64 decode of the query group; {secs:.1f} s wall on {procs} "
-                         f"processes, same byte model"}
+        cpu = oracle_baseline(args.workload, w, bm, procs)
+        cpu["single_core"] = oracle_baseline(args.workload, w, bm, 1, pairs=oracle_pairs(w, 1))
 
-    # quantize; append (when there are rows to append); decode = schedule + tiles + merge
-    launches_per_step = 1 + (1 if max_new > 0 else 0) + 3
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": ranks.world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": workload_config(w, ranks.world),
-        "decode": {"gbs": d_gbs, "ms": d_avg, "frac": d_gbs / peak, "tok_per_s": B / (d_avg * 1e-3),
-                   "kv_tok_per_s": bm["kv_tokens"] / (d_avg * 1e-3), "bytes": bm["decode"],
-                   "fp16_bytes_equiv": bm["kv_tokens"] * H * 512},
-        "quantize": {"gbs": q_gbs, "ms": q_avg, "frac": q_gbs / peak, "bytes": bm["quantize"]},
-        "append": {"ms": statistics.mean(a_ms), "bytes": bm["append"]},
-        "roofline": {"bound": "hbm", "kernel": "quantize_tc_kernel", "achieved": q_gbs, "peak": peak,
-                     "peak_kind": peak_kind, "unit": "GB/s", "frac": q_gbs / peak,
+        "decode": dec, "quantize": qu, "append": app,
+        "roofline": {"bound": "hbm", "kernel": "quantize_tc_kernel", "achieved": qu["gbs"], "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": qu["frac"],
                      "traffic": ncu_traffic("quantize_tc_kernel", bm["quant_units"])},
-        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps, "clocks": clk,
+        "cpu_baseline": cpu, "e2e": e2e, "e2e_decode_step": e2e_decode,
+        "gpu_launches": S.launches * args.steps, "clocks": clk,
     }
-    if args.serving_steps > 0:
-        line["serving"] = serving_loop(w, cfg, rows_k, rows_v, args.serving_steps, dev)
     if args.prefill_chunk > 0:
-        line["prefill"] = prefill_leg(w, cfg, args, dev, stream, seq_lens, bt, nblocks, k_pool, v_pool, k_tail,
-                                      v_tail, status, lens1)
+        line["prefill"] = prefill_leg(w, cfg, args, dev, stream, S.seq_lens, S.bt, S.nblocks, S.k_pool, S.v_pool,
+                                      S.k_tail, S.v_tail, S.status, S.lens1, cpu_ok=solo)
         line["gpu_launches_prefill"] = args.steps * line["prefill"]["launches_per_call"]
+    rows_kv = (S.rows_k, S.rows_v)
+    if args.serving_steps > 0:
+        line["serving"] = serving_loop(w, cfg, *rows_kv, args.serving_steps, dev)
+    del S, rows_kv
+    torch.cuda.empty_cache()
+    if solo and not args.headline_only and args.workload == "qwen3_4b" and args.num_seqs == 0:
+        line["workloads"] = other_workloads(args, dev, stream, peak)
     return line
+
+
+def other_workloads(args, dev, stream, peak):
+    """The other four workloads through the same calls (one GPU, after the
+    headline): a few timed steps each (3 warm-up + min(steps, 5) timed), each
+    with its own oracle baseline."""
+    import torch
+    from quantized_paged_kv_tile_b200 import synth
+    steps = max(1, min(args.steps, 5))
+    procs = max(1, min(os.cpu_count() or 1, 8))
+    res = {}
+    for name in ("tiny", "mixed", "qwen3_32b_burst"):
+        w = synth.workload(name)
+        S = StepSetup(w, dev)
+        t = time_steps(S, stream, steps, 3)
+        dec, qu, app = call_objects(S, t, peak)
+        obj = {"config": workload_config(w, 1), "steps": steps, "decode": dec, "quantize": qu, "append": app,
+               "step_ms": t["total"] / steps}
+        if name == "tiny":
+            obj["note"] = "latency-bound: the whole workload fits in L2; a correctness case, not a roofline case"
+        if not args.no_cpu_baseline:
+            pairs = oracle_pairs(w, procs) if name != "mixed" else small_pairs(w, procs)
+            obj["cpu_baseline"] = oracle_baseline(name, w, S.bm, procs, pairs=pairs)
+            if name == "mixed":
+                obj["cpu_baseline"]["sample"] += " (the shortest sequences)"
+        if name == "qwen3_32b_burst":
+            obj["serving"] = serving_loop(w, S.cfg, S.rows_k, S.rows_v, w.decode_steps, dev)
+            obj["serving"]["what"] = (f"{w.decode_steps} steps after the 64 x 16384-token prefill, each one "
+                                      f"CUDA-graph replay of kvq_append_tokens (1 token per sequence) + "
+                                      f"kvq_paged_decode_attention; tile-completion steps (T = 128) apart")
+        res[name] = obj
+        del S
+        torch.cuda.empty_cache()
+    res["prefill_sweep"] = prefill_sweep(args, dev, stream, peak, procs)
+    return res
+
+
+def prefill_sweep(args, dev, stream, peak, procs):
+    """The 27 (T, b, n) points of the prefill sweep: kvq_quantize_tiles over all
+    32 x 16384 new tokens of 8 KV heads, GB/s, and the method's reconstruction
+    MSE against plain per-token RTN on a seeded sample of K tiles."""
+    import torch
+    from quantized_paged_kv_tile_b200 import kvq, synth
+    w0 = synth.workload("prefill_sweep")
+    total = int(sum(w0.lens))
+    rows_k = synth.kv_rows(w0, "k", total, device=dev)
+    rows_v = synth.kv_rows(w0, "v", total, device=dev)
+    starts = np.concatenate([[0], np.cumsum(w0.lens)[:-1]]).astype(np.int64)
+    rng = np.random.default_rng(4444)
+    points = []
+    for T in (32, 64, 128):
+        for b in (2, 3, 4):
+            for n in (1, 4, 8):
+                w = synth.workload("prefill_sweep", tile_tokens=T, bits_k=b, bits_v=b, iters=n)
+                cfg = kvq.Config(num_kv_heads=w.num_kv_heads, group_size=w.group_size, tile_tokens=T, bits_k=b,
+                                 bits_v=b, iters=n)
+                lay = kvq.get_layout(cfg)
+                bps = int(math.ceil(max(w.lens) / 16))
+                bt = torch.from_numpy(synth.block_table(w, bps)).to(dev)
+                nblocks = w.num_seqs * bps
+                k_pool = torch.zeros((nblocks, w.num_kv_heads, lay["page_bytes_k"]), dtype=torch.uint8, device=dev)
+                v_pool = torch.zeros((nblocks, w.num_kv_heads, lay["page_bytes_v"]), dtype=torch.uint8, device=dev)
+                desc = torch.from_numpy(np.asarray([(starts[s] + i * T, s, i) for s in range(w.num_seqs)
+                                                    for i in range(w.lens[s] // T)], dtype=np.int32)).to(dev)
+                status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+                def call():
+                    kvq.quantize_tiles(cfg, rows_k, rows_v, desc, bt, k_pool, v_pool, num_blocks=nblocks,
+                                       dev_status=status, stream=stream)
+                for _ in range(2):
+                    call()
+                torch.cuda.synchronize(dev)
+                e = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(3)]
+                for e0, e1 in e:
+                    e0.record(stream)
+                    call()
+                    e1.record(stream)
+                torch.cuda.synchronize(dev)
+                if int(status.item()) != 0:
+                    raise RuntimeError(f"device status {int(status.item())} in the sweep at T={T} b={b} n={n}")
+                ms = statistics.mean(a.elapsed_time(c) for a, c in e)
+                nbytes = byte_model(w, 0, 0)["quantize"]
+                gbs = nbytes / (ms * 1e-3) / 1e9
+                # reconstruction of sampled K tiles: the GPU's pages read back
+                # (original domain) against the fp16 rows, and plain per-token
+                # RTN (fp16 scale and zero, no rotation or normalization) of the
+                # same rows
+                picks = [(int(rng.integers(w.num_seqs)), int(rng.integers(w.lens[0] // T))) for _ in range(4)]
+                td = torch.tensor(picks, dtype=torch.int32, device=dev)
+                orig = torch.empty((len(picks), w.num_kv_heads, T, 128), dtype=torch.float32, device=dev)
+                kvq.unpack_tiles(cfg, td, bt, k_pool, False, out_orig=orig, num_blocks=nblocks, dev_status=status)
+                x = torch.stack([rows_k[starts[s] + i * T:starts[s] + (i + 1) * T].permute(1, 0, 2)
+                                 for s, i in picks]).double()
+                mse_m = float(((orig.double() - x) ** 2).mean())
+                mse_p = float(((plain_rtn(x, b) - x) ** 2).mean())
+                points.append({"T": T, "b": b, "n": n, "ms": ms, "gbs": gbs, "frac": gbs / peak, "bytes": nbytes,
+                               "mse_method": mse_m, "mse_plain_rtn": mse_p, "mse_ratio": mse_m / mse_p})
+                del k_pool, v_pool
+    head = next(p for p in points if (p["T"], p["b"], p["n"]) == (64, 4, 4))
+    res = {"points": points, "headline_point": head,
+           "what": "32 seqs x 16384 new tokens, 8 KV heads, K and V, outlier channels 1-5% x[5, 50]; 2 warm-up "
+                   "+ 3 timed kvq_quantize_tiles calls per point; MSE on 4 seeded K tiles x 8 heads per point"}
+    if not args.no_cpu_baseline:
+        res["cpu_baseline"] = oracle_baseline("prefill_sweep", w0, byte_model(w0, 0, 0), procs)
+    del rows_k, rows_v
+    torch.cuda.empty_cache()
+    return res
+
+
+def plain_rtn(x, bits):
+    """Plain per-token asymmetric RTN of fp16 rows x[..., d] (no rotation, no
+    normalization): codes from the exact scale, reconstruction with fp16
+    scale and zero (the comparator of the method-value check)."""
+    import torch
+    qmax = (1 << bits) - 1
+    z = x.amin(dim=-1, keepdim=True)
+    s = (x.amax(dim=-1, keepdim=True) - z) / qmax
+    code = torch.where(s > 0, torch.clamp(torch.round((x - z) / torch.where(s > 0, s, torch.ones_like(s))), 0, qmax),
+                       torch.zeros_like(x))
+    return code * s.half().double() + z.half().double()
 
 
 def prefill_cpu_sample(w, chunk: int, ctx_tokens: int = 16384, tokens: int = 64):
@@ -464,7 +689,8 @@ def prefill_cpu_sample(w, chunk: int, ctx_tokens: int = 16384, tokens: int = 64)
     return prefill_flops([ctx_tokens], tokens, w.group_size), secs
 
 
-def prefill_leg(w, cfg, args, dev, stream, seq_lens, bt, nblocks, k_pool, v_pool, k_tail, v_tail, status, lens1):
+def prefill_leg(w, cfg, args, dev, stream, seq_lens, bt, nblocks, k_pool, v_pool, k_tail, v_tail, status, lens1,
+                cpu_ok=True):
     """Chunked prefill over the step's cache: every sequence gets
     ``--prefill-chunk`` new tokens attending to its cached tokens and
     causally to themselves (one library call, inputs resident in HBM)."""
@@ -505,7 +731,7 @@ def prefill_leg(w, cfg, args, dev, stream, seq_lens, bt, nblocks, k_pool, v_pool
     peak, kind = tensor_peak()
     tflops = flops / (ms * 1e-3) / 1e12
     cpu = None
-    if not args.no_cpu_baseline and os.environ.get("RANK", "0") == "0" and os.environ.get("WORLD_SIZE", "1") == "1":
+    if not args.no_cpu_baseline and cpu_ok:
         sflops, secs = prefill_cpu_sample(w, n)
         cpu = {"value": sflops / secs / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
                "sample": f"1 (sequence, KV head), a 16384-token context quantized by the oracle (untimed), then "
@@ -599,8 +825,11 @@ def main():
                     help="override the workload's sequence count (smaller inputs for profiler captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--prefill-chunk", type=int, default=0,
-                    help="also time chunked-prefill attention of this many new tokens per sequence over the cache")
+    ap.add_argument("--prefill-chunk", type=int, default=512,
+                    help="also time chunked-prefill attention of this many new tokens per sequence over the cache "
+                         "(0: off)")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="only the headline workload (no sub-objects for the other workloads)")
     ap.add_argument("--serving-steps", type=int, default=0,
                     help="after the measurement, time this many graph-replayed append+decode serving steps")
     args = ap.parse_args()

@@ -32,3 +32,30 @@ def test_prefill_cpu_sample_runs_the_oracle():
     w = synth.workload("qwen3_4b")
     flops, secs = bench.prefill_cpu_sample(w, 512, ctx_tokens=128, tokens=4)
     assert flops == bench.prefill_flops([128], 4, w.group_size) and secs > 0
+
+
+def test_plain_rtn_comparator_matches_the_oracle():
+    # bench.py computes the sweep's plain-RTN MSE with torch on the device;
+    # on the CPU it must equal the oracle's plain_rtn_baseline exactly
+    import numpy as np
+    import torch
+    import bench
+    from oracle import kvq_oracle as o
+    rng = np.random.default_rng(12)
+    for bits in (2, 3, 4):
+        x = (rng.standard_normal((64, 128)) * rng.uniform(0.1, 30, size=(64, 1))).astype(np.float16)
+        got = bench.plain_rtn(torch.from_numpy(x).double(), bits).numpy()
+        np.testing.assert_array_equal(got, o.plain_rtn_baseline(x, bits))
+
+
+def test_pair_bytes_add_up_to_the_step():
+    # per-(sequence, KV head) bytes summed over every pair give the step's bytes
+    import numpy as np
+    import bench
+    from quantized_paged_kv_tile_b200 import synth
+    for name in ("qwen3_4b", "mixed", "qwen3_32b_burst", "tiny"):
+        w = synth.workload(name)
+        bm = bench.byte_model(w, 0, 0)
+        total = bm["quantize"] + bm["append"] + bm["decode"]
+        per = bench.pair_bytes(w, bm)
+        assert abs(float(np.sum(per)) * w.num_kv_heads - total) <= 1e-9 * total, name
