@@ -112,6 +112,53 @@ def ncu_traffic(kernel: str, units_now: float):
     return rec["dram_bytes_per_launch"] * units_now / rec["units_per_launch"]
 
 
+TRAFFIC_UNITS = {
+    "quantize_tc_kernel": ("quant_units", "element of the fp16 K/V rows quantized (token x KV head x K|V x channel)"),
+    "decode_tiles_kernel": ("decode", "algorithmic byte of the decode call (the byte model's decode figure)"),
+}
+
+
+def record_traffic(csv_path: str, workload: str, num_seqs: int, command: str, out_path: str = None):
+    """Write the traffic record of every kernel of KERNEL_SOURCES found in an
+    `ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum
+    --csv` capture of `command` (run on `workload` with `num_seqs` sequences):
+    DRAM bytes per launch (the mean over the captured launches), the units that
+    launch processed by the byte model, and the digest of the kernel's sources."""
+    import csv
+    from quantized_paged_kv_tile_b200 import synth
+    with open(csv_path) as f:
+        lines = [ln for ln in f if ln.startswith('"')]
+    rows = list(csv.DictReader(lines))
+    over = {"num_seqs": num_seqs} if num_seqs > 0 else {}
+    bm = byte_model(synth.workload(workload, **over), 0, 0)
+    out_path = out_path or os.path.join(ROOT, "profiles", "traffic.json")
+    rec = {}
+    for kernel, (unit_key, unit_text) in TRAFFIC_UNITS.items():
+        launches = {}
+        for r in rows:
+            if kernel in r["Kernel Name"]:
+                launches.setdefault(r["ID"], {})[r["Metric Name"]] = float(r["Metric Value"].replace(",", ""))
+        if not launches:
+            continue
+        need = ("dram__bytes_read.sum", "dram__bytes_write.sum", "gpu__time_duration.sum")
+        if any(m not in l for l in launches.values() for m in need):
+            raise ValueError(f"{csv_path}: a {kernel} launch lacks one of {need}")
+        n = len(launches)
+        rd = sum(l["dram__bytes_read.sum"] for l in launches.values()) / n
+        wr = sum(l["dram__bytes_write.sum"] for l in launches.values()) / n
+        rec[kernel] = {"source_digest": source_digest(kernel), "dram_bytes_per_launch": rd + wr,
+                       "units_per_launch": bm[unit_key], "unit": unit_text, "capture": command,
+                       "launches_captured": n, "dram_bytes_read": rd, "dram_bytes_write": wr,
+                       "duration_ns_under_ncu": sum(l["gpu__time_duration.sum"] for l in launches.values()) / n,
+                       "workload": f"{workload}, num_seqs={num_seqs or 'default'}"}
+    if not rec:
+        raise ValueError(f"{csv_path}: no launch of {sorted(TRAFFIC_UNITS)}")
+    with open(out_path, "w") as f:
+        json.dump(rec, f, indent=1)
+        f.write("\n")
+    return rec
+
+
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -306,7 +353,7 @@ class StepSetup:
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         self.max_new = int(counts.max())
         self.bm = byte_model(w, lay["page_bytes_k"], lay["page_bytes_v"])
-        # quantize; append (when there are rows to append); decode = schedule + tiles + merge
+        # quantize; append (when there are rows to append); decode = schedule + tiles (the merge runs inside)
         self.launches = (1 if len(desc_np) else 0) + (1 if self.max_new > 0 else 0) + DECODE_LAUNCHES
 
     def quantize(self, stream):
@@ -463,9 +510,9 @@ def run_kvq(args, ranks):
     all_bytes = ranks.sum(step_bytes) * args.steps
     value = all_bytes / (max_ms * 1e-3) / 1e9
     dec, qu, app = call_objects(S, t, peak)
-    dec["roofline"] = {"bound": "hbm", "kernel": "decode (schedule + tiles + merge)", "achieved": dec["gbs"],
+    dec["roofline"] = {"bound": "hbm", "kernel": "decode (schedule + tiles)", "achieved": dec["gbs"],
                        "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": dec["frac"],
-                       "traffic": None}
+                       "traffic": ncu_traffic("decode_tiles_kernel", bm["decode"])}
 
     # end to end through the public calls with host buffers.  (1) the whole
     # step: H2D of its inputs (fp16 rows, new rows, q) from pinned memory,
@@ -568,10 +615,13 @@ def other_workloads(args, dev, stream, peak):
             if name == "mixed":
                 obj["cpu_baseline"]["sample"] += " (the shortest sequences)"
         if name == "qwen3_32b_burst":
-            obj["serving"] = serving_loop(w, S.cfg, S.rows_k, S.rows_v, w.decode_steps, dev)
+            obj["serving"] = serving_loop(w, S.cfg, S.rows_k, S.rows_v, w.decode_steps, dev, fused=True)
             obj["serving"]["what"] = (f"{w.decode_steps} steps after the 64 x 16384-token prefill, each one "
-                                      f"CUDA-graph replay of kvq_append_tokens (1 token per sequence) + "
-                                      f"kvq_paged_decode_attention; tile-completion steps (T = 128) apart")
+                                      f"CUDA-graph replay: kvq_append_decode_step (one launch) on steps that "
+                                      f"complete no tile, kvq_append_tokens + kvq_paged_decode_attention on the "
+                                      f"tile-completion steps (T = 128), reported apart")
+            obj["serving_unfused"] = serving_loop(w, S.cfg, S.rows_k, S.rows_v, w.decode_steps, dev, fused=False)
+            obj["serving_unfused"]["what"] = "the same loop with every step as append + length update + decode"
         res[name] = obj
         del S
         torch.cuda.empty_cache()
@@ -746,18 +796,21 @@ def prefill_leg(w, cfg, args, dev, stream, seq_lens, bt, nblocks, k_pool, v_pool
                                  "so its tensor-core work is twice this"}}
 
 
-def serving_loop(w, cfg, rows_k, rows_v, steps, dev):
+def serving_loop(w, cfg, rows_k, rows_v, steps, dev, fused=False):
     """The serving loop of the workload after its prefill: ``steps`` graph-
     replayed steps of one appended token per sequence plus a decode, each
-    timed with CUDA events; tile-completion steps reported apart."""
+    timed with CUDA events; tile-completion steps reported apart.  With
+    ``fused`` the steps that complete no tile are one launch
+    (kvq_append_decode_step)."""
     import torch
-    from quantized_paged_kv_tile_b200 import synth
+    from quantized_paged_kv_tile_b200 import kvq, synth
     from quantized_paged_kv_tile_b200.paged import DecodeStepGraph, PagedKVCache
     lens0 = np.asarray(w.lens, dtype=np.int64)
     bps = int(math.ceil((lens0.max() + steps) / 16))
     cache = PagedKVCache(cfg, w.num_seqs, bps * 16, device=dev, block_table=synth.block_table(w, bps))
     cache.prefill(rows_k, rows_v, lens0)
-    graph = DecodeStepGraph(cache)
+    splits = kvq.step_splits(cfg, w.num_seqs, torch.cuda.get_device_properties(dev).multi_processor_count)
+    graph = DecodeStepGraph(cache, num_splits=splits, fused=fused)
     ms, done = [], []
     for i in range(steps):
         graph.new_k.copy_(synth.kv_rows(w, "k", w.num_seqs, device=dev, stream_id=1 + i))
@@ -775,7 +828,10 @@ def serving_loop(w, cfg, rows_k, rows_v, steps, dev):
     t = np.array([a.elapsed_time(b) for a, b in ms])
     comp = t[np.array(done)]
     plain = t[~np.array(done)]
-    return {"steps": steps, "graph": True, "mean_ms": float(t.mean()), "p50_ms": float(np.percentile(t, 50)),
+    return {"steps": steps, "graph": True, "fused": fused, "num_splits": splits,
+            "launches_per_step": "1 (2 + 1 length update on tile-completion steps)" if fused else
+            f"{1 + 1 + DECODE_LAUNCHES} (append, length update, decode)",
+            "mean_ms": float(t.mean()), "p50_ms": float(np.percentile(t, 50)),
             "p99_ms": float(np.percentile(t, 99)), "completion_steps": int(comp.size),
             "completion_step_ms": float(comp.mean()) if comp.size else None,
             "other_step_ms": float(plain.mean()) if plain.size else None,
@@ -832,7 +888,16 @@ def main():
                     help="only the headline workload (no sub-objects for the other workloads)")
     ap.add_argument("--serving-steps", type=int, default=0,
                     help="after the measurement, time this many graph-replayed append+decode serving steps")
+    ap.add_argument("--record-traffic", metavar="CSV",
+                    help="write profiles/traffic.json from an ncu --csv capture (dram bytes read/write and duration) "
+                         "of the command given by --traffic-command on --workload/--num-seqs, then exit (no GPU)")
+    ap.add_argument("--traffic-command", default="")
     args = ap.parse_args()
+    if args.record_traffic:
+        sys.path.insert(0, ROOT)
+        rec = record_traffic(args.record_traffic, args.workload, args.num_seqs, args.traffic_command)
+        print(json.dumps({k: v["dram_bytes_per_launch"] for k, v in rec.items()}))
+        return 0
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     sys.path.insert(0, ROOT)

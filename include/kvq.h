@@ -114,7 +114,7 @@ extern "C" {
 typedef enum {
   KVQ_OK = 0,
   KVQ_ERR_INVALID_ARG = 1,   /* bad pointer, size, or configuration value   */
-  KVQ_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. decode b=3) */
+  KVQ_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. d = 64)     */
   KVQ_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed        */
   KVQ_ERR_WORKSPACE = 4,     /* decode workspace smaller than required      */
   KVQ_ERR_DEVICE_BOUNDS = 5, /* device saw a block id out of range          */
@@ -203,8 +203,10 @@ KVQ_API kvq_status kvq_append_tokens(const kvq_config* cfg, const void* new_k, c
  *   num_splits   : split-K factor over tiles per (sequence, KV head); 0 picks
  *                  one from the device size.  The output does not depend on it
  *                  beyond rounding.
- * Decode supports b in {2, 4} for K and V, and 8 for both
- * (KVQ_ERR_UNSUPPORTED for 3). */
+ * Decode reads b in {2, 3, 4} for K and V (any combination), and 8 for
+ * both.  3-bit pages are read code by code (their V layout is a plain
+ * bitstream), so a 3-bit decode costs more instructions per byte than the
+ * 2- and 4-bit ones. */
 KVQ_API kvq_status kvq_paged_decode_attention(const kvq_config* cfg, const void* q, void* out,
                                       const int32_t* seq_lens, int num_seqs,
                                       const int32_t* block_tables, int max_blocks_per_seq,
@@ -213,6 +215,43 @@ KVQ_API kvq_status kvq_paged_decode_attention(const kvq_config* cfg, const void*
                                       float softmax_scale, void* workspace,
                                       size_t workspace_bytes, int num_splits,
                                       int32_t* dev_status, void* stream);
+
+/* One serving step in one launch: append one token per sequence and decode.
+ * The pages say the per-step read path decides the serving gain (aitrends.kr
+ * article 74976, "TL;DR"); this call folds the step's append into the
+ * decode launch, for steps in which no sequence completes a tile.
+ *   new_k, new_v : device fp16 [num_seqs][num_kv_heads][d], the step's token
+ *                  of every sequence.
+ *   seq_lens     : device int32 [num_seqs], tokens cached BEFORE the step;
+ *                  the call advances every entry by one when it finishes.
+ *   q, out       : as kvq_paged_decode_attention (attention over the cache
+ *                  including the step's token).
+ *   k_tail, v_tail: device fp16 tails; the token goes to row seq_len mod T.
+ *   num_splits   : 1..65535 chunks per (sequence, KV head), fixed (no
+ *                  schedule launch); units past a short sequence's tiles are
+ *                  empty.
+ *   workspace    : device, >= kvq_decode_workspace_bytes(cfg, num_seqs,
+ *                  num_splits) bytes, ZERO-FILLED before its first use (for
+ *                  example cudaMemset at allocation).  Every call that
+ *                  completes leaves its counters at zero again, so the same
+ *                  workspace serves the next step without a clear; after a
+ *                  call that reported a device error, zero it again.  Do not
+ *                  share it with kvq_paged_decode_attention calls.
+ * The result (out, tails, seq_lens) equals kvq_append_tokens of the same
+ * rows, the lengths advanced by one, then kvq_paged_decode_attention with the
+ * same num_splits (bit for bit).  Precondition: no sequence's token completes
+ * a tile (seq_len + 1 is not a multiple of T); such a token has to be
+ * quantized into pages, which this launch does not do: it is not written,
+ * KVQ_ERR_DEVICE_BOUNDS is reported, and that sequence's output is not
+ * valid.  Use kvq_append_tokens then kvq_paged_decode_attention for those
+ * steps.  Host-side errors as kvq_paged_decode_attention; the call is
+ * asynchronous on stream. */
+KVQ_API kvq_status kvq_append_decode_step(const kvq_config* cfg, const void* new_k, const void* new_v,
+                                          const void* q, void* out, int32_t* seq_lens, int num_seqs,
+                                          const int32_t* block_tables, int max_blocks_per_seq, int num_blocks,
+                                          const void* k_pool, const void* v_pool, void* k_tail, void* v_tail,
+                                          float softmax_scale, void* workspace, size_t workspace_bytes,
+                                          int num_splits, int32_t* dev_status, void* stream);
 
 /* Bytes of device workspace kvq_paged_prefill_attention needs with num_splits
  * context splits (0 for num_splits = 1).  cfg, bytes: host pointers. */
@@ -264,7 +303,7 @@ KVQ_API kvq_status kvq_prefill_workspace_bytes(const kvq_config* cfg, int num_se
  * longer than max_chunk_tokens, or negative, is reported through dev_status
  * (KVQ_ERR_DEVICE_BOUNDS) and only its first max_chunk_tokens tokens are
  * written; pages outside the pool likewise (the tile is skipped).  b in
- * {2, 4} for K and V, or 8 for both (KVQ_ERR_UNSUPPORTED for 3). */
+ * {2, 3, 4} for K and V (any combination), or 8 for both. */
 KVQ_API kvq_status kvq_paged_prefill_attention(const kvq_config* cfg, const void* q, void* out,
                                        const void* k_new, const void* v_new, const int32_t* cu_chunk,
                                        const int32_t* ctx_lens, int num_seqs, int max_chunk_tokens,

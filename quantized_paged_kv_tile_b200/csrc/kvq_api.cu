@@ -220,8 +220,6 @@ kvq_status kvq_paged_decode_attention(const kvq_config* cfg, const void* q, void
                                       const void* v_tail, float softmax_scale, void* workspace,
                                       size_t workspace_bytes, int num_splits, int32_t* dev_status, void* stream) {
   KVQ_TRY(check_config(cfg));
-  if (cfg->bits_k == 3 || cfg->bits_v == 3)
-    return fail(KVQ_ERR_UNSUPPORTED, "decode reads 2-, 4- or 8-bit codes only (3-bit pages are storage-only)");
   if (num_seqs < 0 || num_splits < 0) return fail(KVQ_ERR_INVALID_ARG, "negative num_seqs or num_splits");
   if (num_seqs == 0) return ok();
   if (num_seqs > 65535) return fail(KVQ_ERR_INVALID_ARG, "num_seqs > 65535");
@@ -266,6 +264,63 @@ kvq_status kvq_paged_decode_attention(const kvq_config* cfg, const void* q, void
                      "kvq_paged_decode_attention launch");
 }
 
+kvq_status kvq_append_decode_step(const kvq_config* cfg, const void* new_k, const void* new_v, const void* q,
+                                  void* out, int32_t* seq_lens, int num_seqs, const int32_t* block_tables,
+                                  int max_blocks_per_seq, int num_blocks, const void* k_pool, const void* v_pool,
+                                  void* k_tail, void* v_tail, float softmax_scale, void* workspace,
+                                  size_t workspace_bytes, int num_splits, int32_t* dev_status, void* stream) {
+  KVQ_TRY(check_config(cfg));
+  if (num_seqs < 0) return fail(KVQ_ERR_INVALID_ARG, "negative num_seqs");
+  if (num_seqs == 0) return ok();
+  if (num_seqs > 65535) return fail(KVQ_ERR_INVALID_ARG, "num_seqs > 65535");
+  if (num_splits < 1 || num_splits > 65535)
+    return fail(KVQ_ERR_INVALID_ARG, "num_splits must be 1..65535 for the serving step (got %d)", num_splits);
+  if (static_cast<long long>(num_seqs) * cfg->num_kv_heads * num_splits > 0x7fffffffLL)
+    return fail(KVQ_ERR_INVALID_ARG, "num_seqs x num_kv_heads x num_splits too large for one launch");
+  if (!(softmax_scale > 0.f) || !(softmax_scale < 1e30f))
+    return fail(KVQ_ERR_INVALID_ARG, "softmax_scale must be a positive finite float");
+  KVQ_TRY(check_ptr(new_k, "new_k"));
+  KVQ_TRY(check_ptr(new_v, "new_v"));
+  KVQ_TRY(check_ptr(q, "q"));
+  KVQ_TRY(check_ptr(out, "out"));
+  KVQ_TRY(check_ptr(seq_lens, "seq_lens"));
+  KVQ_TRY(check_tables(block_tables, max_blocks_per_seq, num_blocks));
+  KVQ_TRY(check_ptr(k_pool, "k_pool"));
+  KVQ_TRY(check_ptr(v_pool, "v_pool"));
+  KVQ_TRY(check_ptr(k_tail, "k_tail"));
+  KVQ_TRY(check_ptr(v_tail, "v_tail"));
+  KVQ_TRY(check_ptr(workspace, "workspace"));
+  KVQ_TRY(check_ptr(dev_status, "dev_status", true));
+  const size_t need = kvq::decode_workspace_bytes(*cfg, num_seqs, num_splits, 0);
+  if (workspace_bytes < need)
+    return fail(KVQ_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, need);
+  kvq::DecodeArgs a{};
+  a.cfg = *cfg;
+  a.gk = kvq::pool_geom(*cfg, false);
+  a.gv = kvq::pool_geom(*cfg, true);
+  a.q = q;
+  a.out = out;
+  a.seq_lens = seq_lens;
+  a.seq_lens_rw = seq_lens;
+  a.num_seqs = num_seqs;
+  a.block_tables = block_tables;
+  a.max_blocks_per_seq = max_blocks_per_seq;
+  a.num_blocks = num_blocks;
+  a.k_pool = k_pool;
+  a.v_pool = v_pool;
+  a.k_tail = k_tail;
+  a.v_tail = v_tail;
+  a.softmax_scale = softmax_scale;
+  a.workspace = workspace;
+  a.num_splits_fixed = num_splits;
+  a.dev_status = dev_status;
+  a.step = 1;
+  a.new_k = new_k;
+  a.new_v = new_v;
+  return cuda_status(kvq::launch_append_decode_step(a, static_cast<cudaStream_t>(stream)),
+                     "kvq_append_decode_step launch");
+}
+
 kvq_status kvq_prefill_workspace_bytes(const kvq_config* cfg, int num_seqs, int max_chunk_tokens, int num_splits,
                                        size_t* bytes) {
   KVQ_TRY(check_config(cfg));
@@ -284,8 +339,6 @@ kvq_status kvq_paged_prefill_attention(const kvq_config* cfg, const void* q, voi
                                        float softmax_scale, int num_splits, void* workspace,
                                        size_t workspace_bytes, int32_t* dev_status, void* stream) {
   KVQ_TRY(check_config(cfg));
-  if (cfg->bits_k == 3 || cfg->bits_v == 3)
-    return fail(KVQ_ERR_UNSUPPORTED, "prefill attention reads 2-, 4- or 8-bit codes only (3-bit pages are storage-only)");
   if (num_splits < 1 || num_splits > 64) return fail(KVQ_ERR_INVALID_ARG, "num_splits must be 1..64");
   if (num_seqs < 0 || max_chunk_tokens < 0) return fail(KVQ_ERR_INVALID_ARG, "negative num_seqs or max_chunk_tokens");
   if (num_seqs == 0 || max_chunk_tokens == 0) return ok();

@@ -8,10 +8,11 @@
 //   acc'_j += C~V_tj (sum_i p_i s~V_i codeV_ij + sum_i p_i z~V_i)
 // which equals softmax(q' . K^'_i) P V^' exactly in real arithmetic.
 //
-// Kernels (three launches per call):
+// Kernels (two launches per call):
 //   decode_schedule_kernel  one CTA: tiles per sequence, chunk size, the
-//                           prefix of work units (sequence, KV head, chunk)
-//   decode_tiles_kernel     persistent warps, one work unit at a time:
+//                           prefix of work units (sequence, KV head, chunk);
+//                           resets the unit queue and the arrival counters
+//   decode_tiles_kernel     persistent warps taking work units from a queue:
 //                           per-warp double-buffered cp.async.bulk staging
 //                           of whole tiles (all pages, K and V) into shared
 //                           memory; scores and P.V on the legacy tensor
@@ -19,10 +20,12 @@
 //                           16 MMA rows = 8 query heads x {hi, lo} fp16
 //                           halves (fp32-accurate operands at no extra MMA)
 //                           and the packed codes unpacked in registers;
-//                           online softmax per tile; rotated-domain partial
-//   decode_merge_kernel     per (sequence, KV head): raw fp16 tail, log-sum-
-//                           exp merge of the chunks, the one inverse rotation,
-//                           fp16 output
+//                           online softmax per tile; rotated-domain partial.
+//                           The unit with chunk 0 of a (sequence, KV head)
+//                           also runs the raw fp16 tail; the last of its
+//                           units to finish merges the partials by
+//                           log-sum-exp, applies the one inverse rotation and
+//                           writes the fp16 output.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -39,23 +42,36 @@ namespace {
 // 132 floats = 528 bytes, so every record and its acc start 16-byte aligned.
 constexpr int kPartFloats = 4 + kHeadDim;
 constexpr int kPartAcc = 4;
+constexpr int kTailScratch = 13 * 1024;  // warp scratch: the tail's staged V rows; the merge's weights and staging
 constexpr int kUnitsPerSm = 32;            // work-unit budget of the automatic split
 constexpr long long kWaitLimitNs = 2000000000LL;  // bounded mbarrier waits: 2 s
 
 // ------------------------------------------------------------------ workspace
 // [0]        int32 U (total work units)
-// [4..]      int32 prefix[B+1]: chunks of sequences 0..b-1 (per KV head)
+// [4]        int32 next unit to hand out (dynamic schedule)
+// [8]        int32 CTAs finished (fused serving step)
+// [16..]     int32 prefix[B+1]: chunks of sequences 0..b-1 (per KV head)
 // then       int32 chunk[B]: tiles per chunk of each sequence
-// at 256-B   float partial[U][G][4 + d]  (m, l, pad, pad, acc)
+// then       int32 arrivals[B][H]: finished units of each (sequence, KV head)
+// at 256-B   float tails[B][H][G][4 + d]  (m, l, pad, pad, acc) of the raw tail
+// then       float partial[U][G][4 + d]  (m, l, pad, pad, acc) of the units
+// then       int32 group[U]: finished chunks of each merge group, at the
+//            slot of the group's first unit
 struct WsLayout {
-  size_t prefix_off, chunk_off, part_off;
+  size_t prefix_off, chunk_off, arrive_off, tail_off, part_off;
 };
-__host__ __device__ inline WsLayout ws_layout(int num_seqs) {
+__host__ __device__ inline WsLayout ws_layout(int num_seqs, int num_heads, int group) {
   WsLayout l;
-  l.prefix_off = 4;
+  l.prefix_off = 16;
   l.chunk_off = l.prefix_off + 4 * static_cast<size_t>(num_seqs + 1);
-  l.part_off = (l.chunk_off + 4 * static_cast<size_t>(num_seqs) + 255) / 256 * 256;
+  l.arrive_off = l.chunk_off + 4 * static_cast<size_t>(num_seqs);
+  l.tail_off = (l.arrive_off + 4 * static_cast<size_t>(num_seqs) * num_heads + 255) / 256 * 256;
+  l.part_off = l.tail_off + static_cast<size_t>(num_seqs) * num_heads * group * kPartFloats * sizeof(float);
   return l;
+}
+
+__host__ __device__ inline int32_t* group_counters(float* parts, size_t units, int group) {
+  return reinterpret_cast<int32_t*>(parts + units * group * kPartFloats);
 }
 
 // ------------------------------------------------------------------ PTX helpers
@@ -110,27 +126,45 @@ __device__ __forceinline__ void mma16816(float d[4], const uint32_t a[4], uint32
 // b = 4: word p/4, nibbles (p%4, p%4+4) -> channels 32t + 8(p/4) + p%4 + {0, 4}
 // b = 2: word p/8, fields (p%8, p%8+8) -> channels 32t + 16(p/8) + p%8 + {0, 8}
 // b = 8: word p/2, bytes (p%2, p%2+2) -> channels 32t + 4(p/2) + p%2 + {0, 2}
+// b = 3: pair p = channels 32t + p + {0, 16} (codes at bits 3p and 3p + 48 of the lane's 96)
 template <int B>
 __device__ __forceinline__ constexpr int pair_ch0(int p) {
-  return B == 8 ? 4 * (p / 2) + (p % 2) : (B == 4 ? 8 * (p / 4) + (p % 4) : 16 * (p / 8) + (p % 8));
+  return B == 3 ? p : (B == 8 ? 4 * (p / 2) + (p % 2) : (B == 4 ? 8 * (p / 4) + (p % 4) : 16 * (p / 8) + (p % 8)));
 }
 template <int B>
 __device__ __forceinline__ constexpr int pair_gap() {
-  return B == 8 ? 2 : (B == 4 ? 4 : 8);
+  return B == 3 ? 16 : (B == 8 ? 2 : (B == 4 ? 4 : 8));
+}
+
+// 3-bit field k (compile-time after unrolling) of a little-endian run of
+// 32-bit words: bits 3k .. 3k + 2, possibly straddling two words
+template <int N>
+__device__ __forceinline__ uint32_t field3(const uint32_t (&w)[N], int k) {
+  const int o = 3 * k, i = o >> 5, sh = o & 31;
+  if (sh <= 29) return (w[i] >> sh) & 7u;
+  return __funnelshift_r(w[i], w[i + 1], sh) & 7u;
+}
+// two codes as an fp16 pair of exact small integers (low half `lo`)
+__device__ __forceinline__ uint32_t code_pair_f16(uint32_t lo, uint32_t hi) {
+  return h2_as_u32(__hsub2(u32_as_h2(lo | (hi << 16) | 0x64006400u), __float2half2_rn(1024.f)));
 }
 
 // ------------------------------------------------------------------ schedule
 __global__ void __launch_bounds__(1024) decode_schedule_kernel(const int32_t* seq_lens, int num_seqs, int tile_tokens,
-                                                               int num_kv_heads, int num_splits, int target_units,
-                                                               void* workspace) {
+                                                               int num_kv_heads, int group, int num_splits,
+                                                               int target_units, void* workspace) {
   __shared__ long long s_total;
   __shared__ int s_scan[1024];
   __shared__ int s_carry;
-  const WsLayout wl = ws_layout(num_seqs);
+  const WsLayout wl = ws_layout(num_seqs, num_kv_heads, group);
   int32_t* ws_i = static_cast<int32_t*>(workspace);
   int32_t* prefix = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + wl.prefix_off);
   int32_t* chunk = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + wl.chunk_off);
+  int32_t* arrivals = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + wl.arrive_off);
   const int tid = threadIdx.x;
+  // the arrival counters and the unit queue start at zero on every call
+  for (int i = tid; i < num_seqs * num_kv_heads; i += blockDim.x) arrivals[i] = 0;
+  if (tid == 0) ws_i[1] = 0;
   if (tid == 0) {
     s_total = 0;
     s_carry = 0;
@@ -156,7 +190,10 @@ __global__ void __launch_bounds__(1024) decode_schedule_kernel(const int32_t* se
       } else {
         ch = static_cast<int>(std::min<long long>(ch_auto, 1 << 30));
       }
-      units = f > 0 ? (f + ch - 1) / ch : 0;
+      // every (sequence, KV head) gets a unit, even with no full tile: the
+      // unit with chunk 0 also takes the raw tail, and the last unit to
+      // finish merges and writes the output
+      units = f > 0 ? (f + ch - 1) / ch : 1;
       chunk[b] = ch;
     }
     s_scan[tid] = units;
@@ -176,6 +213,382 @@ __global__ void __launch_bounds__(1024) decode_schedule_kernel(const int32_t* se
     prefix[num_seqs] = s_carry;
     ws_i[0] = s_carry * num_kv_heads;
   }
+  // the merge-group counters after this call's partial records start at zero
+  const size_t units = static_cast<size_t>(s_carry) * num_kv_heads;
+  int32_t* gcount = group_counters(reinterpret_cast<float*>(static_cast<char*>(workspace) + wl.part_off), units, group);
+  for (size_t i = tid; i < units; i += blockDim.x) gcount[i] = 0;
+}
+
+// ------------------------------------------------------------------ raw tail and merge
+__device__ __forceinline__ float ld_cg(const float* p) { return __ldcg(p); }
+__device__ __forceinline__ float4 ld_cg4(const float* p) { return __ldcg(reinterpret_cast<const float4*>(p)); }
+
+// One warp, serving step: the step's K and V rows of (sequence b, KV head h)
+// into tail row (L - 1) mod T, L the length after the step.  A token that
+// completes a tile (L mod T == 0) would have to be quantized into pages, which
+// this launch does not do: it is reported and not written.
+template <int T>
+__device__ void step_append_warp(const DecodeArgs& a, int b, int h, int L, int lane) {
+  if (L % T == 0) {
+    if (lane == 0) report_error(a.dev_status, KVQ_ERR_DEVICE_BOUNDS);
+    return;
+  }
+  const size_t bh = static_cast<size_t>(b) * a.cfg.num_kv_heads + h;
+  const size_t row = (bh * T + (L - 1) % T) * kHeadDim;
+  const uint2* nk = reinterpret_cast<const uint2*>(static_cast<const __half*>(a.new_k) + bh * kHeadDim);
+  const uint2* nv = reinterpret_cast<const uint2*>(static_cast<const __half*>(a.new_v) + bh * kHeadDim);
+  uint2* tk = reinterpret_cast<uint2*>(const_cast<__half*>(static_cast<const __half*>(a.k_tail)) + row);
+  uint2* tv = reinterpret_cast<uint2*>(const_cast<__half*>(static_cast<const __half*>(a.v_tail)) + row);
+  tk[lane] = nk[lane];
+  tv[lane] = nv[lane];
+  __syncwarp();
+}
+
+// Four 8x8 fp16 matrices from shared memory, transposed: lanes 8i..8i+7 give
+// the row addresses of matrix i; register i of lane (g, t) receives elements
+// (2t, g) and (2t + 1, g) of matrix i (the m16n8k16 B-fragment order).
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+constexpr int kTailRowBytes = 2 * kHeadDim + 16;  // staged V row, padded: 8 rows hit 8 distinct bank groups
+static_assert(16 * kTailRowBytes <= kTailScratch, "16 staged tail rows fit the warp scratch");
+
+// One warp: the raw fp16 tail (tau < T tokens) of (sequence b, KV head h)
+// for its g query heads, in the original domain, on the tensor cores
+// (mma.sync m16n8k16, rows = query heads).  Scores: q and the raw K rows are
+// fp16, so the products are exact and sum in fp32; lane (g, t) loads 16-byte
+// runs of q and K, and k-block 2j + u takes channels 32j + 8t + 4u + {0, 1}
+// (fragment columns 2t, 2t + 1) and 32j + 8t + 4u + {2, 3} (columns 2t + 8,
+// 2t + 9) on both sides.  A softmax per head over the tail alone, then P V:
+// the score fragments are the A fragments of P (rows g / g + 8 = hi / lo fp16
+// halves of p), V comes through shared memory in 16-token chunks as
+// transposed 8x8 fp16 tiles.  Writes the tail record (m, l, acc) of every
+// query head; scratch: 16 padded V rows (4352 bytes) of the warp's shared
+// memory, whose copies must all have landed.
+template <int T>
+__device__ __noinline__ void decode_tail_warp(const DecodeArgs& a, int b, int h, int tau, float* tails, float* scratch, int lane) {
+  constexpr int NB = T / 8;  // 8-token score blocks
+  const int G = a.cfg.group_size, nh = a.cfg.num_kv_heads;
+  const int g = lane >> 2, t = lane & 3;
+  const float qscale = a.softmax_scale * kLog2e;
+  const size_t bh = static_cast<size_t>(b) * nh + h;
+  float* rec = tails + bh * G * kPartFloats;
+  if (tau <= 0) {
+    for (int hh = 0; hh < G; ++hh) {
+      if (lane == 0) {
+        rec[hh * kPartFloats] = -INFINITY;
+        rec[hh * kPartFloats + 1] = 0.f;
+      }
+      *reinterpret_cast<float4*>(rec + hh * kPartFloats + kPartAcc + 4 * lane) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    return;
+  }
+  const bool live = g < G;
+  uint4 qa[4];
+  {
+    const __half* qrow = static_cast<const __half*>(a.q) + (bh * G + (live ? g : 0)) * kHeadDim + 8 * t;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      qa[j] = live ? *reinterpret_cast<const uint4*>(qrow + 32 * j) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  const __half* kt = static_cast<const __half*>(a.k_tail) + bh * T * kHeadDim;
+  const __half* vt = static_cast<const __half*>(a.v_tail) + bh * T * kHeadDim;
+
+  // -- scores (log2 domain) of tokens 8nb + 2t, 8nb + 2t + 1 for head g
+  float sc[NB][2];
+  float m = -INFINITY;
+#pragma unroll
+  for (int nb = 0; nb < NB; ++nb) {
+    sc[nb][0] = sc[nb][1] = -INFINITY;
+    if (8 * nb < tau) {  // warp-uniform
+      const int tk = 8 * nb + g;
+      uint4 kr[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        kr[j] = tk < tau ? *reinterpret_cast<const uint4*>(kt + static_cast<size_t>(tk) * kHeadDim + 32 * j + 8 * t)
+                         : make_uint4(0u, 0u, 0u, 0u);
+      float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t a0[4] = {qa[j].x, 0u, qa[j].y, 0u};
+        const uint32_t a1[4] = {qa[j].z, 0u, qa[j].w, 0u};
+        mma16816(d, a0, kr[j].x, kr[j].y);
+        mma16816(d, a1, kr[j].z, kr[j].w);
+      }
+      const int i0 = 8 * nb + 2 * t;
+      if (i0 < tau) sc[nb][0] = d[0] * qscale;
+      if (i0 + 1 < tau) sc[nb][1] = d[1] * qscale;
+      m = fmaxf(m, fmaxf(sc[nb][0], sc[nb][1]));
+    }
+  }
+  m = fmaxf(m, __shfl_xor_sync(kFull, m, 1));
+  m = fmaxf(m, __shfl_xor_sync(kFull, m, 2));
+  float l = 0.f;
+#pragma unroll
+  for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const float p = sc[nb][e] == -INFINITY ? 0.f : exp2f(sc[nb][e] - m);
+      sc[nb][e] = p;
+      l += p;
+    }
+  l += __shfl_xor_sync(kFull, l, 1);
+  l += __shfl_xor_sync(kFull, l, 2);
+
+  // -- P V: D[16 rows][8 channels] per n-block nv; rows g / g + 8 = hi / lo of p
+  float acc[16][4];
+#pragma unroll
+  for (int nv = 0; nv < 16; ++nv)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) acc[nv][k] = 0.f;
+  unsigned char* vs = reinterpret_cast<unsigned char*>(scratch);
+  const uint32_t vs_addr = smem_u32(vs);
+#pragma unroll
+  for (int kb = 0; kb < NB / 2; ++kb) {
+    if (16 * kb >= tau) break;  // warp-uniform
+    // stage tokens 16kb .. 16kb + 15 (zeros past the tail: p is 0 there, and
+    // 0 times a stale non-finite value would not be)
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int idx = lane + 32 * k, row = idx >> 4, c16 = idx & 15;
+      const int tk = 16 * kb + row;
+      const uint4 v = tk < tau ? *reinterpret_cast<const uint4*>(vt + static_cast<size_t>(tk) * kHeadDim + 8 * c16)
+                               : make_uint4(0u, 0u, 0u, 0u);
+      *reinterpret_cast<uint4*>(vs + row * kTailRowBytes + 16 * c16) = v;
+    }
+    __syncwarp();
+    uint32_t pa[4];
+    {
+      const float x0 = sc[2 * kb][0], x1 = sc[2 * kb][1], y0 = sc[2 * kb + 1][0], y1 = sc[2 * kb + 1][1];
+      const __half2 hx = __floats2half2_rn(x0, x1), hy = __floats2half2_rn(y0, y1);
+      const float2 fx = __half22float2(hx), fy = __half22float2(hy);
+      pa[0] = h2_as_u32(hx);
+      pa[1] = h2_as_u32(__floats2half2_rn(x0 - fx.x, x1 - fx.y));
+      pa[2] = h2_as_u32(hy);
+      pa[3] = h2_as_u32(__floats2half2_rn(y0 - fy.x, y1 - fy.y));
+    }
+    // lane 8i + r: row r of matrix i = token r + 8 (i & 1), channels 8 (nv + (i >> 1)) ..
+    const int mi = lane >> 3, mr = lane & 7;
+    const uint32_t lane_addr = vs_addr + (mr + 8 * (mi & 1)) * kTailRowBytes + 16 * (mi >> 1);
+#pragma unroll
+    for (int nv = 0; nv < 16; nv += 2) {
+      uint32_t bf[4];
+      ldsm_x4_trans(lane_addr + 16 * nv, bf);
+      mma16816(acc[nv], pa, bf[0], bf[1]);
+      mma16816(acc[nv + 1], pa, bf[2], bf[3]);
+    }
+    __syncwarp();
+  }
+  if (live) {
+    float* r = rec + g * kPartFloats;
+    if (t == 0) {
+      r[0] = m;
+      r[1] = l;
+    }
+#pragma unroll
+    for (int nv = 0; nv < 16; ++nv)
+      *reinterpret_cast<float2*>(r + kPartAcc + 8 * nv + 2 * t) =
+          make_float2(acc[nv][0] + acc[nv][2], acc[nv][1] + acc[nv][3]);
+  }
+  __syncwarp();
+}
+
+// Log-sum-exp merge of n partial records of (sequence b, KV head h) by one
+// warp: the records at unit slots first + s * stride (s < n), written by
+// other warps and read through L2.  Two levels keep every merge short: the
+// chunks of a (sequence, KV head) form groups of kMergeGroup consecutive
+// chunks; the last chunk of a group to finish merges the group into a record
+// at the group's first slot (final = false), and the last group to finish
+// merges those records with the raw tail record, applies the one inverse
+// rotation of the rotated-domain accumulator and writes the fp16 output
+// (final = true; a single group goes straight to this step).  The G query
+// heads go together while records are read: the maxima (lanes stride over
+// the records), each record's weight into the scratch, then the weighted sums
+// with R records x G heads (about 16) loads in flight per lane (lane L owns
+// channels 4L .. 4L+3 of every head).  The output (inverse rotation, tail,
+// 1/l) then runs as one loop over the heads from the scratch, which keeps the
+// code small: the tile loop of the warps that share the SM stays in the
+// instruction cache.
+// Scratch layout (bytes): [0, 4096) weights of kBlock records, then the
+// sums [G][32 lanes] float4, the tail accumulators [G][32] float4, and
+// (et, 1/l) per head.
+constexpr int kMergeGroup = 16;
+constexpr int kMergeWBytes = 4096;
+template <int G>
+__device__ __noinline__ void decode_merge_warp_g(const DecodeArgs& a, int b, int h, int n_rec, size_t first,
+                                                 int stride, bool final, float* parts, const float* tails,
+                                                 float* scratch, int lane) {
+  constexpr int R = 16 / G > 1 ? 16 / G : 1;     // records per round
+  constexpr int kBlock = kMergeWBytes / 4 / G;   // records whose weights fit the scratch
+  static_assert(kMergeWBytes + 2 * G * 512 + 8 * G <= kTailScratch, "merge scratch");
+  float* wsc = scratch;
+  float4* acc_s = reinterpret_cast<float4*>(reinterpret_cast<unsigned char*>(scratch) + kMergeWBytes);
+  float4* tail_s = acc_s + G * 32;
+  float* scal = reinterpret_cast<float*>(tail_s + G * 32);
+  const int nh = a.cfg.num_kv_heads;
+  const size_t bh = static_cast<size_t>(b) * nh + h;
+  const float* trec = tails + bh * G * kPartFloats;
+  auto rec = [&](int s, int hh) { return parts + ((first + static_cast<size_t>(s) * stride) * G + hh) * kPartFloats; };
+  float mm[G], ll[G], mt[G], lt[G];
+#pragma unroll
+  for (int hh = 0; hh < G; ++hh) {
+    mt[hh] = -INFINITY;
+    lt[hh] = 0.f;
+    if (final) {
+      mt[hh] = ld_cg(trec + hh * kPartFloats);
+      lt[hh] = ld_cg(trec + hh * kPartFloats + 1);
+      tail_s[hh * 32 + lane] = ld_cg4(trec + hh * kPartFloats + kPartAcc + 4 * lane);
+    }
+    mm[hh] = lt[hh] > 0.f ? mt[hh] : -INFINITY;
+    ll[hh] = 0.f;
+  }
+  for (int s = lane; s < n_rec; s += 32) {
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) {
+      const float2 ml = __ldcg(reinterpret_cast<const float2*>(rec(s, hh)));
+      if (ml.y > 0.f) mm[hh] = fmaxf(mm[hh], ml.x);
+    }
+  }
+#pragma unroll
+  for (int hh = 0; hh < G; ++hh) mm[hh] = warp_max(mm[hh]);
+  float4 acc[G];
+#pragma unroll
+  for (int hh = 0; hh < G; ++hh) acc[hh] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s0 = 0; s0 < n_rec; s0 += kBlock) {
+    const int n = min(kBlock, n_rec - s0);
+    __syncwarp();
+    for (int s = lane; s < n; s += 32) {
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) {
+        const float2 ml = __ldcg(reinterpret_cast<const float2*>(rec(s0 + s, hh)));
+        const float w = ml.y > 0.f ? exp2f(ml.x - mm[hh]) : 0.f;
+        ll[hh] += w * ml.y;
+        wsc[s * G + hh] = w;
+      }
+    }
+    __syncwarp();
+    for (int s = 0; s < n; s += R) {
+      float4 v[R][G];
+#pragma unroll
+      for (int k = 0; k < R; ++k)
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh)
+          v[k][hh] = s + k < n ? ld_cg4(rec(s0 + s + k, hh) + kPartAcc + 4 * lane) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int k = 0; k < R; ++k)
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh) {
+          const float w = s + k < n ? wsc[(s + k) * G + hh] : 0.f;
+          acc[hh].x += w * v[k][hh].x;
+          acc[hh].y += w * v[k][hh].y;
+          acc[hh].z += w * v[k][hh].z;
+          acc[hh].w += w * v[k][hh].w;
+        }
+    }
+  }
+  if (!final) {  // the group's record (m, l, acc), at its first slot, whose reads are all done
+    __syncwarp();
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) {
+      float* r = rec(0, hh);
+      const float l = warp_sum(ll[hh]);
+      if (lane == 0) {
+        r[0] = mm[hh];
+        r[1] = l;
+      }
+      *reinterpret_cast<float4*>(r + kPartAcc + 4 * lane) = acc[hh];
+    }
+    __syncwarp();
+    return;
+  }
+#pragma unroll
+  for (int hh = 0; hh < G; ++hh) {
+    acc_s[hh * 32 + lane] = acc[hh];
+    const float l = warp_sum(ll[hh]);
+    const float et = lt[hh] > 0.f ? exp2f(mt[hh] - mm[hh]) : 0.f;
+    const float ltot = l + lt[hh] * et;
+    if (lane == 0) {
+      scal[2 * hh] = et;
+      scal[2 * hh + 1] = ltot > 0.f ? 1.f / ltot : 0.f;
+    }
+  }
+  __syncwarp();
+  __half* out = static_cast<__half*>(a.out) + bh * G * kHeadDim;
+  const uint32_t seed = a.cfg.rotation_seed;
+  float sg[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) sg[k] = rotation_sign(seed, 4 * lane + k) / kSqrtHeadDim;
+#pragma unroll 1
+  for (int hh = 0; hh < G; ++hh) {
+    const float4 va = acc_s[hh * 32 + lane], tl = tail_s[hh * 32 + lane];
+    const float et = scal[2 * hh], inv_l = scal[2 * hh + 1];
+    float v[4] = {va.x, va.y, va.z, va.w};
+    fwht128_warp(v, lane);  // the one inverse rotation (H = H^T = H^-1)
+    const __half2 o0 = __floats2half2_rn((v[0] * sg[0] + et * tl.x) * inv_l, (v[1] * sg[1] + et * tl.y) * inv_l);
+    const __half2 o1 = __floats2half2_rn((v[2] * sg[2] + et * tl.z) * inv_l, (v[3] * sg[3] + et * tl.w) * inv_l);
+    *reinterpret_cast<uint2*>(out + hh * kHeadDim + 4 * lane) = make_uint2(h2_as_u32(o0), h2_as_u32(o1));
+  }
+  __syncwarp();
+}
+
+__device__ __noinline__ void decode_merge_warp(const DecodeArgs& a, int b, int h, int n_rec, size_t first, int stride,
+                                               bool final, float* parts, const float* tails, float* scratch,
+                                               int lane) {
+  switch (a.cfg.group_size) {
+    case 1: decode_merge_warp_g<1>(a, b, h, n_rec, first, stride, final, parts, tails, scratch, lane); break;
+    case 2: decode_merge_warp_g<2>(a, b, h, n_rec, first, stride, final, parts, tails, scratch, lane); break;
+    case 3: decode_merge_warp_g<3>(a, b, h, n_rec, first, stride, final, parts, tails, scratch, lane); break;
+    case 4: decode_merge_warp_g<4>(a, b, h, n_rec, first, stride, final, parts, tails, scratch, lane); break;
+    case 5: decode_merge_warp_g<5>(a, b, h, n_rec, first, stride, final, parts, tails, scratch, lane); break;
+    case 6: decode_merge_warp_g<6>(a, b, h, n_rec, first, stride, final, parts, tails, scratch, lane); break;
+    case 7: decode_merge_warp_g<7>(a, b, h, n_rec, first, stride, final, parts, tails, scratch, lane); break;
+    default: decode_merge_warp_g<8>(a, b, h, n_rec, first, stride, final, parts, tails, scratch, lane); break;
+  }
+}
+
+// Where work unit u sits: sequence b, KV head h, chunk c of the S chunks of
+// (b, h), ch tiles per chunk, L tokens, its first partial record at ubase.
+// Decode: from the schedule (binary search of the prefix).  Serving step: a
+// fixed grid of num_splits units per (b, h) over the lengths after the step;
+// units with c >= S (past a short sequence's last chunk) are empty.
+struct UnitLoc {
+  int b, h, c, S, L, ch;
+  size_t ubase;
+};
+template <int T>
+__device__ __forceinline__ UnitLoc locate_unit(const DecodeArgs& a, int u, const int32_t* prefix,
+                                               const int32_t* chunk) {
+  const int nh = a.cfg.num_kv_heads;
+  UnitLoc l;
+  if (a.step) {
+    const int sx = a.num_splits_fixed;
+    l.b = u / (nh * sx);
+    const int r = u - l.b * nh * sx;
+    l.h = r / sx;
+    l.c = r % sx;
+    l.L = max(a.seq_lens[l.b], 0) + 1;
+    const int f = l.L / T;
+    l.ch = f > 0 ? (f + sx - 1) / sx : 1;
+    l.S = f > 0 ? (f + l.ch - 1) / l.ch : 1;
+    l.ubase = (static_cast<size_t>(l.b) * nh + l.h) * sx;
+  } else {
+    int lo = 0, hi = a.num_seqs;  // find the largest b with nh*prefix[b] <= u
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (nh * prefix[mid] <= u) lo = mid; else hi = mid;
+    }
+    l.b = lo;
+    l.S = prefix[l.b + 1] - prefix[l.b];
+    const int r = u - nh * prefix[l.b];
+    l.h = r / l.S;
+    l.c = r % l.S;
+    l.L = max(a.seq_lens[l.b], 0);
+    l.ch = chunk[l.b];
+    l.ubase = static_cast<size_t>(nh) * prefix[l.b] + static_cast<size_t>(l.h) * l.S;
+  }
+  return l;
 }
 
 // ------------------------------------------------------------------ main decode
@@ -189,9 +602,12 @@ struct DecodeGeom {
   static constexpr int kPageK = kCodesK + 64 + kCsBytes;
   static constexpr int kPageV = kCodesV + 64 + kCsBytes;
   static constexpr int kStage = kPages * (kPageK + kPageV);    // one tile, K pages then V pages
+  // per warp: two stages, at least the 8 KB the raw tail and the merge use
+  // as scratch (q [8][128] and p [8][T] in fp32) once its copies have landed
+  static constexpr int kWarpBytes = 2 * kStage > kTailScratch ? 2 * kStage : kTailScratch;
   // warps per CTA: 4, fewer when two stages per warp would not fit (8-bit codes)
-  static constexpr int kWarps = 4 * (2 * kStage + 16) <= 200 * 1024 ? 4 : (2 * (2 * kStage + 16) <= 200 * 1024 ? 2 : 1);
-  static constexpr int kSmem = kWarps * (2 * kStage + 16);
+  static constexpr int kWarps = 4 * (kWarpBytes + 16) <= 200 * 1024 ? 4 : (2 * (kWarpBytes + 16) <= 200 * 1024 ? 2 : 1);
+  static constexpr int kSmem = kWarps * (kWarpBytes + 16);
 };
 
 template <int T, int BK, int BV>
@@ -203,8 +619,8 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
   extern __shared__ __align__(128) unsigned char smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
-  unsigned char* stage_base = smem + warp * 2 * Geo::kStage;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kDecWarps * 2 * Geo::kStage) + 2 * warp;
+  unsigned char* stage_base = smem + warp * Geo::kWarpBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kDecWarps * Geo::kWarpBytes) + 2 * warp;
   if (lane == 0) {
     mbar_init(&bars[0], 1);
     mbar_init(&bars[1], 1);
@@ -213,12 +629,16 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
   __syncwarp();
 
   const int G = a.cfg.group_size, nh = a.cfg.num_kv_heads;
-  const WsLayout wl = ws_layout(a.num_seqs);
-  const int32_t* ws_i = static_cast<const int32_t*>(a.workspace);
-  const int32_t* prefix = reinterpret_cast<const int32_t*>(static_cast<const char*>(a.workspace) + wl.prefix_off);
-  const int32_t* chunk = reinterpret_cast<const int32_t*>(static_cast<const char*>(a.workspace) + wl.chunk_off);
-  float* parts = reinterpret_cast<float*>(static_cast<char*>(a.workspace) + wl.part_off);
-  const int U = ws_i[0];
+  const WsLayout wl = ws_layout(a.num_seqs, nh, G);
+  char* ws = static_cast<char*>(a.workspace);
+  int32_t* ws_i = reinterpret_cast<int32_t*>(ws);
+  const int32_t* prefix = reinterpret_cast<const int32_t*>(ws + wl.prefix_off);
+  const int32_t* chunk = reinterpret_cast<const int32_t*>(ws + wl.chunk_off);
+  int32_t* arrivals = reinterpret_cast<int32_t*>(ws + wl.arrive_off);
+  float* tails = reinterpret_cast<float*>(ws + wl.tail_off);
+  float* parts = reinterpret_cast<float*>(ws + wl.part_off);
+  const int U = a.step ? a.num_seqs * nh * a.num_splits_fixed : ws_i[0];
+  int32_t* gcount = group_counters(parts, U, G);
   const uint8_t* kpool = static_cast<const uint8_t*>(a.k_pool);
   const uint8_t* vpool = static_cast<const uint8_t*>(a.v_pool);
   const float qscale = a.softmax_scale * kLog2e / kSqrtHeadDim;
@@ -227,21 +647,22 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
   bool pending[2] = {false, false};  // copies issued into the stage and not yet waited for
   bool failed = false;
 
-  const int total_warps = gridDim.x * kDecWarps;
-  for (int u = blockIdx.x * kDecWarps + warp; u < U && !failed; u += total_warps) {
-    // ---- locate the unit: sequence b (binary search), head h, chunk c
-    int lo = 0, hi = a.num_seqs;  // find the largest b with nh*prefix[b] <= u
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (nh * prefix[mid] <= u) lo = mid; else hi = mid;
-    }
-    const int b = lo;
-    const int S = prefix[b + 1] - prefix[b];
-    const int r = u - nh * prefix[b];
-    const int h = r / S, c = r % S;
-    const int F = max(a.seq_lens[b], 0) / T;
-    const int ch = chunk[b];
-    const int t0 = c * ch, t1 = min(F, t0 + ch);
+  // units are handed out in order (sequence, KV head, chunk) from a queue, so
+  // the chunks of one (sequence, KV head) run at about the same time and its
+  // merge happens early
+  while (!failed) {
+    int u = 0;
+    if (lane == 0) u = atomicAdd(&ws_i[1], 1);
+    u = __shfl_sync(kFull, u, 0);
+    if (u >= U) break;
+    // ---- locate the unit: sequence b, head h, chunk c of the S chunks of
+    // (b, h) over L tokens (the coordinates are located again after the
+    // tile loop, so that only what the loop needs stays live through it)
+    UnitLoc loc = locate_unit<T>(a, u, prefix, chunk);
+    if (loc.c >= loc.S) continue;  // serving step: past a short sequence's last chunk
+    const int b = loc.b, h = loc.h;
+    const int F = loc.L / T;
+    const int t0 = loc.c * loc.ch, t1 = min(F, t0 + loc.ch);
 
     // ---- rotated, scaled query: lane (g, t) holds channels 32t..32t+31 of head g
     float qs[32];
@@ -345,7 +766,8 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
       // up to 4 so that one chunk's code words and accumulators are live; the
       // chunk's scores (log2 domain, tokens 8nb + 2t, 8nb + 2t + 1 of each page)
       // are kept.
-      constexpr int kPcMax = BK == 8 ? 2 : 4;
+      // (two at T = 128, where the scores of 8 pages stay live as well)
+      constexpr int kPcMax = (BK == 8 || BK == 3 || NP >= 8) ? 2 : 4;
       constexpr int kPc = NP < kPcMax ? NP : kPcMax;
       float sig = 0.f;
       float sc[NP][2][2];
@@ -381,19 +803,34 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
             } else if constexpr (BK == 4) {
               const uint4 v = *reinterpret_cast<const uint4*>(src);
               rec[pg][nb][0] = v.x; rec[pg][nb][1] = v.y; rec[pg][nb][2] = v.z; rec[pg][nb][3] = v.w;
+            } else if constexpr (BK == 3) {  // 12 bytes at a 4-byte aligned offset
+              const uint32_t* w = reinterpret_cast<const uint32_t*>(src);
+              rec[pg][nb][0] = w[0]; rec[pg][nb][1] = w[1]; rec[pg][nb][2] = w[2];
             } else {
               const uint2 v = *reinterpret_cast<const uint2*>(src);
               rec[pg][nb][0] = v.x; rec[pg][nb][1] = v.y;
             }
           }
-        constexpr int kbPerWord = 8 / BK;  // k-blocks per word: 2 (b=4) or 4 (b=2)
+        // k-blocks per word: 2 (b=4), 4 (b=2), 1 (b=8); at b=3 the lane's 96
+        // bits are taken as one run and every k-block extracts its 4 codes
+        constexpr int kbPerWord = BK == 3 ? 8 : 8 / BK;
+        constexpr int kWords = BK == 3 ? 1 : BK;
 #pragma unroll
-        for (int wd = 0; wd < BK; ++wd) {
-          uint32_t pr[kPc][2][16 / BK];
+        for (int wd = 0; wd < kWords; ++wd) {
+          constexpr int kPairs = BK == 3 ? 16 : 16 / BK;
+          uint32_t pr[kPc][2][kPairs];
 #pragma unroll
           for (int pg = 0; pg < kPc; ++pg)
 #pragma unroll
-            for (int nb = 0; nb < 2; ++nb) unpack_pairs<BK>(rec[pg][nb][wd], pr[pg][nb]);
+            for (int nb = 0; nb < 2; ++nb) {
+              if constexpr (BK == 3) {
+#pragma unroll
+                for (int pp = 0; pp < 16; ++pp)
+                  pr[pg][nb][pp] = code_pair_f16(field3(rec[pg][nb], pp), field3(rec[pg][nb], pp + 16));
+              } else {
+                unpack_pairs<BK>(rec[pg][nb][wd], pr[pg][nb]);
+              }
+            }
 #pragma unroll
           for (int j = 0; j < kbPerWord; ++j) {
             const int kb = wd * kbPerWord + j;
@@ -464,6 +901,35 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
       // words 2q, 2q+1 (token pairs {2t,2t+1} and {2t+8,2t+9}) hold the n-blocks
       // kPairsV*q .. kPairsV*q + kPairsV-1; a group's accumulators are folded
       // into acc' (times C~V) as soon as all pages of the tile are in.
+      if constexpr (BV == 3) {
+        // 3-bit V pages are a token-major bitstream: code (token p, channel c)
+        // at bit 3 (128 p + c).  Lane (g, t) needs channel 8 nv + g of tokens
+        // 2t, 2t+1 (B register 0) and 2t+8, 2t+9 (register 1); one read of
+        // two words and a funnel shift per code.
+#pragma unroll 2
+        for (int nv = 0; nv < 16; ++nv) {
+          const int bit = 24 * nv + 3 * g, wo = bit >> 5, sh = bit & 31;
+          float dv[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int pg = 0; pg < NP; ++pg) {
+            const uint32_t afr[4] = {pa[pg][0], pa[pg][1], pa[pg][2], pa[pg][3]};
+            const uint32_t* cw = reinterpret_cast<const uint32_t*>(sV + pg * Geo::kPageV);
+            uint32_t c[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int p = 2 * t + (k & 1) + 8 * (k >> 1);
+              c[k] = __funnelshift_r(cw[12 * p + wo], cw[12 * p + wo + 1], sh) & 7u;
+            }
+            mma16816(dv, afr, code_pair_f16(c[0], c[1]), code_pair_f16(c[2], c[3]));
+          }
+          const int c0 = 8 * nv + 2 * t;
+          const __half2 cvh = *reinterpret_cast<const __half2*>(sV + (c0 / Geo::kCs) * Geo::kPageV + Geo::kCodesV +
+                                                                64 + 2 * (c0 % Geo::kCs));
+          const float2 cv = __half22float2(cvh);
+          acc[2 * nv] = alpha * acc[2 * nv] + cv.x * (dv[0] + dv[2] + wsum);
+          acc[2 * nv + 1] = alpha * acc[2 * nv + 1] + cv.y * (dv[1] + dv[3] + wsum);
+        }
+      } else {
       constexpr int kPairsV = 16 / BV;      // n-blocks per word pair
       constexpr int kGroups = 16 / kPairsV;  // word pairs per lane (4 at b=4, 2 at b=2)
 #pragma unroll
@@ -497,6 +963,7 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
           acc[2 * nv + 1] = alpha * acc[2 * nv + 1] + cv.y * (dv[e][1] + dv[e][3] + wsum);
         }
       }
+      }
       __syncwarp();
       if (i + 2 < t1) issue(i + 2, st);
     }
@@ -517,10 +984,72 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
         *reinterpret_cast<float2*>(part + kPartAcc + c0) = make_float2(acc[2 * nv], acc[2 * nv + 1]);
       }
     }
+    // the raw tail goes with chunk 0 (the warp's stages are idle now: every
+    // copy it issued has landed); in a serving step its warp first writes the
+    // step's token into the tail row (L - 1) mod T
+    loc = locate_unit<T>(a, u, prefix, chunk);
+    if (loc.c == 0) {
+      if (a.step) step_append_warp<T>(a, loc.b, loc.h, loc.L, lane);
+      decode_tail_warp<T>(a, loc.b, loc.h, loc.L % T, tails, reinterpret_cast<float*>(stage_base), lane);
+    }
+    // publish this unit's records; the last chunk of its group to finish
+    // merges the group, the last group of (b, h) merges the groups
+    __threadfence();
+    __syncwarp();
+    const int bh = loc.b * nh + loc.h;
+    const int n_groups = (loc.S + kMergeGroup - 1) / kMergeGroup;
+    float* scratch = reinterpret_cast<float*>(stage_base);
+    bool to_final = n_groups == 1;
+    if (n_groups > 1) {
+      const int j = loc.c / kMergeGroup, gsz = min(kMergeGroup, loc.S - j * kMergeGroup);
+      const size_t gfirst = loc.ubase + static_cast<size_t>(j) * kMergeGroup;
+      int last = 0;
+      if (lane == 0) last = atomicAdd(&gcount[gfirst], 1) == gsz - 1;
+      last = __shfl_sync(kFull, last, 0);
+      if (last) {
+        __threadfence();
+        decode_merge_warp(a, loc.b, loc.h, gsz, gfirst, 1, false, parts, tails, scratch, lane);
+        if (a.step && lane == 0) gcount[gfirst] = 0;  // the step leaves its counters at zero
+        __threadfence();
+        __syncwarp();
+        to_final = true;
+      }
+    }
+    if (to_final) {
+      int last = 0;
+      // the counter counts units when there is one group, else groups
+      if (lane == 0) last = atomicAdd(&arrivals[bh], 1) == (n_groups == 1 ? loc.S : n_groups) - 1;
+      last = __shfl_sync(kFull, last, 0);
+      if (last) {
+        __threadfence();
+        decode_merge_warp(a, loc.b, loc.h, n_groups == 1 ? loc.S : n_groups, loc.ubase,
+                          n_groups == 1 ? 1 : kMergeGroup, true, parts, tails, scratch, lane);
+        if (a.step && lane == 0) arrivals[bh] = 0;  // the step leaves its counters at zero
+      }
+    }
   }
   if (failed) {  // let copies already in flight land before the CTA's shared memory is released
     for (int st = 0; st < 2; ++st)
       if (pending[st]) (void)mbar_wait_bounded(&bars[st], phase[st]);
+  }
+  if (a.step) {
+    // the last CTA to finish resets the unit queue and the CTA count and
+    // advances every sequence's length by the step's token
+    __shared__ int s_last;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      __threadfence();
+      s_last = atomicAdd(&ws_i[2], 1) == static_cast<int>(gridDim.x) - 1;
+    }
+    __syncthreads();
+    if (s_last) {
+      __threadfence();
+      for (int i = threadIdx.x; i < a.num_seqs; i += blockDim.x) a.seq_lens_rw[i] = max(a.seq_lens[i], 0) + 1;
+      if (threadIdx.x == 0) {
+        ws_i[1] = 0;
+        ws_i[2] = 0;
+      }
+    }
   }
 }
 
@@ -533,139 +1062,6 @@ __global__ void selftest_wait_decode_kernel(int32_t* dev_status) {
   if (!mbar_wait_bounded(&bar, 0)) report_error(dev_status, KVQ_ERR_DEVICE_TIMEOUT);
 }
 
-// ------------------------------------------------------------------ merge
-constexpr int kMergeThreads = 256;
-
-template <int T>
-struct __align__(16) MergeSmem {
-  float qraw[kMaxGroup][kHeadDim];
-  float sc[kMaxGroup][T];
-  float tl[kMaxGroup][kHeadDim];                 // raw-domain tail accumulator
-  float red[kMergeThreads / 32][kHeadDim];       // per-warp partial sums of one head
-  float big_m[kMaxGroup], inv_l[kMaxGroup], et[kMaxGroup], mt[kMaxGroup], lt[kMaxGroup];
-};
-
-// One CTA of 256 threads per (sequence, KV head): raw fp16 tail, log-sum-
-// exp merge of the chunk partials (warps split the chunks, lanes own four
-// channels), the inverse rotation of the merged accumulator, fp16 output.
-template <int T>
-__global__ void __launch_bounds__(kMergeThreads) decode_merge_kernel(DecodeArgs a) {
-  __shared__ MergeSmem<T> sm;
-  constexpr int kWarps = kMergeThreads / 32;
-  const int h = blockIdx.x, b = blockIdx.y;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int G = a.cfg.group_size, nh = a.cfg.num_kv_heads;
-  const int L = max(a.seq_lens[b], 0);
-  const int F = L / T, tau = L - F * T;
-  const WsLayout wl = ws_layout(a.num_seqs);
-  const int32_t* prefix = reinterpret_cast<const int32_t*>(static_cast<const char*>(a.workspace) + wl.prefix_off);
-  const float* parts = reinterpret_cast<const float*>(static_cast<const char*>(a.workspace) + wl.part_off);
-  const int S = prefix[b + 1] - prefix[b];
-  const size_t ubase = static_cast<size_t>(nh) * prefix[b] + static_cast<size_t>(h) * S;
-  const float qscale = a.softmax_scale * kLog2e;
-  const __half* q = static_cast<const __half*>(a.q) + (static_cast<size_t>(b) * nh + h) * G * kHeadDim;
-  const __half* kt = static_cast<const __half*>(a.k_tail) + (static_cast<size_t>(b) * nh + h) * T * kHeadDim;
-  const __half* vt = static_cast<const __half*>(a.v_tail) + (static_cast<size_t>(b) * nh + h) * T * kHeadDim;
-
-  // 1. raw tail: scores (thread = token), softmax (warp = head), P V (thread = channel)
-  for (int idx = tid; idx < G * kHeadDim; idx += kMergeThreads)
-    sm.qraw[idx / kHeadDim][idx % kHeadDim] = __half2float(q[idx]) * qscale;
-  __syncthreads();
-  for (int i = tid; i < tau; i += kMergeThreads) {
-    float dot[kMaxGroup];
-#pragma unroll
-    for (int hh = 0; hh < kMaxGroup; ++hh) dot[hh] = 0.f;
-    for (int c = 0; c < kHeadDim; ++c) {
-      const float kv = __half2float(kt[i * kHeadDim + c]);
-#pragma unroll
-      for (int hh = 0; hh < kMaxGroup; ++hh)
-        if (hh < G) dot[hh] += sm.qraw[hh][c] * kv;
-    }
-    for (int hh = 0; hh < G; ++hh) sm.sc[hh][i] = dot[hh];
-  }
-  __syncthreads();
-  for (int hh = warp; hh < G; hh += kWarps) {
-    float m = -INFINITY;
-    for (int i = lane; i < tau; i += 32) m = fmaxf(m, sm.sc[hh][i]);
-    m = warp_max(m);
-    float ps = 0.f;
-    for (int i = lane; i < tau; i += 32) {
-      const float p = exp2f(sm.sc[hh][i] - m);
-      sm.sc[hh][i] = p;
-      ps += p;
-    }
-    ps = warp_sum(ps);
-    // merge statistics over the chunks: the warp's lanes stride over them
-    float mm = m;
-    for (int s = lane; s < S; s += 32) {
-      const float* pp = parts + ((ubase + s) * G + hh) * kPartFloats;
-      if (pp[1] > 0.f) mm = fmaxf(mm, pp[0]);
-    }
-    mm = warp_max(mm);
-    float ll = 0.f;
-    for (int s = lane; s < S; s += 32) {
-      const float* pp = parts + ((ubase + s) * G + hh) * kPartFloats;
-      if (pp[1] > 0.f) ll += pp[1] * exp2f(pp[0] - mm);
-    }
-    ll = warp_sum(ll);
-    if (lane == 0) {
-      const float et = ps > 0.f ? exp2f(m - mm) : 0.f;
-      const float l = ll + ps * et;
-      sm.big_m[hh] = mm;
-      sm.et[hh] = et;
-      sm.inv_l[hh] = l > 0.f ? 1.f / l : 0.f;
-    }
-  }
-  __syncthreads();  // tail weights in sm.sc are read by every thread below
-  for (int idx = tid; idx < G * kHeadDim; idx += kMergeThreads) {
-    const int hh = idx / kHeadDim, c = idx % kHeadDim;
-    float at = 0.f;
-    for (int i = 0; i < tau; ++i) at += sm.sc[hh][i] * __half2float(vt[i * kHeadDim + c]);
-    sm.tl[hh][c] = at;
-  }
-  __syncthreads();
-
-  // 2. per head: warps split the chunks, lane owns channels 4*lane .. 4*lane+3
-  __half* out = static_cast<__half*>(a.out) + (static_cast<size_t>(b) * nh + h) * G * kHeadDim;
-  for (int hh = 0; hh < G; ++hh) {
-    const float mm = sm.big_m[hh];
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-    for (int s = warp; s < S; s += kWarps) {
-      const float* pp = parts + ((ubase + s) * G + hh) * kPartFloats;
-      const float2 ml = *reinterpret_cast<const float2*>(pp);
-      const float4 v = *reinterpret_cast<const float4*>(pp + kPartAcc + 4 * lane);
-      if (ml.y > 0.f) {
-        const float wgt = exp2f(ml.x - mm);
-        acc.x += wgt * v.x;
-        acc.y += wgt * v.y;
-        acc.z += wgt * v.z;
-        acc.w += wgt * v.w;
-      }
-    }
-    *reinterpret_cast<float4*>(&sm.red[warp][4 * lane]) = acc;
-    __syncthreads();
-    if (warp == 0) {
-      float v[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        float x = 0.f;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) x += sm.red[w][4 * lane + k];
-        v[k] = x;
-      }
-      fwht128_warp(v, lane);  // the one inverse rotation (H = H^T = H^-1)
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int c = 4 * lane + k;
-        out[hh * kHeadDim + c] = __float2half_rn(
-            (v[k] / kSqrtHeadDim * rotation_sign(a.cfg.rotation_seed, c) + sm.et[hh] * sm.tl[hh][c]) * sm.inv_l[hh]);
-      }
-    }
-    __syncthreads();
-  }
-}
-
 int device_sms() {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -673,7 +1069,7 @@ int device_sms() {
 }
 
 template <int T, int BK, int BV>
-cudaError_t launch_tiles_t(const DecodeArgs& a, cudaStream_t s, int grid) {
+cudaError_t launch_decode_bits(const DecodeArgs& a, cudaStream_t s, int sms) {
   using Geo = DecodeGeom<T, BK, BV>;
   auto kern = decode_tiles_kernel<T, BK, BV>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Geo::kSmem);
@@ -681,47 +1077,79 @@ cudaError_t launch_tiles_t(const DecodeArgs& a, cudaStream_t s, int grid) {
   int per_sm = 0;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, Geo::kWarps * 32, Geo::kSmem);
   if (e != cudaSuccess) return e;
-  kern<<<grid * std::max(per_sm, 1), Geo::kWarps * 32, Geo::kSmem, s>>>(a);
+  per_sm = std::max(per_sm, 1);
+  // automatic split: 32 units per SM whatever the residency (8 per warp at
+  // T = 128, where one CTA fits an SM; the warps take units from a queue, so
+  // short units even out the ragged last chunks), as the workspace holds
+  const int target = kUnitsPerSm * sms;
+  decode_schedule_kernel<<<1, 1024, 0, s>>>(a.seq_lens, a.num_seqs, T, a.cfg.num_kv_heads, a.cfg.group_size,
+                                            a.num_splits_fixed, target, a.workspace);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  kern<<<sms * per_sm, Geo::kWarps * 32, Geo::kSmem, s>>>(a);
   return cudaGetLastError();
 }
 
-template <int T>
-cudaError_t launch_tiles_bits(const DecodeArgs& a, cudaStream_t s, int grid) {
-  if (a.cfg.bits_k == 4 && a.cfg.bits_v == 4) return launch_tiles_t<T, 4, 4>(a, s, grid);
-  if (a.cfg.bits_k == 4 && a.cfg.bits_v == 2) return launch_tiles_t<T, 4, 2>(a, s, grid);
-  if (a.cfg.bits_k == 2 && a.cfg.bits_v == 4) return launch_tiles_t<T, 2, 4>(a, s, grid);
-  if (a.cfg.bits_k == 8 && a.cfg.bits_v == 8) return launch_tiles_t<T, 8, 8>(a, s, grid);
-  return launch_tiles_t<T, 2, 2>(a, s, grid);
+// the fused serving step: no schedule kernel (a fixed grid of num_splits
+// units per (sequence, KV head)), one launch
+template <int T, int BK, int BV>
+cudaError_t launch_step_bits(const DecodeArgs& a, cudaStream_t s, int sms) {
+  using Geo = DecodeGeom<T, BK, BV>;
+  auto kern = decode_tiles_kernel<T, BK, BV>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Geo::kSmem);
+  if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, Geo::kWarps * 32, Geo::kSmem);
+  if (e != cudaSuccess) return e;
+  kern<<<sms * std::max(per_sm, 1), Geo::kWarps * 32, Geo::kSmem, s>>>(a);
+  return cudaGetLastError();
 }
+
+template <int T, template <int, int, int> class L>
+cudaError_t dispatch_decode_bits(const DecodeArgs& a, cudaStream_t s, int sms) {
+  const int bk = a.cfg.bits_k, bv = a.cfg.bits_v;
+  if (bk == 4 && bv == 4) return L<T, 4, 4>::run(a, s, sms);
+  if (bk == 4 && bv == 2) return L<T, 4, 2>::run(a, s, sms);
+  if (bk == 4 && bv == 3) return L<T, 4, 3>::run(a, s, sms);
+  if (bk == 2 && bv == 4) return L<T, 2, 4>::run(a, s, sms);
+  if (bk == 2 && bv == 3) return L<T, 2, 3>::run(a, s, sms);
+  if (bk == 3 && bv == 4) return L<T, 3, 4>::run(a, s, sms);
+  if (bk == 3 && bv == 2) return L<T, 3, 2>::run(a, s, sms);
+  if (bk == 3 && bv == 3) return L<T, 3, 3>::run(a, s, sms);
+  if (bk == 8 && bv == 8) return L<T, 8, 8>::run(a, s, sms);
+  return L<T, 2, 2>::run(a, s, sms);
+}
+template <int T, int BK, int BV>
+struct DecodeLauncher {
+  static cudaError_t run(const DecodeArgs& a, cudaStream_t s, int sms) { return launch_decode_bits<T, BK, BV>(a, s, sms); }
+};
+template <int T, int BK, int BV>
+struct StepLauncher {
+  static cudaError_t run(const DecodeArgs& a, cudaStream_t s, int sms) { return launch_step_bits<T, BK, BV>(a, s, sms); }
+};
 
 template <int T>
 cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t s) {
-  const int sms = device_sms();
-  decode_schedule_kernel<<<1, 1024, 0, s>>>(a.seq_lens, a.num_seqs, T, a.cfg.num_kv_heads, a.num_splits_fixed,
-                                            kUnitsPerSm * sms, a.workspace);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  e = launch_tiles_bits<T>(a, s, sms);
-  if (e != cudaSuccess) return e;
-  dim3 g2(a.cfg.num_kv_heads, a.num_seqs);
-  decode_merge_kernel<T><<<g2, kMergeThreads, 0, s>>>(a);
-  return cudaGetLastError();
+  return a.step ? dispatch_decode_bits<T, StepLauncher>(a, s, device_sms())
+                : dispatch_decode_bits<T, DecodeLauncher>(a, s, device_sms());
 }
 
 }  // namespace
 
 size_t decode_workspace_bytes(const kvq_config& cfg, int num_seqs, int num_splits, int num_sms) {
-  const WsLayout wl = ws_layout(num_seqs);
+  const WsLayout wl = ws_layout(num_seqs, cfg.num_kv_heads, cfg.group_size);
   const size_t units = num_splits > 0
                            ? static_cast<size_t>(num_seqs) * cfg.num_kv_heads * num_splits
                            : static_cast<size_t>(kUnitsPerSm) * num_sms + static_cast<size_t>(num_seqs) * cfg.num_kv_heads;
-  return wl.part_off + units * cfg.group_size * kPartFloats * sizeof(float);
+  return wl.part_off + units * cfg.group_size * kPartFloats * sizeof(float) + units * sizeof(int32_t);
 }
 
 cudaError_t launch_selftest_wait_decode(int32_t* dev_status, cudaStream_t s) {
   selftest_wait_decode_kernel<<<1, 1, 0, s>>>(dev_status);
   return cudaGetLastError();
 }
+
+cudaError_t launch_append_decode_step(const DecodeArgs& a, cudaStream_t s) { return launch_paged_decode(a, s); }
 
 cudaError_t launch_paged_decode(const DecodeArgs& a, cudaStream_t s) {
   if (a.num_seqs == 0) return cudaSuccess;

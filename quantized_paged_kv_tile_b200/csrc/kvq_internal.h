@@ -105,10 +105,21 @@ struct DecodeArgs {
   void* workspace;
   int num_splits_fixed;  // > 0: chunks per (sequence, KV head); 0: automatic
   int32_t* dev_status;
+  // fused serving step (kvq_append_decode_step): seq_lens hold the lengths
+  // before the step; the step's K and V rows (one token per sequence) go into
+  // the tails, attention runs over one more token, and the lengths advance
+  int step;
+  const void* new_k;       // [B][H_kv][d] fp16
+  const void* new_v;
+  int32_t* seq_lens_rw;    // the same array as seq_lens, written at the end of the step
 };
 // Workspace bytes for a split setting on a device with num_sms SMs.
 size_t decode_workspace_bytes(const kvq_config& cfg, int num_seqs, int num_splits, int num_sms);
 cudaError_t launch_paged_decode(const DecodeArgs& a, cudaStream_t s);
+// the fused serving step: one launch (append one token per sequence, decode,
+// advance the lengths); the workspace counters must be zero on entry and are
+// left zero
+cudaError_t launch_append_decode_step(const DecodeArgs& a, cudaStream_t s);
 
 struct PrefillArgs {
   kvq_config cfg;

@@ -125,11 +125,24 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
 // (field e, field e + W/2), so MMA position 2e + s of the word's group holds
 // channel e + s W/2.  q'' is written in the same order (the dot product does
 // not care which order, only that both operands share it).
+// At 3 bits the codes are extracted one by one and the order is the
+// natural one (position k holds channel k).
 template <int B>
 __device__ __forceinline__ constexpr int qk_channel(int kpos) {
-  constexpr int W = 32 / B;
+  if (B == 3) return kpos;
+  constexpr int W = 32 / (B == 3 ? 4 : B);
   const int p = kpos % W;
   return kpos - p + (p >> 1) + (p & 1) * (W / 2);
+}
+
+// b-bit field at bit `bit` of a little-endian run of 32-bit words (b <= 8)
+template <int B>
+__device__ __forceinline__ uint32_t field_at(const uint32_t* w, int bit) {
+  return __funnelshift_r(w[bit >> 5], w[(bit >> 5) + 1], bit & 31) & ((1u << B) - 1u);
+}
+// two codes as an fp16 pair of exact small integers (low half `lo`)
+__device__ __forceinline__ uint32_t code_pair_f16(uint32_t lo, uint32_t hi) {
+  return h2_as_u32(__hsub2(u32_as_h2(lo | (hi << 16) | 0x64006400u), __float2half2_rn(1024.f)));
 }
 
 // Byte offset of (row r, position k) in a K-major fp16 operand of `rows` rows
@@ -563,7 +576,12 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
       const int tok = i >> 4, pc = i & 15;
       const unsigned char* rec = sK + (pg0 + tok / kPageTokens) * Geo::kPageK + (tok % kPageTokens) * (16 * BK);
       uint32_t pr[4];
-      if constexpr (BK == 4) {
+      if constexpr (BK == 3) {  // channels 8 pc .. 8 pc + 7: bits 24 pc .. 24 pc + 23 of the record
+        const uint32_t* rw = reinterpret_cast<const uint32_t*>(rec);
+        const uint32_t x = field_at<24>(rw, 24 * pc);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) pr[k] = code_pair_f16((x >> (6 * k)) & 7u, (x >> (6 * k + 3)) & 7u);
+      } else if constexpr (BK == 4) {
         unpack_pairs<4>(*reinterpret_cast<const uint32_t*>(rec + 4 * pc), pr);
       } else if constexpr (BK == 2) {
         uint32_t all[8];
@@ -578,6 +596,20 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
       *reinterpret_cast<uint4*>(smem + kOffBk + sw_off(tok, 8 * pc, kNS)) = make_uint4(pr[0], pr[1], pr[2], pr[3]);
     }
     unsigned char* bv = smem + kOffBv + (gb & 1) * 16384;
+    if constexpr (BV == 3) {
+      // 3-bit V pages are a token-major bitstream: code (token p, channel c)
+      // at bit 3 (128 p + c); each unit is one channel of one token pair
+      constexpr int kUnits3 = (Geo::kValid / kPageTokens) * kHeadDim * (kPageTokens / 2);
+      for (int i = tid; i < kUnits3; i += kPfThreads) {
+        const int pgl = i / (kHeadDim * (kPageTokens / 2)), rem = i % (kHeadDim * (kPageTokens / 2));
+        const int c = rem % kHeadDim, j = rem / kHeadDim;
+        const uint32_t* cw = reinterpret_cast<const uint32_t*>(sV + (pg0 + pgl) * Geo::kPageV);
+        const int bit = 3 * (kHeadDim * 2 * j + c);
+        *reinterpret_cast<uint32_t*>(bv + sw_off(c, kPageTokens * pgl + 2 * j, kHeadDim)) =
+            code_pair_f16(field_at<3>(cw, bit), field_at<3>(cw, bit + 3 * kHeadDim));
+      }
+      return;
+    }
     constexpr int kRowsPerLane = BV / 2;  // 16-byte rows per lane (2 b words / 4)
     constexpr int kVUnits = (Geo::kValid / kPageTokens) * 32 * kRowsPerLane;
     for (int i = tid; i < kVUnits; i += kPfThreads) {
@@ -1045,10 +1077,16 @@ cudaError_t launch_t(const PrefillArgs& a, cudaStream_t s, long long units) {
 
 template <int T>
 cudaError_t launch_bits(const PrefillArgs& a, cudaStream_t s, long long units) {
-  if (a.cfg.bits_k == 4 && a.cfg.bits_v == 4) return launch_t<T, 4, 4>(a, s, units);
-  if (a.cfg.bits_k == 4 && a.cfg.bits_v == 2) return launch_t<T, 4, 2>(a, s, units);
-  if (a.cfg.bits_k == 2 && a.cfg.bits_v == 4) return launch_t<T, 2, 4>(a, s, units);
-  if (a.cfg.bits_k == 8 && a.cfg.bits_v == 8) return launch_t<T, 8, 8>(a, s, units);
+  const int bk = a.cfg.bits_k, bv = a.cfg.bits_v;
+  if (bk == 4 && bv == 4) return launch_t<T, 4, 4>(a, s, units);
+  if (bk == 4 && bv == 2) return launch_t<T, 4, 2>(a, s, units);
+  if (bk == 4 && bv == 3) return launch_t<T, 4, 3>(a, s, units);
+  if (bk == 2 && bv == 4) return launch_t<T, 2, 4>(a, s, units);
+  if (bk == 2 && bv == 3) return launch_t<T, 2, 3>(a, s, units);
+  if (bk == 3 && bv == 4) return launch_t<T, 3, 4>(a, s, units);
+  if (bk == 3 && bv == 2) return launch_t<T, 3, 2>(a, s, units);
+  if (bk == 3 && bv == 3) return launch_t<T, 3, 3>(a, s, units);
+  if (bk == 8 && bv == 8) return launch_t<T, 8, 8>(a, s, units);
   return launch_t<T, 2, 2>(a, s, units);
 }
 

@@ -30,7 +30,7 @@ EXPORTED_SYMBOLS = (
     "kvq_get_layout", "kvq_decode_workspace_bytes", "kvq_quantize_tiles", "kvq_append_tokens",
     "kvq_paged_decode_attention", "kvq_paged_decode_attention_static_scratch", "kvq_unpack_tiles",
     "kvq_selftest_bounded_wait", "kvq_status_string", "kvq_last_error", "kvq_version",
-    "kvq_prefill_workspace_bytes", "kvq_paged_prefill_attention",
+    "kvq_prefill_workspace_bytes", "kvq_paged_prefill_attention", "kvq_append_decode_step",
 )
 
 
@@ -94,6 +94,8 @@ _SIGNATURES = {
     "kvq_append_tokens": [_cfgp, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp],
     "kvq_paged_decode_attention": [_cfgp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _vp, _vp, _vp, _vp, _f32, _vp,
                                    _sz, _i32, _vp, _vp],
+    "kvq_append_decode_step": [_cfgp, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _vp, _vp, _vp, _vp, _f32,
+                               _vp, _sz, _i32, _vp, _vp],
     "kvq_paged_decode_attention_static_scratch": [_cfgp, _vp, _vp, _vp, _i32, _vp, _i32, _i32, _vp, _vp, _vp,
                                                   _vp, _f32, _i32, _vp, _vp],
     "kvq_selftest_bounded_wait": [_vp, _vp],
@@ -228,6 +230,37 @@ def paged_decode_attention(cfg: Config, q, out, seq_lens, block_tables, k_pool, 
         _ptr(workspace, "workspace", torch.uint8), workspace.numel(), num_splits,
         _ptr(dev_status, "dev_status", torch.int32), _stream(stream))
     _check(st, "kvq_paged_decode_attention")
+
+
+def append_decode_step(cfg: Config, new_k, new_v, q, out, seq_lens, block_tables, k_pool, v_pool, k_tail, v_tail,
+                       workspace, num_splits: int, softmax_scale: float | None = None, num_blocks: int | None = None,
+                       dev_status=None, stream=None) -> None:
+    """One serving step in one launch: the step's token rows (new_k, new_v
+    fp16 [B][H_kv][d]) into the tails, decode over the cache including them,
+    ``seq_lens`` (the lengths before the step) advanced by one.  No sequence
+    may complete a tile in the step.  ``workspace``: uint8, at least
+    ``decode_workspace_bytes(cfg, B, num_splits)`` bytes, zero-filled before
+    its first use (each call leaves its counters at zero again)."""
+    if softmax_scale is None:
+        softmax_scale = cfg.head_dim ** -0.5
+    nb = k_pool.shape[0] if num_blocks is None else num_blocks
+    st = load_library().kvq_append_decode_step(
+        ctypes.byref(cfg.c()), _ptr(new_k, "new_k", torch.float16), _ptr(new_v, "new_v", torch.float16),
+        _ptr(q, "q", torch.float16), _ptr(out, "out", torch.float16), _ptr(seq_lens, "seq_lens", torch.int32),
+        seq_lens.shape[0], _ptr(block_tables, "block_tables", torch.int32), block_tables.shape[1], nb,
+        _ptr(k_pool, "k_pool", torch.uint8), _ptr(v_pool, "v_pool", torch.uint8),
+        _ptr(k_tail, "k_tail", torch.float16), _ptr(v_tail, "v_tail", torch.float16), float(softmax_scale),
+        _ptr(workspace, "workspace", torch.uint8), workspace.numel(), num_splits,
+        _ptr(dev_status, "dev_status", torch.int32), _stream(stream))
+    _check(st, "kvq_append_decode_step")
+
+
+def step_splits(cfg: Config, num_seqs: int, num_sms: int) -> int:
+    """Chunks per (sequence, KV head) for the fused serving step: about 32
+    work units per SM (the granularity the automatic decode split uses), at
+    least one per (sequence, KV head)."""
+    pairs = max(1, num_seqs * cfg.num_kv_heads)
+    return min(65535, max(1, -(-32 * num_sms // pairs)))
 
 
 def prefill_workspace_bytes(cfg: Config, num_seqs: int, max_chunk_tokens: int, num_splits: int) -> int:

@@ -203,14 +203,24 @@ class DecodeStepGraph:
     Stage the step's rows in ``new_k`` / ``new_v`` ([B][H_kv][d] fp16) and its
     queries in ``q`` ([B][H_q][d] fp16), call ``replay()``, read ``out``.  The
     sequence lengths advance on the device inside the graph (the append reads
-    them as the lengths before the step, then they grow by one); the host only
+    them as the lengths before the step, then they grow by one); the host
     tracks them to refuse a step past the allocated pages.  The first decode
     and append calls happen eagerly before capture.
+
+    ``fused=True``: steps in which no sequence completes a tile replay a graph
+    of one launch (kvq_append_decode_step: the token into the tails, the
+    decode, the lengths advanced); steps that complete a tile replay the
+    append + decode graph (the completed tile has to be quantized first).
+    Both use the same split count, so the outputs are those of the unfused
+    step bit for bit.
     """
 
-    def __init__(self, cache: PagedKVCache, num_splits: int | None = None):
+    def __init__(self, cache: PagedKVCache, num_splits: int | None = None, fused: bool = False):
         self.cache = cache
         cfg, b, dev = cache.cfg, cache.num_seqs, cache.device
+        self.fused = fused
+        if fused and num_splits is None:
+            num_splits = kvq.step_splits(cfg, b, torch.cuda.get_device_properties(dev).multi_processor_count)
         self.num_splits = cache.num_splits if num_splits is None else num_splits
         self.new_k = torch.zeros((b, cfg.num_kv_heads, cfg.head_dim), dtype=torch.float16, device=dev)
         self.new_v = torch.zeros_like(self.new_k)
@@ -220,6 +230,8 @@ class DecodeStepGraph:
         need = kvq.decode_workspace_bytes(cfg, b, self.num_splits)
         if cache.workspace.numel() < need:
             cache.workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        # the fused step's own workspace: zero-filled once, left zero by every step
+        self.step_workspace = torch.zeros(need, dtype=torch.uint8, device=dev) if fused else None
         self.graph = torch.cuda.CUDAGraph()
         side = torch.cuda.Stream(device=dev)
         side.wait_stream(torch.cuda.current_stream(dev))
@@ -230,6 +242,11 @@ class DecodeStepGraph:
         torch.cuda.synchronize(dev)
         with torch.cuda.graph(self.graph):
             self._step()
+        self.graph_fused = None
+        if fused:
+            self.graph_fused = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(self.graph_fused):
+                self._fused_step()
 
     def _decode(self) -> None:
         c = self.cache
@@ -244,10 +261,24 @@ class DecodeStepGraph:
         c.seq_lens.add_(1)
         self._decode()
 
+    def _fused_step(self) -> None:
+        c = self.cache
+        kvq.append_decode_step(c.cfg, self.new_k, self.new_v, self.q, self.out, c.seq_lens, c.block_tables,
+                               c.k_pool, c.v_pool, c.k_tail, c.v_tail, self.step_workspace, self.num_splits,
+                               num_blocks=c.num_blocks, dev_status=c.dev_status)
+
+    def completes_tile(self) -> bool:
+        """Whether the next step completes a tile of some sequence."""
+        c = self.cache
+        return bool(np.any((c.host_lens + 1) % c.cfg.tile_tokens == 0))
+
     def replay(self) -> torch.Tensor:
         c = self.cache
         if np.any(c.host_lens + 1 > c.blocks_per_seq * c.cfg.page_tokens):
             raise ValueError("append past the allocated pages")
-        self.graph.replay()
+        if self.fused and not self.completes_tile():
+            self.graph_fused.replay()
+        else:
+            self.graph.replay()
         c.host_lens = c.host_lens + 1
         return self.out

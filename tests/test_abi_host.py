@@ -88,14 +88,24 @@ def test_argument_errors_launch_nothing(lib):
     # misaligned pointer
     st = lib.kvq_quantize_tiles(ctypes.byref(c), 17, None, 10, 16, 1, 16, 1, 4, 8, 16, 16, None, None)
     assert st == kvq.KVQ_ERR_INVALID_ARG and "aligned" in kvq.load_library().kvq_last_error().decode()
-    # 3-bit decode is storage-only
-    c3 = kvq.Config(num_kv_heads=2, group_size=4, tile_tokens=64, bits_k=3, bits_v=4, iters=4).c()
-    st = lib.kvq_paged_decode_attention(ctypes.byref(c3), 16, 16, 16, 1, 16, 4, 8, 16, 16, 16, 16, 0.1, 16,
+    # a head size without kernels is refused before any launch
+    c64 = kvq.Config(num_kv_heads=2, group_size=4, tile_tokens=64, bits_k=4, bits_v=4, iters=4, head_dim=64).c()
+    st = lib.kvq_paged_decode_attention(ctypes.byref(c64), 16, 16, 16, 1, 16, 4, 8, 16, 16, 16, 16, 0.1, 16,
                                         1 << 20, 1, None, None)
     assert st == kvq.KVQ_ERR_UNSUPPORTED
+    # 3-bit pages are read: the call gets past the configuration checks (here
+    # to the workspace check, with no device query for an explicit split count)
+    c3 = kvq.Config(num_kv_heads=2, group_size=4, tile_tokens=64, bits_k=3, bits_v=4, iters=4).c()
+    st = lib.kvq_paged_decode_attention(ctypes.byref(c3), 16, 16, 16, 1, 16, 4, 8, 16, 16, 16, 16, 0.1, 16,
+                                        1, 1, None, None)
+    assert st == kvq.KVQ_ERR_WORKSPACE
     # workspace too small (explicit split count: no device query)
     need = kvq.decode_workspace_bytes(cfg, 3, 2)
-    assert need == 256 + 3 * 2 * 2 * 4 * 132 * 4      # schedule header, then 528-byte partial records
+    # schedule header and counters (256 B), one 528-byte raw-tail record per
+    # (sequence, KV head, query head), then one 528-byte partial record per
+    # (unit, query head): 3 sequences x 2 KV heads x 2 splits x 4 query heads,
+    # then one int32 merge-group counter per unit
+    assert need == 256 + 3 * 2 * 4 * 132 * 4 + 3 * 2 * 2 * 4 * 132 * 4 + 3 * 2 * 2 * 4
     st = lib.kvq_paged_decode_attention(ctypes.byref(c), 16, 16, 16, 3, 16, 4, 8, 16, 16, 16, 16, 0.1, 16,
                                         need - 1, 2, None, None)
     assert st == kvq.KVQ_ERR_WORKSPACE
@@ -111,8 +121,11 @@ def test_prefill_argument_errors_launch_nothing(lib):
         return lib.kvq_paged_prefill_attention(ctypes.byref(conf), q, 16, 16, 16, 16, 16, num_seqs, max_chunk,
                                                tables, 4, 8, 16, 16, 16, 16, scale, splits, ws, ws_bytes, None,
                                                None)
+    c64 = kvq.Config(num_kv_heads=2, group_size=4, tile_tokens=64, bits_k=4, bits_v=4, iters=4, head_dim=64).c()
+    assert call(c64) == kvq.KVQ_ERR_UNSUPPORTED
+    # 3-bit pages are read: past the configuration checks, to the workspace check
     c3 = kvq.Config(num_kv_heads=2, group_size=4, tile_tokens=64, bits_k=4, bits_v=3, iters=4).c()
-    assert call(c3) == kvq.KVQ_ERR_UNSUPPORTED
+    assert call(c3, splits=2, ws=16, ws_bytes=16) == kvq.KVQ_ERR_WORKSPACE
     assert call(c, num_seqs=-1) == kvq.KVQ_ERR_INVALID_ARG
     assert call(c, max_chunk=-2) == kvq.KVQ_ERR_INVALID_ARG
     assert call(c, q=None) == kvq.KVQ_ERR_INVALID_ARG

@@ -59,3 +59,33 @@ def test_pair_bytes_add_up_to_the_step():
         total = bm["quantize"] + bm["append"] + bm["decode"]
         per = bench.pair_bytes(w, bm)
         assert abs(float(np.sum(per)) * w.num_kv_heads - total) <= 1e-9 * total, name
+
+
+def test_record_traffic_reads_an_ncu_csv(tmp_path):
+    # two decode launches and one quantize launch in ncu's --csv layout (with a
+    # profiler line mixed in): per-launch means, units from the byte model
+    import json
+    import bench
+    from quantized_paged_kv_tile_b200 import synth
+    head = '"ID","Process ID","Process Name","Host Name","Kernel Name","Context","Stream","Block Size",' \
+           '"Grid Size","Device","CC","Section Name","Metric Name","Metric Unit","Metric Value"\n'
+    rows = []
+    for i, (kern, rd, wr, ns) in enumerate([("quantize_tc_kernel<64, 4, 4>", 100, 20, 7),
+                                             ("decode_tiles_kernel<64, 4, 4>", "1,000", 10, 3),
+                                             ("decode_tiles_kernel<64, 4, 4>", "3,000", 30, 5)]):
+        for m, v in (("dram__bytes_read.sum", rd), ("dram__bytes_write.sum", wr), ("gpu__time_duration.sum", ns)):
+            rows.append(f'"{i}","1","python3","h","void {kern}(Args)","1","7","(128, 1, 1)","(444, 1, 1)","0",'
+                        f'"10.0","Command line profiler metrics","{m}","byte","{v}"\n')
+    p = tmp_path / "cap.csv"
+    p.write_text("==PROF== Connected to process 1\n" + head + "".join(rows))
+    out = tmp_path / "traffic.json"
+    rec = bench.record_traffic(str(p), "qwen3_4b", 1, "cmd", str(out))
+    bm = bench.byte_model(synth.workload("qwen3_4b", num_seqs=1), 0, 0)
+    assert rec["quantize_tc_kernel"]["dram_bytes_per_launch"] == 120
+    assert rec["decode_tiles_kernel"]["dram_bytes_per_launch"] == 2000 + 20
+    assert rec["decode_tiles_kernel"]["launches_captured"] == 2
+    assert rec["quantize_tc_kernel"]["units_per_launch"] == bm["quant_units"]
+    assert rec["decode_tiles_kernel"]["units_per_launch"] == bm["decode"]
+    assert json.loads(out.read_text()) == rec
+    # the record scales to another launch by units, and only while the sources are unchanged
+    assert rec["decode_tiles_kernel"]["source_digest"] == bench.source_digest("decode_tiles_kernel")

@@ -167,6 +167,8 @@ DECODE_CASES = [
     dict(num_seqs=3, lens=(700, 64, 30), num_kv_heads=2, group_size=4, bits_v=2),
     dict(num_seqs=2, lens=(520, 1), num_kv_heads=2, group_size=1, tile_tokens=128, bits_k=2, bits_v=4, iters=2),
     dict(num_seqs=2, lens=(333, 257), num_kv_heads=1, group_size=3, tile_tokens=32, bits_k=4, bits_v=2, iters=1),
+    dict(num_seqs=2, lens=(700, 90), num_kv_heads=2, group_size=4, bits_k=3, bits_v=3),   # 3-bit pages
+    dict(num_seqs=1, lens=(600,), num_kv_heads=1, group_size=8, tile_tokens=128, bits_k=3, bits_v=4, iters=2),
 ]
 
 
@@ -188,7 +190,7 @@ def test_decode_matches_oracle(over):
             assert err <= ATTN_REL_L2_MAX, (s, hq, err)
 
 
-DECODE_SWEEP = ([(t, bk, bv, g) for t in (32, 64, 128) for bk in (2, 4) for bv in (2, 4) for g in (2, 8)]
+DECODE_SWEEP = ([(t, bk, bv, g) for t in (32, 64, 128) for bk in (2, 3, 4) for bv in (2, 3, 4) for g in (2, 8)]
                 + [(t, 8, 8, g) for t in (32, 64, 128) for g in (2, 8)])
 
 
@@ -264,10 +266,12 @@ def test_decode_only_on_oracle_packed_pages():
 
 
 def test_decode_independent_of_split_count():
-    w = synth.workload("tiny", num_seqs=2, lens=(2048 + 7, 640), num_kv_heads=2, group_size=4)
+    # 40 tiles in sequence 0: 20 and 40 splits merge in two levels (groups of
+    # 16 chunks, then the groups), the others in one
+    w = synth.workload("tiny", num_seqs=2, lens=(64 * 40 + 7, 640), num_kv_heads=2, group_size=4)
     cfg, cache, rk, rv = _prefilled(w)
     q = synth.queries(w, device="cuda")
-    outs = [cache.decode(q, num_splits=s).float().cpu().numpy() for s in (1, 2, 5, 13, 0)]
+    outs = [cache.decode(q, num_splits=s).float().cpu().numpy() for s in (1, 2, 5, 13, 20, 40, 0)]
     for other in outs[1:]:
         assert rel_l2(other, outs[0]) <= 1e-4
 

@@ -84,6 +84,9 @@ CASES = [
     (128, 8, 8, 4, (256, 300), (9, 50)),
     (64, 2, 2, 4, (513, 77), (64, 0)),              # a sequence with an empty chunk
     (32, 8, 8, 2, (100, 0), (64, 3)),
+    (64, 3, 3, 4, (300, 70), (40, 17)),             # 3-bit codes (token-major bitstreams)
+    (128, 3, 4, 2, (260,), (30,)),
+    (32, 4, 3, 8, (97, 64), (21, 40)),
 ]
 
 
