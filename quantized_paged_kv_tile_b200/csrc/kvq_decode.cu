@@ -257,19 +257,19 @@ static_assert(16 * kTailRowBytes <= kTailScratch, "16 staged tail rows fit the w
 
 // One warp: the raw fp16 tail (tau < T tokens) of (sequence b, KV head h)
 // for its g query heads, in the original domain, on the tensor cores
-// (mma.sync m16n8k16, rows = query heads).  Scores: q and the raw K rows are
-// fp16, so the products are exact and sum in fp32; lane (g, t) loads 16-byte
-// runs of q and K, and k-block 2j + u takes channels 32j + 8t + 4u + {0, 1}
-// (fragment columns 2t, 2t + 1) and 32j + 8t + 4u + {2, 3} (columns 2t + 8,
-// 2t + 9) on both sides.  A softmax per head over the tail alone, then P V:
-// the score fragments are the A fragments of P (rows g / g + 8 = hi / lo fp16
-// halves of p), V comes through shared memory in 16-token chunks as
-// transposed 8x8 fp16 tiles.  Writes the tail record (m, l, acc) of every
+// (mma.sync m16n8k16, rows = query heads), 16 tokens at a time with a running
+// (online) softmax per head.  Scores: q and the raw K rows are fp16, so the
+// products are exact and sum in fp32; lane (g, t) loads 16-byte runs of q and
+// K, and k-block 2j + u takes channels 32j + 8t + 4u + {0, 1} (fragment
+// columns 2t, 2t + 1) and 32j + 8t + 4u + {2, 3} (columns 2t + 8, 2t + 9) on
+// both sides.  P V: the score fragments are the A fragments of P (rows g /
+// g + 8 = hi / lo fp16 halves of p), V comes through shared memory as
+// transposed 8x8 fp16 tiles.  The loop body is emitted once, so the code stays
+// small next to the tile loop.  Writes the tail record (m, l, acc) of every
 // query head; scratch: 16 padded V rows (4352 bytes) of the warp's shared
 // memory, whose copies must all have landed.
 template <int T>
 __device__ __noinline__ void decode_tail_warp(const DecodeArgs& a, int b, int h, int tau, float* tails, float* scratch, int lane) {
-  constexpr int NB = T / 8;  // 8-token score blocks
   const int G = a.cfg.group_size, nh = a.cfg.num_kv_heads;
   const int g = lane >> 2, t = lane & 3;
   const float qscale = a.softmax_scale * kLog2e;
@@ -295,15 +295,35 @@ __device__ __noinline__ void decode_tail_warp(const DecodeArgs& a, int b, int h,
   }
   const __half* kt = static_cast<const __half*>(a.k_tail) + bh * T * kHeadDim;
   const __half* vt = static_cast<const __half*>(a.v_tail) + bh * T * kHeadDim;
+  unsigned char* vs = reinterpret_cast<unsigned char*>(scratch);
+  // ldmatrix lane 8i + r: row r of matrix i = token r + 8 (i & 1), channels 8 (nv + (i >> 1)) ..
+  const uint32_t lane_addr = smem_u32(vs) + ((lane & 7) + 8 * ((lane >> 3) & 1)) * kTailRowBytes + 16 * (lane >> 4);
 
-  // -- scores (log2 domain) of tokens 8nb + 2t, 8nb + 2t + 1 for head g
-  float sc[NB][2];
-  float m = -INFINITY;
+  float m = -INFINITY, l = 0.f;  // running max and this lane's share of the sum, head g
+  float acc[16][4];
 #pragma unroll
-  for (int nb = 0; nb < NB; ++nb) {
-    sc[nb][0] = sc[nb][1] = -INFINITY;
-    if (8 * nb < tau) {  // warp-uniform
-      const int tk = 8 * nb + g;
+  for (int nv = 0; nv < 16; ++nv)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) acc[nv][k] = 0.f;
+#pragma unroll 1
+  for (int t0 = 0; t0 < tau; t0 += 16) {
+    // stage V rows t0 .. t0 + 15 (zeros past the tail: p is 0 there, and
+    // 0 times a stale non-finite value would not be); the loads are in
+    // flight while the scores are computed
+    __syncwarp();
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int idx = lane + 32 * k, row = idx >> 4, c16 = idx & 15;
+      const int tk = t0 + row;
+      const uint4 v = tk < tau ? *reinterpret_cast<const uint4*>(vt + static_cast<size_t>(tk) * kHeadDim + 8 * c16)
+                               : make_uint4(0u, 0u, 0u, 0u);
+      *reinterpret_cast<uint4*>(vs + row * kTailRowBytes + 16 * c16) = v;
+    }
+    // scores of tokens t0 + 8e + 2t, t0 + 8e + 2t + 1 (e = 0, 1) for head g
+    float sc[2][2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int tk = t0 + 8 * e + g;
       uint4 kr[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j)
@@ -317,61 +337,39 @@ __device__ __noinline__ void decode_tail_warp(const DecodeArgs& a, int b, int h,
         mma16816(d, a0, kr[j].x, kr[j].y);
         mma16816(d, a1, kr[j].z, kr[j].w);
       }
-      const int i0 = 8 * nb + 2 * t;
-      if (i0 < tau) sc[nb][0] = d[0] * qscale;
-      if (i0 + 1 < tau) sc[nb][1] = d[1] * qscale;
-      m = fmaxf(m, fmaxf(sc[nb][0], sc[nb][1]));
+      const int i0 = t0 + 8 * e + 2 * t;
+      sc[e][0] = i0 < tau ? d[0] * qscale : -INFINITY;
+      sc[e][1] = i0 + 1 < tau ? d[1] * qscale : -INFINITY;
     }
-  }
-  m = fmaxf(m, __shfl_xor_sync(kFull, m, 1));
-  m = fmaxf(m, __shfl_xor_sync(kFull, m, 2));
-  float l = 0.f;
+    float cm = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
+    cm = fmaxf(cm, __shfl_xor_sync(kFull, cm, 1));
+    cm = fmaxf(cm, __shfl_xor_sync(kFull, cm, 2));
+    const float m_new = fmaxf(m, cm);  // finite: token t0 is in the tail
+    const float alpha = exp2f(m - m_new);
+    m = m_new;
+    l *= alpha;
 #pragma unroll
-  for (int nb = 0; nb < NB; ++nb)
+    for (int nv = 0; nv < 16; ++nv)
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const float p = sc[nb][e] == -INFINITY ? 0.f : exp2f(sc[nb][e] - m);
-      sc[nb][e] = p;
-      l += p;
-    }
-  l += __shfl_xor_sync(kFull, l, 1);
-  l += __shfl_xor_sync(kFull, l, 2);
-
-  // -- P V: D[16 rows][8 channels] per n-block nv; rows g / g + 8 = hi / lo of p
-  float acc[16][4];
+      for (int k = 0; k < 4; ++k) acc[nv][k] *= alpha;
 #pragma unroll
-  for (int nv = 0; nv < 16; ++nv)
+    for (int e = 0; e < 2; ++e)
 #pragma unroll
-    for (int k = 0; k < 4; ++k) acc[nv][k] = 0.f;
-  unsigned char* vs = reinterpret_cast<unsigned char*>(scratch);
-  const uint32_t vs_addr = smem_u32(vs);
-#pragma unroll
-  for (int kb = 0; kb < NB / 2; ++kb) {
-    if (16 * kb >= tau) break;  // warp-uniform
-    // stage tokens 16kb .. 16kb + 15 (zeros past the tail: p is 0 there, and
-    // 0 times a stale non-finite value would not be)
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int idx = lane + 32 * k, row = idx >> 4, c16 = idx & 15;
-      const int tk = 16 * kb + row;
-      const uint4 v = tk < tau ? *reinterpret_cast<const uint4*>(vt + static_cast<size_t>(tk) * kHeadDim + 8 * c16)
-                               : make_uint4(0u, 0u, 0u, 0u);
-      *reinterpret_cast<uint4*>(vs + row * kTailRowBytes + 16 * c16) = v;
-    }
-    __syncwarp();
+      for (int k = 0; k < 2; ++k) {
+        const float p = sc[e][k] == -INFINITY ? 0.f : exp2f(sc[e][k] - m_new);
+        sc[e][k] = p;
+        l += p;
+      }
     uint32_t pa[4];
     {
-      const float x0 = sc[2 * kb][0], x1 = sc[2 * kb][1], y0 = sc[2 * kb + 1][0], y1 = sc[2 * kb + 1][1];
-      const __half2 hx = __floats2half2_rn(x0, x1), hy = __floats2half2_rn(y0, y1);
+      const __half2 hx = __floats2half2_rn(sc[0][0], sc[0][1]), hy = __floats2half2_rn(sc[1][0], sc[1][1]);
       const float2 fx = __half22float2(hx), fy = __half22float2(hy);
       pa[0] = h2_as_u32(hx);
-      pa[1] = h2_as_u32(__floats2half2_rn(x0 - fx.x, x1 - fx.y));
+      pa[1] = h2_as_u32(__floats2half2_rn(sc[0][0] - fx.x, sc[0][1] - fx.y));
       pa[2] = h2_as_u32(hy);
-      pa[3] = h2_as_u32(__floats2half2_rn(y0 - fy.x, y1 - fy.y));
+      pa[3] = h2_as_u32(__floats2half2_rn(sc[1][0] - fy.x, sc[1][1] - fy.y));
     }
-    // lane 8i + r: row r of matrix i = token r + 8 (i & 1), channels 8 (nv + (i >> 1)) ..
-    const int mi = lane >> 3, mr = lane & 7;
-    const uint32_t lane_addr = vs_addr + (mr + 8 * (mi & 1)) * kTailRowBytes + 16 * (mi >> 1);
+    __syncwarp();
 #pragma unroll
     for (int nv = 0; nv < 16; nv += 2) {
       uint32_t bf[4];
@@ -379,8 +377,9 @@ __device__ __noinline__ void decode_tail_warp(const DecodeArgs& a, int b, int h,
       mma16816(acc[nv], pa, bf[0], bf[1]);
       mma16816(acc[nv + 1], pa, bf[2], bf[3]);
     }
-    __syncwarp();
   }
+  l += __shfl_xor_sync(kFull, l, 1);
+  l += __shfl_xor_sync(kFull, l, 2);
   if (live) {
     float* r = rec + g * kPartFloats;
     if (t == 0) {
