@@ -17,7 +17,7 @@
  *
  * Definitions (the pages give the outline only; these are the concrete
  * readings the library implements):
- *   d = head_dim = 128, P = page_tokens = 16, T = tile_tokens in {32,64,128},
+ *   d = head_dim in {64,128,256}, P = page_tokens = 16, T = tile_tokens in {32,64,128},
  *   b = bits in {2,3,4,8} (8 for K and V together), n = iters >= 0,
  *   eps = std_eps (1e-6).
  *   H = orthonormal Sylvester Hadamard, H[j][k] = (-1)^popcount(j&k)/sqrt(d).
@@ -55,23 +55,34 @@
  *     uint8 pool[num_blocks][num_kv_heads][page_bytes]
  *   One page region (block, head) holds P tokens of one KV head:
  *     [codes | meta | C slice], each region starting on a 16-byte boundary.
- *   codes: P*d*b/8 bytes (2048 at b=8, 1024 at b=4, 768 at b=3, 512 at b=2), a little-
+ *   codes: P*d*b/8 bytes (at d=128: 2048 at b=8, 1024 at b=4, 768 at b=3, 512 at b=2), a little-
  *     endian bitstream; a code occupies b bits at the bit offset below.
  *   meta:  P entries of {fp16 s~, fp16 z~} (64 bytes), token-major.
  *   C slice: page k of its tile (k = logical block index mod T/P) carries
  *     fp16 C~ of channels [k*d*P/T, (k+1)*d*P/T)  (2*d*P/T bytes).
- *   page_bytes = codes + 64 + 2*d*P/T  (1152 for T=64, b=4).
+ *   page_bytes = codes + 64 + 2*d*P/T rounded up to 16  (1152 for d=128, T=64, b=4).
  *   Bit offset of the code of (channel c, token p of the page):
  *     K, and V at b=3:   (p*d + c) * b                (token-major)
  *     V at b in {2,4,8}: the decode kernel's grouped order.  With
  *       n = c/8, g = c%8, t = (p%8)/2, u = p/8, s = p%2, F = 32/b,
- *       h = F/2, k = 2*(n/h) + u, e = n%h, lane = 4*g + t:
- *       byte of word = ((k/4)*32 + lane)*16 + (k%4)*4,
+ *       h = F/2, k = 2*(n/h) + u, e = n%h, lane = 4*g + t, W = d*b/64
+ *       words per lane in rows of R = min(4, W) words (R = 4 except d=64, b=2):
+ *       byte of word = ((k/R)*32 + lane)*4R + (k%R)*4,
  *       bit offset   = 8*(byte of word) + b*(e + h*s).
  *   Tails: fp16 [num_seqs][num_kv_heads][T][d], one for K and one for V;
  *     token position q of a sequence lives in row q mod T.
  *   Query / output: fp16 [num_seqs][num_kv_heads*group_size][d]; query head
  *     h reads KV head h / group_size.
+ *
+ * Head sizes
+ * ----------
+ *   d = 128 runs the tuned path (tensor-core rotation in the quantizer,
+ *   mma.sync decode, tensor-core chunked prefill, the one-launch serving
+ *   step).  d = 64 and d = 256 run kvq_quantize_tiles, kvq_append_tokens,
+ *   kvq_paged_decode_attention (and its static-scratch form) and
+ *   kvq_unpack_tiles on CUDA-core kernels with the same format and the same
+ *   method; kvq_paged_prefill_attention, kvq_prefill_workspace_bytes and
+ *   kvq_append_decode_step return KVQ_ERR_UNSUPPORTED for them.
  *
  * Conventions
  * -----------
@@ -122,7 +133,7 @@ typedef enum {
 } kvq_status;
 
 typedef struct {
-  int head_dim;      /* d: must be 128                                   */
+  int head_dim;      /* d: 64, 128 or 256 (see the head-size note)       */
   int num_kv_heads;  /* H_kv >= 1                                        */
   int group_size;    /* g = query heads per KV head, 1..8                */
   int tile_tokens;   /* T: 32, 64 or 128                                 */

@@ -38,7 +38,8 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 kvq_status check_config(const kvq_config* c) {
   if (c == nullptr) return fail(KVQ_ERR_INVALID_ARG, "config is NULL");
-  if (c->head_dim != kvq::kHeadDim) return fail(KVQ_ERR_UNSUPPORTED, "head_dim must be 128 (got %d)", c->head_dim);
+  if (c->head_dim != 64 && c->head_dim != 128 && c->head_dim != 256)
+    return fail(KVQ_ERR_UNSUPPORTED, "head_dim must be 64, 128 or 256 (got %d)", c->head_dim);
   if (c->page_tokens != kvq::kPageTokens)
     return fail(KVQ_ERR_UNSUPPORTED, "page_tokens must be 16 (got %d)", c->page_tokens);
   if (c->tile_tokens != 32 && c->tile_tokens != 64 && c->tile_tokens != 128)
@@ -113,7 +114,7 @@ kvq_status kvq_get_layout(const kvq_config* cfg, kvq_layout* out) {
   out->cslice_off_v = gv.cslice_off;
   out->block_stride_k = static_cast<size_t>(cfg->num_kv_heads) * gk.page_bytes;
   out->block_stride_v = static_cast<size_t>(cfg->num_kv_heads) * gv.page_bytes;
-  out->tail_bytes = static_cast<size_t>(cfg->num_kv_heads) * cfg->tile_tokens * kvq::kHeadDim * 2;
+  out->tail_bytes = static_cast<size_t>(cfg->num_kv_heads) * cfg->tile_tokens * cfg->head_dim * 2;
   out->cslice_channels = gk.cs_channels;
   out->pages_per_tile = gk.pages_per_tile;
   return ok();
@@ -270,6 +271,8 @@ kvq_status kvq_append_decode_step(const kvq_config* cfg, const void* new_k, cons
                                   void* k_tail, void* v_tail, float softmax_scale, void* workspace,
                                   size_t workspace_bytes, int num_splits, int32_t* dev_status, void* stream) {
   KVQ_TRY(check_config(cfg));
+  if (cfg->head_dim != kvq::kHeadDim)
+    return fail(KVQ_ERR_UNSUPPORTED, "the one-launch serving step is built for head_dim 128 (got %d)", cfg->head_dim);
   if (num_seqs < 0) return fail(KVQ_ERR_INVALID_ARG, "negative num_seqs");
   if (num_seqs == 0) return ok();
   if (num_seqs > 65535) return fail(KVQ_ERR_INVALID_ARG, "num_seqs > 65535");
@@ -324,6 +327,8 @@ kvq_status kvq_append_decode_step(const kvq_config* cfg, const void* new_k, cons
 kvq_status kvq_prefill_workspace_bytes(const kvq_config* cfg, int num_seqs, int max_chunk_tokens, int num_splits,
                                        size_t* bytes) {
   KVQ_TRY(check_config(cfg));
+  if (cfg->head_dim != kvq::kHeadDim)
+    return fail(KVQ_ERR_UNSUPPORTED, "chunked prefill is built for head_dim 128 (got %d)", cfg->head_dim);
   if (bytes == nullptr) return fail(KVQ_ERR_INVALID_ARG, "bytes is NULL");
   if (num_seqs < 0 || max_chunk_tokens < 0) return fail(KVQ_ERR_INVALID_ARG, "negative num_seqs or max_chunk_tokens");
   if (num_splits < 1 || num_splits > 64) return fail(KVQ_ERR_INVALID_ARG, "num_splits must be 1..64");
@@ -339,6 +344,8 @@ kvq_status kvq_paged_prefill_attention(const kvq_config* cfg, const void* q, voi
                                        float softmax_scale, int num_splits, void* workspace,
                                        size_t workspace_bytes, int32_t* dev_status, void* stream) {
   KVQ_TRY(check_config(cfg));
+  if (cfg->head_dim != kvq::kHeadDim)
+    return fail(KVQ_ERR_UNSUPPORTED, "chunked prefill is built for head_dim 128 (got %d)", cfg->head_dim);
   if (num_splits < 1 || num_splits > 64) return fail(KVQ_ERR_INVALID_ARG, "num_splits must be 1..64");
   if (num_seqs < 0 || max_chunk_tokens < 0) return fail(KVQ_ERR_INVALID_ARG, "negative num_seqs or max_chunk_tokens");
   if (num_seqs == 0 || max_chunk_tokens == 0) return ok();

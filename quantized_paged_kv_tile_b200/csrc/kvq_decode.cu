@@ -1136,6 +1136,7 @@ cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t s) {
 }  // namespace
 
 size_t decode_workspace_bytes(const kvq_config& cfg, int num_seqs, int num_splits, int num_sms) {
+  if (cfg.head_dim != kHeadDim) return generic_decode_workspace_bytes(cfg, num_seqs, num_splits, num_sms);
   const WsLayout wl = ws_layout(num_seqs, cfg.num_kv_heads, cfg.group_size);
   const size_t units = num_splits > 0
                            ? static_cast<size_t>(num_seqs) * cfg.num_kv_heads * num_splits
@@ -1151,6 +1152,7 @@ cudaError_t launch_selftest_wait_decode(int32_t* dev_status, cudaStream_t s) {
 cudaError_t launch_append_decode_step(const DecodeArgs& a, cudaStream_t s) { return launch_paged_decode(a, s); }
 
 cudaError_t launch_paged_decode(const DecodeArgs& a, cudaStream_t s) {
+  if (a.cfg.head_dim != kHeadDim) return launch_generic_decode(a, s);
   if (a.num_seqs == 0) return cudaSuccess;
   switch (a.cfg.tile_tokens) {
     case 32: return launch_decode_t<32>(a, s);

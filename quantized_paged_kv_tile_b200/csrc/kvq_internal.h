@@ -11,14 +11,14 @@
 
 namespace kvq {
 
-constexpr int kHeadDim = 128;
+constexpr int kHeadDim = 128;  // the head size of the tensor-core path
 constexpr int kPageTokens = 16;
 constexpr int kMaxGroup = 8;
 
 // Layout numbers of one pool (K or V), derived from the config.
 struct PoolGeom {
   int bits;            // code width
-  int codes_bytes;     // P*d*b/8
+  int codes_bytes;     // P*d*b/8 (d = cfg.head_dim)
   int meta_off;        // == codes_bytes
   int cslice_off;      // codes_bytes + 64
   int page_bytes;      // one (block, head) region
@@ -148,6 +148,14 @@ struct PrefillArgs {
 int prefill_row_tiles(const kvq_config& cfg, int max_chunk);
 size_t prefill_workspace_bytes(const kvq_config& cfg, int num_seqs, int max_chunk, int num_splits);
 cudaError_t launch_paged_prefill(const PrefillArgs& a, cudaStream_t s);
+
+// Head sizes 64 and 256 (kvq_generic.cu): the same calls on the CUDA cores;
+// the launchers above hand configurations with head_dim != 128 to these.
+cudaError_t launch_generic_quantize(const QuantizeArgs& a, cudaStream_t s);
+cudaError_t launch_generic_append(const AppendArgs& a, cudaStream_t s);
+cudaError_t launch_generic_decode(const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_generic_unpack(const UnpackArgs& a, cudaStream_t s);
+size_t generic_decode_workspace_bytes(const kvq_config& cfg, int num_seqs, int num_splits, int num_sms);
 
 // Self-tests of the bounded mbarrier waits (one per kernel file): a wait on
 // a barrier nothing arrives at gives up after its limit and records

@@ -1039,11 +1039,13 @@ cudaError_t launch_selftest_wait_quantize(int32_t* dev_status, cudaStream_t s) {
 }
 
 cudaError_t launch_quantize_tiles(const QuantizeArgs& a, cudaStream_t s) {
+  if (a.cfg.head_dim != kHeadDim) return launch_generic_quantize(a, s);
   if (a.num_tiles == 0) return cudaSuccess;
   return dispatch_bits<QuantizeLauncher>(a, s);
 }
 
 cudaError_t launch_append_tokens(const AppendArgs& a, cudaStream_t s) {
+  if (a.cfg.head_dim != kHeadDim) return launch_generic_append(a, s);
   if (a.num_seqs == 0) return cudaSuccess;
   return dispatch_bits<AppendLauncher>(a, s);
 }

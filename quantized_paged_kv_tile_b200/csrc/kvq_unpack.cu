@@ -80,9 +80,9 @@ __global__ void __launch_bounds__(kThreads) unpack_tiles_kernel(UnpackArgs a) {
 PoolGeom pool_geom(const kvq_config& cfg, bool is_v) {
   PoolGeom g;
   g.bits = is_v ? cfg.bits_v : cfg.bits_k;
-  g.codes_bytes = kPageTokens * kHeadDim * g.bits / 8;
+  g.codes_bytes = kPageTokens * cfg.head_dim * g.bits / 8;
   g.meta_off = g.codes_bytes;
-  g.cs_channels = kHeadDim * kPageTokens / cfg.tile_tokens;
+  g.cs_channels = cfg.head_dim * kPageTokens / cfg.tile_tokens;
   g.cslice_off = g.codes_bytes + 4 * kPageTokens;
   g.page_bytes = g.cslice_off + ((2 * g.cs_channels + 15) / 16) * 16;
   g.pages_per_tile = cfg.tile_tokens / kPageTokens;
@@ -90,6 +90,7 @@ PoolGeom pool_geom(const kvq_config& cfg, bool is_v) {
 }
 
 cudaError_t launch_unpack_tiles(const UnpackArgs& a, cudaStream_t s) {
+  if (a.cfg.head_dim != kHeadDim) return launch_generic_unpack(a, s);
   if (a.num_tiles == 0) return cudaSuccess;
   dim3 grid(a.num_tiles, a.cfg.num_kv_heads);
   switch (a.cfg.tile_tokens) {

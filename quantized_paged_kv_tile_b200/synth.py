@@ -56,6 +56,7 @@ class Workload:
     append_tokens: int = 0     # tokens appended per sequence by the step
     decode_steps: int = 1
     replica: int = 0           # independent replica batch (multi-GPU weak scaling)
+    head_dim: int = HEAD_DIM   # d: 128 in every named workload; 64 and 256 for the variant tests
 
     @property
     def seed(self) -> int:
@@ -104,7 +105,7 @@ def channel_scales(w: Workload, which: str) -> np.ndarray:
     """Per (KV head, channel) multipliers of the N(0,1) draws, float32 [H_kv][d]."""
     salt = {"k": 11, "v": 23}[which]
     rng = np.random.Generator(np.random.PCG64([w.seed, salt]))
-    h, d = w.num_kv_heads, HEAD_DIM
+    h, d = w.num_kv_heads, w.head_dim
     if w.kv_dist == "tiny":
         # the same 4 channels for K and V: draw them from a stream shared by both
         shared = np.random.Generator(np.random.PCG64([w.seed, 5]))
@@ -144,7 +145,7 @@ def kv_rows(w: Workload, which: str, num_rows: int, device="cpu", stream_id: int
     1.. = appended tokens of later steps)."""
     salt = {"k": 1, "v": 2}[which]
     g = _generator(device, (w.seed * 1000 + salt) * 4099 + stream_id)
-    x = torch.randn((num_rows, w.num_kv_heads, HEAD_DIM), generator=g, device=device, dtype=torch.float32)
+    x = torch.randn((num_rows, w.num_kv_heads, w.head_dim), generator=g, device=device, dtype=torch.float32)
     x *= torch.from_numpy(channel_scales(w, which)).to(device)[None]
     return x.to(torch.float16)
 
@@ -155,7 +156,7 @@ def kv_rows_one_head(w: Workload, which: str, num_rows: int, head: int, stream_i
     need one head of a long sequence without drawing all heads)."""
     salt = {"k": 1, "v": 2}[which]
     rng = np.random.Generator(np.random.PCG64([w.seed, salt, head, stream_id]))
-    x = rng.standard_normal((num_rows, HEAD_DIM), dtype=np.float32)
+    x = rng.standard_normal((num_rows, w.head_dim), dtype=np.float32)
     x *= channel_scales(w, which)[head][None, :]
     return x.astype(np.float16)
 
@@ -163,7 +164,7 @@ def kv_rows_one_head(w: Workload, which: str, num_rows: int, head: int, stream_i
 def queries(w: Workload, device="cpu", step: int = 0) -> torch.Tensor:
     """fp16 [B][H_q][d] ~ N(0,1)."""
     g = _generator(device, (w.seed * 1000 + 3) * 4099 + step)
-    return torch.randn((w.num_seqs, w.num_q_heads, HEAD_DIM), generator=g, device=device,
+    return torch.randn((w.num_seqs, w.num_q_heads, w.head_dim), generator=g, device=device,
                        dtype=torch.float32).to(torch.float16)
 
 

@@ -56,7 +56,7 @@ def rel_l2(a, b) -> float:
 def make_cache(w: synth.Workload, extra_tokens: int = 0, device="cuda", num_splits: int = 0):
     from quantized_paged_kv_tile_b200.paged import PagedKVCache
     cfg = kvq.Config(num_kv_heads=w.num_kv_heads, group_size=w.group_size, tile_tokens=w.tile_tokens,
-                     bits_k=w.bits_k, bits_v=w.bits_v, iters=w.iters)
+                     bits_k=w.bits_k, bits_v=w.bits_v, iters=w.iters, head_dim=w.head_dim)
     max_tokens = max(w.lens) + max(extra_tokens, w.append_tokens)
     bps = -(-max(max_tokens, 1) // 16)
     cache = PagedKVCache(cfg, w.num_seqs, bps * 16, device=device, block_table=synth.block_table(w, bps),
@@ -217,7 +217,8 @@ def gpu_pages_kv_hat(cfg: kvq.Config, cache, seq: int, head: int, length: int, i
     pool = cache.v_pool if is_v else cache.k_pool
     ids = cache.block_tables[seq, :n_full * (t // p)].long()
     host = pool.index_select(0, ids)[:, head:head + 1].cpu().numpy()
-    tiles = [o.read_tile_pages(host, range(i * (t // p), (i + 1) * (t // p)), 0, bits, t, is_v) for i in range(n_full)]
+    tiles = [o.read_tile_pages(host, range(i * (t // p), (i + 1) * (t // p)), 0, bits, t, is_v, d=cfg.head_dim)
+             for i in range(n_full)]
     tail = (cache.v_tail if is_v else cache.k_tail)[seq, head, :tau].cpu().numpy()
     return o.sequence_kv_hat(tiles, tail, cfg.rotation_seed)
 

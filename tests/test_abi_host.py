@@ -63,8 +63,20 @@ def test_layout_matches_oracle(lib, t, bk, bv):
     assert lay["block_stride_v"] == 8 * ov["page_bytes"]
 
 
+@pytest.mark.parametrize("d", [64, 256])
+@pytest.mark.parametrize("t", [32, 64, 128])
+@pytest.mark.parametrize("bk,bv", [(4, 4), (2, 3), (8, 8)])
+def test_layout_matches_oracle_other_head_sizes(lib, d, t, bk, bv):
+    cfg = kvq.Config(num_kv_heads=3, group_size=4, tile_tokens=t, bits_k=bk, bits_v=bv, iters=4, head_dim=d)
+    lay = kvq.get_layout(cfg)
+    ok_, ov = o.page_layout(bk, t, d), o.page_layout(bv, t, d)
+    assert lay["page_bytes_k"] == ok_["page_bytes"] and lay["page_bytes_v"] == ov["page_bytes"]
+    assert lay["codes_bytes_v"] == ov["codes"] and lay["cslice_off_v"] == ov["cslice_off"]
+    assert lay["cslice_channels"] == ok_["cslice_channels"] and lay["tail_bytes"] == 3 * t * d * 2
+
+
 @pytest.mark.parametrize("field,value,status", [
-    ("head_dim", 64, kvq.KVQ_ERR_UNSUPPORTED), ("tile_tokens", 48, kvq.KVQ_ERR_UNSUPPORTED),
+    ("head_dim", 96, kvq.KVQ_ERR_UNSUPPORTED), ("tile_tokens", 48, kvq.KVQ_ERR_UNSUPPORTED),
     ("bits_k", 5, kvq.KVQ_ERR_UNSUPPORTED), ("bits_k", 8, kvq.KVQ_ERR_UNSUPPORTED),  # 8 only with bits_v = 8
     ("group_size", 9, kvq.KVQ_ERR_UNSUPPORTED),
     ("iters", -1, kvq.KVQ_ERR_INVALID_ARG), ("std_eps", 0.0, kvq.KVQ_ERR_INVALID_ARG),
@@ -88,11 +100,18 @@ def test_argument_errors_launch_nothing(lib):
     # misaligned pointer
     st = lib.kvq_quantize_tiles(ctypes.byref(c), 17, None, 10, 16, 1, 16, 1, 4, 8, 16, 16, None, None)
     assert st == kvq.KVQ_ERR_INVALID_ARG and "aligned" in kvq.load_library().kvq_last_error().decode()
-    # a head size without kernels is refused before any launch
-    c64 = kvq.Config(num_kv_heads=2, group_size=4, tile_tokens=64, bits_k=4, bits_v=4, iters=4, head_dim=64).c()
-    st = lib.kvq_paged_decode_attention(ctypes.byref(c64), 16, 16, 16, 1, 16, 4, 8, 16, 16, 16, 16, 0.1, 16,
-                                        1 << 20, 1, None, None)
-    assert st == kvq.KVQ_ERR_UNSUPPORTED
+    # head sizes 64 and 256 decode (to the workspace check here: one split of
+    # 2 sequences x 2 KV heads x 4 query heads x (4 + d) floats); the one-launch
+    # serving step is built for d = 128 only and refuses them before any launch
+    for d in (64, 256):
+        cd = kvq.Config(num_kv_heads=2, group_size=4, tile_tokens=64, bits_k=4, bits_v=4, iters=4, head_dim=d)
+        assert kvq.decode_workspace_bytes(cd, 2, 1) == 2 * 2 * 1 * 4 * (4 + d) * 4
+        st = lib.kvq_paged_decode_attention(ctypes.byref(cd.c()), 16, 16, 16, 2, 16, 4, 8, 16, 16, 16, 16, 0.1, 16,
+                                            16, 1, None, None)
+        assert st == kvq.KVQ_ERR_WORKSPACE
+        st = lib.kvq_append_decode_step(ctypes.byref(cd.c()), 16, 16, 16, 16, 16, 1, 16, 4, 8, 16, 16, 16, 16, 0.1,
+                                        16, 1 << 20, 1, None, None)
+        assert st == kvq.KVQ_ERR_UNSUPPORTED
     # 3-bit pages are read: the call gets past the configuration checks (here
     # to the workspace check, with no device query for an explicit split count)
     c3 = kvq.Config(num_kv_heads=2, group_size=4, tile_tokens=64, bits_k=3, bits_v=4, iters=4).c()

@@ -1,0 +1,159 @@
+"""Head sizes d = 64 and 256 (the method's rotation along the head-dim
+channels of any head size: axbrief.com KVarN article, "What differs from
+existing methods"): quantize, append and decode through the C ABI against the
+oracle, with the same bars as the d = 128 tests."""
+
+import numpy as np
+import pytest
+import torch
+
+from quantized_paged_kv_tile_b200 import kvq, synth
+from quantized_paged_kv_tile_b200.paged import PagedKVCache
+
+from parity_helpers import (ATTN_REL_L2_MAX, TileStats, compare_sequence_tiles, decode_over_gpu_pages, make_cache,
+                            rel_l2)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    kvq.load_library()
+
+
+def _starts(lens):
+    return np.concatenate([[0], np.cumsum(lens)[:-1]]).astype(np.int64)
+
+
+def _prefilled(w, num_splits=0, extra_tokens=0, rotation_seed=0):
+    if rotation_seed:
+        cfg = kvq.Config(num_kv_heads=w.num_kv_heads, group_size=w.group_size, tile_tokens=w.tile_tokens,
+                         bits_k=w.bits_k, bits_v=w.bits_v, iters=w.iters, head_dim=w.head_dim,
+                         rotation_seed=rotation_seed)
+        bps = -(-(max(w.lens) + extra_tokens) // 16)
+        cache = PagedKVCache(cfg, w.num_seqs, bps * 16, block_table=synth.block_table(w, bps), num_splits=num_splits)
+    else:
+        cfg, cache = make_cache(w, extra_tokens=extra_tokens, num_splits=num_splits)
+    total = int(sum(w.lens))
+    rk = synth.kv_rows(w, "k", total, device="cuda")
+    rv = synth.kv_rows(w, "v", total, device="cuda")
+    cache.prefill(rk, rv, w.lens)
+    torch.cuda.synchronize()
+    assert cache.status() == 0
+    return cfg, cache, rk, rv
+
+
+QUANT_CASES = [
+    # (d, T, bits_k, bits_v, iters, heads, lens, rotation seed)
+    (64, 64, 4, 4, 4, 2, (300, 129), 0),
+    (64, 32, 2, 3, 1, 1, (200, 96), 0),
+    (64, 128, 8, 8, 2, 1, (260,), 0),
+    (64, 64, 4, 2, 8, 1, (192,), 0x9E37),   # randomized rotation
+    (256, 64, 4, 4, 4, 2, (200, 70), 0),
+    (256, 128, 3, 4, 2, 1, (300,), 0),
+    (256, 32, 2, 2, 0, 1, (100,), 0),       # n = 0
+    (256, 64, 8, 8, 1, 1, (130,), 0x51),    # 8-bit codes, randomized rotation
+]
+
+
+@pytest.mark.parametrize("d,t,bk,bv,n,h,lens,seed", QUANT_CASES)
+def test_quantize_matches_oracle(d, t, bk, bv, n, h, lens, seed):
+    w = synth.workload("prefill_sweep", num_seqs=len(lens), lens=lens, num_kv_heads=h, tile_tokens=t,
+                       bits_k=bk, bits_v=bv, iters=n, head_dim=d)
+    cfg, cache, rk, rv = _prefilled(w, rotation_seed=seed)
+    rk_h, rv_h = rk.cpu().numpy(), rv.cpu().numpy()
+    tiles = [(s, i) for s in range(len(lens)) for i in range(lens[s] // t)]
+    sk, sv = TileStats(), TileStats()
+    compare_sequence_tiles(cfg, cache, rk_h, rv_h, _starts(lens), tiles, sk, sv)
+    sk.check()
+    sv.check()
+    kt, vt = cache.k_tail.cpu().numpy(), cache.v_tail.cpu().numpy()
+    for s, L in enumerate(lens):
+        tau = L % t
+        r0 = _starts(lens)[s] + L - tau
+        for hh in range(h):
+            np.testing.assert_array_equal(kt[s, hh, :tau], rk_h[r0:r0 + tau, hh])
+            np.testing.assert_array_equal(vt[s, hh, :tau], rv_h[r0:r0 + tau, hh])
+
+
+@pytest.mark.parametrize("d,t,chunks", [(64, 32, [1] * 40), (256, 64, [3, 100, 1, 70]), (64, 128, [130, 7, 1])])
+def test_append_equals_prefill(d, t, chunks):
+    # tokens appended in chunks (tiles completing inside appends, several per
+    # call) give pages bit-identical to quantizing the same tokens directly
+    l0 = 2 * t + 5
+    total = l0 + sum(chunks)
+    w = synth.workload("qwen3_32b_burst", num_seqs=2, lens=(l0, l0), num_kv_heads=2, group_size=4,
+                       tile_tokens=t, head_dim=d)
+    cfg, a = make_cache(w, extra_tokens=total)
+    _, b = make_cache(w, extra_tokens=total)
+    rk = synth.kv_rows(w, "k", 2 * total, device="cuda")
+    rv = synth.kv_rows(w, "v", 2 * total, device="cuda")
+    seq_rows = lambda r, s, lo, hi: r[s * total + lo:s * total + hi]  # noqa: E731
+    a.prefill(torch.cat([seq_rows(rk, s, 0, l0) for s in range(2)]),
+              torch.cat([seq_rows(rv, s, 0, l0) for s in range(2)]), [l0, l0])
+    pos = l0
+    for c in chunks:
+        a.append(torch.cat([seq_rows(rk, s, pos, pos + c) for s in range(2)]),
+                 torch.cat([seq_rows(rv, s, pos, pos + c) for s in range(2)]), [c, c])
+        pos += c
+    b.prefill(rk, rv, [total, total])
+    torch.cuda.synchronize()
+    assert a.status() == 0 and b.status() == 0
+    bt = a.block_tables.cpu().numpy()
+    used = bt[:, :(total // t) * (t // 16)].ravel()
+    assert torch.equal(a.k_pool[used], b.k_pool[used])
+    assert torch.equal(a.v_pool[used], b.v_pool[used])
+    tau = total % t
+    assert torch.equal(a.k_tail[:, :, :tau], b.k_tail[:, :, :tau])
+    assert torch.equal(a.v_tail[:, :, :tau], b.v_tail[:, :, :tau])
+    q = synth.queries(w, device="cuda")
+    assert torch.equal(a.decode(q), b.decode(q))
+
+
+DECODE_CASES = [
+    # (d, T, bits_k, bits_v, g, lens, splits)
+    (64, 64, 4, 4, 4, (3 * 64 + 9, 64 * 5), 0),
+    (64, 32, 2, 3, 8, (7 * 32 + 31,), 3),
+    (64, 128, 8, 8, 2, (2 * 128 + 1, 50), 1),
+    (256, 64, 4, 2, 8, (4 * 64 + 17, 3 * 64), 0),
+    (256, 128, 3, 3, 4, (3 * 128 + 127,), 2),
+    (256, 32, 4, 4, 1, (9 * 32 + 5, 31, 0), 4),
+]
+
+
+@pytest.mark.parametrize("d,t,bk,bv,g,lens,splits", DECODE_CASES)
+def test_decode_matches_oracle(d, t, bk, bv, g, lens, splits):
+    # decode over the cache is held to 1e-3 against fp64 attention over the
+    # GPU's own pages (read by the oracle) and raw tail; the pages themselves
+    # are held to the quantize bars above (every differing code a rounding tie)
+    w = synth.workload("tiny", num_seqs=len(lens), lens=lens, num_kv_heads=2, group_size=g, tile_tokens=t,
+                       bits_k=bk, bits_v=bv, iters=2, head_dim=d)
+    cfg, cache, rk, rv = _prefilled(w, num_splits=splits)
+    q = synth.queries(w, device="cuda")
+    out = cache.decode(q)
+    torch.cuda.synchronize()
+    assert cache.status() == 0
+    out_h, q_h = out.float().cpu().numpy(), q.cpu().numpy()
+    for s, L in enumerate(lens):
+        if L == 0:
+            assert not out_h[s].any()
+            continue
+        ref = decode_over_gpu_pages(cfg, cache, s, L, q_h[s])
+        for hq in range(w.num_q_heads):
+            assert rel_l2(out_h[s, hq], ref[hq]) <= ATTN_REL_L2_MAX, (s, hq)
+    tiles = [(s, i) for s in range(len(lens)) for i in range(lens[s] // t)]
+    sk, sv = TileStats(), TileStats()
+    compare_sequence_tiles(cfg, cache, rk.cpu().numpy(), rv.cpu().numpy(), _starts(lens), tiles, sk, sv)
+    sk.check()
+    sv.check()
+
+
+@pytest.mark.parametrize("d", [64, 256])
+def test_decode_independent_of_split_count(d):
+    w = synth.workload("tiny", num_seqs=2, lens=(64 * 20 + 7, 300), num_kv_heads=2, group_size=4, head_dim=d)
+    cfg, cache, rk, rv = _prefilled(w)
+    q = synth.queries(w, device="cuda")
+    outs = [cache.decode(q, num_splits=s).float().cpu().numpy() for s in (1, 2, 7, 20, 0)]
+    for other in outs[1:]:
+        assert rel_l2(other, outs[0]) <= 1e-4
