@@ -589,6 +589,20 @@ __device__ __forceinline__ UnitLoc locate_unit(const DecodeArgs& a, int u, const
   }
   return l;
 }
+// The first unit (chunk 0) of (sequence b, KV head h).
+template <int T>
+__device__ __forceinline__ UnitLoc locate_pair(const DecodeArgs& a, int b, int h, const int32_t* prefix,
+                                               const int32_t* chunk) {
+  const int nh = a.cfg.num_kv_heads;
+  const int u = a.step ? (b * nh + h) * a.num_splits_fixed : nh * prefix[b] + h * (prefix[b + 1] - prefix[b]);
+  return locate_unit<T>(a, u, prefix, chunk);
+}
+// Arrivals that complete (sequence, KV head) at its counter: its raw-tail unit
+// plus its chunk units (one merge group) or its merge groups.
+__device__ __forceinline__ int pair_arrivals(int S) {
+  const int n_groups = (S + kMergeGroup - 1) / kMergeGroup;
+  return 1 + (n_groups == 1 ? S : n_groups);
+}
 
 // ------------------------------------------------------------------ main decode
 template <int T, int BK, int BV>
@@ -636,8 +650,12 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
   int32_t* arrivals = reinterpret_cast<int32_t*>(ws + wl.arrive_off);
   float* tails = reinterpret_cast<float*>(ws + wl.tail_off);
   float* parts = reinterpret_cast<float*>(ws + wl.part_off);
-  const int U = a.step ? a.num_seqs * nh * a.num_splits_fixed : ws_i[0];
-  int32_t* gcount = group_counters(parts, U, G);
+  // work items: one raw-tail unit per (sequence, KV head) first, then the
+  // chunk units; the tails run as one burst ahead of the tile loop (their code
+  // would otherwise interleave with it in the instruction cache)
+  const int P = a.num_seqs * nh;
+  const int U = P + (a.step ? a.num_seqs * nh * a.num_splits_fixed : ws_i[0]);
+  int32_t* gcount = group_counters(parts, U - P, G);
   const uint8_t* kpool = static_cast<const uint8_t*>(a.k_pool);
   const uint8_t* vpool = static_cast<const uint8_t*>(a.v_pool);
   const float qscale = a.softmax_scale * kLog2e / kSqrtHeadDim;
@@ -654,6 +672,28 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
     if (lane == 0) u = atomicAdd(&ws_i[1], 1);
     u = __shfl_sync(kFull, u, 0);
     if (u >= U) break;
+    if (u < P) {
+      // ---- raw tail of (sequence u / nh, KV head u % nh): in a serving step,
+      // first the step's token into tail row (L - 1) mod T
+      const int b = u / nh, h = u % nh;
+      const UnitLoc loc = locate_pair<T>(a, b, h, prefix, chunk);
+      if (a.step) step_append_warp<T>(a, b, h, loc.L, lane);
+      decode_tail_warp<T>(a, b, h, loc.L % T, tails, reinterpret_cast<float*>(stage_base), lane);
+      __threadfence();
+      __syncwarp();
+      int last = 0;
+      if (lane == 0) last = atomicAdd(&arrivals[u], 1) == pair_arrivals(loc.S) - 1;
+      last = __shfl_sync(kFull, last, 0);
+      if (last) {
+        __threadfence();
+        const int n_groups = (loc.S + kMergeGroup - 1) / kMergeGroup;
+        decode_merge_warp(a, b, h, n_groups == 1 ? loc.S : n_groups, loc.ubase, n_groups == 1 ? 1 : kMergeGroup,
+                          true, parts, tails, reinterpret_cast<float*>(stage_base), lane);
+        if (a.step && lane == 0) arrivals[u] = 0;  // the step leaves its counters at zero
+      }
+      continue;
+    }
+    u -= P;
     // ---- locate the unit: sequence b, head h, chunk c of the S chunks of
     // (b, h) over L tokens (the coordinates are located again after the
     // tile loop, so that only what the loop needs stays live through it)
@@ -983,14 +1023,7 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
         *reinterpret_cast<float2*>(part + kPartAcc + c0) = make_float2(acc[2 * nv], acc[2 * nv + 1]);
       }
     }
-    // the raw tail goes with chunk 0 (the warp's stages are idle now: every
-    // copy it issued has landed); in a serving step its warp first writes the
-    // step's token into the tail row (L - 1) mod T
     loc = locate_unit<T>(a, u, prefix, chunk);
-    if (loc.c == 0) {
-      if (a.step) step_append_warp<T>(a, loc.b, loc.h, loc.L, lane);
-      decode_tail_warp<T>(a, loc.b, loc.h, loc.L % T, tails, reinterpret_cast<float*>(stage_base), lane);
-    }
     // publish this unit's records; the last chunk of its group to finish
     // merges the group, the last group of (b, h) merges the groups
     __threadfence();
@@ -1016,8 +1049,8 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
     }
     if (to_final) {
       int last = 0;
-      // the counter counts units when there is one group, else groups
-      if (lane == 0) last = atomicAdd(&arrivals[bh], 1) == (n_groups == 1 ? loc.S : n_groups) - 1;
+      // the counter counts the tail unit and the chunk units (one group) or the groups
+      if (lane == 0) last = atomicAdd(&arrivals[bh], 1) == pair_arrivals(loc.S) - 1;
       last = __shfl_sync(kFull, last, 0);
       if (last) {
         __threadfence();

@@ -514,7 +514,7 @@ __global__ void __launch_bounds__(kGThreads) gen_decode_merge_kernel(DecodeArgs 
   float* ts = qs + kMaxGroup * D;
   float* hs = ts + kMaxGroup * T;  // [G][8]: tail m, tail l, merged m, total l, tail weight
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int pair = blockIdx.x, b = pair / nh, h = pair % nh;
+  const int pair = blockIdx.x, b = pair / nh;
   const int L = max(a.seq_lens[b], 0), tau = L % T;
   const float qscale = a.softmax_scale * kLog2e;
   const __half* kt = static_cast<const __half*>(a.k_tail) + static_cast<size_t>(pair) * T * D;
