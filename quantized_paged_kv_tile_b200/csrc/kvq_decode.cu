@@ -597,11 +597,12 @@ __device__ __forceinline__ UnitLoc locate_pair(const DecodeArgs& a, int b, int h
   const int u = a.step ? (b * nh + h) * a.num_splits_fixed : nh * prefix[b] + h * (prefix[b + 1] - prefix[b]);
   return locate_unit<T>(a, u, prefix, chunk);
 }
-// Arrivals that complete (sequence, KV head) at its counter: its raw-tail unit
-// plus its chunk units (one merge group) or its merge groups.
+// Arrivals that complete (sequence, KV head) at its counter: its raw-tail
+// unit, its final-merge unit, and its chunk units (one merge group) or its
+// merge groups.
 __device__ __forceinline__ int pair_arrivals(int S) {
   const int n_groups = (S + kMergeGroup - 1) / kMergeGroup;
-  return 1 + (n_groups == 1 ? S : n_groups);
+  return 2 + (n_groups == 1 ? S : n_groups);
 }
 
 // ------------------------------------------------------------------ main decode
@@ -651,11 +652,15 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
   float* tails = reinterpret_cast<float*>(ws + wl.tail_off);
   float* parts = reinterpret_cast<float*>(ws + wl.part_off);
   // work items: one raw-tail unit per (sequence, KV head) first, then the
-  // chunk units; the tails run as one burst ahead of the tile loop (their code
-  // would otherwise interleave with it in the instruction cache)
+  // chunk units, then one final-merge unit per (sequence, KV head).  The tails
+  // and most final merges run as bursts before and after the tile loop (their
+  // code would otherwise interleave with it in the instruction cache).  Nothing
+  // waits: every unit arrives at its pair's counter and whichever arrives
+  // last merges (usually the final-merge unit, else a chunk still running).
   const int P = a.num_seqs * nh;
-  const int U = P + (a.step ? a.num_seqs * nh * a.num_splits_fixed : ws_i[0]);
-  int32_t* gcount = group_counters(parts, U - P, G);
+  const int UC = a.step ? a.num_seqs * nh * a.num_splits_fixed : ws_i[0];
+  const int U = P + UC + P;
+  int32_t* gcount = group_counters(parts, UC, G);
   const uint8_t* kpool = static_cast<const uint8_t*>(a.k_pool);
   const uint8_t* vpool = static_cast<const uint8_t*>(a.v_pool);
   const float qscale = a.softmax_scale * kLog2e / kSqrtHeadDim;
@@ -672,14 +677,19 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
     if (lane == 0) u = atomicAdd(&ws_i[1], 1);
     u = __shfl_sync(kFull, u, 0);
     if (u >= U) break;
-    if (u < P) {
-      // ---- raw tail of (sequence u / nh, KV head u % nh): in a serving step,
-      // first the step's token into tail row (L - 1) mod T
+    if (u < P || u >= P + UC) {
+      // ---- raw tail of (sequence, KV head) p = (b, h): in a serving step,
+      // first the step's token into tail row (L - 1) mod T; or its final-merge
+      // unit, which only arrives
+      const bool tail_unit = u < P;
+      if (!tail_unit) u -= P + UC;
       const int b = u / nh, h = u % nh;
       const UnitLoc loc = locate_pair<T>(a, b, h, prefix, chunk);
-      if (a.step) step_append_warp<T>(a, b, h, loc.L, lane);
-      decode_tail_warp<T>(a, b, h, loc.L % T, tails, reinterpret_cast<float*>(stage_base), lane);
-      __threadfence();
+      if (tail_unit) {
+        if (a.step) step_append_warp<T>(a, b, h, loc.L, lane);
+        decode_tail_warp<T>(a, b, h, loc.L % T, tails, reinterpret_cast<float*>(stage_base), lane);
+        __threadfence();
+      }
       __syncwarp();
       int last = 0;
       if (lane == 0) last = atomicAdd(&arrivals[u], 1) == pair_arrivals(loc.S) - 1;
