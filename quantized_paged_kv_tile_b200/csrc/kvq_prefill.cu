@@ -361,6 +361,15 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(PrefillArgs
   // chunk token of this thread's row (rows past the chunk take the last one)
   const int i_row = (rt * kRows + min(row, rows_valid - 1)) / G;
   const int i_max = (rt * kRows + rows_valid - 1) / G;
+  if (a.mode == 1 && Fr == 0) {  // no context tile in this split: an empty partial, and no set-up at all
+    if (row < rows_valid) {
+      float* part = a.partials + (static_cast<size_t>(blockIdx.x) * kRows + row) * (4 + kHeadDim);
+      if (eta == 0) *reinterpret_cast<float2*>(part) = make_float2(-INFINITY, 0.f);
+#pragma unroll
+      for (int i = 0; i < 64; i += 4) *reinterpret_cast<float4*>(part + 4 + 64 * eta + i) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    return;
+  }
 
   const uint32_t s_base = smem_u32(smem);
   const uint32_t bar_stage0 = s_base + kOffBar, bar_mma = s_base + kOffBar + 16;
