@@ -237,6 +237,10 @@ kvq_status kvq_paged_decode_attention(const kvq_config* cfg, const void* q, void
   KVQ_TRY(check_ptr(workspace, "workspace"));
   KVQ_TRY(check_ptr(dev_status, "dev_status", true));
   if (num_splits > 65535) return fail(KVQ_ERR_INVALID_ARG, "num_splits > 65535");
+  // the device counts work units in 32-bit ints: (num_seqs x num_kv_heads) x (splits + 2) stays below 2^30
+  if (static_cast<long long>(num_seqs) * cfg->num_kv_heads * (num_splits + 2) >= (1LL << 30))
+    return fail(KVQ_ERR_INVALID_ARG, "num_seqs x num_kv_heads x num_splits too large (%d x %d x %d)", num_seqs,
+                cfg->num_kv_heads, num_splits);
   int sms = 0;
   if (num_splits == 0) KVQ_TRY(device_sm_count(&sms));
   const size_t need = kvq::decode_workspace_bytes(*cfg, num_seqs, num_splits, sms);
@@ -278,6 +282,9 @@ kvq_status kvq_append_decode_step(const kvq_config* cfg, const void* new_k, cons
   if (num_seqs > 65535) return fail(KVQ_ERR_INVALID_ARG, "num_seqs > 65535");
   if (num_splits < 1 || num_splits > 65535)
     return fail(KVQ_ERR_INVALID_ARG, "num_splits must be 1..65535 for the serving step (got %d)", num_splits);
+  if (static_cast<long long>(num_seqs) * cfg->num_kv_heads * (num_splits + 2) >= (1LL << 30))
+    return fail(KVQ_ERR_INVALID_ARG, "num_seqs x num_kv_heads x num_splits too large (%d x %d x %d)", num_seqs,
+                cfg->num_kv_heads, num_splits);
   if (static_cast<long long>(num_seqs) * cfg->num_kv_heads * num_splits > 0x7fffffffLL)
     return fail(KVQ_ERR_INVALID_ARG, "num_seqs x num_kv_heads x num_splits too large for one launch");
   if (!(softmax_scale > 0.f) || !(softmax_scale < 1e30f))

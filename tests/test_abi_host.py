@@ -128,6 +128,10 @@ def test_argument_errors_launch_nothing(lib):
     st = lib.kvq_paged_decode_attention(ctypes.byref(c), 16, 16, 16, 3, 16, 4, 8, 16, 16, 16, 16, 0.1, 16,
                                         need - 1, 2, None, None)
     assert st == kvq.KVQ_ERR_WORKSPACE
+    # a split count whose work units would not fit the device's 32-bit counters is refused on the host
+    st = lib.kvq_paged_decode_attention(ctypes.byref(c), 16, 16, 16, 60000, 16, 4, 8, 16, 16, 16, 16, 0.1, 16,
+                                        1 << 62, 65535, None, None)
+    assert st == kvq.KVQ_ERR_INVALID_ARG and "too large" in kvq.load_library().kvq_last_error().decode()
     # zero-sized work is a no-op
     assert lib.kvq_quantize_tiles(ctypes.byref(c), 16, None, 0, None, 0, None, 0, 0, 0, None, None, None,
                                   None) == kvq.KVQ_OK
