@@ -269,7 +269,7 @@ static_assert(16 * kTailRowBytes <= kTailScratch, "16 staged tail rows fit the w
 // query head; scratch: 16 padded V rows (4352 bytes) of the warp's shared
 // memory, whose copies must all have landed.
 template <int T>
-__device__ __noinline__ void decode_tail_warp(const DecodeArgs& a, int b, int h, int tau, float* tails, float* scratch, int lane) {
+__device__ __forceinline__ void decode_tail_warp(const DecodeArgs& a, int b, int h, int tau, float* tails, float* scratch, int lane) {
   const int G = a.cfg.group_size, nh = a.cfg.num_kv_heads;
   const int g = lane >> 2, t = lane & 3;
   const float qscale = a.softmax_scale * kLog2e;
@@ -416,7 +416,7 @@ __device__ __noinline__ void decode_tail_warp(const DecodeArgs& a, int b, int h,
 constexpr int kMergeGroup = 16;
 constexpr int kMergeWBytes = 4096;
 template <int G>
-__device__ __noinline__ void decode_merge_warp_g(const DecodeArgs& a, int b, int h, int n_rec, size_t first,
+__device__ __forceinline__ void decode_merge_warp_g(const DecodeArgs& a, int b, int h, int n_rec, size_t first,
                                                  int stride, bool final, float* parts, const float* tails,
                                                  float* scratch, int lane) {
   constexpr int R = 16 / G > 1 ? 16 / G : 1;     // records per round
@@ -532,7 +532,7 @@ __device__ __noinline__ void decode_merge_warp_g(const DecodeArgs& a, int b, int
   __syncwarp();
 }
 
-__device__ __noinline__ void decode_merge_warp(const DecodeArgs& a, int b, int h, int n_rec, size_t first, int stride,
+__device__ __forceinline__ void decode_merge_warp(const DecodeArgs& a, int b, int h, int n_rec, size_t first, int stride,
                                                bool final, float* parts, const float* tails, float* scratch,
                                                int lane) {
   switch (a.cfg.group_size) {
@@ -597,6 +597,27 @@ __device__ __forceinline__ UnitLoc locate_pair(const DecodeArgs& a, int b, int h
   const int u = a.step ? (b * nh + h) * a.num_splits_fixed : nh * prefix[b] + h * (prefix[b + 1] - prefix[b]);
   return locate_unit<T>(a, u, prefix, chunk);
 }
+// A merge a unit found itself last for: kind 1 = the merge group of chunks
+// [first, first + n) into the record at `first`; kind 2 = the final merge of
+// (b, h) over its n records (chunks or groups, `stride` apart from `ubase`).
+struct PendingMerge {
+  int kind = 0, b = 0, h = 0, S = 0, n = 0, stride = 1;
+  size_t first = 0, ubase = 0;
+  __device__ static PendingMerge group_of(int b, int h, int S, size_t ubase, size_t first, int n) {
+    PendingMerge m;
+    m.kind = 1; m.b = b; m.h = h; m.S = S; m.ubase = ubase; m.first = first; m.n = n; m.stride = 1;
+    return m;
+  }
+  __device__ static PendingMerge final_of(int b, int h, int S, size_t ubase) {
+    PendingMerge m;
+    const int n_groups = (S + kMergeGroup - 1) / kMergeGroup;
+    m.kind = 2; m.b = b; m.h = h; m.S = S; m.ubase = ubase; m.first = ubase;
+    m.n = n_groups == 1 ? S : n_groups;
+    m.stride = n_groups == 1 ? 1 : kMergeGroup;
+    return m;
+  }
+};
+
 // Arrivals that complete (sequence, KV head) at its counter: its raw-tail
 // unit, its final-merge unit, and its chunk units (one merge group) or its
 // merge groups.
@@ -677,6 +698,7 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
     if (lane == 0) u = atomicAdd(&ws_i[1], 1);
     u = __shfl_sync(kFull, u, 0);
     if (u >= U) break;
+    PendingMerge pend{};
     if (u < P || u >= P + UC) {
       // ---- raw tail of (sequence, KV head) p = (b, h): in a serving step,
       // first the step's token into tail row (L - 1) mod T; or its final-merge
@@ -694,15 +716,8 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
       int last = 0;
       if (lane == 0) last = atomicAdd(&arrivals[u], 1) == pair_arrivals(loc.S) - 1;
       last = __shfl_sync(kFull, last, 0);
-      if (last) {
-        __threadfence();
-        const int n_groups = (loc.S + kMergeGroup - 1) / kMergeGroup;
-        decode_merge_warp(a, b, h, n_groups == 1 ? loc.S : n_groups, loc.ubase, n_groups == 1 ? 1 : kMergeGroup,
-                          true, parts, tails, reinterpret_cast<float*>(stage_base), lane);
-        if (a.step && lane == 0) arrivals[u] = 0;  // the step leaves its counters at zero
-      }
-      continue;
-    }
+      if (last) pend = PendingMerge::final_of(b, h, loc.S, loc.ubase);
+    } else {
     u -= P;
     // ---- locate the unit: sequence b, head h, chunk c of the S chunks of
     // (b, h) over L tokens (the coordinates are located again after the
@@ -1035,38 +1050,43 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
     }
     loc = locate_unit<T>(a, u, prefix, chunk);
     // publish this unit's records; the last chunk of its group to finish
-    // merges the group, the last group of (b, h) merges the groups
+    // merges the group, the last group (or unit) of (b, h) merges the pair
     __threadfence();
     __syncwarp();
-    const int bh = loc.b * nh + loc.h;
     const int n_groups = (loc.S + kMergeGroup - 1) / kMergeGroup;
-    float* scratch = reinterpret_cast<float*>(stage_base);
-    bool to_final = n_groups == 1;
     if (n_groups > 1) {
       const int j = loc.c / kMergeGroup, gsz = min(kMergeGroup, loc.S - j * kMergeGroup);
       const size_t gfirst = loc.ubase + static_cast<size_t>(j) * kMergeGroup;
       int last = 0;
       if (lane == 0) last = atomicAdd(&gcount[gfirst], 1) == gsz - 1;
       last = __shfl_sync(kFull, last, 0);
-      if (last) {
-        __threadfence();
-        decode_merge_warp(a, loc.b, loc.h, gsz, gfirst, 1, false, parts, tails, scratch, lane);
-        if (a.step && lane == 0) gcount[gfirst] = 0;  // the step leaves its counters at zero
+      if (last) pend = PendingMerge::group_of(loc.b, loc.h, loc.S, loc.ubase, gfirst, gsz);
+    } else {
+      int last = 0;
+      if (lane == 0) last = atomicAdd(&arrivals[loc.b * nh + loc.h], 1) == pair_arrivals(loc.S) - 1;
+      last = __shfl_sync(kFull, last, 0);
+      if (last) pend = PendingMerge::final_of(loc.b, loc.h, loc.S, loc.ubase);
+    }
+    }
+    // ---- the merges this unit completed, from one call site (inlined once):
+    // a group, which may complete its (sequence, KV head); a final merge
+    while (pend.kind != 0) {
+      __threadfence();
+      decode_merge_warp(a, pend.b, pend.h, pend.n, pend.first, pend.stride, pend.kind == 2, parts, tails,
+                        reinterpret_cast<float*>(stage_base), lane);
+      const int bh = pend.b * nh + pend.h;
+      if (pend.kind == 1) {
+        if (a.step && lane == 0) gcount[pend.first] = 0;  // the step leaves its counters at zero
         __threadfence();
         __syncwarp();
-        to_final = true;
-      }
-    }
-    if (to_final) {
-      int last = 0;
-      // the counter counts the tail unit and the chunk units (one group) or the groups
-      if (lane == 0) last = atomicAdd(&arrivals[bh], 1) == pair_arrivals(loc.S) - 1;
-      last = __shfl_sync(kFull, last, 0);
-      if (last) {
-        __threadfence();
-        decode_merge_warp(a, loc.b, loc.h, n_groups == 1 ? loc.S : n_groups, loc.ubase,
-                          n_groups == 1 ? 1 : kMergeGroup, true, parts, tails, scratch, lane);
+        int last = 0;
+        // the pair counter counts its tail unit, its final-merge unit and its groups
+        if (lane == 0) last = atomicAdd(&arrivals[bh], 1) == pair_arrivals(pend.S) - 1;
+        last = __shfl_sync(kFull, last, 0);
+        pend = last ? PendingMerge::final_of(pend.b, pend.h, pend.S, pend.ubase) : PendingMerge{};
+      } else {
         if (a.step && lane == 0) arrivals[bh] = 0;  // the step leaves its counters at zero
+        pend = PendingMerge{};
       }
     }
   }
