@@ -296,9 +296,19 @@ __device__ void quantize_group_from_tmem(unsigned char* smem, uint32_t tbase, in
     }
     return frexp_exponent(m);
   };
+  // The (C, R) renormalization by a power of two leaves Y, every std and every
+  // clamp decision unchanged, so it runs after every second iteration and
+  // after the last: the final (C, R) are those of renormalizing after every
+  // iteration (both have max C in [1, 2) and differ from the unrenormalized
+  // pair by exact powers of two).  Two iterations move c by at most eps^-2 =
+  // 1e12, so the squared deviations of x c stay below 1e36 even for a tile of
+  // identical tokens at the fp16 range (three would overflow).  cur: the
+  // buffer of c this iteration reads.
+  int cur = 0;
   for (int it = 0; it < iters; ++it) {
-    cc = cc_buf + (it & 1) * (4 * kRows);
-    float* cc_next = cc_buf + ((it + 1) & 1) * (4 * kRows);
+    const bool renorm = it == iters - 1 || (it & 1) == 1;  // uniform
+    cc = cc_buf + cur * (4 * kRows);
+    float* cc_next = cc_buf + (cur ^ 1) * (4 * kRows);
     // ---- channel step: channel `row`, token columns 64hf..64hf+63.  The new
     // c_j are published with the per-warp maxima of C for the renormalization.
     if constexpr (T <= 64) {
@@ -345,11 +355,13 @@ __device__ void quantize_group_from_tmem(unsigned char* smem, uint32_t tbase, in
       pair_sync(qd);  // both halves have read cc[row]
       if (hf == 0) cc[row] = fminf(div_fast(c, sigma), FLT_MAX);
     }
+    if (renorm) {
 #pragma unroll
-    for (int lt = 0; lt < kLocal; ++lt) {
-      // C_j > 0: the float order is the order of the bit patterns
-      const float m = __uint_as_float(__reduce_max_sync(kFull, __float_as_uint(Cj[lt])));
-      if (lane == 0) red[warp * 4 + ch_tile(lt)] = m;
+      for (int lt = 0; lt < kLocal; ++lt) {
+        // C_j > 0: the float order is the order of the bit patterns
+        const float m = __uint_as_float(__reduce_max_sync(kFull, __float_as_uint(Cj[lt])));
+        if (lane == 0) red[warp * 4 + ch_tile(lt)] = m;
+      }
     }
     math_sync();
     // ---- token step with this iteration's c (before the renormalization,
@@ -383,6 +395,11 @@ __device__ void quantize_group_from_tmem(unsigned char* smem, uint32_t tbase, in
         r_new = fminf(div_fast(r, rho), FLT_MAX);  // a zero token keeps a finite factor
       }
     }
+    if (!renorm) {  // c stays in this buffer; the new r replaces the old after the pair barrier
+      if (tok_live && hf == 0) rr[row] = r_new;
+      math_sync();
+      continue;
+    }
     // ---- (C, R) -> (C / 2^k, R 2^k) per tile, max C in [1, 2): every thread
     // rescales what it owns; cc and rr are read again only after the barrier
     // (the exponent of the token's tile is reused when that tile is one of
@@ -405,11 +422,12 @@ __device__ void quantize_group_from_tmem(unsigned char* smem, uint32_t tbase, in
       Ri = scale_pow2(Ri, e - 1);
       if (tok_live && hf == 0) rr[row] = fminf(scale_pow2(r_new, 1 - e), FLT_MAX);
     }
+    cur ^= 1;
     math_sync();
   }
 
   // ---- RTN on D1: token `row`, channels 64hf..64hf+63
-  cc = cc_buf + (iters & 1) * (4 * kRows);
+  cc = cc_buf + cur * (4 * kRows);
   constexpr int qmax = (1 << bits) - 1;
   constexpr bool kGrouped = is_v && bits != 3;  // V in the decode lane order
   const int local = row % T, page_in_tile = local / kPageTokens, p = local % kPageTokens;
