@@ -43,7 +43,9 @@ namespace {
 constexpr int kPartFloats = 4 + kHeadDim;
 constexpr int kPartAcc = 4;
 constexpr int kTailScratch = 13 * 1024;  // warp scratch: the tail's staged V rows; the merge's weights and staging
-constexpr int kUnitsPerSm = 32;            // work-unit budget of the automatic split
+// work-unit budget of the automatic split, per SM: about two units per
+// resident warp at T <= 64 (12 warps per SM), four at T = 128 (8 warps)
+__host__ __device__ constexpr int units_per_sm(int T) { return T == 128 ? 32 : 24; }
 constexpr long long kWaitLimitNs = 2000000000LL;  // bounded mbarrier waits: 2 s
 
 // ------------------------------------------------------------------ workspace
@@ -1140,10 +1142,10 @@ cudaError_t launch_decode_bits(const DecodeArgs& a, cudaStream_t s, int sms) {
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, Geo::kWarps * 32, Geo::kSmem);
   if (e != cudaSuccess) return e;
   per_sm = std::max(per_sm, 1);
-  // automatic split: 32 units per SM whatever the residency (8 per warp at
-  // T = 128, where one CTA fits an SM; the warps take units from a queue, so
-  // short units even out the ragged last chunks), as the workspace holds
-  const int target = kUnitsPerSm * sms;
+  // automatic split: units_per_sm(T) units per SM (the warps take units from
+  // a queue, so short units even out the ragged last chunks), as the
+  // workspace holds
+  const int target = units_per_sm(T) * sms;
   decode_schedule_kernel<<<1, 1024, 0, s>>>(a.seq_lens, a.num_seqs, T, a.cfg.num_kv_heads, a.cfg.group_size,
                                             a.num_splits_fixed, target, a.workspace);
   e = cudaGetLastError();
@@ -1203,7 +1205,8 @@ size_t decode_workspace_bytes(const kvq_config& cfg, int num_seqs, int num_split
   const WsLayout wl = ws_layout(num_seqs, cfg.num_kv_heads, cfg.group_size);
   const size_t units = num_splits > 0
                            ? static_cast<size_t>(num_seqs) * cfg.num_kv_heads * num_splits
-                           : static_cast<size_t>(kUnitsPerSm) * num_sms + static_cast<size_t>(num_seqs) * cfg.num_kv_heads;
+                           : static_cast<size_t>(units_per_sm(cfg.tile_tokens)) * num_sms +
+                                 static_cast<size_t>(num_seqs) * cfg.num_kv_heads;
   return wl.part_off + units * cfg.group_size * kPartFloats * sizeof(float) + units * sizeof(int32_t);
 }
 
