@@ -832,8 +832,7 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
       // up to 4 so that one chunk's code words and accumulators are live; the
       // chunk's scores (log2 domain, tokens 8nb + 2t, 8nb + 2t + 1 of each page)
       // are kept.
-      // (two at T = 128, where the scores of 8 pages stay live as well)
-      constexpr int kPcMax = (BK == 8 || BK == 3 || NP >= 8) ? 2 : 4;
+      constexpr int kPcMax = (BK == 8 || BK == 3) ? 2 : 4;
       constexpr int kPc = NP < kPcMax ? NP : kPcMax;
       float sig = 0.f;
       float sc[NP][2][2];
