@@ -52,21 +52,26 @@ constexpr long long kWaitLimitNs = 2000000000LL;  // bounded mbarrier waits: 2 s
 // [0]        int32 U (total work units)
 // [4]        int32 next unit to hand out (dynamic schedule)
 // [8]        int32 CTAs finished (fused serving step)
-// [16..]     int32 prefix[B+1]: chunks of sequences 0..b-1 (per KV head)
+// [16..]     int32 prefix[B+1]: chunks of the sequences before position i of
+//            the dispatch order (per KV head)
 // then       int32 chunk[B]: tiles per chunk of each sequence
+// then       int32 order[B]: the sequence at position i of the dispatch order
+// then       int32 rank[B]: the position of sequence b in it
 // then       int32 arrivals[B][H]: finished units of each (sequence, KV head)
 // at 256-B   float tails[B][H][G][4 + d]  (m, l, pad, pad, acc) of the raw tail
 // then       float partial[U][G][4 + d]  (m, l, pad, pad, acc) of the units
 // then       int32 group[U]: finished chunks of each merge group, at the
 //            slot of the group's first unit
 struct WsLayout {
-  size_t prefix_off, chunk_off, arrive_off, tail_off, part_off;
+  size_t prefix_off, chunk_off, order_off, rank_off, arrive_off, tail_off, part_off;
 };
 __host__ __device__ inline WsLayout ws_layout(int num_seqs, int num_heads, int group) {
   WsLayout l;
   l.prefix_off = 16;
   l.chunk_off = l.prefix_off + 4 * static_cast<size_t>(num_seqs + 1);
-  l.arrive_off = l.chunk_off + 4 * static_cast<size_t>(num_seqs);
+  l.order_off = l.chunk_off + 4 * static_cast<size_t>(num_seqs);
+  l.rank_off = l.order_off + 4 * static_cast<size_t>(num_seqs);
+  l.arrive_off = l.rank_off + 4 * static_cast<size_t>(num_seqs);
   l.tail_off = (l.arrive_off + 4 * static_cast<size_t>(num_seqs) * num_heads + 255) / 256 * 256;
   l.part_off = l.tail_off + static_cast<size_t>(num_seqs) * num_heads * group * kPartFloats * sizeof(float);
   return l;
@@ -152,16 +157,26 @@ __device__ __forceinline__ uint32_t code_pair_f16(uint32_t lo, uint32_t hi) {
 }
 
 // ------------------------------------------------------------------ schedule
+// Work units of the automatic (or fixed) split: chunk sizes, the dispatch
+// order and its unit prefix, and the counters reset.  With up to 1024
+// sequences they are dispatched longest first (a bitonic sort of the tile
+// counts, ties by index), so the queue ends on short units and the warps
+// finish together; the order does not change any result (each pair's records
+// are merged in chunk order).
 __global__ void __launch_bounds__(1024) decode_schedule_kernel(const int32_t* seq_lens, int num_seqs, int tile_tokens,
                                                                int num_kv_heads, int group, int num_splits,
                                                                int target_units, void* workspace) {
   __shared__ long long s_total;
   __shared__ int s_scan[1024];
+  __shared__ int s_key[1024];
+  __shared__ int s_idx[1024];
   __shared__ int s_carry;
   const WsLayout wl = ws_layout(num_seqs, num_kv_heads, group);
   int32_t* ws_i = static_cast<int32_t*>(workspace);
   int32_t* prefix = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + wl.prefix_off);
   int32_t* chunk = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + wl.chunk_off);
+  int32_t* order = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + wl.order_off);
+  int32_t* rank = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + wl.rank_off);
   int32_t* arrivals = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + wl.arrive_off);
   const int tid = threadIdx.x;
   // the arrival counters and the unit queue start at zero on every call
@@ -175,26 +190,61 @@ __global__ void __launch_bounds__(1024) decode_schedule_kernel(const int32_t* se
   long long part = 0;
   for (int b = tid; b < num_seqs; b += blockDim.x) part += max(seq_lens[b], 0) / tile_tokens;
   atomicAdd(reinterpret_cast<unsigned long long*>(&s_total), static_cast<unsigned long long>(part));
+  // dispatch order: longest first when the sequences fit one sort, else as given
+  const bool sorted = num_seqs <= static_cast<int>(blockDim.x);
+  if (sorted) {
+    s_key[tid] = tid < num_seqs ? max(seq_lens[tid], 0) / tile_tokens : -1;
+    s_idx[tid] = tid;
+    int n = 1;  // the sort spans the next power of two of the sequence count
+    while (n < num_seqs) n <<= 1;
+    __syncthreads();
+    for (int k = 2; k <= n; k <<= 1) {
+      for (int jj = k >> 1; jj > 0; jj >>= 1) {
+        const int p = tid ^ jj;
+        if (p > tid) {
+          // descending by key, ascending by index on ties, in the (tid & k) == 0 halves
+          const bool first_wins = s_key[tid] > s_key[p] || (s_key[tid] == s_key[p] && s_idx[tid] < s_idx[p]);
+          if (((tid & k) == 0) != first_wins) {
+            const int tk = s_key[tid], ti = s_idx[tid];
+            s_key[tid] = s_key[p];
+            s_idx[tid] = s_idx[p];
+            s_key[p] = tk;
+            s_idx[p] = ti;
+          }
+        }
+        __syncthreads();
+      }
+    }
+    if (tid < num_seqs) {
+      order[tid] = s_idx[tid];
+      rank[s_idx[tid]] = tid;
+    }
+  } else {
+    for (int b = tid; b < num_seqs; b += blockDim.x) {
+      order[b] = b;
+      rank[b] = b;
+    }
+  }
   __syncthreads();
   const long long total = s_total;
   long long ch_auto = 1;
   if (num_splits == 0 && total > 0)
     ch_auto = std::max(1LL, (total * num_kv_heads + target_units - 1) / target_units);
   for (int base = 0; base < num_seqs; base += blockDim.x) {
-    const int b = base + tid;
+    const int i = base + tid;  // position in the dispatch order
     int units = 0;
-    if (b < num_seqs) {
+    if (i < num_seqs) {
+      const int b = sorted ? s_idx[i] : i;
       const int f = max(seq_lens[b], 0) / tile_tokens;
       int ch;
       if (num_splits > 0) {
-        const int s = min(num_splits, f);
-        ch = s > 0 ? (f + s - 1) / s : 1;
+        const int sp = min(num_splits, f);
+        ch = sp > 0 ? (f + sp - 1) / sp : 1;
       } else {
         ch = static_cast<int>(std::min<long long>(ch_auto, 1 << 30));
       }
-      // every (sequence, KV head) gets a unit, even with no full tile: the
-      // unit with chunk 0 also takes the raw tail, and the last unit to
-      // finish merges and writes the output
+      // every (sequence, KV head) gets a unit, even with no full tile (its
+      // records say so; the raw tail and the merge are separate units)
       units = f > 0 ? (f + ch - 1) / ch : 1;
       chunk[b] = ch;
     }
@@ -206,7 +256,7 @@ __global__ void __launch_bounds__(1024) decode_schedule_kernel(const int32_t* se
       s_scan[tid] += v;
       __syncthreads();
     }
-    if (b < num_seqs) prefix[b] = s_carry + s_scan[tid] - units;
+    if (i < num_seqs) prefix[i] = s_carry + s_scan[tid] - units;
     __syncthreads();
     if (tid == blockDim.x - 1) s_carry += s_scan[tid];
     __syncthreads();
@@ -575,19 +625,20 @@ __device__ __forceinline__ UnitLoc locate_unit(const DecodeArgs& a, int u, const
     l.S = f > 0 ? (f + l.ch - 1) / l.ch : 1;
     l.ubase = (static_cast<size_t>(l.b) * nh + l.h) * sx;
   } else {
-    int lo = 0, hi = a.num_seqs;  // find the largest b with nh*prefix[b] <= u
+    int lo = 0, hi = a.num_seqs;  // find the largest position i with nh*prefix[i] <= u
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
       if (nh * prefix[mid] <= u) lo = mid; else hi = mid;
     }
-    l.b = lo;
-    l.S = prefix[l.b + 1] - prefix[l.b];
-    const int r = u - nh * prefix[l.b];
+    const int32_t* order = chunk + a.num_seqs;
+    l.b = order[lo];
+    l.S = prefix[lo + 1] - prefix[lo];
+    const int r = u - nh * prefix[lo];
     l.h = r / l.S;
     l.c = r % l.S;
     l.L = max(a.seq_lens[l.b], 0);
     l.ch = chunk[l.b];
-    l.ubase = static_cast<size_t>(nh) * prefix[l.b] + static_cast<size_t>(l.h) * l.S;
+    l.ubase = static_cast<size_t>(nh) * prefix[lo] + static_cast<size_t>(l.h) * l.S;
   }
   return l;
 }
@@ -596,8 +647,9 @@ template <int T>
 __device__ __forceinline__ UnitLoc locate_pair(const DecodeArgs& a, int b, int h, const int32_t* prefix,
                                                const int32_t* chunk) {
   const int nh = a.cfg.num_kv_heads;
-  const int u = a.step ? (b * nh + h) * a.num_splits_fixed : nh * prefix[b] + h * (prefix[b + 1] - prefix[b]);
-  return locate_unit<T>(a, u, prefix, chunk);
+  if (a.step) return locate_unit<T>(a, (b * nh + h) * a.num_splits_fixed, prefix, chunk);
+  const int i = chunk[2 * a.num_seqs + b];  // rank of b in the dispatch order
+  return locate_unit<T>(a, nh * prefix[i] + h * (prefix[i + 1] - prefix[i]), prefix, chunk);
 }
 // A merge a unit found itself last for: kind 1 = the merge group of chunks
 // [first, first + n) into the record at `first`; kind 2 = the final merge of
