@@ -79,10 +79,13 @@
  *   d = 128 runs the tuned path (tensor-core rotation in the quantizer,
  *   mma.sync decode, tensor-core chunked prefill, the one-launch serving
  *   step).  d = 64 and d = 256 run kvq_quantize_tiles, kvq_append_tokens,
- *   kvq_paged_decode_attention (and its static-scratch form) and
- *   kvq_unpack_tiles on CUDA-core kernels with the same format and the same
- *   method; kvq_paged_prefill_attention, kvq_prefill_workspace_bytes and
- *   kvq_append_decode_step return KVQ_ERR_UNSUPPORTED for them.
+ *   kvq_paged_decode_attention (and its static-scratch form),
+ *   kvq_paged_prefill_attention and kvq_unpack_tiles on CUDA-core kernels
+ *   with the same format and the same method (chunked prefill there runs one
+ *   launch over the whole context and needs no workspace:
+ *   kvq_prefill_workspace_bytes gives 0 for every num_splits, which is
+ *   checked and otherwise ignored); kvq_append_decode_step returns
+ *   KVQ_ERR_UNSUPPORTED for them.
  *
  * Conventions
  * -----------
@@ -265,7 +268,8 @@ KVQ_API kvq_status kvq_append_decode_step(const kvq_config* cfg, const void* new
                                           int num_splits, int32_t* dev_status, void* stream);
 
 /* Bytes of device workspace kvq_paged_prefill_attention needs with num_splits
- * context splits (0 for num_splits = 1).  cfg, bytes: host pointers. */
+ * context splits (0 for num_splits = 1, and 0 at d = 64 / 256).  cfg, bytes:
+ * host pointers. */
 KVQ_API kvq_status kvq_prefill_workspace_bytes(const kvq_config* cfg, int num_seqs, int max_chunk_tokens,
                                                int num_splits, size_t* bytes);
 

@@ -334,12 +334,12 @@ kvq_status kvq_append_decode_step(const kvq_config* cfg, const void* new_k, cons
 kvq_status kvq_prefill_workspace_bytes(const kvq_config* cfg, int num_seqs, int max_chunk_tokens, int num_splits,
                                        size_t* bytes) {
   KVQ_TRY(check_config(cfg));
-  if (cfg->head_dim != kvq::kHeadDim)
-    return fail(KVQ_ERR_UNSUPPORTED, "chunked prefill is built for head_dim 128 (got %d)", cfg->head_dim);
   if (bytes == nullptr) return fail(KVQ_ERR_INVALID_ARG, "bytes is NULL");
   if (num_seqs < 0 || max_chunk_tokens < 0) return fail(KVQ_ERR_INVALID_ARG, "negative num_seqs or max_chunk_tokens");
   if (num_splits < 1 || num_splits > 64) return fail(KVQ_ERR_INVALID_ARG, "num_splits must be 1..64");
-  *bytes = kvq::prefill_workspace_bytes(*cfg, num_seqs, max_chunk_tokens, num_splits);
+  // d = 64 / 256: one launch over the whole context, no workspace
+  *bytes = cfg->head_dim == kvq::kHeadDim ? kvq::prefill_workspace_bytes(*cfg, num_seqs, max_chunk_tokens, num_splits)
+                                          : 0;
   return ok();
 }
 
@@ -351,15 +351,16 @@ kvq_status kvq_paged_prefill_attention(const kvq_config* cfg, const void* q, voi
                                        float softmax_scale, int num_splits, void* workspace,
                                        size_t workspace_bytes, int32_t* dev_status, void* stream) {
   KVQ_TRY(check_config(cfg));
-  if (cfg->head_dim != kvq::kHeadDim)
-    return fail(KVQ_ERR_UNSUPPORTED, "chunked prefill is built for head_dim 128 (got %d)", cfg->head_dim);
+  const bool generic = cfg->head_dim != kvq::kHeadDim;  // d = 64 / 256: CUDA-core kernel, context not split
   if (num_splits < 1 || num_splits > 64) return fail(KVQ_ERR_INVALID_ARG, "num_splits must be 1..64");
   if (num_seqs < 0 || max_chunk_tokens < 0) return fail(KVQ_ERR_INVALID_ARG, "negative num_seqs or max_chunk_tokens");
   if (num_seqs == 0 || max_chunk_tokens == 0) return ok();
   if (num_seqs > 65535) return fail(KVQ_ERR_INVALID_ARG, "num_seqs > 65535");
   if (max_chunk_tokens > (1 << 20)) return fail(KVQ_ERR_INVALID_ARG, "max_chunk_tokens > 2^20");
-  const long long units = static_cast<long long>(num_seqs) * cfg->num_kv_heads * kvq::prefill_row_tiles(*cfg, max_chunk_tokens);
-  if (units * num_splits > 0x7fffffffLL)
+  const long long units = generic ? kvq::generic_prefill_ctas(*cfg, num_seqs, max_chunk_tokens)
+                                  : static_cast<long long>(num_seqs) * cfg->num_kv_heads *
+                                        kvq::prefill_row_tiles(*cfg, max_chunk_tokens) * num_splits;
+  if (units > 0x7fffffffLL)
     return fail(KVQ_ERR_INVALID_ARG, "num_seqs x max_chunk_tokens x num_splits too large for one launch");
   if (!(softmax_scale > 0.f) || !(softmax_scale < 1e30f))
     return fail(KVQ_ERR_INVALID_ARG, "softmax_scale must be a positive finite float");
@@ -374,7 +375,7 @@ kvq_status kvq_paged_prefill_attention(const kvq_config* cfg, const void* q, voi
   KVQ_TRY(check_ptr(v_pool, "v_pool"));
   KVQ_TRY(check_ptr(k_tail, "k_tail"));
   KVQ_TRY(check_ptr(v_tail, "v_tail"));
-  const size_t need = kvq::prefill_workspace_bytes(*cfg, num_seqs, max_chunk_tokens, num_splits);
+  const size_t need = generic ? 0 : kvq::prefill_workspace_bytes(*cfg, num_seqs, max_chunk_tokens, num_splits);
   KVQ_TRY(check_ptr(workspace, "workspace", need == 0));
   if (workspace_bytes < need)
     return fail(KVQ_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", workspace_bytes, need);
@@ -401,6 +402,9 @@ kvq_status kvq_paged_prefill_attention(const kvq_config* cfg, const void* q, voi
   a.num_splits = num_splits;
   a.partials = static_cast<float*>(workspace);
   a.dev_status = dev_status;
+  if (generic)
+    return cuda_status(kvq::launch_generic_prefill(a, static_cast<cudaStream_t>(stream)),
+                       "kvq_paged_prefill_attention launch");
   return cuda_status(kvq::launch_paged_prefill(a, static_cast<cudaStream_t>(stream)),
                      "kvq_paged_prefill_attention launch");
 }

@@ -600,6 +600,286 @@ __global__ void __launch_bounds__(kGThreads) gen_decode_merge_kernel(DecodeArgs 
   }
 }
 
+// ------------------------------------------------------------------ prefill
+// Chunked prefill attention (aitrends.kr article 74976, "TL;DR": every phase
+// of attention reads the compressed pages directly): chunk token i of a
+// sequence attends to its cached context (full tiles from the pages, in the
+// rotated domain, as the decode split kernel reads them; then the raw fp16
+// tail) and, causally, to the chunk's own raw rows 0..i.  One CTA per
+// (sequence, KV head, run of chunk tokens); its query rows are those tokens
+// x the g query heads of the KV head, token-major (row r: token r / g, head
+// r % g).  Two running softmax states per row, one per domain: the context
+// tiles in the rotated domain, the tail and chunk rows in the original one;
+// the rotated accumulator goes back through one inverse rotation, then the
+// two states are merged by their log-sum-exp weights.
+
+constexpr int kPfRawBlk = 16;  // raw keys per block of the original-domain phase
+
+template <int D>
+constexpr int gen_pf_rows() {
+  return D == 64 ? 32 : 16;  // query rows per CTA
+}
+
+struct GenPfSmem {
+  size_t qr, qq, acc, acc2, sc, ck, cv, mk, mv, hs, kc, vc, total;
+};
+__host__ __device__ inline GenPfSmem gen_pf_smem(int D, int T, int R) {
+  GenPfSmem m;
+  const size_t rd = static_cast<size_t>(R) * D * 4;
+  m.qr = 0;                                  // q' (then the scaled raw q) [R][D] fp32
+  m.qq = m.qr + rd;                          // q'' [R][D]
+  m.acc = m.qq + rd;                         // acc' (rotated domain) [R][D]
+  m.acc2 = m.acc + rd;                       // acc (original domain) [R][D]
+  m.sc = m.acc2 + rd;                        // scores / p [R][T]
+  m.ck = m.sc + static_cast<size_t>(R) * T * 4;
+  m.cv = m.ck + D * 4;
+  m.mk = m.cv + D * 4;                       // (s~, z~) of K [T] float2
+  m.mv = m.mk + T * 8;
+  m.hs = m.mv + T * 8;                       // per row [R][8]: m, l, alpha, sigma, w, m2, l2, -
+  m.kc = m.hs + static_cast<size_t>(R) * 8 * 4;  // K codes [T][D + 4] bytes, or raw K rows [16][D] fp16
+  m.vc = m.kc + static_cast<size_t>(T) * (D + 4);
+  m.total = m.vc + static_cast<size_t>(T) * (D + 4);
+  return m;
+}
+
+// CTAs of a prefill launch: (sequences x KV heads) x runs of chunk tokens
+long long gen_pf_ctas(const kvq_config& cfg, int num_seqs, int max_chunk) {
+  const int R = cfg.head_dim == 64 ? gen_pf_rows<64>() : gen_pf_rows<256>();
+  const long long toks = std::max(1, R / cfg.group_size);
+  return static_cast<long long>(num_seqs) * cfg.num_kv_heads * ((max_chunk + toks - 1) / toks);
+}
+
+// Running softmax over one block of `n` score columns per row (log2 domain):
+// new maximum, alpha = 2^(m_old - m_new), p = 2^(s - m_new) written back, row
+// sums added into l; masked columns hold -inf and give p = 0.
+__device__ __forceinline__ void pf_softmax_rows(float* sc, int ld, int n, int rows, float* hs, int im, int il) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int r = warp; r < rows; r += kGWarps) {
+    float tm = -INFINITY;
+    for (int i = lane; i < n; i += 32) tm = fmaxf(tm, sc[r * ld + i]);
+    tm = warp_max(tm);
+    const float m_old = hs[8 * r + im], m_new = fmaxf(m_old, tm);
+    const float alpha = m_new == -INFINITY ? 1.f : exp2f(m_old - m_new);
+    float ls = 0.f;
+    for (int i = lane; i < n; i += 32) {
+      const float s = sc[r * ld + i];
+      const float pv = s == -INFINITY ? 0.f : exp2f(s - m_new);
+      sc[r * ld + i] = pv;
+      ls += pv;
+    }
+    ls = warp_sum(ls);
+    if (lane == 0) {
+      hs[8 * r + im] = m_new;
+      hs[8 * r + il] = hs[8 * r + il] * alpha + ls;
+      hs[8 * r + 2] = alpha;
+    }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kGThreads) gen_prefill_kernel(PrefillArgs a, PoolGeom gk, PoolGeom gv) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  __shared__ const uint8_t* kpg[kMaxPages];
+  __shared__ const uint8_t* vpg[kMaxPages];
+  __shared__ int ok;
+  constexpr int R = gen_pf_rows<D>();
+  const int T = a.cfg.tile_tokens, npages = T / kPageTokens;
+  const int nh = a.cfg.num_kv_heads, G = a.cfg.group_size, Hq = nh * G;
+  const int toks = max(1, R / G), rows = toks * G;  // chunk tokens and query rows of this CTA
+  const GenPfSmem L = gen_pf_smem(D, T, R);
+  float* qr = reinterpret_cast<float*>(smem + L.qr);
+  float* qq = reinterpret_cast<float*>(smem + L.qq);
+  float* acc = reinterpret_cast<float*>(smem + L.acc);
+  float* acc2 = reinterpret_cast<float*>(smem + L.acc2);
+  float* sc = reinterpret_cast<float*>(smem + L.sc);
+  float* ck = reinterpret_cast<float*>(smem + L.ck);
+  float* cv = reinterpret_cast<float*>(smem + L.cv);
+  float2* mk = reinterpret_cast<float2*>(smem + L.mk);
+  float2* mv = reinterpret_cast<float2*>(smem + L.mv);
+  float* hs = reinterpret_cast<float*>(smem + L.hs);
+  uint8_t* kc = smem + L.kc;
+  uint8_t* vc = smem + L.vc;
+  const int tid = threadIdx.x;
+  const int runs = (a.max_chunk + toks - 1) / toks;
+  const int pair = static_cast<int>(blockIdx.x / runs), run = static_cast<int>(blockIdx.x % runs);
+  const int b = pair / nh, h = pair % nh;
+  const int c0 = a.cu_chunk[b];
+  const int n = a.cu_chunk[b + 1] - c0;
+  if ((n < 0 || n > a.max_chunk) && tid == 0 && run == 0 && h == 0) report_error(a.dev_status, KVQ_ERR_DEVICE_BOUNDS);
+  const int nc = max(0, min(n, a.max_chunk));  // chunk tokens served
+  const int i0 = run * toks;
+  if (i0 >= nc) return;
+  const int nt = min(toks, nc - i0);  // live tokens of this CTA; rows >= nt * G are idle
+  const int Lc = max(a.ctx_lens[b], 0), F = Lc / T, tau = Lc % T;
+  const float qscale = a.softmax_scale * kLog2e;
+  const __half* q = static_cast<const __half*>(a.q);
+
+  // q' = q D_s H / sqrt(D) times the softmax scale (log2 domain); idle rows 0
+  for (int idx = tid; idx < rows * D; idx += kGThreads) {
+    const int r = idx / D, j = idx % D, ti = r / G;
+    const float v = ti < nt ? __half2float(q[(static_cast<size_t>(c0 + i0 + ti) * Hq + h * G + r % G) * D + j]) : 0.f;
+    qr[idx] = v * rotation_sign(a.cfg.rotation_seed, j);
+    acc[idx] = 0.f;
+    acc2[idx] = 0.f;
+  }
+  for (int r = tid; r < rows; r += kGThreads) {
+    hs[8 * r] = -INFINITY;
+    hs[8 * r + 1] = 0.f;
+    hs[8 * r + 5] = -INFINITY;
+    hs[8 * r + 6] = 0.f;
+  }
+  __syncthreads();
+  fwht_rows<D>(qr, rows, D);
+  for (int idx = tid; idx < rows * D; idx += kGThreads) qr[idx] *= qscale * inv_sqrt_d<D>();
+  __syncthreads();
+
+  // ---- context tiles, rotated domain
+  const uint8_t* kpool = static_cast<const uint8_t*>(a.k_pool);
+  const uint8_t* vpool = static_cast<const uint8_t*>(a.v_pool);
+  for (int tile = 0; tile < F; ++tile) {
+    if (tid == 0) {
+      bool good = (tile + 1) * npages <= a.max_blocks_per_seq;
+      for (int k = 0; good && k < npages; ++k) {
+        const int blk = a.block_tables[static_cast<size_t>(b) * a.max_blocks_per_seq + tile * npages + k];
+        good = blk >= 0 && blk < a.num_blocks;
+        if (good) {
+          kpg[k] = kpool + (static_cast<size_t>(blk) * nh + h) * gk.page_bytes;
+          vpg[k] = vpool + (static_cast<size_t>(blk) * nh + h) * gv.page_bytes;
+        }
+      }
+      if (!good) report_error(a.dev_status, KVQ_ERR_DEVICE_BOUNDS);
+      ok = good;
+    }
+    __syncthreads();
+    const bool tile_ok = ok;
+    __syncthreads();  // every thread has read ok before thread 0 writes the next tile's
+    if (!tile_ok) continue;  // tile skipped (reported)
+    for (int idx = tid; idx < T * D; idx += kGThreads) {
+      const int i = idx / D, j = idx % D, k = i / kPageTokens, p = i % kPageTokens;
+      kc[i * (D + 4) + j] = static_cast<uint8_t>(read_code(kpg[k], code_bit_d<D>(j, p, gk.bits, false), gk.bits));
+      vc[i * (D + 4) + j] = static_cast<uint8_t>(read_code(vpg[k], code_bit_d<D>(j, p, gv.bits, true), gv.bits));
+    }
+    for (int i = tid; i < T; i += kGThreads) {
+      const int k = i / kPageTokens, p = i % kPageTokens;
+      mk[i] = __half22float2(*reinterpret_cast<const __half2*>(kpg[k] + gk.meta_off + 4 * p));
+      mv[i] = __half22float2(*reinterpret_cast<const __half2*>(vpg[k] + gv.meta_off + 4 * p));
+    }
+    for (int j = tid; j < D; j += kGThreads) {
+      ck[j] = __half2float(*reinterpret_cast<const __half*>(kpg[j / gk.cs_channels] + gk.cslice_off +
+                                                            2 * (j % gk.cs_channels)));
+      cv[j] = __half2float(*reinterpret_cast<const __half*>(vpg[j / gv.cs_channels] + gv.cslice_off +
+                                                            2 * (j % gv.cs_channels)));
+    }
+    __syncthreads();
+    for (int idx = tid; idx < rows * D; idx += kGThreads) qq[idx] = qr[idx] * ck[idx % D];
+    __syncthreads();
+    for (int r = threadIdx.x >> 5; r < rows; r += kGWarps) {  // sigma = sum_j q''_j
+      float sg = 0.f;
+      for (int j = threadIdx.x & 31; j < D; j += 32) sg += qq[r * D + j];
+      sg = warp_sum(sg);
+      if ((threadIdx.x & 31) == 0) hs[8 * r + 3] = sg;
+    }
+    __syncthreads();
+    for (int idx = tid; idx < rows * T; idx += kGThreads) {  // scores s~ (q'' . code) + z~ sigma
+      const int r = idx / T, i = idx % T;
+      const float* qh = qq + r * D;
+      const uint8_t* ci = kc + i * (D + 4);
+      float dot = 0.f;
+      for (int j = 0; j < D; j += 4) {
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(ci + j);
+        dot += qh[j] * static_cast<float>(w & 0xffu) + qh[j + 1] * static_cast<float>((w >> 8) & 0xffu) +
+               qh[j + 2] * static_cast<float>((w >> 16) & 0xffu) + qh[j + 3] * static_cast<float>(w >> 24);
+      }
+      sc[r * T + i] = mk[i].x * dot + mk[i].y * hs[8 * r + 3];
+    }
+    __syncthreads();
+    pf_softmax_rows(sc, T, T, rows, hs, 0, 1);
+    __syncthreads();
+    for (int r = threadIdx.x >> 5; r < rows; r += kGWarps) {  // P' = p s~V in place, w = sum p z~V
+      float wz = 0.f;
+      for (int i = threadIdx.x & 31; i < T; i += 32) {
+        const float pv = sc[r * T + i];
+        wz += pv * mv[i].y;
+        sc[r * T + i] = pv * mv[i].x;
+      }
+      wz = warp_sum(wz);
+      if ((threadIdx.x & 31) == 0) hs[8 * r + 4] = wz;
+    }
+    __syncthreads();
+    for (int idx = tid; idx < rows * D; idx += kGThreads) {  // acc' = alpha acc' + C~V (P' code + w)
+      const int r = idx / D, j = idx % D;
+      const float* ph = sc + r * T;
+      float u = 0.f;
+      for (int i = 0; i < T; ++i) u += ph[i] * static_cast<float>(vc[i * (D + 4) + j]);
+      acc[idx] = hs[8 * r + 2] * acc[idx] + cv[j] * (u + hs[8 * r + 4]);
+    }
+    __syncthreads();
+  }
+
+  // ---- raw keys, original domain: the tail (positions F T .. Lc - 1, tail
+  // rows 0 .. tau - 1), then chunk rows 0 .. i0 + nt - 1, causal per row
+  for (int idx = tid; idx < rows * D; idx += kGThreads) {
+    const int r = idx / D, j = idx % D, ti = r / G;
+    qr[idx] = ti < nt ? __half2float(q[(static_cast<size_t>(c0 + i0 + ti) * Hq + h * G + r % G) * D + j]) * qscale
+                      : 0.f;
+  }
+  const __half* kt = static_cast<const __half*>(a.k_tail) + static_cast<size_t>(pair) * T * D;
+  const __half* vt = static_cast<const __half*>(a.v_tail) + static_cast<size_t>(pair) * T * D;
+  const __half* kn = static_cast<const __half*>(a.k_new);
+  const __half* vn = static_cast<const __half*>(a.v_new);
+  __half* kr = reinterpret_cast<__half*>(kc);  // [16][D]
+  __half* vr = reinterpret_cast<__half*>(vc);
+  const int nkeys = tau + i0 + nt;
+  for (int u0 = 0; u0 < nkeys; u0 += kPfRawBlk) {
+    const int nb = min(kPfRawBlk, nkeys - u0);
+    __syncthreads();  // the previous block's rows are no longer read
+    for (int idx = tid; idx < nb * (D / 8); idx += kGThreads) {
+      const int i = idx / (D / 8), piece = idx % (D / 8), u = u0 + i;
+      const size_t src = u < tau ? static_cast<size_t>(u) * D
+                                 : (static_cast<size_t>(c0 + u - tau) * nh + h) * D;
+      const __half* ks = u < tau ? kt : kn;
+      const __half* vs = u < tau ? vt : vn;
+      *reinterpret_cast<uint4*>(kr + i * D + 8 * piece) = *reinterpret_cast<const uint4*>(ks + src + 8 * piece);
+      *reinterpret_cast<uint4*>(vr + i * D + 8 * piece) = *reinterpret_cast<const uint4*>(vs + src + 8 * piece);
+    }
+    __syncthreads();
+    for (int idx = tid; idx < rows * kPfRawBlk; idx += kGThreads) {
+      const int r = idx / kPfRawBlk, i = idx % kPfRawBlk, u = u0 + i;
+      const int ti = i0 + r / G;  // chunk index of the row's token
+      float s = -INFINITY;
+      if (i < nb && (u < tau || u - tau <= ti)) {
+        s = 0.f;
+        for (int j = 0; j < D; ++j) s += qr[r * D + j] * __half2float(kr[i * D + j]);
+      }
+      sc[r * T + i] = s;
+    }
+    __syncthreads();
+    pf_softmax_rows(sc, T, kPfRawBlk, rows, hs, 5, 6);
+    __syncthreads();
+    for (int idx = tid; idx < rows * D; idx += kGThreads) {
+      const int r = idx / D, j = idx % D;
+      float u = 0.f;
+      for (int i = 0; i < nb; ++i) u += sc[r * T + i] * __half2float(vr[i * D + j]);
+      acc2[idx] = hs[8 * r + 2] * acc2[idx] + u;
+    }
+  }
+  __syncthreads();
+
+  // ---- the one inverse rotation of the context part, the log-sum-exp merge, fp16 out
+  fwht_rows<D>(acc, rows, D);
+  __half* out = static_cast<__half*>(a.out);
+  for (int idx = tid; idx < nt * G * D; idx += kGThreads) {
+    const int r = idx / D, j = idx % D;
+    const float m1 = hs[8 * r], l1 = hs[8 * r + 1], m2 = hs[8 * r + 5], l2 = hs[8 * r + 6];
+    const float mm = fmaxf(m1, m2);
+    const float e1 = l1 > 0.f ? exp2f(m1 - mm) : 0.f, e2 = l2 > 0.f ? exp2f(m2 - mm) : 0.f;
+    const float ltot = e1 * l1 + e2 * l2;
+    const float o = e1 * acc[idx] * inv_sqrt_d<D>() * rotation_sign(a.cfg.rotation_seed, j) + e2 * acc2[idx];
+    out[(static_cast<size_t>(c0 + i0 + r / G) * Hq + h * G + r % G) * D + j] =
+        __float2half_rn(ltot > 0.f ? o / ltot : 0.f);
+  }
+}
+
 // ------------------------------------------------------------------ read-back
 // Codes, metadata, C~ and the dequantized tile in both domains, for one
 // (tile, KV head) per CTA.
@@ -688,6 +968,17 @@ cudaError_t launch_generic_decode_d(const DecodeArgs& a, cudaStream_t s, int S) 
 }
 
 template <int D>
+cudaError_t launch_generic_prefill_d(const PrefillArgs& a, cudaStream_t s) {
+  const size_t smem = gen_pf_smem(D, a.cfg.tile_tokens, gen_pf_rows<D>()).total;
+  cudaError_t e = allow_smem(gen_prefill_kernel<D>, smem);
+  if (e != cudaSuccess) return e;
+  const long long ctas = gen_pf_ctas(a.cfg, a.num_seqs, a.max_chunk);
+  gen_prefill_kernel<D><<<static_cast<unsigned>(ctas), kGThreads, smem, s>>>(a, pool_geom(a.cfg, false),
+                                                                             pool_geom(a.cfg, true));
+  return cudaGetLastError();
+}
+
+template <int D>
 cudaError_t launch_generic_unpack_d(const UnpackArgs& a, cudaStream_t s) {
   const size_t smem = static_cast<size_t>(a.cfg.tile_tokens) * D * 4;
   cudaError_t e = allow_smem(gen_unpack_kernel<D>, smem);
@@ -724,6 +1015,15 @@ cudaError_t launch_generic_decode(const DecodeArgs& a, cudaStream_t s) {
   }
   const int S = gen_splits(a.num_seqs, a.cfg.num_kv_heads, a.num_splits_fixed, sms);
   return a.cfg.head_dim == 64 ? launch_generic_decode_d<64>(a, s, S) : launch_generic_decode_d<256>(a, s, S);
+}
+
+long long generic_prefill_ctas(const kvq_config& cfg, int num_seqs, int max_chunk) {
+  return gen_pf_ctas(cfg, num_seqs, max_chunk);
+}
+
+cudaError_t launch_generic_prefill(const PrefillArgs& a, cudaStream_t s) {
+  if (a.num_seqs == 0 || a.max_chunk == 0) return cudaSuccess;
+  return a.cfg.head_dim == 64 ? launch_generic_prefill_d<64>(a, s) : launch_generic_prefill_d<256>(a, s);
 }
 
 cudaError_t launch_generic_unpack(const UnpackArgs& a, cudaStream_t s) {

@@ -156,6 +156,10 @@ cudaError_t launch_generic_append(const AppendArgs& a, cudaStream_t s);
 cudaError_t launch_generic_decode(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_generic_unpack(const UnpackArgs& a, cudaStream_t s);
 size_t generic_decode_workspace_bytes(const kvq_config& cfg, int num_seqs, int num_splits, int num_sms);
+// chunked prefill at d = 64 / 256: one launch, no workspace, any num_splits
+// (the context is not split); CTAs of the launch
+cudaError_t launch_generic_prefill(const PrefillArgs& a, cudaStream_t s);
+long long generic_prefill_ctas(const kvq_config& cfg, int num_seqs, int max_chunk);
 
 // Self-tests of the bounded mbarrier waits (one per kernel file): a wait on
 // a barrier nothing arrives at gives up after its limit and records

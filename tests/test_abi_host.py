@@ -144,8 +144,16 @@ def test_prefill_argument_errors_launch_nothing(lib):
         return lib.kvq_paged_prefill_attention(ctypes.byref(conf), q, 16, 16, 16, 16, 16, num_seqs, max_chunk,
                                                tables, 4, 8, 16, 16, 16, 16, scale, splits, ws, ws_bytes, None,
                                                None)
-    c64 = kvq.Config(num_kv_heads=2, group_size=4, tile_tokens=64, bits_k=4, bits_v=4, iters=4, head_dim=64).c()
-    assert call(c64) == kvq.KVQ_ERR_UNSUPPORTED
+    # head sizes 64 and 256: one launch over the whole context, no workspace
+    # for any split count (checked, then ignored); argument errors as at d = 128
+    for d in (64, 256):
+        cfg_d = kvq.Config(num_kv_heads=2, group_size=4, tile_tokens=64, bits_k=4, bits_v=4, iters=4, head_dim=d)
+        assert all(kvq.prefill_workspace_bytes(cfg_d, 3, 40, s) == 0 for s in (1, 3, 64))
+        c_d = cfg_d.c()
+        assert call(c_d, splits=65) == kvq.KVQ_ERR_INVALID_ARG
+        assert call(c_d, q=None) == kvq.KVQ_ERR_INVALID_ARG
+        assert call(c_d, num_seqs=70000) == kvq.KVQ_ERR_INVALID_ARG
+        assert call(c_d, num_seqs=0) == kvq.KVQ_OK
     # 3-bit pages are read: past the configuration checks, to the workspace check
     c3 = kvq.Config(num_kv_heads=2, group_size=4, tile_tokens=64, bits_k=4, bits_v=3, iters=4).c()
     assert call(c3, splits=2, ws=16, ws_bytes=16) == kvq.KVQ_ERR_WORKSPACE

@@ -1,17 +1,18 @@
 """Head sizes d = 64 and 256 (the method's rotation along the head-dim
 channels of any head size: axbrief.com KVarN article, "What differs from
-existing methods"): quantize, append and decode through the C ABI against the
-oracle, with the same bars as the d = 128 tests."""
+existing methods"): quantize, append, decode and chunked prefill through the
+C ABI against the oracle, with the same bars as the d = 128 tests."""
 
 import numpy as np
 import pytest
 import torch
 
+from oracle import kvq_oracle as o
 from quantized_paged_kv_tile_b200 import kvq, synth
 from quantized_paged_kv_tile_b200.paged import PagedKVCache
 
-from parity_helpers import (ATTN_REL_L2_MAX, TileStats, compare_sequence_tiles, decode_over_gpu_pages, make_cache,
-                            rel_l2)
+from parity_helpers import (ATTN_REL_L2_MAX, TileStats, compare_sequence_tiles, decode_over_gpu_pages,
+                            gpu_pages_kv_hat, make_cache, rel_l2)
 
 pytestmark = pytest.mark.gpu
 
@@ -157,3 +158,79 @@ def test_decode_independent_of_split_count(d):
     outs = [cache.decode(q, num_splits=s).float().cpu().numpy() for s in (1, 2, 7, 20, 0)]
     for other in outs[1:]:
         assert rel_l2(other, outs[0]) <= 1e-4
+
+
+PREFILL_CASES = [
+    # (d, T, bits_k, bits_v, g, context lengths, chunk lengths)
+    (64, 64, 4, 4, 4, (300, 64, 0), (40, 33, 17)),   # ragged tails, a tail-free context, an empty context
+    (64, 32, 2, 3, 8, (100, 31), (20, 1)),           # 3-bit V, a context that is all tail
+    (64, 128, 8, 8, 1, (260,), (70,)),               # g = 1: 32 chunk tokens per CTA, three runs
+    (256, 64, 4, 2, 8, (200, 70), (9, 30)),          # 2 chunk tokens per CTA
+    (256, 128, 3, 4, 2, (300,), (25,)),
+    (256, 32, 2, 2, 4, (97, 64), (0, 40)),           # a sequence with an empty chunk
+]
+
+
+@pytest.mark.parametrize("d,t,bk,bv,g,ctx,chunk", PREFILL_CASES)
+def test_prefill_attention_matches_oracle(d, t, bk, bv, g, ctx, chunk):
+    # chunk token i attends to the cached context (the GPU's own pages, read
+    # back by the oracle, then the raw tail) and to chunk rows 0..i: fp64
+    # attention held to 1e-3 per (chunk token, query head); the result does
+    # not depend on the split count (the context is not split at these sizes)
+    w = synth.workload("tiny", num_seqs=len(ctx), lens=tuple(ctx), num_kv_heads=2, group_size=g, tile_tokens=t,
+                       bits_k=bk, bits_v=bv, iters=2, head_dim=d)
+    cfg, cache, _, _ = _prefilled(w, extra_tokens=max(chunk))
+    n = int(sum(chunk))
+    k_new = synth.kv_rows(w, "k", max(n, 1), device="cuda", stream_id=3)[:n]
+    v_new = synth.kv_rows(w, "v", max(n, 1), device="cuda", stream_id=3)[:n]
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(7100 + d)
+    q = torch.randn((n, w.num_q_heads, d), generator=gen, device="cuda").to(torch.float16)
+    out = cache.prefill_chunk(q, k_new, v_new, chunk, append=False)
+    again = cache.prefill_chunk(q, k_new, v_new, chunk, append=False, num_splits=5)
+    torch.cuda.synchronize()
+    assert cache.status() == 0
+    assert torch.equal(out, again)
+    qh, kh, vh, oh = (x.float().cpu().numpy() for x in (q, k_new, v_new, out))
+    assert np.all(np.isfinite(oh))
+    starts = np.concatenate([[0], np.cumsum(chunk)]).astype(np.int64)
+    for s, c in enumerate(chunk):
+        if c == 0:
+            continue
+        k_hat = [gpu_pages_kv_hat(cfg, cache, s, h, int(ctx[s]), False) for h in range(cfg.num_kv_heads)]
+        v_hat = [gpu_pages_kv_hat(cfg, cache, s, h, int(ctx[s]), True) for h in range(cfg.num_kv_heads)]
+        a, b = starts[s], starts[s] + c
+        ref = o.prefill_chunk_sequence(qh[a:b], k_hat, v_hat, kh[a:b], vh[a:b], cfg.group_size)
+        for i in range(c):
+            for hq in range(cfg.num_q_heads):
+                assert rel_l2(oh[a + i, hq], ref[i, hq]) <= ATTN_REL_L2_MAX, (s, i, hq)
+
+
+@pytest.mark.parametrize("d", [64, 256])
+def test_prefill_chunk_then_append_matches_one_prefill(d):
+    # attention, then the chunk joins the cache (tiles it completes are
+    # quantized): pages and tails equal to one prefill of context + chunk
+    ctx, chunk = (130, 64, 5), (70, 1, 200)
+    w = synth.workload("tiny", num_seqs=3, lens=ctx, num_kv_heads=2, group_size=4, tile_tokens=64, bits_k=4,
+                       bits_v=2, iters=2, head_dim=d)
+    cfg, a, _, _ = _prefilled(w, extra_tokens=max(chunk))
+    n = int(sum(chunk))
+    k_new = synth.kv_rows(w, "k", n, device="cuda", stream_id=4)
+    v_new = synth.kv_rows(w, "v", n, device="cuda", stream_id=4)
+    q = torch.zeros((n, w.num_q_heads, d), dtype=torch.float16, device="cuda")
+    a.prefill_chunk(q, k_new, v_new, chunk)
+    rk = synth.kv_rows(w, "k", int(sum(ctx)), device="cuda")
+    rv = synth.kv_rows(w, "v", int(sum(ctx)), device="cuda")
+    cs, ns = np.concatenate([[0], np.cumsum(ctx)]), np.concatenate([[0], np.cumsum(chunk)])
+    full_k = torch.cat([torch.cat([rk[cs[s]:cs[s + 1]], k_new[ns[s]:ns[s + 1]]]) for s in range(3)])
+    full_v = torch.cat([torch.cat([rv[cs[s]:cs[s + 1]], v_new[ns[s]:ns[s + 1]]]) for s in range(3)])
+    totals = [c + m for c, m in zip(ctx, chunk)]
+    _, b = make_cache(w, extra_tokens=max(chunk))
+    b.prefill(full_k, full_v, totals)
+    torch.cuda.synchronize()
+    assert a.status() == 0 and b.status() == 0
+    for s, L in enumerate(totals):
+        used = a.block_tables[s, :(L // 64) * 4].long()
+        assert torch.equal(a.k_pool[used], b.k_pool[used]) and torch.equal(a.v_pool[used], b.v_pool[used])
+        assert torch.equal(a.k_tail[s, :, :L % 64], b.k_tail[s, :, :L % 64])
+        assert torch.equal(a.v_tail[s, :, :L % 64], b.v_tail[s, :, :L % 64])
