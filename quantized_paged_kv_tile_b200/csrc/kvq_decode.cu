@@ -782,6 +782,17 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
     const int F = loc.L / T;
     const int t0 = loc.c * loc.ch, t1 = min(F, t0 + loc.ch);
 
+    // block id of page `lane` (< NP) of tile `tile` of sequence b, -1 past the table
+    auto tile_blk = [&](int tile) {
+      const int lb = tile * NP + lane;
+      return lane < NP && lb < a.max_blocks_per_seq
+                 ? a.block_tables[static_cast<size_t>(b) * a.max_blocks_per_seq + lb] : -1;
+    };
+    // the first two tiles' block ids are read before the query, so that both
+    // reads are in flight together
+    const int blk0 = t0 < t1 ? tile_blk(t0) : -1;
+    const int blk1 = t0 + 1 < t1 ? tile_blk(t0 + 1) : -1;
+
     // ---- rotated, scaled query: lane (g, t) holds channels 32t..32t+31 of head g
     float qs[32];
     if (head_live) {
@@ -835,13 +846,9 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
 #pragma unroll
     for (int i = 0; i < 32; ++i) acc[i] = 0.f;
 
-    // ---- issue the first two tiles
-    auto issue = [&](int tile, int st) {
-      // lanes 0..NP-1 read and check the block ids of the tile's pages
-      const int lb = tile * NP + lane;
-      int blk = -1;
-      if (lane < NP)
-        blk = lb < a.max_blocks_per_seq ? a.block_tables[static_cast<size_t>(b) * a.max_blocks_per_seq + lb] : -1;
+    // ---- copies of a tile's pages into stage st; lanes 0..NP-1 hold the
+    // block ids of its pages and check them
+    auto issue = [&](int blk, int st) {
       const bool bad = lane < NP && (blk < 0 || blk >= a.num_blocks);
       if (__any_sync(kFull, bad)) {
         if (lane == 0) report_error(a.dev_status, KVQ_ERR_DEVICE_BOUNDS);
@@ -858,13 +865,18 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
       }
       pending[st] = true;
     };
-    if (t0 < t1) issue(t0, 0);
-    if (t0 + 1 < t1) issue(t0 + 1, 1);
+    if (t0 < t1) issue(blk0, 0);
+    if (t0 + 1 < t1) issue(blk1, 1);
 
     for (int i = t0; i < t1; ++i) {
       const int st = (i - t0) & 1;
+      // T <= 64: the block ids of tile i + 2 are read now and used after this
+      // tile's work; at T = 128 the extra live register costs more spills
+      // than the read's latency
+      constexpr bool kEarlyIds = T <= 64;
+      const int blk_next = kEarlyIds && i + 2 < t1 ? tile_blk(i + 2) : -1;
       if (!pending[st]) {  // tile skipped (bad block id, already reported)
-        if (i + 2 < t1) issue(i + 2, st);
+        if (i + 2 < t1) issue(kEarlyIds ? blk_next : tile_blk(i + 2), st);
         continue;
       }
       if (!mbar_wait_bounded(&bars[st], phase[st])) {
@@ -1082,7 +1094,7 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
       }
       }
       __syncwarp();
-      if (i + 2 < t1) issue(i + 2, st);
+      if (i + 2 < t1) issue(kEarlyIds ? blk_next : tile_blk(i + 2), st);
     }
     if (failed) break;
 
