@@ -151,6 +151,12 @@ __device__ __forceinline__ uint32_t field3(const uint32_t (&w)[N], int k) {
   if (sh <= 29) return (w[i] >> sh) & 7u;
   return __funnelshift_r(w[i], w[i + 1], sh) & 7u;
 }
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // two codes as an fp16 pair of exact small integers (low half `lo`)
 __device__ __forceinline__ uint32_t code_pair_f16(uint32_t lo, uint32_t hi) {
   return h2_as_u32(__hsub2(u32_as_h2(lo | (hi << 16) | 0x64006400u), __float2half2_rn(1024.f)));
@@ -793,8 +799,10 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
     const int blk0 = t0 < t1 ? tile_blk(t0) : -1;
     const int blk1 = t0 + 1 < t1 ? tile_blk(t0 + 1) : -1;
 
-    // ---- rotated, scaled query: lane (g, t) holds channels 32t..32t+31 of head g
-    float qs[32];
+    // ---- rotated, scaled query: lane (g, t) holds channels 32t..32t+31 of head g,
+    // as pairs (2i, 2i + 1) for the packed f32x2 arithmetic of the q'' fragments
+    float2 qs[16];
+    auto qch = [&](int i) -> float& { return (i & 1) ? qs[i >> 1].y : qs[i >> 1].x; };
     if (head_live) {
       const __half* qp = static_cast<const __half*>(a.q) +
                          ((static_cast<size_t>(b) * nh + h) * G + g) * kHeadDim + 32 * t;
@@ -803,19 +811,15 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
         const uint4 raw = *reinterpret_cast<const uint4*>(qp + 8 * v);
         const __half2* hp = reinterpret_cast<const __half2*>(&raw);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float2 f = __half22float2(hp[k]);
-          qs[8 * v + 2 * k] = f.x;
-          qs[8 * v + 2 * k + 1] = f.y;
-        }
+        for (int k = 0; k < 4; ++k) qs[4 * v + k] = __half22float2(hp[k]);
       }
     } else {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) qs[i] = 0.f;
+      for (int i = 0; i < 16; ++i) qs[i] = make_float2(0.f, 0.f);
     }
     if (a.cfg.rotation_seed != 0) {  // q' = H D_s q
 #pragma unroll
-      for (int i = 0; i < 32; ++i) qs[i] *= rotation_sign(a.cfg.rotation_seed, 32 * t + i);
+      for (int i = 0; i < 32; ++i) qch(i) *= rotation_sign(a.cfg.rotation_seed, 32 * t + i);
     }
 #pragma unroll
     for (int bit = 0; bit < 5; ++bit) {  // channel bits 0..4: in-register butterflies
@@ -823,9 +827,9 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
 #pragma unroll
       for (int i = 0; i < 32; ++i)
         if (!(i & m)) {
-          const float x = qs[i], y = qs[i | m];
-          qs[i] = x + y;
-          qs[i | m] = x - y;
+          const float x = qch(i), y = qch(i | m);
+          qch(i) = x + y;
+          qch(i | m) = x - y;
         }
     }
 #pragma unroll
@@ -834,17 +838,20 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
       const bool upper = t & m;
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const float o = __shfl_xor_sync(kFull, qs[i], m);
-        qs[i] = upper ? (o - qs[i]) : (qs[i] + o);
+        const float o = __shfl_xor_sync(kFull, qch(i), m);
+        qch(i) = upper ? (o - qch(i)) : (qch(i) + o);
       }
     }
 #pragma unroll
-    for (int i = 0; i < 32; ++i) qs[i] *= qscale;
+    for (int i = 0; i < 16; ++i) qs[i] = __fmul2_rn(qs[i], make_float2(qscale, qscale));
 
-    float m_run = -INFINITY, l_part = 0.f;
-    float acc[32];
+    // running max; the softmax sum and the accumulator (channels 8nv + 2t,
+    // 8nv + 2t + 1 in acc[nv]) as f32x2 pairs
+    float m_run = -INFINITY;
+    float2 l_part = make_float2(0.f, 0.f);
+    float2 acc[16];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+    for (int i = 0; i < 16; ++i) acc[i] = make_float2(0.f, 0.f);
 
     // ---- copies of a tile's pages into stage st; lanes 0..NP-1 hold the
     // block ids of its pages and check them
@@ -898,8 +905,9 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
       // are kept.
       constexpr int kPcMax = (BK == 8 || BK == 3) ? 2 : 4;
       constexpr int kPc = NP < kPcMax ? NP : kPcMax;
+      float2 sig2 = make_float2(0.f, 0.f);
       float sig = 0.f;
-      float sc[NP][2][2];
+      float2 sc[NP][2];  // scores of tokens 8nb + 2t, 8nb + 2t + 1 of each page
       float mt = -INFINITY;
       // C~K of channels 32t + c, c + 1 (c even) within the tile's page slices
       auto ck_pair = [&](int c) {
@@ -965,14 +973,16 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
             const int kb = wd * kbPerWord + j;
             // pairs 2kb, 2kb+1: channels (c0, c1) and (c0+1, c1+1), c0 even
             const int c0 = pair_ch0<BK>(2 * kb), c1 = c0 + pair_gap<BK>();
-            const float2 ka = ck_pair(c0), kc = ck_pair(c1);
-            const float x00 = qs[c0] * ka.x, x01 = qs[c0 + 1] * ka.y;
-            const float x10 = qs[c1] * kc.x, x11 = qs[c1 + 1] * kc.y;
-            if (pc == 0) sig += (x00 + x01) + (x10 + x11);
-            const __half2 h0 = __floats2half2_rn(x00, x10), h1 = __floats2half2_rn(x01, x11);
+            const float2 x0 = __fmul2_rn(qs[c0 >> 1], ck_pair(c0));  // channels c0, c0 + 1
+            const float2 x1 = __fmul2_rn(qs[c1 >> 1], ck_pair(c1));  // channels c1, c1 + 1
+            if (pc == 0) sig2 = __fadd2_rn(sig2, __fadd2_rn(x0, x1));
+            // hi = fp16(x), lo = fp16(x - hi); A rows g / g + 8 take channels (c0, c1) / (c0 + 1, c1 + 1)
+            const __half2 h0 = __floats2half2_rn(x0.x, x1.x), h1 = __floats2half2_rn(x0.y, x1.y);
             const float2 f0 = __half22float2(h0), f1 = __half22float2(h1);
-            const uint32_t afr[4] = {h2_as_u32(h0), h2_as_u32(__floats2half2_rn(x00 - f0.x, x10 - f0.y)),
-                                     h2_as_u32(h1), h2_as_u32(__floats2half2_rn(x01 - f1.x, x11 - f1.y))};
+            const float2 r0 = __fadd2_rn(x0, make_float2(-f0.x, -f1.x));
+            const float2 r1 = __fadd2_rn(x1, make_float2(-f0.y, -f1.y));
+            const uint32_t afr[4] = {h2_as_u32(h0), h2_as_u32(__floats2half2_rn(r0.x, r1.x)),
+                                     h2_as_u32(h1), h2_as_u32(__floats2half2_rn(r0.y, r1.y))};
 #pragma unroll
             for (int pg = 0; pg < kPc; ++pg)
 #pragma unroll
@@ -980,6 +990,7 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
           }
         }
         if (pc == 0) {
+          sig = sig2.x + sig2.y;
           sig += __shfl_xor_sync(kFull, sig, 1);
           sig += __shfl_xor_sync(kFull, sig, 2);
         }
@@ -988,11 +999,14 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
           const unsigned char* meta = sK + (pc + pg) * Geo::kPageK + Geo::kCodesK;
 #pragma unroll
           for (int nb = 0; nb < 2; ++nb) {
+            // (s~, z~) of tokens 2t, 2t + 1 -> (s~, s~) and (z~, z~) pairs
             const uint2 mm = *reinterpret_cast<const uint2*>(meta + 4 * (8 * nb + 2 * t));
-            const float2 m0 = __half22float2(u32_as_h2(mm.x)), m1 = __half22float2(u32_as_h2(mm.y));
-            sc[pc + pg][nb][0] = m0.x * (sd[pg][nb][0] + sd[pg][nb][2]) + m0.y * sig;
-            sc[pc + pg][nb][1] = m1.x * (sd[pg][nb][1] + sd[pg][nb][3]) + m1.y * sig;
-            mt = fmaxf(mt, fmaxf(sc[pc + pg][nb][0], sc[pc + pg][nb][1]));
+            const float2 sk = __half22float2(u32_as_h2(__byte_perm(mm.x, mm.y, 0x5410)));
+            const float2 zk = __half22float2(u32_as_h2(__byte_perm(mm.x, mm.y, 0x7632)));
+            const float2 dot = __fadd2_rn(make_float2(sd[pg][nb][0], sd[pg][nb][1]),
+                                          make_float2(sd[pg][nb][2], sd[pg][nb][3]));  // hi + lo rows
+            sc[pc + pg][nb] = __ffma2_rn(sk, dot, __fmul2_rn(zk, make_float2(sig, sig)));
+            mt = max3f(mt, sc[pc + pg][nb].x, sc[pc + pg][nb].y);
           }
         }
       }
@@ -1001,28 +1015,32 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
       const float m_new = fmaxf(m_run, mt);
       const float alpha = exp2f(m_run - m_new);
       m_run = m_new;
-      l_part *= alpha;
+      l_part = __fmul2_rn(l_part, make_float2(alpha, alpha));
 
       // -- P = p * s~V as hi/lo fp16 A fragments per page; w = sum p z~V
       uint32_t pa[NP][4];
-      float wsum = 0.f;
+      float2 w2 = make_float2(0.f, 0.f);
 #pragma unroll
       for (int pg = 0; pg < NP; ++pg) {
         const unsigned char* meta = sV + pg * Geo::kPageV + Geo::kCodesV;
 #pragma unroll
         for (int nb = 0; nb < 2; ++nb) {
           const uint2 mm = *reinterpret_cast<const uint2*>(meta + 4 * (8 * nb + 2 * t));
-          const float2 m0 = __half22float2(u32_as_h2(mm.x)), m1 = __half22float2(u32_as_h2(mm.y));
-          const float p0 = exp2f(sc[pg][nb][0] - m_new), p1 = exp2f(sc[pg][nb][1] - m_new);
-          l_part += p0 + p1;
-          wsum += p0 * m0.y + p1 * m1.y;
-          const float x0 = p0 * m0.x, x1 = p1 * m1.x;
-          const __half2 hv = __floats2half2_rn(x0, x1);
+          const float2 sv = __half22float2(u32_as_h2(__byte_perm(mm.x, mm.y, 0x5410)));
+          const float2 zv = __half22float2(u32_as_h2(__byte_perm(mm.x, mm.y, 0x7632)));
+          const float2 e = __fadd2_rn(sc[pg][nb], make_float2(-m_new, -m_new));
+          const float2 p = make_float2(exp2f(e.x), exp2f(e.y));
+          l_part = __fadd2_rn(l_part, p);
+          w2 = __ffma2_rn(p, zv, w2);
+          const float2 x = __fmul2_rn(p, sv);
+          const __half2 hv = __floats2half2_rn(x.x, x.y);
           const float2 hf = __half22float2(hv);
+          const float2 r = __fadd2_rn(x, make_float2(-hf.x, -hf.y));
           pa[pg][2 * nb] = h2_as_u32(hv);
-          pa[pg][2 * nb + 1] = h2_as_u32(__floats2half2_rn(x0 - hf.x, x1 - hf.y));
+          pa[pg][2 * nb + 1] = h2_as_u32(__floats2half2_rn(r.x, r.y));
         }
       }
+      float wsum = w2.x + w2.y;
       wsum += __shfl_xor_sync(kFull, wsum, 1);
       wsum += __shfl_xor_sync(kFull, wsum, 2);
 
@@ -1054,9 +1072,9 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
           const int c0 = 8 * nv + 2 * t;
           const __half2 cvh = *reinterpret_cast<const __half2*>(sV + (c0 / Geo::kCs) * Geo::kPageV + Geo::kCodesV +
                                                                 64 + 2 * (c0 % Geo::kCs));
-          const float2 cv = __half22float2(cvh);
-          acc[2 * nv] = alpha * acc[2 * nv] + cv.x * (dv[0] + dv[2] + wsum);
-          acc[2 * nv + 1] = alpha * acc[2 * nv + 1] + cv.y * (dv[1] + dv[3] + wsum);
+          const float2 u = __fadd2_rn(__fadd2_rn(make_float2(dv[0], dv[1]), make_float2(dv[2], dv[3])),
+                                      make_float2(wsum, wsum));
+          acc[nv] = __ffma2_rn(make_float2(alpha, alpha), acc[nv], __fmul2_rn(__half22float2(cvh), u));
         }
       } else {
       constexpr int kPairsV = 16 / BV;      // n-blocks per word pair
@@ -1087,9 +1105,9 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
           const int c0 = 8 * nv + 2 * t;
           const __half2 cvh = *reinterpret_cast<const __half2*>(sV + (c0 / Geo::kCs) * Geo::kPageV + Geo::kCodesV +
                                                                 64 + 2 * (c0 % Geo::kCs));
-          const float2 cv = __half22float2(cvh);
-          acc[2 * nv] = alpha * acc[2 * nv] + cv.x * (dv[e][0] + dv[e][2] + wsum);
-          acc[2 * nv + 1] = alpha * acc[2 * nv + 1] + cv.y * (dv[e][1] + dv[e][3] + wsum);
+          const float2 u = __fadd2_rn(__fadd2_rn(make_float2(dv[e][0], dv[e][1]), make_float2(dv[e][2], dv[e][3])),
+                                      make_float2(wsum, wsum));
+          acc[nv] = __ffma2_rn(make_float2(alpha, alpha), acc[nv], __fmul2_rn(__half22float2(cvh), u));
         }
       }
       }
@@ -1099,7 +1117,8 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
     if (failed) break;
 
     // ---- partial of this unit
-    float l_tot = l_part + __shfl_xor_sync(kFull, l_part, 1);
+    float l_tot = l_part.x + l_part.y;
+    l_tot += __shfl_xor_sync(kFull, l_tot, 1);
     l_tot += __shfl_xor_sync(kFull, l_tot, 2);
     if (head_live) {
       float* part = parts + (static_cast<size_t>(u) * G + g) * kPartFloats;
@@ -1110,7 +1129,7 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
 #pragma unroll
       for (int nv = 0; nv < 16; ++nv) {
         const int c0 = 8 * nv + 2 * t;
-        *reinterpret_cast<float2*>(part + kPartAcc + c0) = make_float2(acc[2 * nv], acc[2 * nv + 1]);
+        *reinterpret_cast<float2*>(part + kPartAcc + c0) = acc[nv];
       }
     }
     loc = locate_unit<T>(a, u, prefix, chunk);
