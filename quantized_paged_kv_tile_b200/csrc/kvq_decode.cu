@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(1024) decode_schedule_kernel(const int32_t* se
                                                                int num_kv_heads, int group, int num_splits,
                                                                int target_units, void* workspace) {
   __shared__ long long s_total;
-  __shared__ int s_scan[1024];
+  __shared__ int s_warp[32];
   __shared__ int s_key[1024];
   __shared__ int s_idx[1024];
   __shared__ int s_carry;
@@ -193,13 +193,16 @@ __global__ void __launch_bounds__(1024) decode_schedule_kernel(const int32_t* se
     s_carry = 0;
   }
   __syncthreads();
-  long long part = 0;
-  for (int b = tid; b < num_seqs; b += blockDim.x) part += max(seq_lens[b], 0) / tile_tokens;
+  // full tiles per sequence, read once (sequences past the block size are
+  // read again below, in the order given)
+  const bool sorted = num_seqs <= static_cast<int>(blockDim.x);
+  const int f_own = tid < num_seqs ? max(seq_lens[tid], 0) / tile_tokens : -1;
+  long long part = f_own > 0 ? f_own : 0;
+  for (int b = tid + blockDim.x; b < num_seqs; b += blockDim.x) part += max(seq_lens[b], 0) / tile_tokens;
   atomicAdd(reinterpret_cast<unsigned long long*>(&s_total), static_cast<unsigned long long>(part));
   // dispatch order: longest first when the sequences fit one sort, else as given
-  const bool sorted = num_seqs <= static_cast<int>(blockDim.x);
   if (sorted) {
-    s_key[tid] = tid < num_seqs ? max(seq_lens[tid], 0) / tile_tokens : -1;
+    s_key[tid] = f_own;
     s_idx[tid] = tid;
     int n = 1;  // the sort spans the next power of two of the sequence count
     while (n < num_seqs) n <<= 1;
@@ -241,7 +244,7 @@ __global__ void __launch_bounds__(1024) decode_schedule_kernel(const int32_t* se
     int units = 0;
     if (i < num_seqs) {
       const int b = sorted ? s_idx[i] : i;
-      const int f = max(seq_lens[b], 0) / tile_tokens;
+      const int f = sorted ? s_key[i] : max(seq_lens[b], 0) / tile_tokens;
       int ch;
       if (num_splits > 0) {
         const int sp = min(num_splits, f);
@@ -254,17 +257,31 @@ __global__ void __launch_bounds__(1024) decode_schedule_kernel(const int32_t* se
       units = f > 0 ? (f + ch - 1) / ch : 1;
       chunk[b] = ch;
     }
-    s_scan[tid] = units;
-    __syncthreads();
-    for (int off = 1; off < static_cast<int>(blockDim.x); off <<= 1) {  // inclusive scan
-      const int v = tid >= off ? s_scan[tid - off] : 0;
-      __syncthreads();
-      s_scan[tid] += v;
-      __syncthreads();
+    // inclusive scan of units over the block: within warps by shuffles, then
+    // over the warp totals
+    const int lane = tid & 31, wid = tid >> 5, nw = blockDim.x >> 5;
+    int incl = units;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(kFull, incl, off);
+      if (lane >= off) incl += v;
     }
-    if (i < num_seqs) prefix[i] = s_carry + s_scan[tid] - units;
+    if (lane == 31) s_warp[wid] = incl;
     __syncthreads();
-    if (tid == blockDim.x - 1) s_carry += s_scan[tid];
+    if (wid == 0) {
+      int w = lane < nw ? s_warp[lane] : 0;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(kFull, w, off);
+        if (lane >= off) w += v;
+      }
+      if (lane < nw) s_warp[lane] = w;  // inclusive over warps
+    }
+    __syncthreads();
+    incl += (wid > 0 ? s_warp[wid - 1] : 0);
+    if (i < num_seqs) prefix[i] = s_carry + incl - units;
+    __syncthreads();
+    if (tid == blockDim.x - 1) s_carry += incl;
     __syncthreads();
   }
   if (tid == 0) {

@@ -292,6 +292,37 @@ def test_decode_edge_lengths():
             assert rel_l2(out[s, hq], ref[hq]) <= ATTN_REL_L2_MAX
 
 
+@pytest.mark.parametrize("num_seqs", [300, 1100])
+def test_decode_many_sequences(num_seqs):
+    # the schedule's longest-first order (a sort over up to 1024 sequences)
+    # and its block-wide scan of the units, past one warp and past one block
+    # (1100 sequences: the order as given); lengths log-uniform with empty
+    # and tail-only sequences; a seeded sample of sequences against fp64
+    # attention over the GPU's own pages
+    rng = np.random.default_rng(4242 + num_seqs)
+    lens = np.floor(np.exp(rng.uniform(0.0, math.log(700.0), num_seqs))).astype(np.int64) - 1
+    lens[:3] = (0, 31, 32)
+    w = synth.workload("tiny", num_seqs=num_seqs, lens=tuple(int(x) for x in lens), num_kv_heads=1, group_size=2,
+                       tile_tokens=32, bits_k=4, bits_v=2, iters=1)
+    cfg, cache, _, _ = _prefilled(w)
+    q = synth.queries(w, device="cuda")
+    out = cache.decode(q)
+    again = cache.decode(q, num_splits=1)
+    torch.cuda.synchronize()
+    assert cache.status() == 0
+    out_h, q_h = out.float().cpu().numpy(), q.cpu().numpy()
+    assert not out_h[0].any()
+    sample = sorted(set([1, 2, num_seqs - 1] + list(rng.choice(num_seqs, 30, replace=False))))
+    for s in sample:
+        if lens[s] == 0:
+            assert not out_h[s].any()
+            continue
+        ref = decode_over_gpu_pages(cfg, cache, s, int(lens[s]), q_h[s])
+        for hq in range(w.num_q_heads):
+            assert rel_l2(out_h[s, hq], ref[hq]) <= ATTN_REL_L2_MAX, (s, hq)
+    assert rel_l2(again.float().cpu().numpy(), out_h) <= 1e-4
+
+
 # ------------------------------------------------------------------- append
 
 @pytest.mark.parametrize("t,chunks", [(64, [1] * 70), (128, [3, 100, 1, 130, 7]), (32, [33, 1, 64, 2])])
