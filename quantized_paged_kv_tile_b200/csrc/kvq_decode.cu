@@ -1096,36 +1096,48 @@ __global__ void __launch_bounds__(DecodeGeom<T, BK, BV>::kWarps * 32, BK == 8 ? 
       } else {
       constexpr int kPairsV = 16 / BV;      // n-blocks per word pair
       constexpr int kGroups = 16 / kPairsV;  // word pairs per lane (4 at b=4, 2 at b=2)
+      // word pairs taken together, so that kQI * kPairsV accumulators chain
+      // across the pages (at least 8 MMAs between two into the same one)
+      constexpr int kQI = kPairsV >= 8 ? 1 : 8 / kPairsV > kGroups ? kGroups : 8 / kPairsV;
 #pragma unroll
-      for (int q = 0; q < kGroups; ++q) {
-        float dv[kPairsV][4];
+      for (int q0 = 0; q0 < kGroups; q0 += kQI) {
+        float dv[kQI][kPairsV][4];
 #pragma unroll
-        for (int e = 0; e < kPairsV; ++e)
+        for (int qi = 0; qi < kQI; ++qi)
 #pragma unroll
-          for (int k = 0; k < 4; ++k) dv[e][k] = 0.f;
+          for (int e = 0; e < kPairsV; ++e)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) dv[qi][e][k] = 0.f;
 #pragma unroll
         for (int pg = 0; pg < NP; ++pg) {
           const uint32_t afr[4] = {pa[pg][0], pa[pg][1], pa[pg][2], pa[pg][3]};
-          // words 2q and 2q+1 sit in the same 16-byte row of the lane; the whole
-          // row is loaded (lanes read consecutive 16-byte rows: no bank conflict)
-          const uint4 row = *reinterpret_cast<const uint4*>(sV + pg * Geo::kPageV + (((2 * q) >> 2) * 32 + lane) * 16);
-          const uint32_t w0 = (q & 1) ? row.z : row.x, w1 = (q & 1) ? row.w : row.y;
-          uint32_t p0[kPairsV], p1[kPairsV];
-          unpack_pairs<BV>(w0, p0);
-          unpack_pairs<BV>(w1, p1);
 #pragma unroll
-          for (int e = 0; e < kPairsV; ++e) mma16816(dv[e], afr, p0[e], p1[e]);
+          for (int qi = 0; qi < kQI; ++qi) {
+            const int q = q0 + qi;
+            // words 2q and 2q+1 sit in the same 16-byte row of the lane; the whole
+            // row is loaded (lanes read consecutive 16-byte rows: no bank conflict)
+            const uint4 row = *reinterpret_cast<const uint4*>(sV + pg * Geo::kPageV + (((2 * q) >> 2) * 32 + lane) * 16);
+            const uint32_t w0 = (q & 1) ? row.z : row.x, w1 = (q & 1) ? row.w : row.y;
+            uint32_t p0[kPairsV], p1[kPairsV];
+            unpack_pairs<BV>(w0, p0);
+            unpack_pairs<BV>(w1, p1);
+#pragma unroll
+            for (int e = 0; e < kPairsV; ++e) mma16816(dv[qi][e], afr, p0[e], p1[e]);
+          }
         }
 #pragma unroll
-        for (int e = 0; e < kPairsV; ++e) {
-          const int nv = kPairsV * q + e;
-          const int c0 = 8 * nv + 2 * t;
-          const __half2 cvh = *reinterpret_cast<const __half2*>(sV + (c0 / Geo::kCs) * Geo::kPageV + Geo::kCodesV +
-                                                                64 + 2 * (c0 % Geo::kCs));
-          const float2 u = __fadd2_rn(__fadd2_rn(make_float2(dv[e][0], dv[e][1]), make_float2(dv[e][2], dv[e][3])),
-                                      make_float2(wsum, wsum));
-          acc[nv] = __ffma2_rn(make_float2(alpha, alpha), acc[nv], __fmul2_rn(__half22float2(cvh), u));
-        }
+        for (int qi = 0; qi < kQI; ++qi)
+#pragma unroll
+          for (int e = 0; e < kPairsV; ++e) {
+            const int nv = kPairsV * (q0 + qi) + e;
+            const int c0 = 8 * nv + 2 * t;
+            const __half2 cvh = *reinterpret_cast<const __half2*>(sV + (c0 / Geo::kCs) * Geo::kPageV + Geo::kCodesV +
+                                                                  64 + 2 * (c0 % Geo::kCs));
+            const float2 u = __fadd2_rn(
+                __fadd2_rn(make_float2(dv[qi][e][0], dv[qi][e][1]), make_float2(dv[qi][e][2], dv[qi][e][3])),
+                make_float2(wsum, wsum));
+            acc[nv] = __ffma2_rn(make_float2(alpha, alpha), acc[nv], __fmul2_rn(__half22float2(cvh), u));
+          }
       }
       }
       __syncwarp();
