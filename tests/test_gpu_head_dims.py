@@ -234,3 +234,72 @@ def test_prefill_chunk_then_append_matches_one_prefill(d):
         assert torch.equal(a.k_pool[used], b.k_pool[used]) and torch.equal(a.v_pool[used], b.v_pool[used])
         assert torch.equal(a.k_tail[s, :, :L % 64], b.k_tail[s, :, :L % 64])
         assert torch.equal(a.v_tail[s, :, :L % 64], b.v_tail[s, :, :L % 64])
+
+
+def _chunk_setup(d, ctx, chunk, g=4, t=64):
+    w = synth.workload("tiny", num_seqs=len(ctx), lens=tuple(ctx), num_kv_heads=2, group_size=g, tile_tokens=t,
+                       bits_k=4, bits_v=4, iters=2, head_dim=d)
+    cfg, cache, _, _ = _prefilled(w, extra_tokens=max(chunk))
+    n = int(sum(chunk))
+    k_new = synth.kv_rows(w, "k", n, device="cuda", stream_id=5)
+    v_new = synth.kv_rows(w, "v", n, device="cuda", stream_id=5)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(7300 + d)
+    q = torch.randn((n, w.num_q_heads, d), generator=gen, device="cuda").to(torch.float16)
+    return w, cfg, cache, q, k_new, v_new
+
+
+@pytest.mark.parametrize("d", [64, 256])
+def test_one_token_chunk_matches_decode_after_append(d):
+    # both GPU paths at this head size: a one-token chunk (the token raw)
+    # against appending it and decoding (the token in the tail, raw too)
+    w, cfg, cache, q, k_new, v_new = _chunk_setup(d, (300, 70, 129), (1, 1, 1))  # no tile completes
+    out = cache.prefill_chunk(q, k_new, v_new, (1, 1, 1), append=True)
+    dec = cache.decode(q)
+    torch.cuda.synchronize()
+    assert cache.status() == 0
+    a, b = out.float().cpu().numpy(), dec.float().cpu().numpy()
+    for s in range(3):
+        for hq in range(w.num_q_heads):
+            assert rel_l2(a[s, hq], b[s, hq]) <= ATTN_REL_L2_MAX
+
+
+@pytest.mark.parametrize("d", [64, 256])
+def test_prefill_chunk_longer_than_bound_is_reported(d):
+    w, cfg, cache, q, k_new, v_new = _chunk_setup(d, (200, 90), (10, 12))
+    cu = torch.tensor([0, 10, 22], dtype=torch.int32, device="cuda")
+    out = torch.full_like(q, float("nan"))
+    kvq.paged_prefill_attention(cfg, q, out, k_new, v_new, cu, cache.seq_lens, 11, cache.block_tables,
+                                cache.k_pool, cache.v_pool, cache.k_tail, cache.v_tail,
+                                num_blocks=cache.num_blocks, dev_status=cache.dev_status)
+    torch.cuda.synchronize()
+    assert cache.status() == kvq.KVQ_ERR_DEVICE_BOUNDS
+    oh = out.float().cpu().numpy()
+    assert np.all(np.isfinite(oh[:21])) and np.all(np.isnan(oh[21]))  # rows past the bound untouched
+    cache.dev_status.zero_()
+    full = cache.prefill_chunk(q, k_new, v_new, (10, 12), append=False)
+    torch.cuda.synchronize()
+    assert torch.equal(full[:21], out[:21])
+
+
+@pytest.mark.parametrize("d", [64, 256])
+def test_prefill_tile_outside_pool_is_skipped_and_reported(d):
+    # one tile of sequence 0 points outside the pool: reported, and the
+    # output is attention over the context without that tile's tokens
+    ctx, chunk = (640, 300), (24, 40)
+    w, cfg, cache, q, k_new, v_new = _chunk_setup(d, ctx, chunk)
+    k_hat = [gpu_pages_kv_hat(cfg, cache, 0, h, ctx[0], False) for h in range(cfg.num_kv_heads)]
+    v_hat = [gpu_pages_kv_hat(cfg, cache, 0, h, ctx[0], True) for h in range(cfg.num_kv_heads)]
+    bad_tile, t, per = 3, cfg.tile_tokens, cfg.tile_tokens // cfg.page_tokens
+    cache.block_tables[0, bad_tile * per + 1] = cache.num_blocks + 7
+    out = cache.prefill_chunk(q, k_new, v_new, chunk, append=False)
+    torch.cuda.synchronize()
+    assert cache.status() == kvq.KVQ_ERR_DEVICE_BOUNDS
+    keep = np.r_[0:bad_tile * t, (bad_tile + 1) * t:ctx[0]]
+    qh, kh, vh, oh = (x.float().cpu().numpy() for x in (q, k_new, v_new, out))
+    ref = o.prefill_chunk_sequence(qh[:24], [k[keep] for k in k_hat], [v[keep] for v in v_hat], kh[:24], vh[:24],
+                                   cfg.group_size)
+    for i in range(24):
+        for hq in range(cfg.num_q_heads):
+            assert rel_l2(oh[i, hq], ref[i, hq]) <= ATTN_REL_L2_MAX
+    assert np.all(np.isfinite(oh))
