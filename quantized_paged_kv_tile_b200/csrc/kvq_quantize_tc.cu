@@ -199,36 +199,46 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
 }
 
 // Shifted sums of 32 values x_k * w_k - shift with packed f32x2 arithmetic
-// (four independent accumulator chains per statistic).
-__device__ __forceinline__ void shifted_sums(const float* x, const float* w, float shift, float2 (&s1)[4],
-                                             float2 (&s2)[4]) {
+// (kChains independent accumulator chains per statistic).
+constexpr int kChains = 2;
+__device__ __forceinline__ void shifted_sums(const float* x, const float* w, float shift, float2 (&s1)[kChains],
+                                             float2 (&s2)[kChains]) {
   const float2 nk = make_float2(-shift, -shift);
 #pragma unroll
-  for (int k = 0; k < 32; k += 8) {
-    const float4 w0 = *reinterpret_cast<const float4*>(w + k);
-    const float4 w1 = *reinterpret_cast<const float4*>(w + k + 4);
-    const float2 d0 = __ffma2_rn(make_float2(x[k], x[k + 1]), make_float2(w0.x, w0.y), nk);
-    const float2 d1 = __ffma2_rn(make_float2(x[k + 2], x[k + 3]), make_float2(w0.z, w0.w), nk);
-    const float2 d2 = __ffma2_rn(make_float2(x[k + 4], x[k + 5]), make_float2(w1.x, w1.y), nk);
-    const float2 d3 = __ffma2_rn(make_float2(x[k + 6], x[k + 7]), make_float2(w1.z, w1.w), nk);
-    s1[0] = __fadd2_rn(s1[0], d0);
-    s1[1] = __fadd2_rn(s1[1], d1);
-    s1[2] = __fadd2_rn(s1[2], d2);
-    s1[3] = __fadd2_rn(s1[3], d3);
-    s2[0] = __ffma2_rn(d0, d0, s2[0]);
-    s2[1] = __ffma2_rn(d1, d1, s2[1]);
-    s2[2] = __ffma2_rn(d2, d2, s2[2]);
-    s2[3] = __ffma2_rn(d3, d3, s2[3]);
+  for (int k = 0; k < 32; k += 2 * kChains) {
+    float2 d[kChains];
+#pragma unroll
+    for (int c = 0; c < kChains; c += 2) {
+      const float4 wv = *reinterpret_cast<const float4*>(w + k + 2 * c);
+      d[c] = __ffma2_rn(make_float2(x[k + 2 * c], x[k + 2 * c + 1]), make_float2(wv.x, wv.y), nk);
+      d[c + 1] = __ffma2_rn(make_float2(x[k + 2 * c + 2], x[k + 2 * c + 3]), make_float2(wv.z, wv.w), nk);
+    }
+#pragma unroll
+    for (int c = 0; c < kChains; ++c) s1[c] = __fadd2_rn(s1[c], d[c]);
+#pragma unroll
+    for (int c = 0; c < kChains; ++c) s2[c] = __ffma2_rn(d[c], d[c], s2[c]);
   }
+}
+
+__device__ __forceinline__ float2 sum_chains(const float2 (&s)[kChains]) {
+  float2 v[kChains];
+#pragma unroll
+  for (int c = 0; c < kChains; ++c) v[c] = s[c];
+#pragma unroll
+  for (int h = kChains / 2; h > 0; h >>= 1)
+#pragma unroll
+    for (int c = 0; c < h; ++c) v[c] = __fadd2_rn(v[c], v[c + h]);
+  return v[0];
 }
 
 // (mean, M2) of n values from shifted sums (shift k): mean = k + S1/n, M2 = S2 - S1^2/n
 struct Moments {
   float mean, m2;
 };
-__device__ __forceinline__ Moments moments(const float2 (&s1)[4], const float2 (&s2)[4], float shift, float n) {
-  const float2 a2 = __fadd2_rn(__fadd2_rn(s1[0], s1[1]), __fadd2_rn(s1[2], s1[3]));
-  const float2 q2 = __fadd2_rn(__fadd2_rn(s2[0], s2[1]), __fadd2_rn(s2[2], s2[3]));
+__device__ __forceinline__ Moments moments(const float2 (&s1)[kChains], const float2 (&s2)[kChains], float shift,
+                                           float n) {
+  const float2 a2 = sum_chains(s1);
+  const float2 q2 = sum_chains(s2);
   const float a = a2.x + a2.y, q = q2.x + q2.y;
   Moments m;
   m.mean = shift + a / n;
@@ -316,8 +326,9 @@ __device__ void quantize_group_from_tmem(unsigned char* smem, uint32_t tbase, in
       for (int lt = 0; lt < kLocal; ++lt) {
         const int t = ch_tile(lt);
         if (!((valid >> t) & 1)) continue;
-        float2 s1[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-        float2 s2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        float2 s1[kChains], s2[kChains];
+#pragma unroll
+        for (int c = 0; c < kChains; ++c) s1[c] = s2[c] = make_float2(0.f, 0.f);
         float shift = 0.f;
 #pragma unroll
         for (int ch = 0; ch < T / 32; ++ch) {
@@ -333,8 +344,9 @@ __device__ void quantize_group_from_tmem(unsigned char* smem, uint32_t tbase, in
         cc[t * kRows + row] = fminf(div_fast(c, sigma), FLT_MAX);  // a zero channel keeps a finite factor
       }
     } else {
-      float2 s1[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-      float2 s2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      float2 s1[kChains], s2[kChains];
+#pragma unroll
+      for (int c = 0; c < kChains; ++c) s1[c] = s2[c] = make_float2(0.f, 0.f);
       float shift = 0.f;
 #pragma unroll
       for (int ch = 0; ch < 2; ++ch) {
@@ -371,8 +383,9 @@ __device__ void quantize_group_from_tmem(unsigned char* smem, uint32_t tbase, in
       Moments mo = {0.f, 0.f};
       const float r = rr[row];  // read before the pair barrier: the owner rewrites it below
       if (tok_live) {
-        float2 s1[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-        float2 s2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        float2 s1[kChains], s2[kChains];
+#pragma unroll
+        for (int c = 0; c < kChains; ++c) s1[c] = s2[c] = make_float2(0.f, 0.f);
         const float* cvec = cc + my_tile * kRows + 64 * hf;
         float shift = 0.f;
 #pragma unroll
