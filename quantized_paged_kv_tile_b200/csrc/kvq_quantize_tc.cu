@@ -22,8 +22,9 @@
 //           per thread) and token statistics stream D1 rows (one token per
 //           thread) out of TMEM with packed f32x2 arithmetic; the tile itself
 //           is never rewritten: Y = X' * c_j * r_i with the channel / token
-//           reciprocals c, r (exact power-of-two renormalization of (C, R)
-//           after every iteration, as in the definition)
+//           reciprocals c, r (the exact power-of-two renormalization of
+//           (C, R) runs after every second iteration and after the last:
+//           the same final (C, R) as renormalizing after every one)
 //   RTN     from D1: per-token min / max, codes, packing (K token-major, V in
 //           the decode lane order), fp16 metadata and C slices into a staging
 //           copy of the group's 8 pages, written out with cp.async.bulk.
