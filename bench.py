@@ -46,6 +46,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 METRIC = "paged decode attn GB/s & tok/s over quantized KV (% HBM peak); quantize GB/s"
 DECODE_LAUNCHES = 2  # kvq_paged_decode_attention: schedule, tiles (the merge runs inside the tiles kernel)
+E2E_CHUNKS = 8  # pieces of the fp16 rows in the end-to-end step (copy of piece k+1 overlaps quantize of piece k)
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -356,10 +357,10 @@ class StepSetup:
         # quantize; append (when there are rows to append); decode = schedule + tiles (the merge runs inside)
         self.launches = (1 if len(desc_np) else 0) + (1 if self.max_new > 0 else 0) + DECODE_LAUNCHES
 
-    def quantize(self, stream):
+    def quantize(self, stream, desc=None):
         from quantized_paged_kv_tile_b200 import kvq
-        kvq.quantize_tiles(self.cfg, self.rows_k, self.rows_v, self.desc, self.bt, self.k_pool, self.v_pool,
-                           num_blocks=self.nblocks, dev_status=self.status, stream=stream)
+        kvq.quantize_tiles(self.cfg, self.rows_k, self.rows_v, self.desc if desc is None else desc, self.bt,
+                           self.k_pool, self.v_pool, num_blocks=self.nblocks, dev_status=self.status, stream=stream)
 
     def append(self, stream):
         from quantized_paged_kv_tile_b200 import kvq
@@ -544,10 +545,77 @@ def run_kvq(args, ranks):
             ranks.barrier()
             return ranks.max(e0.elapsed_time(e1)), sum(host[nm].numel() * host[nm].element_size() for nm in names)
 
+        # the step's fp16 rows go up in E2E_CHUNKS pieces on a copy stream; each
+        # piece's tiles are quantized as soon as it has landed, so the
+        # quantization overlaps the transfer of the next piece (every copy and
+        # call is still inside the timed region)
+        copy_stream = torch.cuda.Stream(device=dev)
+        T = w.tile_tokens
+        desc_all = S.desc
+        n_desc = int(desc_all.shape[0])
+        cuts = [n_desc * c // E2E_CHUNKS for c in range(E2E_CHUNKS + 1)]
+        pieces = []
+        rows_total = int(S.rows_k.shape[0])
+        desc_host = desc_all.cpu().numpy()
+        for c in range(E2E_CHUNKS):
+            lo_d, hi_d = cuts[c], cuts[c + 1]
+            if hi_d <= lo_d:
+                continue
+            lo = 0 if not pieces else pieces[-1][1]
+            hi = rows_total if c == E2E_CHUNKS - 1 else int(desc_host[hi_d - 1, 0]) + T
+            pieces.append((lo, hi, desc_all[lo_d:hi_d].clone()))  # own allocation: 16-byte aligned
+        if pieces and pieces[-1][1] < rows_total:
+            lo, _, d = pieces[-1]
+            pieces[-1] = (lo, rows_total, d)
+
+        def step_pipelined():
+            start = torch.cuda.Event()
+            start.record(stream)
+            copy_stream.wait_event(start)
+            landed = []
+            with torch.cuda.stream(copy_stream):
+                for lo, hi, _ in pieces:
+                    S.rows_k[lo:hi].copy_(host["rows_k"][lo:hi], non_blocking=True)
+                    S.rows_v[lo:hi].copy_(host["rows_v"][lo:hi], non_blocking=True)
+                    ev = torch.cuda.Event()
+                    ev.record(copy_stream)
+                    landed.append(ev)
+                for nm in ("new_k", "new_v", "q"):
+                    getattr(S, nm).copy_(host[nm], non_blocking=True)
+                rest = torch.cuda.Event()
+                rest.record(copy_stream)
+            for (lo, hi, d), ev in zip(pieces, landed):
+                stream.wait_event(ev)
+                S.quantize(stream, desc=d)
+            stream.wait_event(rest)
+            S.append(stream)
+            S.decode(stream)
+            out_host.copy_(S.out, non_blocking=True)
+
         n = max(1, min(args.steps, 3))
-        e_ms, h2d = e2e_run(("rows_k", "rows_v", "new_k", "new_v", "q"), lambda: S.step(stream), n)
+        step_pipelined()
+        torch.cuda.synchronize(dev)
+        ranks.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            step_pipelined()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ranks.barrier()
+        e_ms = ranks.max(e0.elapsed_time(e1))
+        # the pieced step computes what the plain step computes
+        piped = out_host.clone()
+        S.step(stream)
+        torch.cuda.synchronize(dev)
+        if not torch.equal(piped, S.out.cpu()):
+            raise RuntimeError("the pieced end-to-end step differs from the plain step")
+        h2d = sum(host[nm].numel() * host[nm].element_size() for nm in ("rows_k", "rows_v", "new_k", "new_v", "q"))
         e2e = {"value": ranks.sum(step_bytes) * n / (e_ms * 1e-3) / 1e9, "unit": "GB/s",
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": n, "ms_per_step": e_ms / n}
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": n, "ms_per_step": e_ms / n,
+               "what": f"full step with its inputs from pinned host memory: the fp16 rows in {len(pieces)} pieces on a "
+                       "copy stream, each piece's tiles quantized once it has landed, then append + decode, output "
+                       "back to the host"}
         n = max(3, args.steps)
         e_ms, h2d = e2e_run(("new_k", "new_v", "q"), lambda: (S.append(stream), S.decode(stream)), n)
         dbytes = ranks.sum(bm["append"] + bm["decode"])
