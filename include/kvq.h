@@ -78,14 +78,13 @@
  * ----------
  *   d = 128 runs the tuned path (tensor-core rotation in the quantizer,
  *   mma.sync decode, tensor-core chunked prefill, the one-launch serving
- *   step).  d = 64 and d = 256 run kvq_quantize_tiles, kvq_append_tokens,
- *   kvq_paged_decode_attention (and its static-scratch form),
- *   kvq_paged_prefill_attention and kvq_unpack_tiles on CUDA-core kernels
- *   with the same format and the same method (chunked prefill there runs one
- *   launch over the whole context and needs no workspace:
- *   kvq_prefill_workspace_bytes gives 0 for every num_splits, which is
- *   checked and otherwise ignored); kvq_append_decode_step returns
- *   KVQ_ERR_UNSUPPORTED for them.
+ *   step).  d = 64 and d = 256 run every call on CUDA-core kernels with the
+ *   same format, the same method and the same contracts, with two
+ *   differences: chunked prefill runs one launch over the whole context and
+ *   needs no workspace (kvq_prefill_workspace_bytes gives 0 for every
+ *   num_splits, which is checked and otherwise ignored), and
+ *   kvq_append_decode_step runs as three launches (the tokens into the tails
+ *   and the lengths advanced, then the split-K decode and its merge).
  *
  * Conventions
  * -----------
@@ -230,7 +229,8 @@ KVQ_API kvq_status kvq_paged_decode_attention(const kvq_config* cfg, const void*
                                       size_t workspace_bytes, int num_splits,
                                       int32_t* dev_status, void* stream);
 
-/* One serving step in one launch: append one token per sequence and decode.
+/* One serving step in one launch (d = 128; three at d = 64 / 256): append one
+ * token per sequence and decode.
  * The pages say the per-step read path decides the serving gain (aitrends.kr
  * article 74976, "TL;DR"); this call folds the step's append into the
  * decode launch, for steps in which no sequence completes a tile.

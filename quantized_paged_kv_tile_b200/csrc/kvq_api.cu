@@ -275,8 +275,6 @@ kvq_status kvq_append_decode_step(const kvq_config* cfg, const void* new_k, cons
                                   void* k_tail, void* v_tail, float softmax_scale, void* workspace,
                                   size_t workspace_bytes, int num_splits, int32_t* dev_status, void* stream) {
   KVQ_TRY(check_config(cfg));
-  if (cfg->head_dim != kvq::kHeadDim)
-    return fail(KVQ_ERR_UNSUPPORTED, "the one-launch serving step is built for head_dim 128 (got %d)", cfg->head_dim);
   if (num_seqs < 0) return fail(KVQ_ERR_INVALID_ARG, "negative num_seqs");
   if (num_seqs == 0) return ok();
   if (num_seqs > 65535) return fail(KVQ_ERR_INVALID_ARG, "num_seqs > 65535");
@@ -327,6 +325,9 @@ kvq_status kvq_append_decode_step(const kvq_config* cfg, const void* new_k, cons
   a.step = 1;
   a.new_k = new_k;
   a.new_v = new_v;
+  if (cfg->head_dim != kvq::kHeadDim)  // d = 64 / 256: tail write and length update, then the decode
+    return cuda_status(kvq::launch_generic_step(a, static_cast<cudaStream_t>(stream)),
+                       "kvq_append_decode_step launch");
   return cuda_status(kvq::launch_append_decode_step(a, static_cast<cudaStream_t>(stream)),
                      "kvq_append_decode_step launch");
 }

@@ -600,6 +600,35 @@ __global__ void __launch_bounds__(kGThreads) gen_decode_merge_kernel(DecodeArgs 
   }
 }
 
+// ------------------------------------------------------------------ serving step
+// The step's token of every sequence into its tail, then the lengths advanced
+// by one (one CTA per sequence: every thread reads the length before thread 0
+// rewrites it).  A token that would complete a tile is refused (reported and
+// not written), as in the one-launch step at d = 128; the length still
+// advances.  The decode of the step follows as its own launches.
+template <int D>
+__global__ void __launch_bounds__(kGThreads) gen_step_append_kernel(DecodeArgs a) {
+  const int b = blockIdx.x, T = a.cfg.tile_tokens, nh = a.cfg.num_kv_heads;
+  const int L = max(a.seq_lens[b], 0) + 1;  // length with the step's token
+  __syncthreads();
+  if (L % T == 0) {
+    if (threadIdx.x == 0) report_error(a.dev_status, KVQ_ERR_DEVICE_BOUNDS);
+  } else {
+    const int row = (L - 1) % T;
+    for (int idx = threadIdx.x; idx < nh * (D / 8); idx += kGThreads) {
+      const int h = idx / (D / 8), piece = idx % (D / 8);
+      const size_t bh = static_cast<size_t>(b) * nh + h;
+      const size_t src = bh * D + 8 * piece, dst = (bh * T + row) * D + 8 * piece;
+      *reinterpret_cast<uint4*>(static_cast<__half*>(const_cast<void*>(a.k_tail)) + dst) =
+          *reinterpret_cast<const uint4*>(static_cast<const __half*>(a.new_k) + src);
+      *reinterpret_cast<uint4*>(static_cast<__half*>(const_cast<void*>(a.v_tail)) + dst) =
+          *reinterpret_cast<const uint4*>(static_cast<const __half*>(a.new_v) + src);
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) a.seq_lens_rw[b] = L;
+}
+
 // ------------------------------------------------------------------ prefill
 // Chunked prefill attention (aitrends.kr article 74976, "TL;DR": every phase
 // of attention reads the compressed pages directly): chunk token i of a
@@ -1019,6 +1048,17 @@ cudaError_t launch_generic_decode(const DecodeArgs& a, cudaStream_t s) {
 
 long long generic_prefill_ctas(const kvq_config& cfg, int num_seqs, int max_chunk) {
   return gen_pf_ctas(cfg, num_seqs, max_chunk);
+}
+
+cudaError_t launch_generic_step(const DecodeArgs& a, cudaStream_t s) {
+  if (a.num_seqs == 0) return cudaSuccess;
+  if (a.cfg.head_dim == 64)
+    gen_step_append_kernel<64><<<a.num_seqs, kGThreads, 0, s>>>(a);
+  else
+    gen_step_append_kernel<256><<<a.num_seqs, kGThreads, 0, s>>>(a);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_generic_decode(a, s);
 }
 
 cudaError_t launch_generic_prefill(const PrefillArgs& a, cudaStream_t s) {

@@ -159,6 +159,9 @@ size_t generic_decode_workspace_bytes(const kvq_config& cfg, int num_seqs, int n
 // chunked prefill at d = 64 / 256: one launch, no workspace, any num_splits
 // (the context is not split); CTAs of the launch
 cudaError_t launch_generic_prefill(const PrefillArgs& a, cudaStream_t s);
+// the serving step at d = 64 / 256: the step's tokens into the tails and the
+// lengths advanced (one launch), then the decode (split-K and merge launches)
+cudaError_t launch_generic_step(const DecodeArgs& a, cudaStream_t s);
 long long generic_prefill_ctas(const kvq_config& cfg, int num_seqs, int max_chunk);
 
 // Self-tests of the bounded mbarrier waits (one per kernel file): a wait on

@@ -100,9 +100,9 @@ def test_argument_errors_launch_nothing(lib):
     # misaligned pointer
     st = lib.kvq_quantize_tiles(ctypes.byref(c), 17, None, 10, 16, 1, 16, 1, 4, 8, 16, 16, None, None)
     assert st == kvq.KVQ_ERR_INVALID_ARG and "aligned" in kvq.load_library().kvq_last_error().decode()
-    # head sizes 64 and 256 decode (to the workspace check here: one split of
-    # 2 sequences x 2 KV heads x 4 query heads x (4 + d) floats); the one-launch
-    # serving step is built for d = 128 only and refuses them before any launch
+    # head sizes 64 and 256: decode and the serving step (to the workspace
+    # check here: one split of 2 sequences x 2 KV heads x 4 query heads x
+    # (4 + d) floats; 1 sequence for the step)
     for d in (64, 256):
         cd = kvq.Config(num_kv_heads=2, group_size=4, tile_tokens=64, bits_k=4, bits_v=4, iters=4, head_dim=d)
         assert kvq.decode_workspace_bytes(cd, 2, 1) == 2 * 2 * 1 * 4 * (4 + d) * 4
@@ -110,8 +110,11 @@ def test_argument_errors_launch_nothing(lib):
                                             16, 1, None, None)
         assert st == kvq.KVQ_ERR_WORKSPACE
         st = lib.kvq_append_decode_step(ctypes.byref(cd.c()), 16, 16, 16, 16, 16, 1, 16, 4, 8, 16, 16, 16, 16, 0.1,
-                                        16, 1 << 20, 1, None, None)
-        assert st == kvq.KVQ_ERR_UNSUPPORTED
+                                        16, 1 * 2 * 1 * 4 * (4 + d) * 4 - 1, 1, None, None)
+        assert st == kvq.KVQ_ERR_WORKSPACE
+        st = lib.kvq_append_decode_step(ctypes.byref(cd.c()), 16, 16, 16, 16, 16, 1, 16, 4, 8, 16, 16, 16, 16, 0.1,
+                                        16, 1 << 20, 0, None, None)
+        assert st == kvq.KVQ_ERR_INVALID_ARG  # split count 0
     # 3-bit pages are read: the call gets past the configuration checks (here
     # to the workspace check, with no device query for an explicit split count)
     c3 = kvq.Config(num_kv_heads=2, group_size=4, tile_tokens=64, bits_k=3, bits_v=4, iters=4).c()

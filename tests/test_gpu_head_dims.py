@@ -303,3 +303,48 @@ def test_prefill_tile_outside_pool_is_skipped_and_reported(d):
         for hq in range(cfg.num_q_heads):
             assert rel_l2(oh[i, hq], ref[i, hq]) <= ATTN_REL_L2_MAX
     assert np.all(np.isfinite(oh))
+
+
+@pytest.mark.parametrize("d", [64, 256])
+def test_serving_step_equals_append_then_decode(d):
+    # the serving step at this head size (tail write and length update, then
+    # the decode) against kvq_append_tokens, the lengths advanced, and
+    # kvq_paged_decode_attention with the same split count: identical outputs,
+    # tails and lengths, step after step
+    w = synth.workload("tiny", num_seqs=2, lens=(64 * 9 + 3, 64 * 4 + 9), num_kv_heads=2, group_size=4,
+                       head_dim=d)
+    cfg, a, _, _ = _prefilled(w, extra_tokens=8)
+    _, b, _, _ = _prefilled(w, extra_tokens=8)
+    ws = torch.zeros(kvq.decode_workspace_bytes(cfg, 2, 3), dtype=torch.uint8, device="cuda")
+    for i in range(8):
+        nk = synth.kv_rows(w, "k", 2, device="cuda", stream_id=1 + i)
+        nv = synth.kv_rows(w, "v", 2, device="cuda", stream_id=1 + i)
+        q = synth.queries(w, device="cuda", step=i)
+        a.append(nk, nv)
+        out_a = a.decode(q, num_splits=3)
+        out_b = torch.empty_like(q)
+        kvq.append_decode_step(cfg, nk, nv, q, out_b, b.seq_lens, b.block_tables, b.k_pool, b.v_pool, b.k_tail,
+                               b.v_tail, ws, 3, num_blocks=b.num_blocks, dev_status=b.dev_status)
+        assert torch.equal(out_a, out_b), i
+    torch.cuda.synchronize()
+    assert a.status() == 0 and b.status() == 0
+    assert torch.equal(a.seq_lens, b.seq_lens)
+    assert torch.equal(a.k_tail, b.k_tail) and torch.equal(a.v_tail, b.v_tail)
+
+
+@pytest.mark.parametrize("d", [64, 256])
+def test_serving_step_refuses_a_tile_completion(d):
+    w = synth.workload("tiny", num_seqs=2, lens=(63, 40), num_kv_heads=1, group_size=2, head_dim=d)
+    cfg, c, _, _ = _prefilled(w, extra_tokens=2)
+    ws = torch.zeros(kvq.decode_workspace_bytes(cfg, 2, 2), dtype=torch.uint8, device="cuda")
+    nk = torch.ones((2, 1, d), dtype=torch.float16, device="cuda")
+    q = synth.queries(w, device="cuda")
+    out = torch.empty_like(q)
+    tail_before = c.k_tail.clone()
+    kvq.append_decode_step(cfg, nk, nk, q, out, c.seq_lens, c.block_tables, c.k_pool, c.v_pool, c.k_tail, c.v_tail,
+                           ws, 2, num_blocks=c.num_blocks, dev_status=c.dev_status)
+    torch.cuda.synchronize()
+    assert c.status() == kvq.KVQ_ERR_DEVICE_BOUNDS
+    assert torch.equal(c.k_tail[0], tail_before[0])      # sequence 0 (63 -> 64) not written
+    assert torch.equal(c.k_tail[1, 0, 40], nk[1, 0])     # sequence 1 appended at row 40
+    assert c.seq_lens.tolist() == [64, 41]
