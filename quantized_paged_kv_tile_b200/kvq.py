@@ -274,7 +274,7 @@ def prefill_splits(cfg: Config, num_seqs: int, max_chunk_tokens: int, max_contex
                    num_sms: int) -> int:
     """A context split count for kvq_paged_prefill_attention: the smallest S
     (each split keeping at least 16 tiles) whose CTA count fills its last wave
-    to 95%, else the best fill found."""
+    to 99%, else the best fill found."""
     units = num_seqs * cfg.num_kv_heads * -(-max_chunk_tokens * cfg.group_size // 128)
     if units == 0:
         return 1
@@ -285,7 +285,7 @@ def prefill_splits(cfg: Config, num_seqs: int, max_chunk_tokens: int, max_contex
             break
         n = units * s
         fill = n / (-(-n // num_sms) * num_sms)
-        if fill >= 0.95:
+        if fill >= 0.99:
             return s
         if fill > best_fill + 1e-9:
             best, best_fill = s, fill

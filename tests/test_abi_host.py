@@ -245,11 +245,11 @@ def test_prefill_split_heuristic():
     # one sequence, 512-token chunk: 128 units on 148 SMs -> a split count that fills whole waves
     s = kvq.prefill_splits(cfg, 1, 512, 131073, 148)
     n = 128 * s
-    assert n / (-(-n // 148) * 148) >= 0.95 and 2048 // s >= 16
+    assert n / (-(-n // 148) * 148) >= 0.99 and 2048 // s >= 16
     # six sequences: 768 units (5.19 waves) -> more CTAs
     s6 = kvq.prefill_splits(cfg, 6, 512, 131073, 148)
     n6 = 768 * s6
-    assert s6 > 1 and n6 / (-(-n6 // 148) * 148) >= 0.95
+    assert s6 > 1 and n6 / (-(-n6 // 148) * 148) >= 0.99
     # short contexts are not split (each split keeps >= 16 tiles)
     assert kvq.prefill_splits(cfg, 1, 512, 1500, 148) == 1
     # no chunk tokens: nothing to split
