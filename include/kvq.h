@@ -127,7 +127,7 @@ extern "C" {
 typedef enum {
   KVQ_OK = 0,
   KVQ_ERR_INVALID_ARG = 1,   /* bad pointer, size, or configuration value   */
-  KVQ_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. d = 64)     */
+  KVQ_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. d = 96)     */
   KVQ_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed        */
   KVQ_ERR_WORKSPACE = 4,     /* decode workspace smaller than required      */
   KVQ_ERR_DEVICE_BOUNDS = 5, /* device saw a block id out of range          */
